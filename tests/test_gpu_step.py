@@ -1,0 +1,159 @@
+"""Whole denoising steps through the engine (dllm_begin_step / dllm_layer_forward /
+dllm_select_active / dllm_unmask / dllm_step) against the oracle.
+
+End-to-end trajectories of a bf16 path and an fp64 oracle part at near-tied
+confidences, so the step-level comparison is teacher-forced: the oracle runs
+the step first, the GPU step takes the oracle's selection scores, and after
+the step the oracle's tokens and confidences are written into the GPU state.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle.steps import OracleRun
+from synth import get_config, make_tokens, make_weights
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from token_skip_denoising_b200.engine import Engine
+
+DEV = "cuda"
+TINY = get_config("tiny")
+TOL_HIDDEN = 2e-2
+
+
+def _rowrel(a, b):
+    a = np.asarray(a, np.float64).reshape(len(a), -1)
+    b = np.asarray(b, np.float64).reshape(len(b), -1)
+    return float((np.abs(a - b).max(1) / np.maximum(np.abs(b).max(1), 1e-30)).max())
+
+
+@pytest.fixture(scope="module")
+def tiny_w_cpu():
+    return make_weights(TINY.model)
+
+
+def _to_dev(w):
+    return {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in w.items()}
+
+
+def _flat(b_idx, pos, N):
+    return np.asarray(b_idx) * N + np.asarray(pos)
+
+
+def _engine(cfg, w, tokens):
+    return Engine(cfg, _to_dev(w), tokens.to(DEV).contiguous())
+
+
+@pytest.mark.parametrize("cfg", [TINY, TINY.replace(batch=2), TINY.replace(policy="vanilla"),
+                                 TINY.replace(tokens_per_step=1, block_len=8)])
+def test_generation_unmasks_each_position_once(cfg, tiny_w_cpu):
+    tok0 = make_tokens(cfg)
+    eng = _engine(cfg, tiny_w_cpu, tok0)
+    seen = np.zeros((cfg.batch, cfg.seq_len), int)
+    steps = 0
+    width = cfg.tokens_per_step                     # pos_out / tok_out are [B, n] for top-n unmasking
+    pos = torch.full((cfg.batch, width), -1, dtype=torch.int32, device=DEV)
+    tk = torch.full((cfg.batch, width), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros(cfg.batch, dtype=torch.int32, device=DEV)
+    while not eng.done:
+        eng.begin_step()
+        ls = cfg.skip_layer if cfg.policy == "es" else cfg.model.n_layers
+        for l in range(cfg.model.n_layers):
+            if l == ls:
+                eng.select_active()
+            eng.layer_forward(l)
+        eng.unmask(pos, tk, cnt)
+        for b in range(cfg.batch):
+            for i in range(int(cnt[b])):
+                seen[b, int(pos[b, i])] += 1
+        steps += 1
+    tok = eng.tokens.cpu().numpy()
+    assert steps == cfg.gen_len // cfg.tokens_per_step
+    assert np.all(seen[:, cfg.prompt_len:] == 1) and np.all(seen[:, :cfg.prompt_len] == 0)
+    assert not np.any(tok == cfg.model.mask_id)
+    np.testing.assert_array_equal(tok[:, :cfg.prompt_len], tok0.numpy()[:, :cfg.prompt_len])
+
+
+def test_es_steps_match_oracle_teacher_forced(tiny_w_cpu):
+    cfg = TINY
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, tiny_w_cpu, tok0.numpy())
+    eng = _engine(cfg, tiny_w_cpu, tok0)
+    N, L, ls = cfg.seq_len, cfg.model.n_layers, cfg.skip_layer
+    kc, vc = eng.buffer("kcache"), eng.buffer("vcache")
+    hid, conf, amax = eng.buffer("hidden"), eng.buffer("conf"), eng.buffer("argmax")
+    n_skip = 0
+    while not orc.done:
+        rec = orc.step()
+        kind = eng.begin_step()
+        assert kind == ("full" if rec["kind"] == "refresh" else "skip")
+        for l in range(L):
+            if l == ls:
+                if kind == "skip":
+                    b_idx, pos = rec["cand"]
+                    # hidden state of the candidates at the skip layer (Eq. 1 input)
+                    hc = hid[torch.tensor(_flat(b_idx, pos, N), device=DEV)].cpu().numpy()
+                    assert _rowrel(hc, rec["h_skip"]) < TOL_HIDDEN
+                    forced = torch.tensor(rec["scores"], dtype=torch.float32, device=DEV)
+                    eng.select_active(forced)
+                    gpu_scores = eng.buffer("scores")[:len(rec["scores"])].cpu().numpy()
+                    # Eq. 1 on the bf16 path: the variation term differences two nearby states,
+                    # so compare against the score scale rather than element-wise
+                    assert np.abs(gpu_scores - rec["scores"]).max() <= 0.1 * np.abs(rec["scores"]).max()
+                    n_skip += 1
+                else:
+                    eng.select_active()
+            eng.layer_forward(l)
+        rows = eng.buffer("rows")
+        nrows = int(eng.buffer("nrows")[0])
+        flat = _flat(*rec["rows"], N)
+        np.testing.assert_array_equal(rows[:nrows].cpu().numpy(), flat)      # same active set, bit-exact
+        assert _rowrel(hid[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
+        eng.unmask()
+        torch.cuda.synchronize()
+        lm = flat[rec["lm_rows"]]
+        np.testing.assert_allclose(conf[torch.tensor(lm, device=DEV)].cpu().numpy(), orc.conf.reshape(-1)[lm],
+                                   rtol=5e-2, atol=1e-5)
+        # caches: every layer, every row the oracle holds
+        for l in range(L):
+            assert _rowrel(kc[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
+                           orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
+        # teacher forcing of the decisions
+        eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
+        conf.copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
+        amax.copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
+    assert n_skip == 7
+    assert eng.done
+
+
+def test_keep_all_equals_vanilla_on_gpu(tiny_w_cpu):
+    tok0 = make_tokens(TINY)
+    a = _engine(TINY.replace(keep_ratio=1.0, cand_scope="all"), tiny_w_cpu, tok0)
+    b = _engine(TINY.replace(policy="vanilla"), tiny_w_cpu, tok0)
+    a.generate()
+    b.generate()
+    torch.cuda.synchronize()
+    assert torch.equal(a.tokens, b.tokens)
+    assert torch.equal(a.buffer("kcache"), b.buffer("kcache"))
+    assert torch.equal(a.buffer("vcache"), b.buffer("vcache"))
+
+
+def test_skip_step_rewrites_only_active_rows(tiny_w_cpu):
+    cfg = TINY
+    eng = _engine(cfg, tiny_w_cpu, make_tokens(cfg))
+    eng.step()                                      # refresh
+    torch.cuda.synchronize()
+    k0, v0 = eng.buffer("kcache").clone(), eng.buffer("vcache").clone()
+    info = eng.step(info=True)                      # skip step
+    assert info["kind_name"] == "skip" and info["rows_first"] == 32 and info["rows_last"] == 8
+    act = eng.buffer("rows")[:8].cpu().numpy()
+    k1, v1 = eng.buffer("kcache"), eng.buffer("vcache")
+    ls = cfg.skip_layer
+    changed = (k1[ls:] != k0[ls:]).any(dim=-1).any(dim=0).any(dim=1)[0].cpu().numpy()   # [N]
+    assert set(np.nonzero(changed)[0]) <= set(act.tolist())
+    # the prompt is never rewritten in a skip step, at any layer
+    assert torch.equal(k1[:, :, :, :cfg.prompt_len], k0[:, :, :, :cfg.prompt_len])
+    assert torch.equal(v1[:, :, :, :cfg.prompt_len], v0[:, :, :, :cfg.prompt_len])
+    assert info["lm_rows"] <= 8

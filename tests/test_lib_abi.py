@@ -1,0 +1,78 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+and validates configurations on the host (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from synth import get_config
+from token_skip_denoising_b200 import _lib
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _lib.header_symbols()
+    assert len(declared) >= 25
+    missing = [s for s in declared if not hasattr(lib, s)]
+    assert not missing, missing
+    # and the binding declares a prototype for each of them
+    assert set(declared) <= set(_lib._SIGS)
+
+
+def test_status_strings(lib):
+    assert lib.dllm_status_string(0) == b"ok"
+    assert lib.dllm_status_string(3) == b"unsupported"
+    assert lib.dllm_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("name", ["tiny", "micro", "llada_es", "dream_surelock", "llada_cache_dus"])
+def test_state_bytes_for_every_workload(lib, name):
+    cfg = _lib.make_config(get_config(name))
+    sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb)) == 0, \
+        lib.dllm_last_error()
+    assert sb.value > 0 and wb.value > 0
+    assert sb.value < 120e9 and wb.value < 20e9      # fits beside the weights in 180 GB
+
+
+def test_state_bytes_covers_kv_cache(lib):
+    run = get_config("llada_es")
+    m = run.model
+    cfg = _lib.make_config(run)
+    sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+    lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb))
+    kv = 2 * m.n_layers * run.batch * m.n_kv_heads * run.seq_len * m.head_dim * 2
+    assert sb.value >= kv
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 96, 3), ("gen_len", 33, 2), ("n_kv_heads", 3, 2), ("mask_id", 5000, 1),
+    ("policy", 9, 1), ("keep_ratio", 0.0, 1), ("skip_layer", 99, 1), ("vocab", 1000, 3),
+])
+def test_invalid_configs_are_rejected(lib, field, value, status):
+    cfg = _lib.make_config(get_config("tiny"))
+    setattr(cfg, field, value)
+    if field == "vocab":
+        cfg.mask_id = value - 1
+    sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+    rc = lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb))
+    assert rc == status, (rc, lib.dllm_last_error())
+    assert lib.dllm_last_error()
+
+
+def test_dus_block_of_two_rejected(lib):
+    run = get_config("tiny").replace(unmask="dus", block_len=2)
+    cfg = _lib.make_config(run)
+    sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb)) == 3
+
+
+def test_null_arguments_are_rejected_without_a_gpu(lib):
+    assert lib.dllm_state_bytes(None, None, None) == 1
+    h = ctypes.c_void_p()
+    cfg = _lib.make_config(get_config("tiny"))
+    assert lib.dllm_step_init(ctypes.byref(h), ctypes.byref(cfg), None, None, None, None, None) == 1
+    assert lib.dllm_op_select(None, 1, 4, 0, 2, 0.0, 0, 4, None, None, 0, None, None, None, None) == 1

@@ -1,0 +1,101 @@
+// Shared declarations of the CUDA path: status codes, launch-side structs and
+// the host entry points of each kernel family.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+
+#include "../../include/dllm.h"
+
+namespace dllm {
+
+constexpr int kNumSMs = 148;
+
+#define DLLM_CUDA_TRY(expr)                                                   \
+  do {                                                                        \
+    cudaError_t _e = (expr);                                                  \
+    if (_e != cudaSuccess) {                                                  \
+      dllm::set_last_error(cudaGetErrorString(_e), __FILE__, __LINE__);      \
+      return DLLM_ERR_CUDA;                                                   \
+    }                                                                         \
+  } while (0)
+
+void set_last_error(const char* msg, const char* file, int line);
+
+// Kernels launched by this library in the process (reported by dllm_kernel_launches).
+extern std::atomic<int64_t> g_kernel_launches;
+inline void count_launch(int n = 1) { g_kernel_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ------------------------------------------------------------------ GEMM
+// C[j, n] = sum_k X[j, k] * W[n, k]: X holds the active rows (K-major), W the
+// weight matrix [out, in] (K-major).  One CTA computes a 128 (W rows) x BN
+// (rows of X) tile with tcgen05 into TMEM; the epilogue is fused.
+enum EpiKind : int {
+  EPI_STORE_F32 = 0,   // out_f32[j * ldo + n]
+  EPI_STORE_BF16 = 1,  // out_bf16[j * ldo + n]
+  EPI_QKV_ROPE = 2,    // RoPE on q/k, q -> q_out, k/v -> cache rows of row_map[j]
+  EPI_RESID_ADD = 3,   // h[row_map[j] * ldh + n] += C
+  EPI_SWIGLU = 4,      // act[j * F + f] = silu(gate) * up   (W tile = 64 gate + 64 up rows)
+  EPI_LMHEAD = 5,      // per (row, 128-vocab tile): max, sum exp, argmax (mask id excluded)
+};
+
+struct EpiParams {
+  int kind = EPI_STORE_F32;
+  void* out = nullptr;
+  int64_t ldo = 0;
+  // QKV + RoPE + K/V scatter
+  __nv_bfloat16* q_out = nullptr;   // [rows, q_dim]
+  __nv_bfloat16* kcache = nullptr;  // this layer: [B, Hkv, N, hd]
+  __nv_bfloat16* vcache = nullptr;
+  const int* row_map = nullptr;     // row j -> b * N + pos
+  int seq_n = 0, n_kv = 0, head_dim = 0, q_dim = 0, kv_dim = 0;
+  const float* rope_cos = nullptr;  // [N, hd/2]
+  const float* rope_sin = nullptr;
+  // residual
+  float* h = nullptr;
+  int64_t ldh = 0;
+  // SwiGLU
+  __nv_bfloat16* act = nullptr;
+  int ffn = 0;
+  // LM head partials: [rows, n_vtiles] of {max, sumexp, best value, best id}
+  float4* lm_part = nullptr;
+  int n_vtiles = 0;
+  int mask_id = -1;
+};
+
+struct GemmArgs {
+  const void* W = nullptr;       // bf16 [w_rows_total, K]
+  int64_t w_rows_total = 0;
+  const void* X = nullptr;       // bf16 [rows_cap, K]
+  int rows_cap = 0;              // host bound on the number of X rows
+  const int* rows_dev = nullptr; // device count of valid rows (nullable: rows_cap)
+  int K = 0;
+  int n_tiles_w = 0;             // 128-row output tiles (SwiGLU: F / 64)
+  bool swiglu = false;
+  EpiParams epi;
+};
+
+struct GemmScratch {
+  float* partial = nullptr;      // split-K partial tiles
+  size_t partial_floats = 0;
+  int* counters = nullptr;       // one per output tile, zero between launches
+  int n_counters = 0;
+};
+
+// Launch one fused GEMM; returns a DLLM_* status.
+int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int force_splits = 0,
+                int force_bn = 0);
+// Scratch floats a launch with these sizes needs (upper bound over tile choices).
+size_t gemm_partial_floats(int rows_cap, int n_tiles_w, int K);
+int gemm_counters_needed(int rows_cap, int n_tiles_w);
+
+// Combine LM-head partials into conf / argmax / lse per row; rows are written at
+// out_index[j] (nullable: j).
+int lmhead_combine_launch(const float4* part, int n_vtiles, int rows_cap, const int* rows_dev,
+                          const int* out_index, float* conf, int* amax, float* lse, cudaStream_t st);
+
+}  // namespace dllm

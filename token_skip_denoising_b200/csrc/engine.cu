@@ -1,0 +1,808 @@
+// The step engine behind the C ABI: validation, carving of caller memory,
+// the generation schedule and the kernel sequence of one denoising step.
+//
+// Step kinds (the pages' denoising iteration with its four row policies):
+//   FULL    every row through every layer: the vanilla step, ES-dLLM's
+//           periodic refresh (ES-dLLM summary sec. 2.2), dLLM-Cache's prompt
+//           refresh (dLLM-Cache explainer sec. 3).
+//   SKIP    ES-dLLM (sec. 2.1): the candidates run the layers below the skip
+//           layer, Eq. 1 scores them, the top k run the remaining layers.
+//   LOCKED  SureLock (sec. 2.1): the unlocked rows run every layer; locked
+//           rows keep their frozen K/V; unmasked rows are checked for locking.
+//   PARTIAL dLLM-Cache: per layer, response rows whose value vectors moved
+//           (cosine < tau, at most ceil(rho * n)) are recomputed; the rest
+//           keep their cached layer output and K/V.
+// No step synchronises the host: row counts live in device memory and the
+// schedule (block, round) is known on the host in advance.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace dllm {
+
+static thread_local std::string g_last_error;
+
+void set_last_error(const char* msg, const char* file, int line) {
+  char buf[512];
+  snprintf(buf, sizeof buf, "%s (%s:%d)", msg, file, line);
+  g_last_error = buf;
+}
+
+#define DLLM_FAIL(code, msg)                              \
+  do {                                                    \
+    dllm::set_last_error((msg), __FILE__, __LINE__);      \
+    return (code);                                        \
+  } while (0)
+
+#define DLLM_TRY(expr)             \
+  do {                             \
+    int _rc = (expr);              \
+    if (_rc != DLLM_OK) return _rc; \
+  } while (0)
+
+namespace {
+
+// Bump allocator over caller memory (256-byte aligned pieces).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+int dus_rounds_for(int block) {
+  if (block <= 1) return 1;
+  int r = 0;
+  while ((1 << r) < block) ++r;
+  return r;
+}
+
+int keep_count(float ratio, int n) {
+  if (n <= 0) return 0;
+  const double k = std::ceil(static_cast<double>(ratio) * n - 1e-9);
+  return std::max(1, std::min(n, static_cast<int>(k)));
+}
+
+int rho_cap_count(float rho, int n) {
+  if (rho >= 1.f) return n;
+  const double k = std::ceil(static_cast<double>(rho) * n - 1e-9);
+  return std::max(0, std::min(n, static_cast<int>(k)));
+}
+
+int validate(const dllm_config* c) {
+  if (!c) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null config");
+  if (c->n_layers <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+      c->ffn_dim <= 0 || c->vocab <= 1 || c->batch <= 0 || c->prompt_len < 0 || c->gen_len <= 0 ||
+      c->block_len <= 0)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "non-positive dimension");
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "mask_id outside the vocabulary");
+  if (c->gen_len % c->block_len) DLLM_FAIL(DLLM_ERR_SHAPE, "gen_len must be a multiple of block_len");
+  if (c->n_heads % c->n_kv_heads) DLLM_FAIL(DLLM_ERR_SHAPE, "n_heads must be a multiple of n_kv_heads");
+  if (c->head_dim != 64 && c->head_dim != 128) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  const int qd = c->n_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
+  if (qd % 128 || kvd % 128) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "q and kv widths must be multiples of 128");
+  if (c->d_model % 128) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "d_model must be a multiple of 128");
+  if (c->ffn_dim % 64) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "ffn_dim must be a multiple of 64");
+  if (c->vocab % 128) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "vocab must be a multiple of 128");
+  if (c->policy < DLLM_POLICY_VANILLA || c->policy > DLLM_POLICY_DLLM_CACHE)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown policy");
+  if (c->unmask != DLLM_UNMASK_TOPCONF && c->unmask != DLLM_UNMASK_DUS) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown unmask");
+  if (c->cand_scope != DLLM_SCOPE_BLOCK && c->cand_scope != DLLM_SCOPE_ALL)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown candidate scope");
+  if (c->unmask == DLLM_UNMASK_TOPCONF && c->tokens_per_step <= 0)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "tokens_per_step must be positive");
+  if (c->unmask == DLLM_UNMASK_DUS && c->block_len == 2)
+    DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "DUS: a block of 2 has no single-round non-adjacent schedule");
+  if (c->block_len > 8192) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "block_len above 8192");
+  if (c->policy == DLLM_POLICY_ES && (c->skip_layer < 0 || c->skip_layer > c->n_layers))
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "skip_layer outside [0, n_layers]");
+  if (c->policy == DLLM_POLICY_ES && !(c->keep_ratio > 0.f && c->keep_ratio <= 1.f))
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "keep_ratio must be in (0, 1]");
+  if (c->policy == DLLM_POLICY_DLLM_CACHE && c->prompt_interval <= 0)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "prompt_interval must be positive");
+  const int N = c->prompt_len + c->gen_len;
+  const int n_cand = c->cand_scope == DLLM_SCOPE_ALL ? N : c->block_len;
+  if (n_cand > 8192 || N > 65536) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "sequence too long for the selection kernel");
+  return DLLM_OK;
+}
+
+}  // namespace
+}  // namespace dllm
+
+using namespace dllm;
+
+std::atomic<int64_t> dllm::g_kernel_launches{0};
+
+// CUDA-event brackets around the fused GEMMs and the attention (roofline reporting).
+struct Prof {
+  struct Rec {
+    cudaEvent_t a, b;
+    int cls;            // 0 GEMM, 1 attention
+    double bytes, flops;
+  };
+  bool on = false;
+  double hbm_gbs = 0, tflops = 0;
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void begin(cudaStream_t st, cudaEvent_t* a) {
+    *a = nullptr;
+    if (!on) return;
+    *a = get();
+    cudaEventRecord(*a, st);
+  }
+  void end(cudaStream_t st, cudaEvent_t a, int cls, double bytes, double flops) {
+    if (!on || !a) return;
+    cudaEvent_t b = get();
+    cudaEventRecord(b, st);
+    recs.push_back({a, b, cls, bytes, flops});
+  }
+  ~Prof() {
+    for (auto& r : recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
+struct dllm_handle {
+  dllm_config c;
+  dllm_weights w;
+  int32_t* tokens;
+  int N, B, L, d, qd, kvd, qkvd, F, V, hd;
+  int n_cand, cand_start, k_keep, steps_per_block, n_rounds, n_resp, resp_start, resp_cap;
+  // state
+  __nv_bfloat16 *kcache, *vcache;
+  float *h, *h_prev, *conf, *lse, *rope_cos, *rope_sin, *hcache;
+  int* amax;
+  uint8_t *masked_prev, *lock;
+  __nv_bfloat16* zstore;   // SureLock: position-indexed bf16 logits, 2 buffers
+  float* lse_store;        // 2 x [B*N]
+  int* has_prev;           // [B*N] step + 1 at which the stored logits were written
+  // workspace
+  int *rows, *rows2, *nrows, *nrows2, *seq_off, *seq_off2, *lm_rows, *n_lm, *act_idx, *act_count;
+  float *scores, *kl;
+  uint8_t* round_masks;    // [R, block_len] (state constants)
+  size_t const_bytes = 0, state_total = 0;
+  Prof prof;
+  __nv_bfloat16 *z, *q, *attn, *act;
+  float* vnew;
+  float4* lm_part;
+  GemmScratch gs;
+  float* attn_opart;
+  float2* attn_ml;
+  size_t attn_floats;
+  // schedule
+  int block = 0, step_in_block = 0, n_steps = 0;
+  // current step
+  int kind = DLLM_STEP_FULL;
+  int cur_rows_cap = 0, cur_rows_per_seq = 0;
+  int* cur_rows = nullptr;
+  int* cur_n = nullptr;
+  int* cur_seq_off = nullptr;
+  int rows_first = 0;
+  bool began = false;
+  std::vector<uint8_t> round_host;
+};
+
+namespace {
+
+int lm_cap_of(const dllm_handle* hd) {
+  const auto& c = hd->c;
+  if (c.policy == DLLM_POLICY_SURELOCK) return hd->B * hd->N;
+  return hd->B * c.block_len;
+}
+
+// Carve state (persistent) and workspace pieces; with null bases only sizes are computed.
+void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* ws_bytes) {
+  const auto& c = x->c;
+  const int64_t BN = static_cast<int64_t>(x->B) * x->N;
+  Carver s(state);
+  // constants (kept by dllm_reset): RoPE tables and DUS round masks
+  x->rope_cos = s.take<float>(static_cast<size_t>(x->N) * x->hd / 2);
+  x->rope_sin = s.take<float>(static_cast<size_t>(x->N) * x->hd / 2);
+  x->round_masks = s.take<uint8_t>(static_cast<size_t>(x->n_rounds) * c.block_len);
+  x->const_bytes = (s.off + 255) & ~size_t(255);
+  const size_t kv = static_cast<size_t>(x->L) * x->B * c.n_kv_heads * x->N * x->hd;
+  x->kcache = s.take<__nv_bfloat16>(kv);
+  x->vcache = s.take<__nv_bfloat16>(kv);
+  x->h = s.take<float>(BN * x->d);
+  x->h_prev = c.policy == DLLM_POLICY_ES ? s.take<float>(BN * x->d) : nullptr;
+  x->conf = s.take<float>(BN);
+  x->lse = s.take<float>(BN);
+  x->amax = s.take<int>(BN);
+  x->masked_prev = s.take<uint8_t>(BN);
+  x->lock = s.take<uint8_t>(BN);
+  x->has_prev = s.take<int>(BN);
+  if (c.policy == DLLM_POLICY_SURELOCK) {
+    x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
+    x->lse_store = s.take<float>(2 * BN);
+  } else {
+    x->zstore = nullptr;
+    x->lse_store = nullptr;
+  }
+  x->hcache = c.policy == DLLM_POLICY_DLLM_CACHE ? s.take<float>(static_cast<size_t>(x->L) * BN * x->d) : nullptr;
+  x->state_total = (s.off + 255) & ~size_t(255);
+  if (state_bytes) *state_bytes = x->state_total;
+
+  Carver w(ws);
+  x->rows = w.take<int>(BN);
+  x->rows2 = w.take<int>(BN);
+  x->nrows = w.take<int>(1);
+  x->nrows2 = w.take<int>(1);
+  x->seq_off = w.take<int>(x->B + 1);
+  x->seq_off2 = w.take<int>(x->B + 1);
+  x->lm_rows = w.take<int>(BN);
+  x->n_lm = w.take<int>(1);
+  x->act_idx = w.take<int>(BN);
+  x->act_count = w.take<int>(x->B);
+  x->scores = w.take<float>(BN);
+  x->kl = w.take<float>(BN);
+  const int64_t R = BN;   // row bound of any step
+  x->z = w.take<__nv_bfloat16>(R * x->d);
+  x->q = w.take<__nv_bfloat16>(R * x->qd);
+  x->attn = w.take<__nv_bfloat16>(R * x->qd);
+  x->act = w.take<__nv_bfloat16>(R * x->F);
+  x->vnew = c.policy == DLLM_POLICY_DLLM_CACHE ? w.take<float>(static_cast<size_t>(x->B) * x->n_resp * x->kvd) : nullptr;
+  const int lm_cap = lm_cap_of(x);
+  x->lm_part = w.take<float4>(static_cast<size_t>(lm_cap) * (x->V / 128));
+  // split-K scratch: the largest need over the row counts a step can use
+  std::vector<int> caps = {static_cast<int>(BN), x->B * x->n_cand, x->B * x->k_keep, x->B * x->n_resp, lm_cap};
+  size_t pf = 0;
+  int ctr = 0;
+  for (int cap : caps) {
+    if (cap <= 0) continue;
+    const int tiles[5] = {x->qkvd / 128, x->d / 128, x->F / 64, x->kvd / 128, x->V / 128};
+    const int Ks[5] = {x->d, x->qd, x->d, x->d, x->d};
+    for (int i = 0; i < 5; ++i) {
+      pf = std::max(pf, gemm_partial_floats(cap, tiles[i], Ks[i]));
+      ctr = std::max(ctr, gemm_counters_needed(cap, tiles[i]));
+    }
+    pf = std::max(pf, gemm_partial_floats(cap, x->d / 128, x->F));
+  }
+  x->gs.partial = w.take<float>(pf);
+  x->gs.partial_floats = pf;
+  x->gs.counters = w.take<int>(ctr);
+  x->gs.n_counters = ctr;
+  size_t af = 0;
+  const int G = c.n_heads / c.n_kv_heads;
+  for (int cap_seq : {x->N, x->n_cand, x->k_keep, x->n_resp}) {
+    if (cap_seq <= 0) continue;
+    const int sp = attn_pick_splits(x->B, c.n_kv_heads, G, cap_seq, x->N);
+    if (sp > 1) af = std::max(af, attn_partial_floats(x->B * cap_seq, c.n_heads, x->hd, sp));
+  }
+  x->attn_opart = w.take<float>(af);
+  x->attn_floats = af;
+  size_t ml = af / std::max(1, x->hd);
+  x->attn_ml = w.take<float2>(ml);
+  if (ws_bytes) *ws_bytes = (w.off + 255) & ~size_t(255);
+}
+
+void fill_dims(dllm_handle* x, const dllm_config* c) {
+  x->c = *c;
+  x->N = c->prompt_len + c->gen_len;
+  x->B = c->batch;
+  x->L = c->n_layers;
+  x->d = c->d_model;
+  x->hd = c->head_dim;
+  x->qd = c->n_heads * c->head_dim;
+  x->kvd = c->n_kv_heads * c->head_dim;
+  x->qkvd = x->qd + 2 * x->kvd;
+  x->F = c->ffn_dim;
+  x->V = c->vocab;
+  x->cand_start = c->cand_scope == DLLM_SCOPE_ALL ? 0 : c->prompt_len;   // plus block offset at run time
+  x->n_cand = c->cand_scope == DLLM_SCOPE_ALL ? x->N : c->block_len;
+  x->k_keep = c->policy == DLLM_POLICY_ES ? keep_count(c->keep_ratio, x->n_cand) : x->n_cand;
+  x->n_rounds = dus_rounds_for(c->block_len);
+  x->steps_per_block = c->unmask == DLLM_UNMASK_DUS ? x->n_rounds : ceil_div(c->block_len, c->tokens_per_step);
+  x->resp_start = c->cand_scope == DLLM_SCOPE_ALL ? 0 : c->prompt_len;
+  x->n_resp = x->N - x->resp_start;
+  x->resp_cap = rho_cap_count(c->rho_cap, x->n_resp);
+}
+
+int blk_start(const dllm_handle* x) { return x->c.prompt_len + x->block * x->c.block_len; }
+
+int cand_first(const dllm_handle* x) {
+  return x->c.cand_scope == DLLM_SCOPE_ALL ? 0 : blk_start(x);
+}
+
+// Everything one transformer layer needs (weights of the layer, its caches, scratch).
+struct LayerCtx {
+  int B, N, d, qd, kvd, qkvd, F, hd, Hq, Hkv;
+  float eps;
+  const __nv_bfloat16 *Wqkv, *Wo, *Wgu, *Wdn;
+  const float *g_attn, *g_ffn;
+  __nv_bfloat16 *kc, *vc;
+  const float *rope_cos, *rope_sin;
+  __nv_bfloat16 *z, *q, *attn, *act;
+  GemmScratch gs;
+  float* attn_opart;
+  float2* attn_ml;
+  size_t attn_floats;
+  Prof* prof = nullptr;
+};
+
+// GEMM launch with optional event bracketing; bytes / flops are the algorithmic figures
+// (weights + activation rows + outputs) for rows_cap rows.
+int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_t st, double out_bytes_per_row) {
+  cudaEvent_t a = nullptr;
+  if (prof) prof->begin(st, &a);
+  const int rc = gemm_launch(g, gs, st);
+  if (prof && prof->on) {
+    const double wrows = g.swiglu ? 2.0 * g.epi.ffn : 128.0 * g.n_tiles_w;
+    const double bytes = wrows * g.K * 2.0 + static_cast<double>(g.rows_cap) * (g.K * 2.0 + out_bytes_per_row);
+    prof->end(st, a, 0, bytes, 2.0 * g.rows_cap * wrows * g.K);
+  }
+  return rc;
+}
+
+// One transformer layer on rows[j] (j < *n) of the position-indexed hidden buffer hbuf:
+// RMSNorm gather -> QKV (+RoPE, K/V scatter) -> attention over all cached keys ->
+// O (+residual) -> RMSNorm -> gate/up (+SwiGLU) -> down (+residual).
+int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, const int* seq_off, int rows_cap,
+              int rows_per_seq, cudaStream_t st) {
+  DLLM_TRY(rmsnorm_rows_launch(hbuf, rows, n, rows_cap, x.d, x.g_attn, x.eps, x.z, x.d, st));
+  GemmArgs g;
+  g.W = x.Wqkv; g.w_rows_total = x.qkvd; g.X = x.z; g.rows_cap = rows_cap; g.rows_dev = n; g.K = x.d;
+  g.n_tiles_w = x.qkvd / 128;
+  g.epi.kind = EPI_QKV_ROPE; g.epi.q_out = x.q; g.epi.kcache = x.kc; g.epi.vcache = x.vc; g.epi.row_map = rows;
+  g.epi.seq_n = x.N; g.epi.n_kv = x.Hkv; g.epi.head_dim = x.hd; g.epi.q_dim = x.qd; g.epi.kv_dim = x.kvd;
+  g.epi.rope_cos = x.rope_cos; g.epi.rope_sin = x.rope_sin;
+  DLLM_TRY(timed_gemm(x.prof, g, x.gs, st, 2.0 * x.qkvd));
+  {
+    cudaEvent_t a = nullptr;
+    if (x.prof) x.prof->begin(st, &a);
+    DLLM_TRY(attn_launch(x.q, x.kc, x.vc, x.attn, seq_off, x.B, rows_cap, rows_per_seq, x.N, x.Hq, x.Hkv, x.hd, 0,
+                         x.attn_opart, x.attn_ml, x.attn_floats, st));
+    if (x.prof && x.prof->on) {
+      const double kvb = 2.0 * x.B * x.Hkv * static_cast<double>(x.N) * x.hd * 2.0;
+      x.prof->end(st, a, 1, kvb + 4.0 * rows_cap * x.qd, 4.0 * rows_cap * x.Hq * static_cast<double>(x.N) * x.hd);
+    }
+  }
+  GemmArgs o;
+  o.W = x.Wo; o.w_rows_total = x.d; o.X = x.attn; o.rows_cap = rows_cap; o.rows_dev = n; o.K = x.qd;
+  o.n_tiles_w = x.d / 128;
+  o.epi.kind = EPI_RESID_ADD; o.epi.h = hbuf; o.epi.ldh = x.d; o.epi.row_map = rows;
+  DLLM_TRY(timed_gemm(x.prof, o, x.gs, st, 8.0 * x.d));
+  DLLM_TRY(rmsnorm_rows_launch(hbuf, rows, n, rows_cap, x.d, x.g_ffn, x.eps, x.z, x.d, st));
+  GemmArgs gu;
+  gu.W = x.Wgu; gu.w_rows_total = 2 * x.F; gu.X = x.z; gu.rows_cap = rows_cap; gu.rows_dev = n; gu.K = x.d;
+  gu.n_tiles_w = x.F / 64; gu.swiglu = true;
+  gu.epi.kind = EPI_SWIGLU; gu.epi.act = x.act; gu.epi.ffn = x.F;
+  DLLM_TRY(timed_gemm(x.prof, gu, x.gs, st, 2.0 * x.F));
+  GemmArgs dn;
+  dn.W = x.Wdn; dn.w_rows_total = x.d; dn.X = x.act; dn.rows_cap = rows_cap; dn.rows_dev = n; dn.K = x.F;
+  dn.n_tiles_w = x.d / 128;
+  dn.epi.kind = EPI_RESID_ADD; dn.epi.h = hbuf; dn.epi.ldh = x.d; dn.epi.row_map = rows;
+  DLLM_TRY(timed_gemm(x.prof, dn, x.gs, st, 8.0 * x.d));
+  return DLLM_OK;
+}
+
+LayerCtx layer_ctx(const dllm_handle* x, int l) {
+  LayerCtx L;
+  const auto& c = x->c;
+  L.B = x->B; L.N = x->N; L.d = x->d; L.qd = x->qd; L.kvd = x->kvd; L.qkvd = x->qkvd; L.F = x->F; L.hd = x->hd;
+  L.Hq = c.n_heads; L.Hkv = c.n_kv_heads; L.eps = c.rms_eps;
+  L.Wqkv = static_cast<const __nv_bfloat16*>(x->w.w_qkv) + static_cast<size_t>(l) * x->qkvd * x->d;
+  L.Wo = static_cast<const __nv_bfloat16*>(x->w.w_o) + static_cast<size_t>(l) * x->d * x->qd;
+  L.Wgu = static_cast<const __nv_bfloat16*>(x->w.w_gu) + static_cast<size_t>(l) * 2 * x->F * x->d;
+  L.Wdn = static_cast<const __nv_bfloat16*>(x->w.w_down) + static_cast<size_t>(l) * x->d * x->F;
+  L.g_attn = x->w.g_attn + static_cast<size_t>(l) * x->d;
+  L.g_ffn = x->w.g_ffn + static_cast<size_t>(l) * x->d;
+  const size_t kvl = static_cast<size_t>(x->B) * c.n_kv_heads * x->N * x->hd;
+  L.kc = x->kcache + l * kvl;
+  L.vc = x->vcache + l * kvl;
+  L.rope_cos = x->rope_cos; L.rope_sin = x->rope_sin;
+  L.z = x->z; L.q = x->q; L.attn = x->attn; L.act = x->act;
+  L.gs = x->gs;
+  L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
+  L.prof = const_cast<Prof*>(&x->prof);
+  return L;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* dllm_status_string(int s) {
+  switch (s) {
+    case DLLM_OK: return "ok";
+    case DLLM_ERR_INVALID_ARG: return "invalid argument";
+    case DLLM_ERR_SHAPE: return "shape mismatch";
+    case DLLM_ERR_UNSUPPORTED: return "unsupported";
+    case DLLM_ERR_CUDA: return "CUDA error";
+    case DLLM_ERR_TIMEOUT: return "device wait timed out";
+    case DLLM_ERR_DEVICE: return "device status set";
+    case DLLM_ERR_STATE: return "call out of order";
+    default: return "unknown status";
+  }
+}
+
+const char* dllm_last_error(void) { return g_last_error.c_str(); }
+
+int dllm_state_bytes(const dllm_config* cfg, size_t* state_bytes, size_t* workspace_bytes) {
+  DLLM_TRY(validate(cfg));
+  dllm_handle x{};
+  fill_dims(&x, cfg);
+  carve(&x, nullptr, nullptr, state_bytes, workspace_bytes);
+  return DLLM_OK;
+}
+
+int dllm_step_init(dllm_handle** out, const dllm_config* cfg, const dllm_weights* w, void* state, void* workspace,
+                   int32_t* tokens, void* stream) {
+  if (!out || !w || !state || !workspace || !tokens) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  DLLM_TRY(validate(cfg));
+  if (!w->embed || !w->lm_head || !w->w_qkv || !w->w_o || !w->w_gu || !w->w_down || !w->g_attn || !w->g_ffn ||
+      !w->g_final)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null weight pointer");
+  if ((reinterpret_cast<uintptr_t>(state) | reinterpret_cast<uintptr_t>(workspace)) & 255)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "state and workspace must be 256-byte aligned");
+  dllm_handle* x = new (std::nothrow) dllm_handle();
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "out of host memory");
+  fill_dims(x, cfg);
+  x->w = *w;
+  x->tokens = tokens;
+  size_t sb = 0, wb = 0;
+  carve(x, state, workspace, &sb, &wb);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto fail = [&](int rc) { delete x; return rc; };
+  if (cudaMemsetAsync(state, 0, sb, st) != cudaSuccess) { set_last_error("memset state", __FILE__, __LINE__); return fail(DLLM_ERR_CUDA); }
+  if (cudaMemsetAsync(workspace, 0, wb, st) != cudaSuccess) { set_last_error("memset workspace", __FILE__, __LINE__); return fail(DLLM_ERR_CUDA); }
+  int rc = rope_table_launch(x->rope_cos, x->rope_sin, x->N, x->hd, cfg->rope_theta, st);
+  if (rc) return fail(rc);
+  // DUS round masks: round r takes positions divisible by 2^(R-1-r) not taken earlier
+  x->round_host.assign(static_cast<size_t>(x->n_rounds) * cfg->block_len, 0);
+  std::vector<uint8_t> taken(cfg->block_len, 0);
+  for (int r = 0; r < x->n_rounds; ++r) {
+    const int stride = 1 << (x->n_rounds - 1 - r);
+    for (int p = 0; p < cfg->block_len; ++p)
+      if (p % stride == 0 && !taken[p]) { taken[p] = 1; x->round_host[static_cast<size_t>(r) * cfg->block_len + p] = 1; }
+  }
+  if (cudaMemcpyAsync(x->round_masks, x->round_host.data(), x->round_host.size(), cudaMemcpyHostToDevice, st) !=
+      cudaSuccess) { set_last_error("round masks", __FILE__, __LINE__); return fail(DLLM_ERR_CUDA); }
+  // the host vector must outlive the copy
+  if (cudaStreamSynchronize(st) != cudaSuccess) { set_last_error("init sync", __FILE__, __LINE__); return fail(DLLM_ERR_CUDA); }
+  *out = x;
+  return DLLM_OK;
+}
+
+int dllm_done(const dllm_handle* h) { return (!h || h->block >= h->c.gen_len / h->c.block_len) ? 1 : 0; }
+
+int dllm_begin_step(dllm_handle* x, int32_t* kind_out, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (dllm_done(x)) DLLM_FAIL(DLLM_ERR_STATE, "generation finished");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto& c = x->c;
+  const int BN = x->B * x->N;
+  int kind = DLLM_STEP_FULL;
+  switch (c.policy) {
+    case DLLM_POLICY_VANILLA: kind = DLLM_STEP_FULL; break;
+    case DLLM_POLICY_ES: {
+      const bool refresh = x->step_in_block == 0 || (c.refresh_period > 0 && x->step_in_block % c.refresh_period == 0);
+      kind = refresh ? DLLM_STEP_FULL : DLLM_STEP_SKIP;
+      break;
+    }
+    case DLLM_POLICY_SURELOCK: kind = DLLM_STEP_LOCKED; break;
+    case DLLM_POLICY_DLLM_CACHE: kind = (x->n_steps % c.prompt_interval == 0) ? DLLM_STEP_FULL : DLLM_STEP_PARTIAL; break;
+  }
+  x->kind = kind;
+  if (kind == DLLM_STEP_FULL) {
+    DLLM_TRY(range_rows_launch(x->B, x->N, 0, x->N, x->rows, x->seq_off, x->nrows, st));
+    x->cur_rows_cap = BN;
+    x->cur_rows_per_seq = x->N;
+  } else if (kind == DLLM_STEP_SKIP) {
+    DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->n_cand, x->rows, x->seq_off, x->nrows, st));
+    x->cur_rows_cap = x->B * x->n_cand;
+    x->cur_rows_per_seq = x->n_cand;
+  } else if (kind == DLLM_STEP_LOCKED) {
+    SelectParams sp;
+    sp.B = x->B; sp.n = x->N; sp.mode = SEL_ALL_ELIGIBLE; sp.cand_start = 0; sp.seq_n = x->N; sp.lock = x->lock;
+    sp.row_map = x->rows; sp.seq_off = x->seq_off; sp.total = x->nrows;
+    DLLM_TRY(select_launch(sp, st));
+    x->cur_rows_cap = BN;
+    x->cur_rows_per_seq = x->N;
+  } else {   // PARTIAL: the response rows enter layer 0
+    DLLM_TRY(range_rows_launch(x->B, x->N, x->resp_start, x->n_resp, x->rows, x->seq_off, x->nrows, st));
+    x->cur_rows_cap = x->B * x->n_resp;
+    x->cur_rows_per_seq = x->n_resp;
+  }
+  x->cur_rows = x->rows;
+  x->cur_n = x->nrows;
+  x->cur_seq_off = x->seq_off;
+  x->rows_first = x->cur_rows_cap;
+  DLLM_TRY(embed_rows_launch(static_cast<const __nv_bfloat16*>(x->w.embed), x->tokens, x->rows, x->nrows,
+                             x->cur_rows_cap, x->d, x->h, st));
+  x->began = true;
+  if (kind_out) *kind_out = kind;
+  return DLLM_OK;
+}
+
+int dllm_layer_forward(dllm_handle* x, int32_t layer, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "layer_forward before begin_step");
+  if (layer < 0 || layer >= x->L) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "layer out of range");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto& c = x->c;
+  const int64_t BNd = static_cast<int64_t>(x->B) * x->N * x->d;
+  if (c.policy == DLLM_POLICY_DLLM_CACHE) {
+    float* out_l = x->hcache + layer * BNd;
+    if (x->kind == DLLM_STEP_FULL) {
+      DLLM_TRY(run_layer(layer_ctx(x, layer), x->h, x->cur_rows, x->cur_n, x->cur_seq_off, x->cur_rows_cap,
+                         x->cur_rows_per_seq, st));
+      DLLM_CUDA_TRY(cudaMemcpyAsync(out_l, x->h, BNd * sizeof(float), cudaMemcpyDeviceToDevice, st));
+      return DLLM_OK;
+    }
+    return DLLM_ERR_UNSUPPORTED;   // partial response updates: see dllm_cache_layer below
+  }
+  return run_layer(layer_ctx(x, layer), x->h, x->cur_rows, x->cur_n, x->cur_seq_off, x->cur_rows_cap,
+                   x->cur_rows_per_seq, st);
+}
+
+int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* active_idx, int32_t* active_count,
+                       void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "select_active before begin_step");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto& c = x->c;
+  if (c.policy != DLLM_POLICY_ES) return DLLM_OK;
+  const int mask = c.mask_id;
+  if (x->kind == DLLM_STEP_FULL) {
+    // refresh: snapshot the candidates' hidden state at the skip layer
+    DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->n_cand, x->rows2, x->seq_off2, x->nrows2, st));
+    DLLM_TRY(snapshot_rows_launch(x->h, x->h_prev, x->tokens, x->masked_prev, mask, x->rows2, x->B * x->n_cand, x->d, st));
+    return DLLM_OK;
+  }
+  if (x->kind != DLLM_STEP_SKIP) DLLM_FAIL(DLLM_ERR_STATE, "select_active outside an ES step");
+  // Eq. 1 (always evaluated: it also rolls h_prev and masked_prev forward)
+  DLLM_TRY(score_es_launch(x->h, x->h_prev, x->conf, x->masked_prev, x->tokens, mask, x->rows, x->B * x->n_cand, x->d,
+                           c.alpha, 1, x->scores, st));
+  SelectParams sp;
+  sp.scores = scores_or_null ? scores_or_null : x->scores;
+  sp.B = x->B; sp.n = x->n_cand; sp.mode = SEL_TOPK_DESC; sp.k = x->k_keep; sp.cand_start = cand_first(x);
+  sp.seq_n = x->N; sp.act_pos = active_idx ? active_idx : x->act_idx; sp.k_max = x->k_keep;
+  sp.count = active_count ? active_count : x->act_count; sp.row_map = x->rows2; sp.seq_off = x->seq_off2;
+  sp.total = x->nrows2;
+  DLLM_TRY(select_launch(sp, st));
+  x->cur_rows = x->rows2;
+  x->cur_n = x->nrows2;
+  x->cur_seq_off = x->seq_off2;
+  x->cur_rows_cap = x->B * x->k_keep;
+  x->cur_rows_per_seq = x->k_keep;
+  return DLLM_OK;
+}
+
+int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "unmask before begin_step");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto& c = x->c;
+  const int bs = blk_start(x);
+  const uint8_t* rmask = nullptr;
+  if (c.unmask == DLLM_UNMASK_DUS)
+    rmask = x->round_masks + static_cast<size_t>(std::min(x->step_in_block, x->n_rounds - 1)) * c.block_len;
+  const float* hsrc = (c.policy == DLLM_POLICY_DLLM_CACHE) ? x->hcache + static_cast<int64_t>(x->L - 1) * x->B * x->N * x->d
+                                                          : x->h;
+  const int lm_cap = std::min(lm_cap_of(x), x->cur_rows_cap);
+  DLLM_TRY(lm_rows_launch(x->cur_rows, x->cur_n, x->cur_rows_cap, x->tokens, c.mask_id, x->N, bs, bs + c.block_len,
+                          rmask, x->lm_rows, x->n_lm, st));
+  DLLM_TRY(rmsnorm_rows_launch(hsrc, x->lm_rows, x->n_lm, lm_cap, x->d, x->w.g_final, c.rms_eps, x->z, x->d, st));
+  GemmArgs g;
+  g.W = x->w.lm_head; g.w_rows_total = x->V; g.X = x->z; g.rows_cap = lm_cap; g.rows_dev = x->n_lm; g.K = x->d;
+  g.n_tiles_w = x->V / 128;
+  g.epi.kind = EPI_LMHEAD; g.epi.lm_part = x->lm_part; g.epi.n_vtiles = x->V / 128; g.epi.mask_id = c.mask_id;
+  DLLM_TRY(timed_gemm(&x->prof, g, x->gs, st, 16.0 * (x->V / 128)));
+  DLLM_TRY(lmhead_combine_launch(x->lm_part, x->V / 128, lm_cap, x->n_lm, x->lm_rows, x->conf, x->amax, x->lse, st));
+  const int max_out = c.unmask == DLLM_UNMASK_DUS ? c.block_len : c.tokens_per_step;
+  DLLM_TRY(unmask_launch(x->tokens, x->conf, x->amax, x->B, x->N, bs, c.block_len, c.mask_id, c.tokens_per_step, rmask,
+                         pos_out, tok_out, n_out, max_out, st));
+  // schedule
+  x->n_steps += 1;
+  x->step_in_block += 1;
+  if (x->step_in_block >= x->steps_per_block) {
+    x->block += 1;
+    x->step_in_block = 0;
+  }
+  x->began = false;
+  return DLLM_OK;
+}
+
+int dllm_step(dllm_handle* x, dllm_step_info* info, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  const int step = x->n_steps, block = x->block, sib = x->step_in_block;
+  int32_t kind = 0;
+  DLLM_TRY(dllm_begin_step(x, &kind, stream));
+  const auto& c = x->c;
+  const int ls = c.policy == DLLM_POLICY_ES ? c.skip_layer : x->L;
+  for (int l = 0; l < x->L; ++l) {
+    if (l == ls) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+    DLLM_TRY(dllm_layer_forward(x, l, stream));
+  }
+  if (ls == x->L && c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+  DLLM_TRY(dllm_unmask(x, nullptr, nullptr, nullptr, stream));
+  if (info) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DLLM_CUDA_TRY(cudaStreamSynchronize(st));
+    int nl = 0, nlm = 0;
+    DLLM_CUDA_TRY(cudaMemcpy(&nl, x->cur_n, sizeof(int), cudaMemcpyDeviceToHost));
+    DLLM_CUDA_TRY(cudaMemcpy(&nlm, x->n_lm, sizeof(int), cudaMemcpyDeviceToHost));
+    info->kind = kind;
+    info->step = step;
+    info->block = block;
+    info->step_in_block = sib;
+    info->rows_first = x->rows_first;
+    info->rows_last = nl;
+    info->lm_rows = nlm;
+    info->n_locked = 0;
+    info->done = dllm_done(x);
+  }
+  return DLLM_OK;
+}
+
+int dllm_get_buffer(dllm_handle* x, int32_t which, void** ptr, size_t* bytes) {
+  if (!x || !ptr) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  const size_t BN = static_cast<size_t>(x->B) * x->N;
+  const size_t kv = static_cast<size_t>(x->L) * x->B * x->c.n_kv_heads * x->N * x->hd;
+  void* p = nullptr;
+  size_t b = 0;
+  switch (which) {
+    case DLLM_BUF_KCACHE: p = x->kcache; b = kv * 2; break;
+    case DLLM_BUF_VCACHE: p = x->vcache; b = kv * 2; break;
+    case DLLM_BUF_HIDDEN: p = x->h; b = BN * x->d * 4; break;
+    case DLLM_BUF_HPREV: p = x->h_prev; b = x->h_prev ? BN * x->d * 4 : 0; break;
+    case DLLM_BUF_CONF: p = x->conf; b = BN * 4; break;
+    case DLLM_BUF_ARGMAX: p = x->amax; b = BN * 4; break;
+    case DLLM_BUF_ROWS: p = x->cur_rows ? x->cur_rows : x->rows; b = BN * 4; break;
+    case DLLM_BUF_NROWS: p = x->cur_n ? x->cur_n : x->nrows; b = 4; break;
+    case DLLM_BUF_SCORES: p = x->scores; b = BN * 4; break;
+    case DLLM_BUF_LOCK: p = x->lock; b = BN; break;
+    case DLLM_BUF_MASKED_PREV: p = x->masked_prev; b = BN; break;
+    case DLLM_BUF_LMROWS: p = x->lm_rows; b = BN * 4; break;
+    case DLLM_BUF_NLMROWS: p = x->n_lm; b = 4; break;
+    case DLLM_BUF_KL: p = x->kl; b = BN * 4; break;
+    case DLLM_BUF_HCACHE: p = x->hcache; b = x->hcache ? static_cast<size_t>(x->L) * BN * x->d * 4 : 0; break;
+    case DLLM_BUF_LSE: p = x->lse; b = BN * 4; break;
+    default: DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown buffer");
+  }
+  *ptr = p;
+  if (bytes) *bytes = b;
+  return DLLM_OK;
+}
+
+void dllm_destroy(dllm_handle* x) { delete x; }
+
+int dllm_reset(dllm_handle* x, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(x->rope_cos);
+  DLLM_CUDA_TRY(cudaMemsetAsync(base + x->const_bytes, 0, x->state_total - x->const_bytes, st));
+  x->block = 0;
+  x->step_in_block = 0;
+  x->n_steps = 0;
+  x->began = false;
+  return DLLM_OK;
+}
+
+int dllm_profile_enable(dllm_handle* x, int32_t enable, double hbm_gbs, double tensor_tflops) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  x->prof.on = enable != 0;
+  x->prof.hbm_gbs = hbm_gbs;
+  x->prof.tflops = tensor_tflops;
+  return DLLM_OK;
+}
+
+int dllm_profile_read(dllm_handle* x, dllm_profile* out) {
+  if (!x || !out) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  std::memset(out, 0, sizeof(*out));
+  for (auto& r : x->prof.recs) {
+    DLLM_CUDA_TRY(cudaEventSynchronize(r.b));
+    float ms = 0.f;
+    DLLM_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    if (r.cls == 0) {
+      out->gemm_launches += 1;
+      out->gemm_ms += ms;
+      out->gemm_bytes += r.bytes;
+      out->gemm_flops += r.flops;
+      if (x->prof.hbm_gbs > 0 && x->prof.tflops > 0)
+        out->gemm_roofline_ms += std::max(r.bytes / (x->prof.hbm_gbs * 1e6), r.flops / (x->prof.tflops * 1e9));
+    } else {
+      out->attn_launches += 1;
+      out->attn_ms += ms;
+      out->attn_bytes += r.bytes;
+      out->attn_flops += r.flops;
+    }
+    x->prof.pool.push_back(r.a);
+    x->prof.pool.push_back(r.b);
+  }
+  x->prof.recs.clear();
+  return DLLM_OK;
+}
+
+int64_t dllm_kernel_launches(void) { return dllm::g_kernel_launches.load(); }
+
+int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t rows_per_seq_cap, size_t* bytes) {
+  if (!cfg || !bytes || rows_cap <= 0) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "bad layer workspace args");
+  const int d = cfg->d_model, qd = cfg->n_heads * cfg->head_dim, kvd = cfg->n_kv_heads * cfg->head_dim;
+  const int qkvd = qd + 2 * kvd, F = cfg->ffn_dim;
+  Carver w(nullptr);
+  w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * d);
+  w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
+  w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
+  w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * F);
+  size_t pf = std::max({gemm_partial_floats(rows_cap, qkvd / 128, d), gemm_partial_floats(rows_cap, d / 128, qd),
+                        gemm_partial_floats(rows_cap, F / 64, d), gemm_partial_floats(rows_cap, d / 128, F)});
+  int ctr = std::max({gemm_counters_needed(rows_cap, qkvd / 128), gemm_counters_needed(rows_cap, d / 128),
+                      gemm_counters_needed(rows_cap, F / 64)});
+  w.take<float>(pf);
+  w.take<int>(ctr);
+  const int B = cfg->batch, N = cfg->prompt_len + cfg->gen_len;
+  const int sp = attn_pick_splits(B, cfg->n_kv_heads, cfg->n_heads / cfg->n_kv_heads, rows_per_seq_cap, N);
+  const size_t af = sp > 1 ? attn_partial_floats(rows_cap, cfg->n_heads, cfg->head_dim, sp) : 0;
+  w.take<float>(af);
+  w.take<float2>(af / cfg->head_dim);
+  *bytes = (w.off + 255) & ~size_t(255);
+  return DLLM_OK;
+}
+
+int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, const void* w_gu, const void* w_down,
+                  const float* g_attn, const float* g_ffn, void* kcache, void* vcache, const float* rope_cos,
+                  const float* rope_sin, float* h, const int32_t* rows, const int32_t* count, const int32_t* seq_off,
+                  int32_t rows_cap, int32_t rows_per_seq_cap, void* workspace, size_t workspace_bytes, void* stream) {
+  DLLM_TRY(validate(cfg));
+  if (!w_qkv || !w_o || !w_gu || !w_down || !g_attn || !g_ffn || !kcache || !vcache || !rope_cos || !rope_sin || !h ||
+      !rows || !seq_off || !workspace)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  size_t need = 0;
+  DLLM_TRY(dllm_op_layer_workspace(cfg, rows_cap, rows_per_seq_cap, &need));
+  if (workspace_bytes < need) DLLM_FAIL(DLLM_ERR_SHAPE, "workspace too small for the layer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LayerCtx L;
+  L.B = cfg->batch; L.N = cfg->prompt_len + cfg->gen_len; L.d = cfg->d_model; L.hd = cfg->head_dim;
+  L.Hq = cfg->n_heads; L.Hkv = cfg->n_kv_heads; L.qd = L.Hq * L.hd; L.kvd = L.Hkv * L.hd; L.qkvd = L.qd + 2 * L.kvd;
+  L.F = cfg->ffn_dim; L.eps = cfg->rms_eps;
+  L.Wqkv = static_cast<const __nv_bfloat16*>(w_qkv); L.Wo = static_cast<const __nv_bfloat16*>(w_o);
+  L.Wgu = static_cast<const __nv_bfloat16*>(w_gu); L.Wdn = static_cast<const __nv_bfloat16*>(w_down);
+  L.g_attn = g_attn; L.g_ffn = g_ffn;
+  L.kc = static_cast<__nv_bfloat16*>(kcache); L.vc = static_cast<__nv_bfloat16*>(vcache);
+  L.rope_cos = rope_cos; L.rope_sin = rope_sin;
+  Carver w(workspace);
+  L.z = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.d);
+  L.q = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
+  L.attn = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
+  L.act = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.F);
+  size_t pf = std::max({gemm_partial_floats(rows_cap, L.qkvd / 128, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.qd),
+                        gemm_partial_floats(rows_cap, L.F / 64, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.F)});
+  int ctr = std::max({gemm_counters_needed(rows_cap, L.qkvd / 128), gemm_counters_needed(rows_cap, L.d / 128),
+                      gemm_counters_needed(rows_cap, L.F / 64)});
+  L.gs.partial = w.take<float>(pf);
+  L.gs.partial_floats = pf;
+  L.gs.counters = w.take<int>(ctr);
+  L.gs.n_counters = ctr;
+  const int sp = attn_pick_splits(L.B, L.Hkv, L.Hq / L.Hkv, rows_per_seq_cap, L.N);
+  L.attn_floats = sp > 1 ? attn_partial_floats(rows_cap, L.Hq, L.hd, sp) : 0;
+  L.attn_opart = w.take<float>(L.attn_floats);
+  L.attn_ml = w.take<float2>(L.attn_floats / L.hd);
+  if (ctr) DLLM_CUDA_TRY(cudaMemsetAsync(L.gs.counters, 0, ctr * sizeof(int), st));
+  return run_layer(L, h, rows, count, seq_off, rows_cap, rows_per_seq_cap, st);
+}
+
+}  // extern "C"

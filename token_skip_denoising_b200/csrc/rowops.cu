@@ -1,0 +1,610 @@
+// Row-wise kernels of the step: embedding gather, RMSNorm gather, the three
+// row scores (ES-dLLM Eq. 1, SureLock KL, dLLM-Cache cosine), radix top-k /
+// threshold selection with compaction, vocabulary-row lists and unmasking.
+// All of them are HBM- or latency-bound; none is a contraction.
+#include <algorithm>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace dllm {
+namespace {
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------ RoPE table
+__global__ void rope_table_kernel(float* cos_t, float* sin_t, int N, int half, double theta, int hd) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= N * half) return;
+  const int pos = idx / half, i = idx % half;
+  const double inv = pow(theta, -2.0 * i / static_cast<double>(hd));
+  const double ang = static_cast<double>(pos) * inv;
+  double s, c;
+  sincos(ang, &s, &c);
+  cos_t[idx] = static_cast<float>(c);
+  sin_t[idx] = static_cast<float>(s);
+}
+
+// ------------------------------------------------------------------ embedding
+// h[row_map[j]] = E[tokens[row_map[j]]] (bf16 -> fp32), j < count
+__global__ void embed_rows_kernel(const __nv_bfloat16* __restrict__ E, const int* __restrict__ tokens,
+                                  const int* __restrict__ row_map, const int* count_dev, int rows_cap, int d,
+                                  float* __restrict__ h) {
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int j = blockIdx.x;
+  if (j >= m) return;
+  const int flat = row_map[j];
+  const int tok = tokens[flat];
+  const __nv_bfloat16* src = E + static_cast<int64_t>(tok) * d;
+  float* dst = h + static_cast<int64_t>(flat) * d;
+  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float4 a, b;
+    float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+    float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+    a = make_float4(f0.x, f0.y, f1.x, f1.y);
+    b = make_float4(f2.x, f2.y, f3.x, f3.y);
+    *reinterpret_cast<float4*>(dst + i) = a;
+    *reinterpret_cast<float4*>(dst + i + 4) = b;
+  }
+}
+
+// ------------------------------------------------------------------ RMSNorm gather
+// z[j] = bf16(h[src(j)] / sqrt(mean(h^2) + eps) * g); src(j) = row_map[j] (or j).
+// One CTA of 256 threads per row.
+__global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int* __restrict__ row_map,
+                                    const int* count_dev, int rows_cap, int d, const float* __restrict__ g,
+                                    float eps, __nv_bfloat16* __restrict__ z, int64_t ldz) {
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int j = blockIdx.x;
+  if (j >= m) return;
+  const int src = row_map ? row_map[j] : j;
+  const float* x = h + static_cast<int64_t>(src) * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  __shared__ float red[32];
+  ss = warp_sum_f(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum_f(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  __nv_bfloat16* out = z + static_cast<int64_t>(j) * ldz;
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    const float4 gg = *reinterpret_cast<const float4*>(g + i);
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r * gg.x, v.y * r * gg.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r * gg.z, v.w * r * gg.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&a);
+    pk.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(out + i) = pk;
+  }
+}
+
+// ------------------------------------------------------------------ ES-dLLM Eq. 1
+// For candidate row j (flat = rows[j]):
+//   c   = masked_prev[flat] ? conf[flat] : 0
+//   var = ||h - h_prev||_1 / (sqrt(d) ||h_prev||_2)   (0 when ||h_prev|| = 0)
+//   score[j] = alpha c + (1 - alpha) var
+// then h_prev[flat] := h[flat] and masked_prev[flat] := (tokens[flat] == mask_id)
+// One warp per row.
+__global__ void score_es_kernel(const float* __restrict__ h, float* __restrict__ h_prev,
+                                const float* __restrict__ conf, uint8_t* __restrict__ masked_prev,
+                                const int* __restrict__ tokens, int mask_id, const int* __restrict__ rows,
+                                int n_rows, int d, float alpha, int update, float* __restrict__ score) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= n_rows) return;
+  const int flat = rows ? rows[wid] : wid;
+  const float* x = h + static_cast<int64_t>(flat) * d;
+  float* xp = h_prev + static_cast<int64_t>(flat) * d;
+  float l1 = 0.f, l2 = 0.f;
+  for (int i = lane * 4; i < d; i += 128) {
+    const float4 a = *reinterpret_cast<const float4*>(x + i);
+    const float4 b = *reinterpret_cast<const float4*>(xp + i);
+    l1 += fabsf(a.x - b.x) + fabsf(a.y - b.y) + fabsf(a.z - b.z) + fabsf(a.w - b.w);
+    l2 += b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+    if (update) *reinterpret_cast<float4*>(xp + i) = a;
+  }
+  l1 = warp_sum_f(l1);
+  l2 = warp_sum_f(l2);
+  if (lane == 0) {
+    const float c = (masked_prev && masked_prev[flat]) ? conf[flat] : 0.f;
+    const float nrm = sqrtf(l2);
+    const float var = nrm > 0.f ? l1 / (sqrtf(static_cast<float>(d)) * nrm) : 0.f;
+    score[wid] = alpha * c + (1.f - alpha) * var;
+    if (update && masked_prev && tokens) masked_prev[flat] = tokens[flat] == mask_id ? 1 : 0;
+  }
+}
+
+// ------------------------------------------------------------------ dLLM-Cache cosine
+// s[j] = <v_new[j], v_cache(rows[j])> / (|v_new| |v_cache|); 1 if both zero, 0 if one is.
+// v_cache for flat = b * N + pos is the concatenation over KV heads of cache[b, kvh, pos, :].
+__global__ void score_cos_kernel(const float* __restrict__ vnew, int64_t ldv, const __nv_bfloat16* __restrict__ vc,
+                                 const int* __restrict__ rows, const int* count_dev, int rows_cap, int N, int Hkv,
+                                 int hd, float* __restrict__ sim) {
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= m) return;
+  const int flat = rows[wid];
+  const int b = flat / N, pos = flat % N;
+  float dot = 0.f, na = 0.f, nb = 0.f;
+  for (int kvh = 0; kvh < Hkv; ++kvh) {
+    const __nv_bfloat16* cv = vc + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd;
+    const float* nv = vnew + static_cast<int64_t>(wid) * ldv + kvh * hd;
+    for (int i = lane; i < hd; i += 32) {
+      const float a = nv[i], c = __bfloat162float(cv[i]);
+      dot += a * c;
+      na += a * a;
+      nb += c * c;
+    }
+  }
+  dot = warp_sum_f(dot);
+  na = warp_sum_f(na);
+  nb = warp_sum_f(nb);
+  if (lane == 0) {
+    float s;
+    if (na > 0.f && nb > 0.f) s = dot / (sqrtf(na) * sqrtf(nb));
+    else s = (na == 0.f && nb == 0.f) ? 1.f : 0.f;
+    sim[wid] = s;
+  }
+}
+
+// ------------------------------------------------------------------ SureLock KL + confidence
+// For LM row j with logits z[j, :] (bf16): lse, conf = p(argmax over v != mask), argmax,
+// and when has_prev: D = sum_v p_t (z_t - lse_t - z_p + lse_p), clamped at 0.
+// One CTA (256 threads) per row.
+__global__ void kl_conf_kernel(const __nv_bfloat16* __restrict__ z, int64_t ldz, const __nv_bfloat16* __restrict__ zp_store,
+                               int64_t ldp, const float* __restrict__ lse_prev, const int* __restrict__ has_prev,
+                               const int* __restrict__ rows, const int* count_dev, int rows_cap, int V, int mask_id,
+                               float* __restrict__ conf, int* __restrict__ amax, float* __restrict__ lse_out,
+                               float* __restrict__ kl_out) {
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int j = blockIdx.x;
+  if (j >= m) return;
+  const int flat = rows ? rows[j] : j;
+  const __nv_bfloat16* zr = z + static_cast<int64_t>(j) * ldz;
+  __shared__ float sf[32];
+  __shared__ int si[32];
+  // pass 1: max and argmax (mask id excluded from the argmax)
+  float mx = -INFINITY, bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float x = __bfloat162float(zr[v]);
+    mx = fmaxf(mx, x);
+    if (v != mask_id && (x > bv || (x == bv && v < bi))) { bv = x; bi = v; }
+  }
+  for (int o = 16; o; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (l == 0) { sf[w] = mx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int i = 0; i < nw; ++i) M = fmaxf(M, sf[i]);
+    sf[31] = M;
+  }
+  __syncthreads();
+  const float M = sf[31];
+  __syncthreads();
+  if (l == 0) { sf[w] = bv; si[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float B = -INFINITY;
+    int I = 0x7fffffff;
+    for (int i = 0; i < nw; ++i)
+      if (sf[i] > B || (sf[i] == B && si[i] < I)) { B = sf[i]; I = si[i]; }
+    sf[30] = B;
+    si[30] = I;
+  }
+  __syncthreads();
+  const float BV = sf[30];
+  const int BI = si[30];
+  __syncthreads();
+  // pass 2: sum exp
+  float se = 0.f;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) se += __expf(__bfloat162float(zr[v]) - M);
+  se = warp_sum_f(se);
+  if (l == 0) sf[w] = se;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float S = 0.f;
+    for (int i = 0; i < nw; ++i) S += sf[i];
+    sf[29] = S;
+  }
+  __syncthreads();
+  const float L = M + logf(sf[29]);
+  const bool hp = has_prev && has_prev[flat];
+  float kl = 0.f;
+  if (hp) {
+    const __nv_bfloat16* pr = zp_store + static_cast<int64_t>(flat) * ldp;
+    const float Lp = lse_prev[flat];
+    for (int v = threadIdx.x; v < V; v += blockDim.x) {
+      const float zt = __bfloat162float(zr[v]) - L;
+      const float zq = __bfloat162float(pr[v]) - Lp;
+      kl += __expf(zt) * (zt - zq);
+    }
+    kl = warp_sum_f(kl);
+    __syncthreads();
+    if (l == 0) sf[w] = kl;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float K = 0.f;
+      for (int i = 0; i < nw; ++i) K += sf[i];
+      sf[28] = fmaxf(K, 0.f);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    conf[flat] = __expf(BV - L);
+    amax[flat] = BI;
+    if (lse_out) lse_out[flat] = L;
+    if (kl_out) kl_out[j] = hp ? sf[28] : NAN;
+  }
+}
+
+// ------------------------------------------------------------------ selection
+constexpr int kSelThreads = 1024;
+constexpr int kSelMaxN = 8192;
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+  if (x != x) return 0u;               // NaN: lowest
+  x = x + 0.0f;                        // -0 -> +0
+  uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// exclusive block scan for 1024 threads; returns the exclusive prefix, total via ref
+__device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int& total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    s_warp[lane] = t;   // inclusive
+  }
+  __syncthreads();
+  const int base = w ? s_warp[w - 1] : 0;
+  total = s_warp[31];
+  __syncthreads();
+  return base + x - v;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
+  __shared__ uint32_t keys[kSelMaxN];
+  __shared__ uint8_t elig[kSelMaxN];
+  __shared__ int hist[256];
+  __shared__ int s_warp[32];
+  __shared__ int s_misc[4];
+  const int tid = threadIdx.x;
+  int off = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const float* sc = p.scores ? p.scores + static_cast<int64_t>(b) * p.n : nullptr;
+    int local_elig = 0;
+    for (int i = tid; i < p.n; i += kSelThreads) {
+      const float s = sc ? sc[i] : 0.f;
+      uint32_t k;
+      bool e;
+      switch (p.mode) {
+        case SEL_TOPK_DESC: k = order_key(s); e = true; break;
+        case SEL_BELOW_CAP_ASC: k = (s != s) ? 0xffffffffu : ~order_key(s); e = (s != s) || (s < p.tau); break;
+        case SEL_FORCED_ASC: k = (s != s) ? 0xffffffffu : ~order_key(s); e = true; break;
+        default: k = 0; e = p.lock ? (p.lock[static_cast<int64_t>(b) * p.seq_n + p.cand_start + i] == 0) : true; break;
+      }
+      keys[i] = k;
+      elig[i] = e ? 1 : 0;
+      local_elig += e ? 1 : 0;
+    }
+    __syncthreads();
+    int n_elig;
+    block_scan_excl(local_elig, s_warp, n_elig);
+    const int kk = (p.mode == SEL_ALL_ELIGIBLE) ? n_elig : min(p.k, n_elig);
+    uint32_t T = 0;
+    int need_eq = 0;
+    const bool take_all = (kk == n_elig);
+    if (!take_all && kk > 0) {
+      uint32_t prefix = 0, mask = 0;
+      int remaining = kk;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < p.n; i += kSelThreads)
+          if (elig[i] && (keys[i] & mask) == prefix) atomicAdd(&hist[(keys[i] >> shift) & 255], 1);
+        __syncthreads();
+        if (tid == 0) {
+          int above = 0, dg = 255;
+          for (; dg >= 0; --dg) {
+            if (above + hist[dg] >= remaining) break;
+            above += hist[dg];
+          }
+          s_misc[0] = dg;
+          s_misc[1] = remaining - above;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(s_misc[0]) << shift;
+        mask |= 255u << shift;
+        remaining = s_misc[1];
+        __syncthreads();
+      }
+      T = prefix;
+      need_eq = remaining;
+    }
+    // flags in index order: eq-rank among keys == T, then compaction
+    int carry_eq = 0, carry_sel = 0;
+    for (int base = 0; base < p.n; base += kSelThreads) {
+      const int i = base + tid;
+      const bool in = i < p.n;
+      const bool e = in && elig[i];
+      const bool eq = e && !take_all && keys[i] == T;
+      int tot_eq;
+      const int eqr = block_scan_excl(eq ? 1 : 0, s_warp, tot_eq) + carry_eq;
+      const bool sel = e && (take_all || keys[i] > T || (eq && eqr < need_eq));
+      int tot_sel;
+      const int o = block_scan_excl(sel ? 1 : 0, s_warp, tot_sel) + carry_sel;
+      if (sel && kk > 0) {
+        const int pos = p.cand_start + i;
+        if (p.act_pos) p.act_pos[static_cast<int64_t>(b) * p.k_max + o] = pos;
+        if (p.row_map) p.row_map[off + o] = b * p.seq_n + pos;
+      }
+      carry_eq += tot_eq;
+      carry_sel += tot_sel;
+    }
+    const int cnt = kk > 0 ? carry_sel : 0;
+    if (tid == 0) {
+      if (p.count) p.count[b] = cnt;
+      if (p.seq_off) p.seq_off[b] = off;
+    }
+    off += cnt;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (p.seq_off) p.seq_off[p.B] = off;
+    if (p.total) *p.total = off;
+  }
+}
+
+// ------------------------------------------------------------------ row lists
+// Rows of a contiguous position range per sequence: row_map = b * N + start + i.
+__global__ void range_rows_kernel(int B, int N, int start, int len, int* row_map, int* seq_off, int* total) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < B * len) row_map[idx] = (idx / len) * N + start + (idx % len);
+  if (idx <= B && seq_off) seq_off[idx] = idx * len;
+  if (idx == 0 && total) *total = B * len;
+}
+
+// LM rows: the recomputed rows that are masked and inside [blk_s, blk_e) (and, with
+// a round mask, inside this round).  Single CTA, order-preserving compaction.
+__global__ void __launch_bounds__(kSelThreads) lm_rows_kernel(const int* __restrict__ rows, const int* count_dev,
+                                                              int rows_cap, const int* __restrict__ tokens, int mask_id,
+                                                              int N, int blk_s, int blk_e,
+                                                              const uint8_t* __restrict__ round_mask,
+                                                              int* __restrict__ lm_rows, int* lm_count) {
+  __shared__ int s_warp[32];
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  int carry = 0;
+  for (int base = 0; base < m; base += kSelThreads) {
+    const int j = base + threadIdx.x;
+    bool keep = false;
+    int flat = 0;
+    if (j < m) {
+      flat = rows[j];
+      const int pos = flat % N;
+      keep = tokens[flat] == mask_id && pos >= blk_s && pos < blk_e &&
+             (!round_mask || round_mask[pos - blk_s]);
+    }
+    int tot;
+    const int o = block_scan_excl(keep ? 1 : 0, s_warp, tot) + carry;
+    if (keep) lm_rows[o] = flat;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) *lm_count = carry;
+}
+
+// h_prev[flat] = h[flat], masked_prev[flat] = (tokens[flat] == mask) for the given rows.
+__global__ void snapshot_rows_kernel(const float* __restrict__ h, float* __restrict__ h_prev,
+                                     const int* __restrict__ tokens, uint8_t* __restrict__ masked_prev, int mask_id,
+                                     const int* __restrict__ rows, int n_rows, int d) {
+  const int j = blockIdx.x;
+  if (j >= n_rows) return;
+  const int flat = rows[j];
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4)
+    *reinterpret_cast<float4*>(h_prev + static_cast<int64_t>(flat) * d + i) =
+        *reinterpret_cast<const float4*>(h + static_cast<int64_t>(flat) * d + i);
+  if (threadIdx.x == 0 && masked_prev) masked_prev[flat] = tokens[flat] == mask_id ? 1 : 0;
+}
+
+// ------------------------------------------------------------------ unmask
+// One CTA per sequence; threads stride over the block positions blk_s + i.
+// TOPCONF: commit the n masked positions with the highest conf (ties: lower position).
+// round_mask (DUS): commit every masked position of this round.
+__global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict__ conf, const int* __restrict__ amax,
+                              int N, int blk_s, int blk_len, int mask_id, int n_commit,
+                              const uint8_t* __restrict__ round_mask, int* __restrict__ pos_out,
+                              int* __restrict__ tok_out, int* __restrict__ n_out, int max_out) {
+  extern __shared__ float s_conf[];
+  uint8_t* s_masked = reinterpret_cast<uint8_t*>(s_conf + blk_len);
+  __shared__ int s_cnt;
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) s_cnt = 0;
+  const int64_t base = static_cast<int64_t>(b) * N + blk_s;
+  for (int i = threadIdx.x; i < blk_len; i += blockDim.x) {
+    s_masked[i] = tokens[base + i] == mask_id ? 1 : 0;
+    float c = conf[base + i];
+    c = (c != c) ? -INFINITY : c + 0.0f;
+    s_conf[i] = c;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < blk_len; i += blockDim.x) {
+    bool commit = false;
+    if (s_masked[i]) {
+      if (round_mask) {
+        commit = round_mask[i] != 0;
+      } else {
+        int rank = 0;
+        const float ci = s_conf[i];
+        for (int q = 0; q < blk_len && rank < n_commit; ++q)
+          if (s_masked[q] && (s_conf[q] > ci || (s_conf[q] == ci && q < i))) ++rank;
+        commit = rank < n_commit;
+      }
+    }
+    if (commit) {
+      const int tok = amax[base + i];
+      tokens[base + i] = tok;
+      if (pos_out) {
+        const int slot = atomicAdd(&s_cnt, 1);
+        if (slot < max_out) {
+          pos_out[static_cast<int64_t>(b) * max_out + slot] = blk_s + i;
+          tok_out[static_cast<int64_t>(b) * max_out + slot] = tok;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && n_out) n_out[b] = min(s_cnt, max_out);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st) {
+  const int half = hd / 2;
+  const int n = N * half;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(cos_t, sin_t, N, half, theta, hd);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int embed_rows_launch(const __nv_bfloat16* E, const int* tokens, const int* row_map, const int* count_dev,
+                      int rows_cap, int d, float* h, cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  if (d % 8) return DLLM_ERR_SHAPE;
+  embed_rows_kernel<<<rows_cap, 128, 0, st>>>(E, tokens, row_map, count_dev, rows_cap, d, h);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
+                        float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  if (d % 4) return DLLM_ERR_SHAPE;
+  rmsnorm_rows_kernel<<<rows_cap, 256, 0, st>>>(h, row_map, count_dev, rows_cap, d, g, eps, z, ldz);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
+                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update, float* score,
+                    cudaStream_t st) {
+  if (n_rows <= 0) return DLLM_OK;
+  if (d % 4) return DLLM_ERR_SHAPE;
+  const int blocks = (n_rows * 32 + 255) / 256;
+  score_es_kernel<<<blocks, 256, 0, st>>>(h, h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
+                                          update, score);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, const int* rows, const int* count_dev,
+                     int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  const int blocks = (rows_cap * 32 + 255) / 256;
+  score_cos_kernel<<<blocks, 256, 0, st>>>(vnew, ldv, vc, rows, count_dev, rows_cap, N, Hkv, hd, sim);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int kl_conf_launch(const __nv_bfloat16* z, int64_t ldz, const __nv_bfloat16* zp_store, int64_t ldp,
+                   const float* lse_prev, const int* has_prev, const int* rows, const int* count_dev, int rows_cap,
+                   int V, int mask_id, float* conf, int* amax, float* lse_out, float* kl_out, cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  kl_conf_kernel<<<rows_cap, 256, 0, st>>>(z, ldz, zp_store, ldp, lse_prev, has_prev, rows, count_dev, rows_cap, V,
+                                           mask_id, conf, amax, lse_out, kl_out);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int select_launch(const SelectParams& p, cudaStream_t st) {
+  if (p.B <= 0) return DLLM_OK;
+  if (p.n < 0 || p.n > kSelMaxN) return DLLM_ERR_UNSUPPORTED;
+  select_kernel<<<1, kSelThreads, 0, st>>>(p);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int range_rows_launch(int B, int N, int start, int len, int* row_map, int* seq_off, int* total, cudaStream_t st) {
+  const int n = std::max(B * len, B + 1);
+  range_rows_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, N, start, len, row_map, seq_off, total);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const int* tokens, int mask_id, int N,
+                   int blk_s, int blk_e, const uint8_t* round_mask, int* lm_rows, int* lm_count, cudaStream_t st) {
+  lm_rows_kernel<<<1, kSelThreads, 0, st>>>(rows, count_dev, rows_cap, tokens, mask_id, N, blk_s, blk_e, round_mask,
+                                            lm_rows, lm_count);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8_t* masked_prev, int mask_id,
+                         const int* rows, int n_rows, int d, cudaStream_t st) {
+  if (n_rows <= 0) return DLLM_OK;
+  snapshot_rows_kernel<<<n_rows, 256, 0, st>>>(h, h_prev, tokens, masked_prev, mask_id, rows, n_rows, d);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N, int blk_s, int blk_len, int mask_id,
+                  int n_commit, const uint8_t* round_mask, int* pos_out, int* tok_out, int* n_out, int max_out,
+                  cudaStream_t st) {
+  if (blk_len <= 0 || blk_len > 8192) return DLLM_ERR_UNSUPPORTED;
+  const int threads = std::min(1024, ((blk_len + 31) / 32) * 32);
+  const size_t smem = blk_len * sizeof(float) + blk_len;
+  unmask_kernel<<<B, threads, smem, st>>>(tokens, conf, amax, N, blk_s, blk_len, mask_id, n_commit, round_mask, pos_out,
+                                          tok_out, n_out, max_out);
+  count_launch();
+  DLLM_CUDA_TRY(cudaGetLastError());
+  return DLLM_OK;
+}
+
+}  // namespace dllm

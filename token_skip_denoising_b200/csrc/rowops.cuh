@@ -1,0 +1,60 @@
+// Host launchers of the row-wise kernels (rowops.cu) and the attention (attention.cu).
+#pragma once
+#include "common.cuh"
+
+namespace dllm {
+
+enum SelMode : int {
+  SEL_TOPK_DESC = 0,       // keep the k highest scores (ties: lower index)
+  SEL_BELOW_CAP_ASC = 1,   // rows with score < tau (NaN counts), at most k lowest
+  SEL_FORCED_ASC = 2,      // exactly min(k, n) lowest scores
+  SEL_ALL_ELIGIBLE = 3,    // every row whose lock flag is 0
+};
+
+struct SelectParams {
+  const float* scores = nullptr;   // [B, n]
+  int B = 0, n = 0;
+  int mode = SEL_TOPK_DESC;
+  int k = 0;
+  float tau = 0.f;
+  int cand_start = 0;              // candidate i is position cand_start + i
+  int seq_n = 0;                   // sequence length N
+  const uint8_t* lock = nullptr;   // [B, N] (SEL_ALL_ELIGIBLE)
+  int* act_pos = nullptr;          // [B, k_max] ascending positions
+  int k_max = 0;
+  int* count = nullptr;            // [B]
+  int* row_map = nullptr;          // flat rows, b-major
+  int* seq_off = nullptr;          // [B + 1]
+  int* total = nullptr;
+};
+
+int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st);
+int embed_rows_launch(const __nv_bfloat16* E, const int* tokens, const int* row_map, const int* count_dev,
+                      int rows_cap, int d, float* h, cudaStream_t st);
+int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
+                        float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st);
+int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
+                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update, float* score,
+                    cudaStream_t st);
+int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, const int* rows, const int* count_dev,
+                     int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st);
+int kl_conf_launch(const __nv_bfloat16* z, int64_t ldz, const __nv_bfloat16* zp_store, int64_t ldp,
+                   const float* lse_prev, const int* has_prev, const int* rows, const int* count_dev, int rows_cap,
+                   int V, int mask_id, float* conf, int* amax, float* lse_out, float* kl_out, cudaStream_t st);
+int select_launch(const SelectParams& p, cudaStream_t st);
+int range_rows_launch(int B, int N, int start, int len, int* row_map, int* seq_off, int* total, cudaStream_t st);
+int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const int* tokens, int mask_id, int N,
+                   int blk_s, int blk_e, const uint8_t* round_mask, int* lm_rows, int* lm_count, cudaStream_t st);
+int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8_t* masked_prev, int mask_id,
+                         const int* rows, int n_rows, int d, cudaStream_t st);
+int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N, int blk_s, int blk_len, int mask_id,
+                  int n_commit, const uint8_t* round_mask, int* pos_out, int* tok_out, int* n_out, int max_out,
+                  cudaStream_t st);
+
+size_t attn_partial_floats(int rows_cap, int Hq, int hd, int splits);
+int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N);
+int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, __nv_bfloat16* out,
+                const int* seq_off, int B, int rows_cap, int rows_per_seq_cap, int N, int Hq, int Hkv, int hd,
+                int splits, float* opart, float2* ml, size_t partial_floats, cudaStream_t st);
+
+}  // namespace dllm
