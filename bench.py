@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Generated tokens/s of the token-skipping denoising generation on B200.
+
+Workload (default): the LLaDA-8B-shaped ES-dLLM generation -- 32 layers,
+d 4096, 32 heads x 128, SwiGLU 12288, vocab 126464, random-init N(0, 0.02)
+bf16 weights; batch 1, a 512-token uniform-random prompt, 256 generated tokens
+in blocks of 32 at 1 token per step; every block starts with a full refresh,
+the other steps recompute the block's 32 rows through layers 0-3, score them
+by Eq. 1 and keep the top 20% (7 rows) for layers 4-31.
+
+One bench step = one whole generation (8 blocks x 32 denoising steps).
+`value` is device-timed (CUDA events, max over ranks) with the weights and
+prompt resident in HBM; `e2e` is the same generation through the public API
+with the prompt copied from pinned host memory and the tokens read back each
+step.  Multi-GPU runs are independent replicas (each rank generates its own
+batch; the path has no exchange step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "generated tokens/s, LLaDA-8B shape, 1×B200; step latency & roofline % vs active ratio"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return dict(PEAKS_FALLBACK, source="fallback")
+
+
+def workload_desc(cfg):
+    m = cfg.model
+    return (f"{cfg.name}: {m.n_layers} layers, d {m.d_model}, {m.n_heads} heads x {m.head_dim} "
+            f"({m.n_kv_heads} KV), SwiGLU {m.ffn_dim}, vocab {m.vocab}; batch {cfg.batch}, prompt {cfg.prompt_len}, "
+            f"gen {cfg.gen_len} in blocks of {cfg.block_len}, {cfg.tokens_per_step} token/step; "
+            f"ES-dLLM skip at layer {cfg.skip_layer} keeping {cfg.keep_ratio:.0%} of the block")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if uuid:
+            cmd += ["-i", uuid]
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from synth import get_config, make_tokens, make_weights
+    from synth.gen import PROMPT_SEED
+    from token_skip_denoising_b200.engine import Engine, kernel_launches
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = get_config(args.workload)
+    peaks = load_peaks()
+    w = make_weights(cfg.model, device=dev)
+    tok0_host = make_tokens(cfg, seed=PROMPT_SEED + rank).pin_memory()
+    tok0 = tok0_host.to(dev)
+    tok = tok0.clone()
+    stream = torch.cuda.current_stream(dev)
+    eng = Engine(cfg, w, tok, stream=stream)
+
+    def one_generation():
+        eng.reset(tok0)
+        eng.generate()
+
+    for _ in range(args.warmup):
+        one_generation()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- device-timed region: K generations, profiling of the GEMMs / attention on
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    eng.profile(True, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"])
+    eng.profile_read()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(uuid)
+    launches0 = kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        one_generation()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = kernel_launches() - launches0
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    prof = eng.profile_read()
+    eng.profile(False)
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_total = cfg.batch * cfg.gen_len * args.steps * world
+    value = tokens_total / (ms_max / 1e3)
+    assert not bool((tok == cfg.model.mask_id).any()), "generation left mask ids"
+
+    # ---- end to end through the public API, host buffers, copies inside the region
+    out_host = torch.empty_like(tok0_host).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for _ in range(args.steps):
+        tok.copy_(tok0_host, non_blocking=True)      # H2D of this step's input
+        eng.reset()
+        eng.generate()
+        out_host.copy_(tok, non_blocking=True)       # D2H of the result
+    torch.cuda.synchronize()
+    e2e_s = time.perf_counter() - w0
+    e2e_t = torch.tensor([e2e_s], device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens_total / float(e2e_t.item())
+
+    # ---- roofline of the dominant kernel (the fused tcgen05 GEMM)
+    gemm_gbs = prof["gemm_bytes"] / (prof["gemm_ms"] / 1e3) / 1e9 if prof["gemm_ms"] > 0 else 0.0
+    roof = {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+            "kernel": "gemm_tc_kernel (all QKV/O/gate-up/down/LM-head launches of the timed region)",
+            "peak_source": peaks["source"],
+            "launches": prof["gemm_launches"],
+            "avg_launch_us": round(1e3 * prof["gemm_ms"] / max(1, prof["gemm_launches"]), 3),
+            "time_share": round(prof["gemm_ms"] / ms, 4),
+            "roofline_time_frac": round(prof["gemm_roofline_ms"] / prof["gemm_ms"], 4) if prof["gemm_ms"] else None,
+            "attention": {"launches": prof["attn_launches"], "ms": round(prof["attn_ms"], 3),
+                          "achieved_gbs": round(prof["attn_bytes"] / (prof["attn_ms"] / 1e3) / 1e9, 1)
+                          if prof["attn_ms"] else None}}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded random-init N(0,0.02) bf16 weights, uniform-random prompt ids",
+        "config": {"workload": workload_desc(cfg), "batch": cfg.batch, "seq_len": cfg.seq_len,
+                   "gen_len": cfg.gen_len, "step": "one whole generation (all blocks and denoising steps)",
+                   "l2": "inputs larger than L2: every denoising step streams all 16 GB of weights",
+                   "parallelism": f"replicas x{world} (no collective)"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(tok0_host.numel() * 4), "d2h_bytes_per_step": int(out_host.numel() * 4)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    return line, eng, w, cfg
+
+
+# ---------------------------------------------------------------- active-ratio sweep (single layer)
+def micro_sweep(peaks, reps=20):
+    """Single-layer step at N = 2048 (d 4096, 32 heads, FFN 12288): score -> top-k ->
+    gathered QKV/O/FFN -> active-query attention -> K/V scatter, for each active ratio."""
+    import torch
+
+    from synth import get_config, make_weights
+    from synth.gen import kv_cache_fill, microbench_active, microbench_hidden
+    from token_skip_denoising_b200 import _lib, ops
+
+    cfg = get_config("micro")
+    m = cfg.model
+    N, d = cfg.seq_len, m.d_model
+    w = make_weights(m, device="cuda")
+    lw = {k: w[k][0] for k in ("w_qkv", "w_o", "w_gu", "w_down", "g_attn", "g_ffn")}
+    kv = kv_cache_fill(1, 1, m.n_kv_heads, N, m.head_dim, device="cuda")
+    kc, vc = kv[0, 0].contiguous(), kv[0, 1].contiguous()
+    hin = microbench_hidden(N, d, device="cuda")
+    cos, sin = ops.rope_table(N, m.head_dim, m.rope_theta)
+    ccfg = _lib.make_config(cfg)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = []
+    P = m.params_per_layer
+    for rho in (0.03, 0.1, 0.25, 0.5, 1.0):
+        k = max(1, math.ceil(rho * N - 1e-9))
+        ws = torch.empty(ops.layer_workspace_bytes(ccfg, k, k), dtype=torch.uint8, device="cuda")
+        for pattern in ("random", "contiguous"):
+            h = hin["h_cur"].clone()
+            hp = hin["h_prev"].clone()
+            act_idx = microbench_active(N, k, pattern).cuda()
+            cnt = torch.tensor([k], dtype=torch.int32, device="cuda")
+            off = torch.tensor([0, k], dtype=torch.int32, device="cuda")
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            times = []
+            for it in range(reps + 3):
+                flush.zero_()
+                ev[0].record()
+                s = ops.score_es(h, hp, hin["conf"], 0.5, masked_prev=hin["masked_prev"])
+                ops.select(s, 1, N, ops.SEL_TOPK_DESC, k)
+                # the layer runs on the fixed index pattern so both patterns are measured
+                ops.layer(ccfg, lw, kc, vc, cos, sin, h, act_idx, cnt, off, k, k, ws=ws)
+                ev[1].record()
+                torch.cuda.synchronize()
+                if it >= 3:
+                    times.append(ev[0].elapsed_time(ev[1]))
+            t = statistics.median(times)
+            kv_bytes = 2 * N * m.kv_dim * 2
+            byts = P * 2 + kv_bytes + k * (2 * m.kv_dim + 2 * d) * 2 + 2 * N * d * 4
+            flops = 2 * k * P + 4 * k * N * m.n_heads * m.head_dim
+            roof_ms = max(byts / (peaks["hbm_gbs"] * 1e6), flops / (peaks["bf16_tflops"] * 1e9))
+            out.append({"rho": rho, "k": k, "pattern": pattern, "ms": round(t, 4),
+                        "roofline_ms": round(roof_ms, 4), "roofline_frac": round(roof_ms / t, 4),
+                        "bound": "hbm" if byts / (peaks["hbm_gbs"] * 1e6) >= flops / (peaks["bf16_tflops"] * 1e9)
+                        else "tensor"})
+    del w
+    return out
+
+
+# ---------------------------------------------------------------- oracle timing (CPU)
+def oracle_sample_timing(cfg, w_dev, seconds_cap=40.0):
+    """Time the oracle on a bounded sample of the workload on the host cores and
+    extrapolate to one whole generation: one layer at the three row counts a
+    generation uses (all rows at a refresh, the block below the skip layer, the
+    kept rows above it) and the vocabulary projection of the kept rows."""
+    import numpy as np
+    import torch
+
+    from oracle.model import OracleModel
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    m = cfg.model
+    N = cfg.seq_len
+    n_c = cfg.block_len
+    k = cfg.keep_count(n_c)
+    rng = np.random.default_rng(0)
+
+    def layer_time(rows, layer):
+        lw = {key: w_dev[key][layer:layer + 1].cpu() for key in ("w_qkv", "w_o", "w_gu", "w_down", "g_attn",
+                                                                 "g_ffn")}
+        lw.update({"embed": w_dev["embed"], "lm_head": w_dev["lm_head"], "g_final": w_dev["g_final"].cpu(),
+                   "layers": [layer]})
+        om = OracleModel(m, lw)
+        K = np.zeros((1, m.n_kv_heads, N, m.head_dim))
+        V = np.zeros_like(K)
+        h = rng.standard_normal((rows, m.d_model))
+        pos = np.sort(rng.choice(N, rows, replace=False))
+        t = time.perf_counter()
+        om.layer(layer, h, np.zeros(rows, dtype=np.int64), pos, K, V)   # includes its lazy weight conversion
+        return time.perf_counter() - t
+
+    def lm_time(rows):
+        om = OracleModel(m, {"lm_head": w_dev["lm_head"], "g_final": w_dev["g_final"].cpu(), "layers": []})
+        h = rng.standard_normal((rows, m.d_model))
+        t = time.perf_counter()
+        om.logits(h)
+        return time.perf_counter() - t
+
+    t_start = time.perf_counter()
+    t_full = layer_time(N, 0)
+    t_pre = layer_time(n_c, 1)
+    t_post = layer_time(k, 2)
+    t_lm = lm_time(k)
+    spent = time.perf_counter() - t_start
+    steps_per_block = math.ceil(cfg.block_len / cfg.tokens_per_step)
+    n_ref = cfg.n_blocks
+    n_skip = cfg.n_blocks * (steps_per_block - 1)
+    L, ls = m.n_layers, cfg.skip_layer
+    gen_s = n_ref * (L * t_full + t_lm) + n_skip * (ls * t_pre + (L - ls) * t_post + t_lm)
+    return {"value": round(cfg.batch * cfg.gen_len / gen_s, 6), "unit": "tokens/s", "cores": int(cores),
+            "kind": "oracle",
+            "sample": (f"fp64 oracle on one layer at {N}, {n_c} and {k} rows and the vocabulary projection of "
+                       f"{k} rows ({spent:.1f} s of host time, weight conversion included), extrapolated to "
+                       f"{n_ref} refresh + {n_skip} skip steps of {L} layers")}
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args):
+    import numpy as np
+
+    from oracle.model import OracleModel
+    from synth import get_config
+
+    cfg = get_config(args.workload)
+    m = cfg.model
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    # weights of the sampled layers only (host, bf16 values), seeded like the GPU arm's draw
+    import torch
+    from synth.gen import make_weights
+    w = make_weights(m, device="cpu", layers=[0], with_vocab=False)
+    N, n_c, k = cfg.seq_len, cfg.block_len, cfg.keep_count(cfg.block_len)
+    rng = np.random.default_rng(0)
+
+    def one_sample():
+        """One skip step's worth of the layer stack, scaled to a whole generation.  Each
+        layer call converts its weights, as the oracle does for every layer of a run."""
+        K = np.zeros((1, m.n_kv_heads, N, m.head_dim))
+        V = np.zeros_like(K)
+        t = time.perf_counter()
+        OracleModel(m, w).layer(0, rng.standard_normal((n_c, m.d_model)), np.zeros(n_c, np.int64),
+                                np.arange(n_c), K, V)
+        t_pre = time.perf_counter() - t
+        t = time.perf_counter()
+        OracleModel(m, w).layer(0, rng.standard_normal((k, m.d_model)), np.zeros(k, np.int64), np.arange(k), K, V)
+        t_post = time.perf_counter() - t
+        steps = cfg.n_blocks * math.ceil(cfg.block_len / cfg.tokens_per_step)
+        return steps * (cfg.skip_layer * t_pre + (m.n_layers - cfg.skip_layer) * t_post)
+
+    for _ in range(args.warmup):
+        one_sample()
+    times = [one_sample() for _ in range(args.steps)]
+    gen_s = sum(times)
+    value = cfg.batch * cfg.gen_len * args.steps / gen_s
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * gen_s / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+            "data": "synthetic: seeded random-init N(0,0.02) bf16 weights, uniform-random prompt ids",
+            "config": {"workload": workload_desc(cfg), "batch": cfg.batch, "seq_len": cfg.seq_len,
+                       "gen_len": cfg.gen_len, "step": "one whole generation, extrapolated from a sample",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+                             "sample": ("per step: one layer of the fp64 oracle at the block's rows and at the "
+                                        "kept rows (weight conversion included), scaled to every skip step "
+                                        "and layer of the generation")},
+            "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llada_es")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3          # timing rule: at least three untimed warm-up steps
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    line, eng, w, cfg = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1:
+        peaks = load_peaks()
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample_timing(cfg, w)
+        del eng
+        if not args.no_sweep:
+            w.clear()
+            torch.cuda.empty_cache()
+            line["active_ratio_sweep"] = micro_sweep(peaks)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

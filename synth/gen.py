@@ -32,7 +32,7 @@ def _normal_bf16(shape, std, seed, device):
 
 
 def make_weights(m: ModelDims, seed: int = WEIGHT_SEED, device="cpu", std: float = 0.02,
-                 gain_jitter: float = 0.0, layers=None) -> dict:
+                 gain_jitter: float = 0.0, layers=None, with_vocab: bool = True) -> dict:
     """All model weights in the library's layout.
 
     embed, lm_head: [V, d] bf16.  w_qkv: [L, Hq*hd + 2*Hkv*hd, d] (q rows, then k,
@@ -40,6 +40,7 @@ def make_weights(m: ModelDims, seed: int = WEIGHT_SEED, device="cpu", std: float
     w_down: [L, d, F].  g_attn, g_ffn: [L, d] fp32, g_final: [d] fp32.
     `layers` restricts generation to a subset of layers (others are omitted);
     each layer is drawn from its own seed so a subset equals the full draw.
+    with_vocab=False omits the two [V, d] matrices.
     """
     dev = torch.device(device)
     L = m.n_layers
@@ -48,10 +49,10 @@ def make_weights(m: ModelDims, seed: int = WEIGHT_SEED, device="cpu", std: float
     def sd(name, layer=0):
         return seed * 100003 + _TENSOR_IDS[name] * 1009 + layer
 
-    w = {
-        "embed": _normal_bf16((m.vocab, m.d_model), std, sd("embed"), dev),
-        "lm_head": _normal_bf16((m.vocab, m.d_model), std, sd("lm_head"), dev),
-    }
+    w = {}
+    if with_vocab:
+        w["embed"] = _normal_bf16((m.vocab, m.d_model), std, sd("embed"), dev)
+        w["lm_head"] = _normal_bf16((m.vocab, m.d_model), std, sd("lm_head"), dev)
     shapes = {"w_qkv": (m.qkv_dim, m.d_model), "w_o": (m.d_model, m.q_dim),
               "w_gu": (2 * m.ffn_dim, m.d_model), "w_down": (m.d_model, m.ffn_dim)}
     for name, shp in shapes.items():

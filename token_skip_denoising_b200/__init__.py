@@ -2,17 +2,6 @@
 
 The compute path is libdllm.so (hand-written sm_100a CUDA behind a C ABI,
 include/dllm.h); this package only marshals torch tensors into it.
+Submodules: `engine` (the generation engine), `ops` (single kernels).
 """
 from ._lib import load, DllmError, make_config  # noqa: F401
-
-__all__ = ["load", "DllmError", "make_config", "Engine", "ops"]
-
-
-def __getattr__(name):
-    if name == "Engine":
-        from .engine import Engine
-        return Engine
-    if name == "ops":
-        from . import ops
-        return ops
-    raise AttributeError(name)
