@@ -171,8 +171,9 @@ int dllm_done(const dllm_handle* h);
 int dllm_reset(dllm_handle* h, void* stream);
 
 /* Per-kernel timing of the fused GEMMs and the attention, for roofline
- * reporting: with enable != 0 every such launch is bracketed by CUDA events on
- * its stream, and its algorithmic bytes and flops are recorded.
+ * reporting: with enable = n > 0 every n-th launch of each kind is bracketed by
+ * CUDA events on its stream, and its algorithmic bytes and flops are recorded
+ * (sampling keeps the event overhead off the timed stream); 0 turns it off.
  * dllm_profile_read synchronises, sums the records since the last read and
  * clears them. */
 typedef struct dllm_profile {
@@ -212,7 +213,10 @@ void dllm_destroy(dllm_handle* h);
 
 /* ------------------------------------------------------------------ ops
  * Single kernels of the path on caller buffers (parity tests, the
- * single-layer microbenchmark).  Device pointers, stream as above.        */
+ * single-layer microbenchmark).  Device pointers, stream as above.
+ * `workspace` (where taken) is caller scratch: zero it before its first use;
+ * its first 256 KB hold GEMM tile counters that every call leaves at zero, so
+ * calls on one stream may share it; calls that overlap on the GPU may not.  */
 
 /* RoPE tables cos/sin fp32 [N, hd/2] with angle pos * theta^(-2i/hd). */
 int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, double theta, void* stream);
@@ -295,7 +299,8 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
                   const float* rope_sin, float* h, const int32_t* rows, const int32_t* count, const int32_t* seq_off,
                   int32_t rows_cap, int32_t rows_per_seq_cap, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes dllm_op_layer needs for rows_cap rows. */
+/* Workspace bytes dllm_op_layer needs for rows_cap rows (zero it before its first use;
+ * the GEMM tile counters at its start are left at zero by every call). */
 int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t rows_per_seq_cap, size_t* bytes);
 
 #ifdef __cplusplus

@@ -73,6 +73,8 @@ struct AttnParams {
 
 template <int HD>
 __global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kChunks = HD / 8;                      // 16-byte chunks per key row
   constexpr int kTileBytes = kKeysPerBlock * HD * 2;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -270,6 +272,8 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
 // One warp per (row, head): merge the split partials.
 template <int HD>
 __global__ void attn_combine_kernel(AttnParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int total = p.seq_off[p.B];
@@ -339,20 +343,19 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
   const size_t smem = 4 * kKeysPerBlock * hd * 2;
   if (hd == 128) {
     DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attn_kernel<128><<<grid, 128, smem, st>>>(p);
+    const int rc = launch_pdl(attn_kernel<128>, grid, dim3(128), smem, st, p);
+    if (rc) return rc;
   } else {
     DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attn_kernel<64><<<grid, 128, smem, st>>>(p);
+    const int rc = launch_pdl(attn_kernel<64>, grid, dim3(128), smem, st, p);
+    if (rc) return rc;
   }
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
   if (splits > 1) {
     const int warps = rows_cap * Hq;
     const int blocks = (warps * 32 + 255) / 256;
-    if (hd == 128) attn_combine_kernel<128><<<blocks, 256, 0, st>>>(p);
-    else attn_combine_kernel<64><<<blocks, 256, 0, st>>>(p);
-    count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+    const int rc = hd == 128 ? launch_pdl(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, p)
+                             : launch_pdl(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, p);
+    if (rc) return rc;
   }
   return DLLM_OK;
 }

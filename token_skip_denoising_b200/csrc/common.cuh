@@ -8,6 +8,8 @@
 #include <atomic>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
+#include <utility>
 
 #include "../../include/dllm.h"
 
@@ -29,6 +31,36 @@ void set_last_error(const char* msg, const char* file, int line);
 // Kernels launched by this library in the process (reported by dllm_kernel_launches).
 extern std::atomic<int64_t> g_kernel_launches;
 inline void count_launch(int n = 1) { g_kernel_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Launch with programmatic dependent launch: the kernel may be scheduled while the
+// previous kernel on the stream is still running; every kernel of this library calls
+// pdl_wait() before it touches memory an earlier kernel produced, and pdl_trigger()
+// as soon as its own dependents may be scheduled.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  static const bool pdl_off = getenv("DLLM_NO_PDL") != nullptr;   // A/B switch for measurements
+  cfg.numAttrs = pdl_off ? 0 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  count_launch();
+  if (e != cudaSuccess) {
+    set_last_error(cudaGetErrorString(e), __FILE__, __LINE__);
+    return DLLM_ERR_CUDA;
+  }
+  return DLLM_OK;
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------ GEMM
 // C[j, n] = sum_k X[j, k] * W[n, k]: X holds the active rows (K-major), W the

@@ -137,6 +137,8 @@ struct Prof {
     double bytes, flops;
   };
   bool on = false;
+  int every = 1;                // bracket every n-th launch of each class
+  int64_t seen[2] = {0, 0};
   double hbm_gbs = 0, tflops = 0;
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -146,9 +148,9 @@ struct Prof {
     cudaEventCreate(&e);
     return e;
   }
-  void begin(cudaStream_t st, cudaEvent_t* a) {
+  void begin(cudaStream_t st, cudaEvent_t* a, int cls) {
     *a = nullptr;
-    if (!on) return;
+    if (!on || (seen[cls]++ % every) != 0) return;
     *a = get();
     cudaEventRecord(*a, st);
   }
@@ -345,9 +347,9 @@ struct LayerCtx {
 // (weights + activation rows + outputs) for rows_cap rows.
 int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_t st, double out_bytes_per_row) {
   cudaEvent_t a = nullptr;
-  if (prof) prof->begin(st, &a);
+  if (prof) prof->begin(st, &a, 0);
   const int rc = gemm_launch(g, gs, st);
-  if (prof && prof->on) {
+  if (prof && a) {
     const double wrows = g.swiglu ? 2.0 * g.epi.ffn : 128.0 * g.n_tiles_w;
     const double bytes = wrows * g.K * 2.0 + static_cast<double>(g.rows_cap) * (g.K * 2.0 + out_bytes_per_row);
     prof->end(st, a, 0, bytes, 2.0 * g.rows_cap * wrows * g.K);
@@ -370,10 +372,10 @@ int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, con
   DLLM_TRY(timed_gemm(x.prof, g, x.gs, st, 2.0 * x.qkvd));
   {
     cudaEvent_t a = nullptr;
-    if (x.prof) x.prof->begin(st, &a);
+    if (x.prof) x.prof->begin(st, &a, 1);
     DLLM_TRY(attn_launch(x.q, x.kc, x.vc, x.attn, seq_off, x.B, rows_cap, rows_per_seq, x.N, x.Hq, x.Hkv, x.hd, 0,
                          x.attn_opart, x.attn_ml, x.attn_floats, st));
-    if (x.prof && x.prof->on) {
+    if (x.prof && a) {
       const double kvb = 2.0 * x.B * x.Hkv * static_cast<double>(x.N) * x.hd * 2.0;
       x.prof->end(st, a, 1, kvb + 4.0 * rows_cap * x.qd, 4.0 * rows_cap * x.Hq * static_cast<double>(x.N) * x.hd);
     }
@@ -704,7 +706,9 @@ int dllm_reset(dllm_handle* x, void* stream) {
 
 int dllm_profile_enable(dllm_handle* x, int32_t enable, double hbm_gbs, double tensor_tflops) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
-  x->prof.on = enable != 0;
+  x->prof.on = enable > 0;
+  x->prof.every = enable > 0 ? enable : 1;
+  x->prof.seen[0] = x->prof.seen[1] = 0;
   x->prof.hbm_gbs = hbm_gbs;
   x->prof.tflops = tensor_tflops;
   return DLLM_OK;
@@ -744,16 +748,16 @@ int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t ro
   const int d = cfg->d_model, qd = cfg->n_heads * cfg->head_dim, kvd = cfg->n_kv_heads * cfg->head_dim;
   const int qkvd = qd + 2 * kvd, F = cfg->ffn_dim;
   Carver w(nullptr);
+  int ctr = std::max({gemm_counters_needed(rows_cap, qkvd / 128), gemm_counters_needed(rows_cap, d / 128),
+                      gemm_counters_needed(rows_cap, F / 64)});
+  w.take<int>(ctr);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * d);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * F);
   size_t pf = std::max({gemm_partial_floats(rows_cap, qkvd / 128, d), gemm_partial_floats(rows_cap, d / 128, qd),
                         gemm_partial_floats(rows_cap, F / 64, d), gemm_partial_floats(rows_cap, d / 128, F)});
-  int ctr = std::max({gemm_counters_needed(rows_cap, qkvd / 128), gemm_counters_needed(rows_cap, d / 128),
-                      gemm_counters_needed(rows_cap, F / 64)});
   w.take<float>(pf);
-  w.take<int>(ctr);
   const int B = cfg->batch, N = cfg->prompt_len + cfg->gen_len;
   const int sp = attn_pick_splits(B, cfg->n_kv_heads, cfg->n_heads / cfg->n_kv_heads, rows_per_seq_cap, N);
   const size_t af = sp > 1 ? attn_partial_floats(rows_cap, cfg->n_heads, cfg->head_dim, sp) : 0;
@@ -785,23 +789,22 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
   L.kc = static_cast<__nv_bfloat16*>(kcache); L.vc = static_cast<__nv_bfloat16*>(vcache);
   L.rope_cos = rope_cos; L.rope_sin = rope_sin;
   Carver w(workspace);
+  int ctr = std::max({gemm_counters_needed(rows_cap, L.qkvd / 128), gemm_counters_needed(rows_cap, L.d / 128),
+                      gemm_counters_needed(rows_cap, L.F / 64)});
+  L.gs.counters = w.take<int>(ctr);
+  L.gs.n_counters = ctr;
   L.z = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.d);
   L.q = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
   L.attn = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
   L.act = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.F);
   size_t pf = std::max({gemm_partial_floats(rows_cap, L.qkvd / 128, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.qd),
                         gemm_partial_floats(rows_cap, L.F / 64, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.F)});
-  int ctr = std::max({gemm_counters_needed(rows_cap, L.qkvd / 128), gemm_counters_needed(rows_cap, L.d / 128),
-                      gemm_counters_needed(rows_cap, L.F / 64)});
   L.gs.partial = w.take<float>(pf);
   L.gs.partial_floats = pf;
-  L.gs.counters = w.take<int>(ctr);
-  L.gs.n_counters = ctr;
   const int sp = attn_pick_splits(L.B, L.Hkv, L.Hq / L.Hkv, rows_per_seq_cap, L.N);
   L.attn_floats = sp > 1 ? attn_partial_floats(rows_cap, L.Hq, L.hd, sp) : 0;
   L.attn_opart = w.take<float>(L.attn_floats);
   L.attn_ml = w.take<float2>(L.attn_floats / L.hd);
-  if (ctr) DLLM_CUDA_TRY(cudaMemsetAsync(L.gs.counters, 0, ctr * sizeof(int), st));
   return run_layer(L, h, rows, count, seq_off, rows_cap, rows_per_seq_cap, st);
 }
 

@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -32,16 +33,28 @@ constexpr int kBK = 64;                      // K elements per stage (128 B rows
 constexpr int kTileM = 128;                  // weight rows per tile
 constexpr uint32_t kABytes = kTileM * kBK * 2;
 
-template <int BN>
+// Pipeline depth and shared memory per tile width.  Weight-streaming widths (BN <= 64)
+// use ~100 KB so a CTA of the next GEMM fits beside the current one on an SM and starts
+// streaming its weights during this kernel's tail (programmatic dependent launch);
+// compute-bound widths take ~200 KB for a deeper ring.  Two TMEM accumulators let the
+// epilogue of one work segment overlap the MMAs of the next.
+template <int BN, int KSUB>
 struct Cfg {
-  static constexpr int kStages = (BN >= 256) ? 4 : 4;
-  static constexpr uint32_t kBBytes = BN * kBK * 2;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
-  static constexpr int kXPitch = 17;         // epilogue exchange buffer pitch (floats)
+  static constexpr uint32_t kBBytes = BN * kBK * 2;                // one 64-wide k block of X
+  static constexpr uint32_t kStageBytes = KSUB * (kABytes + kBBytes);
+  static constexpr uint32_t kBudget = (BN <= 64 ? 100u : 200u) * 1024u;
+  static constexpr int kStagesFit = static_cast<int>(kBudget / kStageBytes);
+  static constexpr int kStages = kStagesFit > 12 ? 12 : (kStagesFit < 2 ? 2 : kStagesFit);
+  static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // TMEM columns per accumulator
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static constexpr int kXPitch = 17;                                 // epilogue exchange pitch (floats)
   static constexpr size_t kSmem = 1024 /*align slack*/ + kStages * kStageBytes + 128 * kXPitch * 4 +
-                                  (2 * kStages + 2) * 8 + 64;
+                                  (2 * kStages + 4) * 8 + 64;
+  static_assert(kSmem <= 227 * 1024, "GEMM stage ring does not fit shared memory");
 };
+
+constexpr int kEpiThreads = 128;     // warps 0-3: epilogue, one thread per TMEM lane
+constexpr int kThreads = 192;        // + warp 4: TMA producer, warp 5: MMA issuer / TMEM owner
 
 struct KParams {
   int K;
@@ -49,14 +62,14 @@ struct KParams {
   const int* rows_dev;
   int n_tiles_w;
   int tiles_act;
-  int splits;
-  int kb_per_split;
   int swiglu;
   int ffn;
-  float* partial;
-  int* counters;
+  float* partial;      // [gridDim.x][2][BN * 128]
+  int* counters;       // [tiles]
   EpiParams epi;
 };
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -78,34 +91,190 @@ __device__ __forceinline__ void warp_argmax(float& v, int& id) {
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(128, 1)
+// Stream-K partition: CTA c owns the k-block iterations [lo(c), lo(c + 1)) of the
+// flattened (tile, k-block) space; first_cta(x) is the CTA whose range holds x.
+__device__ __forceinline__ int64_t sk_lo(int64_t T, int G, int c) { return T * c / G; }
+__device__ __forceinline__ int sk_first_cta(int64_t x, int64_t T, int G) {
+  return static_cast<int>(((x + 1) * G + T - 1) / T - 1);
+}
+
+// Epilogue of one 16-column chunk (columns = activation rows jbase..jbase+15) for the
+// weight row n held by TMEM lane t.  Exchange kinds synchronise the 128 epilogue threads.
+template <int XP>
+__device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[16], int t, int lane, int warp, int n,
+                                          int jbase, int m_rows, int tw, float* xb) {
+  switch (e.kind) {
+    case EPI_STORE_F32: {
+      float* o = static_cast<float*>(e.out);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (jbase + i < m_rows) o[static_cast<int64_t>(jbase + i) * e.ldo + n] = v[i];
+      break;
+    }
+    case EPI_STORE_BF16: {
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(e.out);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (jbase + i < m_rows) o[static_cast<int64_t>(jbase + i) * e.ldo + n] = __float2bfloat16(v[i]);
+      break;
+    }
+    case EPI_RESID_ADD: {
+      // all loads of the chunk are issued before any store (no serialised round trips)
+      int rr[16];
+      float old[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        rr[i] = (jbase + i < m_rows) ? (e.row_map ? __ldg(e.row_map + jbase + i) : jbase + i) : -1;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) old[i] = rr[i] >= 0 ? __ldcg(e.h + static_cast<int64_t>(rr[i]) * e.ldh + n) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (rr[i] >= 0) e.h[static_cast<int64_t>(rr[i]) * e.ldh + n] = old[i] + v[i];
+      break;
+    }
+    case EPI_QKV_ROPE: {
+      // rotate-half pairs (i, i + hd/2) of a head sit in lanes t and t ^ (hd/2)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xb[t * XP + i] = v[i];
+      const int hd = e.head_dim;
+      const int half = hd >> 1;
+      const int i_in_head = n % hd;
+      const int fi = i_in_head % half;
+      const bool lo = i_in_head < half;
+      const int region = n < e.q_dim ? 0 : (n < e.q_dim + e.kv_dim ? 1 : 2);
+      // gather every index and table entry of the chunk first
+      int pos[16], bb[16];
+      float cs[16], sn[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int j = jbase + i;
+        const int flat = j < m_rows ? __ldg(e.row_map + j) : 0;
+        bb[i] = flat / e.seq_n;
+        pos[i] = flat - bb[i] * e.seq_n;
+      }
+      if (region < 2) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          cs[i] = __ldg(e.rope_cos + static_cast<int64_t>(pos[i]) * half + fi);
+          sn[i] = __ldg(e.rope_sin + static_cast<int64_t>(pos[i]) * half + fi);
+        }
+      }
+      epi_bar();
+      const int partner = t ^ half;
+      float out[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float x = v[i];
+        if (region < 2) {
+          const float y = xb[partner * XP + i];
+          x = lo ? (x * cs[i] - y * sn[i]) : (x * cs[i] + y * sn[i]);
+        }
+        out[i] = x;
+      }
+      if (region == 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (jbase + i < m_rows) e.q_out[static_cast<int64_t>(jbase + i) * e.q_dim + n] = __float2bfloat16(out[i]);
+      } else {
+        const int nn = n - e.q_dim - (region == 2 ? e.kv_dim : 0);
+        const int kvh = nn / hd;
+        __nv_bfloat16* dst = region == 1 ? e.kcache : e.vcache;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (jbase + i < m_rows)
+            dst[((static_cast<int64_t>(bb[i]) * e.n_kv + kvh) * e.seq_n + pos[i]) * hd + (nn % hd)] =
+                __float2bfloat16(out[i]);
+      }
+      epi_bar();
+      break;
+    }
+    case EPI_SWIGLU: {
+      // lanes 0-63 hold gate rows, lanes 64-127 the matching up rows
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xb[t * XP + i] = v[i];
+      epi_bar();
+      if (t < 64) {
+        const int f = tw * 64 + t;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = jbase + i;
+          if (j < m_rows) {
+            const float g = v[i];
+            const float u = xb[(t + 64) * XP + i];
+            e.act[static_cast<int64_t>(j) * e.ffn + f] = __float2bfloat16(g / (1.f + __expf(-g)) * u);
+          }
+        }
+      }
+      epi_bar();
+      break;
+    }
+    case EPI_LMHEAD: {
+      // per row j: max, sum exp(x - max) and argmax over this tile's 128 vocabulary ids
+      float4* red = reinterpret_cast<float4*>(xb);   // [4 warps][16 cols]
+#pragma unroll 1
+      for (int i = 0; i < 16; ++i) {
+        const float x = v[i];
+        const float mx = warp_max(x);
+        const float se = warp_sum(__expf(x - mx));
+        float bv = (n == e.mask_id) ? -INFINITY : x;
+        int bi = (n == e.mask_id) ? 0x7fffffff : n;
+        warp_argmax(bv, bi);
+        if (lane == 0) red[warp * 16 + i] = make_float4(mx, se, bv, __int_as_float(bi));
+      }
+      epi_bar();
+      if (t < 16 && jbase + t < m_rows) {
+        float M = -INFINITY, S = 0.f, BV = -INFINITY;
+        int BI = 0x7fffffff;
+        for (int w = 0; w < 4; ++w) {
+          const float4 r = red[w * 16 + t];
+          const float nm = fmaxf(M, r.x);
+          S = S * __expf(M - nm) + r.y * __expf(r.x - nm);
+          M = nm;
+          const int ri = __float_as_int(r.w);
+          if (r.z > BV || (r.z == BV && ri < BI)) { BV = r.z; BI = ri; }
+        }
+        e.lm_part[static_cast<int64_t>(jbase + t) * e.n_vtiles + tw] = make_float4(M, S, BV, __int_as_float(BI));
+      }
+      epi_bar();
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+// Persistent stream-K GEMM: grid = one CTA per SM (or fewer), each CTA walks its
+// contiguous share of the (tile, k-block) iterations; a tile split across CTAs is
+// summed by the last CTA to finish its piece, in k order.
+template <int BN, int KSUB>
+__global__ void __launch_bounds__(kThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, KSUB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* xbuf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(xbuf + 128 * C::kXPitch);
   uint64_t* empty_bar = full_bar + C::kStages;
-  uint64_t* done_bar = empty_bar + C::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* acc_full = empty_bar + C::kStages;     // [2]
+  uint64_t* acc_empty = acc_full + 2;              // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last-piece
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tw = blockIdx.x;             // weight tile
-  const int ta = blockIdx.y;             // activation-row tile
-  const int z = blockIdx.z;              // K split
-  const int act0 = ta * BN;
-  const int m_rows = p.rows_dev ? min(*p.rows_dev, p.rows_cap) : p.rows_cap;
-  if (act0 >= m_rows) return;            // uniform: no valid rows in this tile
-
-  const int KB = p.K / kBK;
-  const int kb0 = z * p.kb_per_split;
-  const int kb1 = min(KB, kb0 + p.kb_per_split);
-  const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
-  const int row1 = p.swiglu ? p.ffn + tw * 64 : tw * kTileM + 64;
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  const int KB = p.K / (kBK * KSUB);                    // k chunks of KSUB x 64
+  const int tiles = p.n_tiles_w * p.tiles_act;
+  const int64_t T = static_cast<int64_t>(tiles) * KB;
+  const int64_t lo = sk_lo(T, G, c), hi = sk_lo(T, G, c + 1);
+  pdl_trigger();
+  if (lo >= hi) return;                                  // uniform: no work for this CTA
+  const int first_tile = static_cast<int>(lo / KB);
+  // With one activation tile every segment is processed (rows past the device count are
+  // masked in the epilogue), so weights can stream before the previous kernel finishes.
+  const bool single = p.tiles_act == 1;
 
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmW);
@@ -114,240 +283,222 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(done_bar, 1);
-    s_flag[0] = 0;   // abort flag
-    s_flag[1] = 0;   // split-K "last CTA" flag
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiThreads);
+    }
+    s_flag[0] = 0;
+    s_flag[1] = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (warp == 5) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    const uint64_t pol_w = policy_evict_first();
-    const uint64_t pol_x = policy_evict_last();
-    for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
-      const int s = i % C::kStages;
-      const uint32_t ph = (i / C::kStages) & 1;
-      if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
-      if (s_flag[0]) break;
-      uint8_t* a = stage_base + s * C::kStageBytes;
-      uint8_t* b = a + kABytes;
-      mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
-      tma_load_2d(a, &tmW, &full_bar[s], kb * kBK, row0, pol_w);
-      tma_load_2d(a + kABytes / 2, &tmW, &full_bar[s], kb * kBK, row1, pol_w);
-      tma_load_2d(b, &tmX, &full_bar[s], kb * kBK, act0, pol_x);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = make_idesc_bf16(kTileM, BN);
-    bool ok = true;
-    for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
-      const int s = i % C::kStages;
-      const uint32_t ph = (i / C::kStages) & 1;
-      if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; ok = false; break; }
-      tc_fence_after();
-      const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
-      const uint32_t b = a + kABytes;
-#pragma unroll
-      for (int k = 0; k < kBK / 16; ++k) {
-        tc_mma_f16(tmem, make_desc_k_sw128(a + k * 32), make_desc_k_sw128(b + k * 32), idesc,
-                   (kb > kb0 || k > 0) ? 1u : 0u);
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- TMA producer: one continuous ring over every segment
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int m_rows = p.rows_cap;
+      // stages whose weight tiles were requested before the grid dependency resolved
+      int pend_x[C::kStages], pend_a[C::kStages], n_pend = 0;
+      bool waited = false;
+      if (!single) {
+        pdl_wait();
+        waited = true;
+        m_rows = p.rows_dev ? min(*p.rows_dev, p.rows_cap) : p.rows_cap;
       }
-      tc_commit(&empty_bar[s]);
-    }
-    (void)ok;
-    tc_commit(done_bar);
-  }
-  __syncwarp();
-
-  // ---------------- epilogue (all 128 threads)
-  const int t = threadIdx.x;
-  if (!mbar_wait(done_bar, 0)) s_flag[0] = 1;
-  tc_fence_after();
-  const uint32_t tbase = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  const EpiParams& e = p.epi;
-  __syncthreads();
-  bool do_epi = !s_flag[0];   // uniform across the CTA
-
-  const int tile_lin = tw * p.tiles_act + ta;
-  if (do_epi && p.splits > 1) {
-    float* mine = p.partial + (static_cast<size_t>(tile_lin) * p.splits + z) * (BN * 128);
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      tmem_ld16(tbase + c, v);
+      int i = 0;
+      for (int64_t it = lo; it < hi && !s_flag[0];) {
+        const int tile = static_cast<int>(it / KB);
+        const int kb0 = static_cast<int>(it % KB);
+        const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+        it += kb1 - kb0;
+        const int tw = tile / p.tiles_act, ta = tile % p.tiles_act;
+        const int act0 = ta * BN;
+        if (!single && act0 >= m_rows) continue;     // tile without valid rows: skipped by every role
+        const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
+        const int row1 = p.swiglu ? p.ffn + tw * 64 : tw * kTileM + 64;
+        for (int kb = kb0; kb < kb1; ++kb, ++i) {
+          const int s = i % C::kStages;
+          const uint32_t ph = (i / C::kStages) & 1;
+          if (!waited && i >= C::kStages) {
+            // the ring is full of weight tiles: now the activations are needed
+            pdl_wait();
+            waited = true;
+            for (int q = 0; q < n_pend; ++q) {
+              uint8_t* bx = stage_base + q * C::kStageBytes + KSUB * kABytes;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) mine[(c + i) * 128 + t] = v[i];
-    }
-    __threadfence();
-    __syncthreads();
-    if (t == 0) {
-      const int old = atomicAdd(&p.counters[tile_lin], 1);
-      s_flag[1] = (old == p.splits - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    do_epi = s_flag[1] != 0;
-    __threadfence();
-  }
-
-  if (do_epi) {
-    const int hd = e.head_dim;
-    const int n = row0 + (t < 64 ? t : (row1 - row0) + t - 64);   // global weight row of this lane
-    float* xb = xbuf;
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      if (p.splits > 1) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        for (int zz = 0; zz < p.splits; ++zz) {
-          if (zz == z) {
-            float w[16];
-            tmem_ld16(tbase + c, w);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] += w[i];
-          } else {
-            const float* src = p.partial + (static_cast<size_t>(tile_lin) * p.splits + zz) * (BN * 128);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] += __ldcg(src + (c + i) * 128 + t);
+              for (int sub = 0; sub < KSUB; ++sub)
+                tma_load_2d(bx + sub * C::kBBytes, &tmX, &full_bar[q], pend_x[q] + sub * kBK, pend_a[q], pol_x);
+            }
+            n_pend = 0;
           }
+          if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
+          uint8_t* a = stage_base + s * C::kStageBytes;
+          uint8_t* bx = a + KSUB * kABytes;
+          mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
+#pragma unroll
+          for (int sub = 0; sub < KSUB; ++sub) {
+            const int x = (kb * KSUB + sub) * kBK;
+            tma_load_2d(a + sub * kABytes, &tmW, &full_bar[s], x, row0, pol_w);
+            tma_load_2d(a + sub * kABytes + kABytes / 2, &tmW, &full_bar[s], x, row1, pol_w);
+          }
+          if (waited) {
+#pragma unroll
+            for (int sub = 0; sub < KSUB; ++sub)
+              tma_load_2d(bx + sub * C::kBBytes, &tmX, &full_bar[s], (kb * KSUB + sub) * kBK, act0, pol_x);
+          } else {
+            pend_x[n_pend] = kb * KSUB * kBK;
+            pend_a[n_pend] = act0;
+            ++n_pend;
+          }
+        }
+      }
+      if (!waited) {
+        pdl_wait();
+        for (int q = 0; q < n_pend; ++q) {
+          uint8_t* bx = stage_base + q * C::kStageBytes + KSUB * kABytes;
+#pragma unroll
+          for (int sub = 0; sub < KSUB; ++sub)
+            tma_load_2d(bx + sub * C::kBBytes, &tmX, &full_bar[q], pend_x[q] + sub * kBK, pend_a[q], pol_x);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: alternates between the two TMEM accumulators
+      constexpr uint32_t idesc = make_idesc_bf16(kTileM, BN);
+      int m_rows = p.rows_cap;
+      if (!single) {
+        pdl_wait();
+        m_rows = p.rows_dev ? min(*p.rows_dev, p.rows_cap) : p.rows_cap;
+      }
+      int i = 0, j = 0;
+      for (int64_t it = lo; it < hi && !s_flag[0];) {
+        const int tile = static_cast<int>(it / KB);
+        const int kb0 = static_cast<int>(it % KB);
+        const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+        it += kb1 - kb0;
+        if (!single && (tile % p.tiles_act) * BN >= m_rows) continue;
+        const int b = j & 1;
+        const uint32_t u = static_cast<uint32_t>(j >> 1);
+        ++j;
+        if (!mbar_wait(&acc_empty[b], (u & 1) ^ 1)) { s_flag[0] = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + b * C::kAccCols;
+        for (int kb = kb0; kb < kb1; ++kb, ++i) {
+          const int s = i % C::kStages;
+          const uint32_t ph = (i / C::kStages) & 1;
+          if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
+          const uint32_t bb = a + KSUB * kABytes;
+#pragma unroll
+          for (int sub = 0; sub < KSUB; ++sub)
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              tc_mma_f16(d, make_desc_k_sw128(a + sub * kABytes + k * 32),
+                         make_desc_k_sw128(bb + sub * C::kBBytes + k * 32), idesc,
+                         (kb > kb0 || sub > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&empty_bar[s]);
+        }
+        tc_commit(&acc_full[b]);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 0-3
+    const int t = threadIdx.x;
+    const EpiParams& e = p.epi;
+    pdl_wait();
+    const int m_rows = p.rows_dev ? min(*p.rows_dev, p.rows_cap) : p.rows_cap;
+    int j = 0;
+    for (int64_t it = lo; it < hi;) {
+      const int tile = static_cast<int>(it / KB);
+      const int kb0 = static_cast<int>(it % KB);
+      const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+      it += kb1 - kb0;
+      const int tw = tile / p.tiles_act, ta = tile % p.tiles_act;
+      const int act0 = ta * BN;
+      if (!single && act0 >= m_rows) continue;
+      const int b = j & 1;
+      const uint32_t u = static_cast<uint32_t>(j >> 1);
+      ++j;
+      if (!mbar_wait(&acc_full[b], u & 1)) s_flag[0] = 1;
+      epi_bar();
+      if (s_flag[0]) break;                            // uniform after the barrier
+      tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * C::kAccCols;
+      const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
+      const int row1 = p.swiglu ? p.ffn + tw * 64 : tw * kTileM + 64;
+      const int n = t < 64 ? row0 + t : row1 + (t - 64);
+      const bool whole = (kb0 == 0 && kb1 == KB);
+      if (whole) {
+        for (int cc = 0; cc < BN; cc += 16) {
+          float v[16];
+          tmem_ld16(tb + cc, v);
+          if (cc + 16 >= BN) {                         // accumulator drained: hand it back
+            tc_fence_before();
+            mbar_arrive(&acc_empty[b]);
+          }
+          epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, act0 + cc, m_rows, tw, xbuf);
         }
       } else {
-        tmem_ld16(tbase + c, v);
-      }
-      const int jbase = act0 + c;
-      switch (e.kind) {
-        case EPI_STORE_F32: {
-          float* o = static_cast<float*>(e.out);
+        // a piece of a split tile: store it, then the last piece to arrive sums all of them
+        const int which = (tile == first_tile) ? 0 : 1;
+        float* mine = p.partial + (static_cast<size_t>(c) * 2 + which) * (BN * 128);
+        for (int cc = 0; cc < BN; cc += 16) {
+          float v[16];
+          tmem_ld16(tb + cc, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (jbase + i < m_rows) o[static_cast<int64_t>(jbase + i) * e.ldo + n] = v[i];
-          break;
+          for (int q = 0; q < 16; ++q) mine[(cc + q) * 128 + t] = v[q];
         }
-        case EPI_STORE_BF16: {
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(e.out);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (jbase + i < m_rows) o[static_cast<int64_t>(jbase + i) * e.ldo + n] = __float2bfloat16(v[i]);
-          break;
+        tc_fence_before();
+        mbar_arrive(&acc_empty[b]);
+        __threadfence();
+        epi_bar();
+        const int64_t x0 = static_cast<int64_t>(tile) * KB;
+        const int c_first = sk_first_cta(x0, T, G);
+        const int c_last = sk_first_cta(x0 + KB - 1, T, G);
+        if (t == 0) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          s_flag[1] = (old == c_last - c_first) ? 1 : 0;
         }
-        case EPI_RESID_ADD: {
+        epi_bar();
+        if (s_flag[1]) {
+          __threadfence();
+          for (int cc = 0; cc < BN; cc += 16) {
+            float v[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (jbase + i < m_rows) {
-              const int r = e.row_map ? __ldg(e.row_map + jbase + i) : jbase + i;
-              float* dst = e.h + static_cast<int64_t>(r) * e.ldh + n;
-              *dst = *dst + v[i];
+            for (int q = 0; q < 16; ++q) v[q] = 0.f;
+            for (int cp = c_first; cp <= c_last; ++cp) {
+              const int wp = (tile == static_cast<int>(sk_lo(T, G, cp) / KB)) ? 0 : 1;
+              const float* src = p.partial + (static_cast<size_t>(cp) * 2 + wp) * (BN * 128);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) v[q] += __ldcg(src + (cc + q) * 128 + t);
             }
+            epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, act0 + cc, m_rows, tw, xbuf);
           }
-          break;
+          if (t == 0) p.counters[tile] = 0;
         }
-        case EPI_QKV_ROPE: {
-          // exchange with the rotate-half partner lane (same head, offset hd/2)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) xb[t * C::kXPitch + i] = v[i];
-          __syncthreads();
-          const int half = hd >> 1;
-          const int partner = t ^ half;
-          const int i_in_head = n % hd;
-          const int fi = i_in_head % half;
-          const bool lo = i_in_head < half;
-          const int region = n < e.q_dim ? 0 : (n < e.q_dim + e.kv_dim ? 1 : 2);
-#pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
-            const int j = jbase + i;
-            if (j < m_rows) {
-              const int flat = __ldg(e.row_map + j);
-              const int b = flat / e.seq_n;
-              const int pos = flat - b * e.seq_n;
-              float x = v[i];
-              if (region < 2) {
-                const float y = xb[partner * C::kXPitch + i];
-                const float cs = __ldg(e.rope_cos + static_cast<int64_t>(pos) * half + fi);
-                const float sn = __ldg(e.rope_sin + static_cast<int64_t>(pos) * half + fi);
-                x = lo ? (x * cs - y * sn) : (x * cs + y * sn);
-              }
-              const __nv_bfloat16 xv = __float2bfloat16(x);
-              if (region == 0) {
-                e.q_out[static_cast<int64_t>(j) * e.q_dim + n] = xv;
-              } else {
-                const int nn = n - e.q_dim - (region == 2 ? e.kv_dim : 0);
-                const int kvh = nn / hd;
-                const int64_t off = ((static_cast<int64_t>(b) * e.n_kv + kvh) * e.seq_n + pos) * hd + (nn % hd);
-                (region == 1 ? e.kcache : e.vcache)[off] = xv;
-              }
-            }
-          }
-          __syncthreads();
-          break;
-        }
-        case EPI_SWIGLU: {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) xb[t * C::kXPitch + i] = v[i];
-          __syncthreads();
-          if (t < 64) {
-            const int f = tw * 64 + t;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int j = jbase + i;
-              if (j < m_rows) {
-                const float g = v[i];
-                const float u = xb[(t + 64) * C::kXPitch + i];
-                const float a = g / (1.f + __expf(-g)) * u;
-                e.act[static_cast<int64_t>(j) * e.ffn + f] = __float2bfloat16(a);
-              }
-            }
-          }
-          __syncthreads();
-          break;
-        }
-        case EPI_LMHEAD: {
-          // per row j: max, sum exp(x - max), argmax over this tile's 128 vocab ids
-          float4* red = reinterpret_cast<float4*>(xb);   // [4 warps][16 cols]
-#pragma unroll 1
-          for (int i = 0; i < 16; ++i) {
-            const float x = v[i];
-            const float mx = warp_max(x);
-            const float se = warp_sum(__expf(x - mx));
-            float bv = (n == e.mask_id) ? -INFINITY : x;
-            int bi = (n == e.mask_id) ? 0x7fffffff : n;
-            warp_argmax(bv, bi);
-            if (lane == 0) red[warp * 16 + i] = make_float4(mx, se, bv, __int_as_float(bi));
-          }
-          __syncthreads();
-          if (t < 16 && jbase + t < m_rows) {
-            float M = -INFINITY, S = 0.f, BV = -INFINITY;
-            int BI = 0x7fffffff;
-            for (int w = 0; w < 4; ++w) {
-              const float4 r = red[w * 16 + t];
-              const float nm = fmaxf(M, r.x);
-              S = S * __expf(M - nm) + r.y * __expf(r.x - nm);
-              M = nm;
-              const int ri = __float_as_int(r.w);
-              if (r.z > BV || (r.z == BV && ri < BI)) { BV = r.z; BI = ri; }
-            }
-            e.lm_part[static_cast<int64_t>(jbase + t) * e.n_vtiles + tw] = make_float4(M, S, BV, __int_as_float(BI));
-          }
-          __syncthreads();
-          break;
-        }
-        default:
-          break;
+        epi_bar();
       }
     }
-    if (p.splits > 1 && t == 0) p.counters[tile_lin] = 0;
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 5) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 __global__ void lmhead_combine_kernel(const float4* __restrict__ part, int n_vtiles, int rows_cap,
                                       const int* rows_dev, const int* out_index, float* conf, int* amax,
                                       float* lse) {
+  pdl_trigger();
+  pdl_wait();
   const int m_rows = rows_dev ? min(*rows_dev, rows_cap) : rows_cap;
   const int j = blockIdx.x;
   if (j >= m_rows) return;
@@ -437,46 +588,60 @@ int pick_bn(int rows) {
   return 256;
 }
 
-int pick_splits(int tiles, int KB) {
-  if (tiles >= kNumSMs) return 1;
-  // aim for about two resident CTAs per SM, at least 4 K blocks per split
-  int best = 1;
-  double best_eff = 0;
-  const int max_s = std::max(1, KB / 4);
-  for (int s = 1; s <= max_s && s <= 32; ++s) {
-    const int total = tiles * s;
-    const int slots = 2 * kNumSMs;
-    const int waves = (total + slots - 1) / slots;
-    const double eff = static_cast<double>(total) / (waves * slots) - 0.01 * s;
-    if (eff > best_eff) { best_eff = eff; best = s; }
-  }
-  return best;
+// Grid of the persistent kernel: one CTA per SM, never more CTAs than k-block iterations.
+int pick_grid(int tiles, int KB) {
+  const int64_t T = static_cast<int64_t>(tiles) * KB;
+  return static_cast<int>(std::min<int64_t>(kNumSMs, T));
 }
 
-template <int BN>
-int launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, cudaStream_t st) {
-  using C = Cfg<BN>;
+template <int BN, int KSUB>
+int launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, cudaStream_t st) {
+  using C = Cfg<BN, KSUB>;
   static bool attr_done = false;
   if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    DLLM_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem)));
     attr_done = true;
   }
-  dim3 grid(kp.n_tiles_w, kp.tiles_act, kp.splits);
-  gemm_tc_kernel<BN><<<grid, 128, C::kSmem, st>>>(tmW, tmX, kp);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  gemm_tc_kernel<BN, KSUB>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
+}
+
+// Widest KSUB whose two-stage ring still fits shared memory for this tile width.
+constexpr int max_ksub(int bn) { return bn <= 64 ? 4 : (bn <= 128 ? 2 : 1); }
+
+template <int BN>
+int launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, int ksub, cudaStream_t st) {
+  if constexpr (max_ksub(BN) >= 4) {
+    if (ksub >= 4) return launch_cfg<BN, 4>(tmW, tmX, kp, grid, st);
+  }
+  if constexpr (max_ksub(BN) >= 2) {
+    if (ksub >= 2) return launch_cfg<BN, 2>(tmW, tmX, kp, grid, st);
+  }
+  return launch_cfg<BN, 1>(tmW, tmX, kp, grid, st);
+}
+
+// k blocks fetched per pipeline stage: consecutive 128-byte pieces of every weight row are
+// requested together, so each DRAM page opened for a row serves several of them.
+int pick_ksub(int K, int bn) {
+  const char* env = getenv("DLLM_GEMM_KSUB");
+  const int KB = K / kBK;
+  int want = std::min(env ? atoi(env) : 4, max_ksub(bn));
+  for (int k : {4, 2, 1})
+    if (k <= want && KB % k == 0) return k;
+  return 1;
 }
 
 }  // namespace
 
 size_t gemm_partial_floats(int rows_cap, int n_tiles_w, int K) {
+  (void)n_tiles_w;
+  (void)K;
   const int bn = pick_bn(rows_cap);
-  const int tiles_act = (rows_cap + bn - 1) / bn;
-  const int s = pick_splits(n_tiles_w * tiles_act, K / kBK);
-  if (s <= 1) return 0;
-  return static_cast<size_t>(n_tiles_w) * tiles_act * s * bn * 128;
+  return static_cast<size_t>(kNumSMs) * 2 * bn * 128;
 }
 
 int gemm_counters_needed(int rows_cap, int n_tiles_w) {
@@ -484,22 +649,22 @@ int gemm_counters_needed(int rows_cap, int n_tiles_w) {
   return n_tiles_w * ((rows_cap + bn - 1) / bn);
 }
 
-int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int force_splits, int force_bn) {
+int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int force_grid, int force_bn) {
   if (a.K <= 0 || a.K % kBK != 0 || a.rows_cap <= 0 || a.n_tiles_w <= 0) return DLLM_ERR_SHAPE;
   const int bn = force_bn ? force_bn : pick_bn(a.rows_cap);
   if (bn != 16 && bn != 32 && bn != 64 && bn != 128 && bn != 256) return DLLM_ERR_INVALID_ARG;
   const int tiles_act = (a.rows_cap + bn - 1) / bn;
-  const int KB = a.K / kBK;
-  int splits = force_splits ? force_splits : pick_splits(a.n_tiles_w * tiles_act, KB);
-  splits = std::max(1, std::min(splits, KB));
-  const int kbps = (KB + splits - 1) / splits;
-  splits = (KB + kbps - 1) / kbps;   // no empty split
-  if (splits > 1) {
-    const size_t need = static_cast<size_t>(a.n_tiles_w) * tiles_act * splits * bn * 128;
-    if (!s.partial || s.partial_floats < need || !s.counters || s.n_counters < a.n_tiles_w * tiles_act) {
-      // not enough scratch for split-K: run unsplit
-      splits = 1;
-    }
+  const int tiles = a.n_tiles_w * tiles_act;
+  const int ksub = pick_ksub(a.K, bn);
+  const int KB = a.K / (kBK * ksub);
+  int grid = force_grid > 0 ? force_grid : pick_grid(tiles, KB);
+  grid = static_cast<int>(std::min<int64_t>(grid, static_cast<int64_t>(tiles) * KB));
+  // split tiles need the partial buffer and one counter per tile; without them every
+  // CTA takes whole tiles only (grid = number of tiles divides the work exactly)
+  const size_t need = static_cast<size_t>(grid) * 2 * bn * 128;
+  if (!s.partial || s.partial_floats < need || !s.counters || s.n_counters < tiles) {
+    if (static_cast<int64_t>(tiles) * KB % grid != 0 || tiles % grid != 0) grid = std::min(grid, tiles);
+    while (grid > 1 && tiles % grid != 0) --grid;
   }
   CUtensorMap tmW, tmX;
   int rc = make_tmap(&tmW, a.W, a.w_rows_total, a.K, 64);
@@ -512,28 +677,27 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   kp.rows_dev = a.rows_dev;
   kp.n_tiles_w = a.n_tiles_w;
   kp.tiles_act = tiles_act;
-  kp.splits = splits;
-  kp.kb_per_split = (KB + splits - 1) / splits;
   kp.swiglu = a.swiglu ? 1 : 0;
   kp.ffn = a.epi.ffn;
   kp.partial = s.partial;
   kp.counters = s.counters;
   kp.epi = a.epi;
   switch (bn) {
-    case 16: return launch_bn<16>(tmW, tmX, kp, st);
-    case 32: return launch_bn<32>(tmW, tmX, kp, st);
-    case 64: return launch_bn<64>(tmW, tmX, kp, st);
-    case 128: return launch_bn<128>(tmW, tmX, kp, st);
-    default: return launch_bn<256>(tmW, tmX, kp, st);
+    case 16: return launch_bn<16>(tmW, tmX, kp, grid, ksub, st);
+    case 32: return launch_bn<32>(tmW, tmX, kp, grid, ksub, st);
+    case 64: return launch_bn<64>(tmW, tmX, kp, grid, ksub, st);
+    case 128: return launch_bn<128>(tmW, tmX, kp, grid, ksub, st);
+    default: return launch_bn<256>(tmW, tmX, kp, grid, ksub, st);
   }
 }
 
 int lmhead_combine_launch(const float4* part, int n_vtiles, int rows_cap, const int* rows_dev,
                           const int* out_index, float* conf, int* amax, float* lse, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
-  lmhead_combine_kernel<<<rows_cap, 256, 0, st>>>(part, n_vtiles, rows_cap, rows_dev, out_index, conf, amax, lse);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  lmhead_combine_kernel, dim3(rows_cap), dim3(256), 0, st, part, n_vtiles, rows_cap, rows_dev, out_index, conf, amax, lse);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 

@@ -31,21 +31,21 @@ struct OpCarver {
   }
 };
 
-// split-K scratch for one GEMM; counters are zeroed on the stream
-int gemm_scratch(OpCarver& cv, int rows_cap, int tiles, int K, int splits, int bn, GemmScratch& gs,
-                 cudaStream_t st) {
-  const int b = bn ? bn : (rows_cap <= 16 ? 16 : rows_cap <= 32 ? 32 : rows_cap <= 64 ? 64 : rows_cap <= 128 ? 128 : 256);
-  const int ta = (rows_cap + b - 1) / b;
-  size_t pf = gemm_partial_floats(rows_cap, tiles, K);
-  if (splits > 1) pf = std::max(pf, static_cast<size_t>(tiles) * ta * splits * b * 128);
-  const int nc = tiles * ta;
-  if (pf == 0) return DLLM_OK;
+// Scratch of one GEMM launched through an op: the tile counters live at the start of the
+// workspace (the caller zeroes the workspace once; every GEMM leaves its counters at zero),
+// the partial tiles of split work follow.
+constexpr int kOpCounters = 65536;
+
+int gemm_scratch(OpCarver& cv, int rows_cap, int tiles, int K, GemmScratch& gs) {
+  const int b = rows_cap <= 16 ? 16 : rows_cap <= 32 ? 32 : rows_cap <= 64 ? 64 : rows_cap <= 128 ? 128 : 256;
+  const int nc = tiles * ((rows_cap + b - 1) / b);
+  if (nc > kOpCounters) OP_FAIL(DLLM_ERR_SHAPE, "too many output tiles for the op workspace");
+  gs.counters = cv.take<int>(kOpCounters);
+  const size_t pf = gemm_partial_floats(rows_cap, tiles, K);
   gs.partial = cv.take<float>(pf);
-  gs.counters = cv.take<int>(nc);
-  if (!cv.ok) OP_FAIL(DLLM_ERR_SHAPE, "workspace too small for split-K partials");
+  if (!cv.ok) OP_FAIL(DLLM_ERR_SHAPE, "workspace too small for the GEMM scratch");
   gs.partial_floats = pf;
   gs.n_counters = nc;
-  DLLM_CUDA_TRY(cudaMemsetAsync(gs.counters, 0, nc * sizeof(int), st));
   return DLLM_OK;
 }
 
@@ -82,7 +82,7 @@ int dllm_op_gemm(int32_t kind, const void* W, int32_t n_out, const void* X, int3
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
-  const int rc = gemm_scratch(cv, rows_cap, n_out / 128, K, splits, bn, gs, st);
+  const int rc = gemm_scratch(cv, rows_cap, n_out / 128, K, gs);
   if (rc) return rc;
   GemmArgs a;
   a.W = W; a.w_rows_total = n_out; a.X = X; a.rows_cap = rows_cap; a.rows_dev = count; a.K = K;
@@ -109,7 +109,7 @@ int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32
   const int qkvd = qd + 2 * kvd;
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
-  const int rc = gemm_scratch(cv, rows_cap, qkvd / 128, d, splits, 0, gs, st);
+  const int rc = gemm_scratch(cv, rows_cap, qkvd / 128, d, gs);
   if (rc) return rc;
   GemmArgs g;
   g.W = W; g.w_rows_total = qkvd; g.X = X; g.rows_cap = rows_cap; g.rows_dev = count; g.K = d;
@@ -128,7 +128,7 @@ int dllm_op_gate_up(const void* W, int32_t F, const void* X, int32_t rows_cap, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
-  const int rc = gemm_scratch(cv, rows_cap, F / 64, d, splits, 0, gs, st);
+  const int rc = gemm_scratch(cv, rows_cap, F / 64, d, gs);
   if (rc) return rc;
   GemmArgs g;
   g.W = W; g.w_rows_total = 2 * F; g.X = X; g.rows_cap = rows_cap; g.rows_dev = count; g.K = d;
@@ -167,15 +167,15 @@ int dllm_op_lm_head(const void* W, int32_t V, const void* X, int32_t rows_cap, c
   if (V % 128 || d % 64) OP_FAIL(DLLM_ERR_SHAPE, "V must be a multiple of 128 and d of 64");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   OpCarver cv(workspace, workspace_bytes);
+  GemmScratch gs;
+  const int rc = gemm_scratch(cv, rows_cap, V / 128, d, gs);
+  if (rc) return rc;
   float4* part = cv.take<float4>(static_cast<size_t>(rows_cap) * (V / 128));
   if (!cv.ok) OP_FAIL(DLLM_ERR_SHAPE, "workspace too small for LM-head partials");
-  GemmScratch gs;
-  const int rc = gemm_scratch(cv, rows_cap, V / 128, d, 0, 0, gs, st);
-  if (rc) return rc;
   GemmArgs g;
   g.W = W; g.w_rows_total = V; g.X = X; g.rows_cap = rows_cap; g.rows_dev = count; g.K = d; g.n_tiles_w = V / 128;
   g.epi.kind = EPI_LMHEAD; g.epi.lm_part = part; g.epi.n_vtiles = V / 128; g.epi.mask_id = mask_id;
-  int r = gemm_launch(g, gs, st, 1, 0);
+  int r = gemm_launch(g, gs, st, 0, 0);
   if (r) return r;
   return lmhead_combine_launch(part, V / 128, rows_cap, count, out_index, conf, argmax, lse, st);
 }

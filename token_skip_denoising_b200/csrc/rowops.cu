@@ -19,6 +19,8 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 
 // ------------------------------------------------------------------ RoPE table
 __global__ void rope_table_kernel(float* cos_t, float* sin_t, int N, int half, double theta, int hd) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= N * half) return;
   const int pos = idx / half, i = idx % half;
@@ -35,6 +37,8 @@ __global__ void rope_table_kernel(float* cos_t, float* sin_t, int N, int half, d
 __global__ void embed_rows_kernel(const __nv_bfloat16* __restrict__ E, const int* __restrict__ tokens,
                                   const int* __restrict__ row_map, const int* count_dev, int rows_cap, int d,
                                   float* __restrict__ h) {
+  pdl_trigger();
+  pdl_wait();
   const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
   const int j = blockIdx.x;
   if (j >= m) return;
@@ -61,6 +65,8 @@ __global__ void embed_rows_kernel(const __nv_bfloat16* __restrict__ E, const int
 __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int* __restrict__ row_map,
                                     const int* count_dev, int rows_cap, int d, const float* __restrict__ g,
                                     float eps, __nv_bfloat16* __restrict__ z, int64_t ldz) {
+  pdl_trigger();
+  pdl_wait();
   const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
   const int j = blockIdx.x;
   if (j >= m) return;
@@ -106,6 +112,8 @@ __global__ void score_es_kernel(const float* __restrict__ h, float* __restrict__
                                 const float* __restrict__ conf, uint8_t* __restrict__ masked_prev,
                                 const int* __restrict__ tokens, int mask_id, const int* __restrict__ rows,
                                 int n_rows, int d, float alpha, int update, float* __restrict__ score) {
+  pdl_trigger();
+  pdl_wait();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= n_rows) return;
@@ -137,6 +145,8 @@ __global__ void score_es_kernel(const float* __restrict__ h, float* __restrict__
 __global__ void score_cos_kernel(const float* __restrict__ vnew, int64_t ldv, const __nv_bfloat16* __restrict__ vc,
                                  const int* __restrict__ rows, const int* count_dev, int rows_cap, int N, int Hkv,
                                  int hd, float* __restrict__ sim) {
+  pdl_trigger();
+  pdl_wait();
   const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -174,6 +184,8 @@ __global__ void kl_conf_kernel(const __nv_bfloat16* __restrict__ z, int64_t ldz,
                                const int* __restrict__ rows, const int* count_dev, int rows_cap, int V, int mask_id,
                                float* __restrict__ conf, int* __restrict__ amax, float* __restrict__ lse_out,
                                float* __restrict__ kl_out) {
+  pdl_trigger();
+  pdl_wait();
   const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
   const int j = blockIdx.x;
   if (j >= m) return;
@@ -301,6 +313,8 @@ __device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int& total) {
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ uint32_t keys[kSelMaxN];
   __shared__ uint8_t elig[kSelMaxN];
   __shared__ int hist[256];
@@ -396,6 +410,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
 // ------------------------------------------------------------------ row lists
 // Rows of a contiguous position range per sequence: row_map = b * N + start + i.
 __global__ void range_rows_kernel(int B, int N, int start, int len, int* row_map, int* seq_off, int* total) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < B * len) row_map[idx] = (idx / len) * N + start + (idx % len);
   if (idx <= B && seq_off) seq_off[idx] = idx * len;
@@ -409,6 +425,8 @@ __global__ void __launch_bounds__(kSelThreads) lm_rows_kernel(const int* __restr
                                                               int N, int blk_s, int blk_e,
                                                               const uint8_t* __restrict__ round_mask,
                                                               int* __restrict__ lm_rows, int* lm_count) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_warp[32];
   const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
   int carry = 0;
@@ -434,6 +452,8 @@ __global__ void __launch_bounds__(kSelThreads) lm_rows_kernel(const int* __restr
 __global__ void snapshot_rows_kernel(const float* __restrict__ h, float* __restrict__ h_prev,
                                      const int* __restrict__ tokens, uint8_t* __restrict__ masked_prev, int mask_id,
                                      const int* __restrict__ rows, int n_rows, int d) {
+  pdl_trigger();
+  pdl_wait();
   const int j = blockIdx.x;
   if (j >= n_rows) return;
   const int flat = rows[j];
@@ -451,6 +471,8 @@ __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict_
                               int N, int blk_s, int blk_len, int mask_id, int n_commit,
                               const uint8_t* __restrict__ round_mask, int* __restrict__ pos_out,
                               int* __restrict__ tok_out, int* __restrict__ n_out, int max_out) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float s_conf[];
   uint8_t* s_masked = reinterpret_cast<uint8_t*>(s_conf + blk_len);
   __shared__ int s_cnt;
@@ -499,9 +521,10 @@ __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict_
 int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st) {
   const int half = hd / 2;
   const int n = N * half;
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(cos_t, sin_t, N, half, theta, hd);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, cos_t, sin_t, N, half, theta, hd);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -509,9 +532,10 @@ int embed_rows_launch(const __nv_bfloat16* E, const int* tokens, const int* row_
                       int rows_cap, int d, float* h, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
   if (d % 8) return DLLM_ERR_SHAPE;
-  embed_rows_kernel<<<rows_cap, 128, 0, st>>>(E, tokens, row_map, count_dev, rows_cap, d, h);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  embed_rows_kernel, dim3(rows_cap), dim3(128), 0, st, E, tokens, row_map, count_dev, rows_cap, d, h);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -519,9 +543,10 @@ int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev
                         float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
   if (d % 4) return DLLM_ERR_SHAPE;
-  rmsnorm_rows_kernel<<<rows_cap, 256, 0, st>>>(h, row_map, count_dev, rows_cap, d, g, eps, z, ldz);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  rmsnorm_rows_kernel, dim3(rows_cap), dim3(256), 0, st, h, row_map, count_dev, rows_cap, d, g, eps, z, ldz);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -531,10 +556,11 @@ int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* m
   if (n_rows <= 0) return DLLM_OK;
   if (d % 4) return DLLM_ERR_SHAPE;
   const int blocks = (n_rows * 32 + 255) / 256;
-  score_es_kernel<<<blocks, 256, 0, st>>>(h, h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
+{
+    const int rc_ = launch_pdl(  score_es_kernel, dim3(blocks), dim3(256), 0, st, h, h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
                                           update, score);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -542,9 +568,10 @@ int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, co
                      int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
   const int blocks = (rows_cap * 32 + 255) / 256;
-  score_cos_kernel<<<blocks, 256, 0, st>>>(vnew, ldv, vc, rows, count_dev, rows_cap, N, Hkv, hd, sim);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  score_cos_kernel, dim3(blocks), dim3(256), 0, st, vnew, ldv, vc, rows, count_dev, rows_cap, N, Hkv, hd, sim);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -552,45 +579,50 @@ int kl_conf_launch(const __nv_bfloat16* z, int64_t ldz, const __nv_bfloat16* zp_
                    const float* lse_prev, const int* has_prev, const int* rows, const int* count_dev, int rows_cap,
                    int V, int mask_id, float* conf, int* amax, float* lse_out, float* kl_out, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
-  kl_conf_kernel<<<rows_cap, 256, 0, st>>>(z, ldz, zp_store, ldp, lse_prev, has_prev, rows, count_dev, rows_cap, V,
+{
+    const int rc_ = launch_pdl(  kl_conf_kernel, dim3(rows_cap), dim3(256), 0, st, z, ldz, zp_store, ldp, lse_prev, has_prev, rows, count_dev, rows_cap, V,
                                            mask_id, conf, amax, lse_out, kl_out);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
 int select_launch(const SelectParams& p, cudaStream_t st) {
   if (p.B <= 0) return DLLM_OK;
   if (p.n < 0 || p.n > kSelMaxN) return DLLM_ERR_UNSUPPORTED;
-  select_kernel<<<1, kSelThreads, 0, st>>>(p);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  select_kernel, dim3(1), dim3(kSelThreads), 0, st, p);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
 int range_rows_launch(int B, int N, int start, int len, int* row_map, int* seq_off, int* total, cudaStream_t st) {
   const int n = std::max(B * len, B + 1);
-  range_rows_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, N, start, len, row_map, seq_off, total);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  range_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, B, N, start, len, row_map, seq_off, total);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
 int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const int* tokens, int mask_id, int N,
                    int blk_s, int blk_e, const uint8_t* round_mask, int* lm_rows, int* lm_count, cudaStream_t st) {
-  lm_rows_kernel<<<1, kSelThreads, 0, st>>>(rows, count_dev, rows_cap, tokens, mask_id, N, blk_s, blk_e, round_mask,
+{
+    const int rc_ = launch_pdl(  lm_rows_kernel, dim3(1), dim3(kSelThreads), 0, st, rows, count_dev, rows_cap, tokens, mask_id, N, blk_s, blk_e, round_mask,
                                             lm_rows, lm_count);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
 int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8_t* masked_prev, int mask_id,
                          const int* rows, int n_rows, int d, cudaStream_t st) {
   if (n_rows <= 0) return DLLM_OK;
-  snapshot_rows_kernel<<<n_rows, 256, 0, st>>>(h, h_prev, tokens, masked_prev, mask_id, rows, n_rows, d);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+{
+    const int rc_ = launch_pdl(  snapshot_rows_kernel, dim3(n_rows), dim3(256), 0, st, h, h_prev, tokens, masked_prev, mask_id, rows, n_rows, d);
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 
@@ -600,10 +632,11 @@ int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N,
   if (blk_len <= 0 || blk_len > 8192) return DLLM_ERR_UNSUPPORTED;
   const int threads = std::min(1024, ((blk_len + 31) / 32) * 32);
   const size_t smem = blk_len * sizeof(float) + blk_len;
-  unmask_kernel<<<B, threads, smem, st>>>(tokens, conf, amax, N, blk_s, blk_len, mask_id, n_commit, round_mask, pos_out,
+{
+    const int rc_ = launch_pdl(  unmask_kernel, dim3(B), dim3(threads), smem, st, tokens, conf, amax, N, blk_s, blk_len, mask_id, n_commit, round_mask, pos_out,
                                           tok_out, n_out, max_out);
-  count_launch();
-  DLLM_CUDA_TRY(cudaGetLastError());
+    if (rc_) return rc_;
+  }
   return DLLM_OK;
 }
 

@@ -96,8 +96,9 @@ class Engine:
             self.tokens.copy_(tokens, non_blocking=True)
         check(self.lib.dllm_reset(self.handle, stream_ptr(self.stream)), "dllm_reset")
 
-    def profile(self, enable: bool, hbm_gbs: float = 0.0, tensor_tflops: float = 0.0):
-        check(self.lib.dllm_profile_enable(self.handle, 1 if enable else 0, hbm_gbs, tensor_tflops),
+    def profile(self, every: int, hbm_gbs: float = 0.0, tensor_tflops: float = 0.0):
+        """Bracket every `every`-th GEMM / attention launch with CUDA events (0: off)."""
+        check(self.lib.dllm_profile_enable(self.handle, int(every), hbm_gbs, tensor_tflops),
               "dllm_profile_enable")
 
     def profile_read(self) -> dict:

@@ -15,7 +15,8 @@ _DEFAULT_WS = 256 << 20
 
 
 def _ws(nbytes=_DEFAULT_WS):
-    return torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    """Op workspace: zeroed once (the GEMM tile counters at its start must begin at 0)."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
 
 
 def _L():
@@ -160,7 +161,7 @@ def layer(cfg, lw: dict, kcache, vcache, rope_cos, rope_sin, h, rows, count, seq
           ws=None):
     """One transformer layer in place on h[rows[j]] (lw: this layer's weights)."""
     if ws is None:
-        ws = torch.empty(layer_workspace_bytes(cfg, rows_cap, rows_per_seq_cap), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(layer_workspace_bytes(cfg, rows_cap, rows_per_seq_cap), dtype=torch.uint8, device="cuda")
     check(_L().dllm_op_layer(ctypes.byref(cfg), ptr(lw["w_qkv"]), ptr(lw["w_o"]), ptr(lw["w_gu"]),
                              ptr(lw["w_down"]), ptr(lw["g_attn"]), ptr(lw["g_ffn"]), ptr(kcache), ptr(vcache),
                              ptr(rope_cos), ptr(rope_sin), ptr(h), ptr(rows), ptr(count), ptr(seq_off), rows_cap,
