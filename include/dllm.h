@@ -236,6 +236,26 @@ int dllm_op_gemm(int32_t kind, const void* W, int32_t n_out, const void* X, int3
                  int32_t K, void* out, const int32_t* rows_map, int32_t splits, int32_t bn, void* workspace,
                  size_t workspace_bytes, void* stream);
 
+/* The same GEMM as dllm_op_gemm for callers that cannot allocate device memory:
+ * a host framework that owns all device memory and hands a plugin only its
+ * input and output buffers, or a hot path that must not call cudaMalloc (it
+ * synchronises the device and can fail under memory pressure).  The paper has
+ * no counterpart; this is a deployment convenience of this library.
+ * Its scratch (tile counters and split-tile partial sums, ~4.9 MB) is a fixed
+ * array in the library's device image, held on every device that loads the
+ * library until the process exits.  The call allocates nothing: no cudaMalloc,
+ * no cudaFree, no allocating library routine.  Limits: rows_cap <= 32 and
+ * n_out <= 524288 (4096 tiles of 128); larger problems return DLLM_ERR_SHAPE
+ * and belong to dllm_op_gemm.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current, so
+ * make that first call before any stream capture.  All calls on a device share
+ * its one array, which keeps what the last call left; each call clears the tile
+ * counters it needs on `stream`.  Calls that can overlap on the GPU (issued on
+ * different streams of one device without ordering between them) race on the
+ * array and must be serialised by the caller. */
+int dllm_op_gemm_noalloc(int32_t kind, const void* W, int32_t n_out, const void* X, int32_t rows_cap,
+                         const int32_t* count, int32_t K, void* out, const int32_t* rows_map, void* stream);
+
 /* Fused QKV projection: RoPE on q and k, q -> q_out bf16 [rows, Hq*hd], k and v -> the
  * cache rows (b, :, pos) of rows_map[j] = b * N + pos.  W = one layer of w_qkv. */
 int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32_t* count, int32_t d,

@@ -84,6 +84,7 @@ _SIGS = {
     "dllm_op_rmsnorm_rows": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_f32, c_vp, c_vp]),
     "dllm_op_gemm": (ctypes.c_int, [c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32,
                                     c_vp, c_sz, c_vp]),
+    "dllm_op_gemm_noalloc": (ctypes.c_int, [c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "dllm_op_qkv_rope": (ctypes.c_int, [c_vp, c_vp, c_i32, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp,
                                         c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_sz, c_vp]),
     "dllm_op_gate_up": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_sz, c_vp]),
