@@ -166,6 +166,13 @@ int dllm_step(dllm_handle* h, dllm_step_info* info_or_null, void* stream);
 /* Host-side schedule: 1 when every block is finished. */
 int dllm_done(const dllm_handle* h);
 
+/* SureLock measurement mode: with a device uint8 [B, N] pattern, a row locks as soon
+ * as it is unmasked and has a previous distribution and pattern[b, pos] != 0,
+ * instead of by the KL / confidence rule (random weights never reach the
+ * confidence threshold).  NULL restores the rule.  The pattern must outlive
+ * the handle's steps. */
+int dllm_set_lock_pattern(dllm_handle* h, const uint8_t* pattern);
+
 /* Starts a new generation on the same handle: zeroes the caches and rewinds
  * the schedule, asynchronously on `stream` (the caller rewrites `tokens`). */
 int dllm_reset(dllm_handle* h, void* stream);
@@ -205,7 +212,9 @@ enum {
   DLLM_BUF_NLMROWS = 12, /* int32 [1] */
   DLLM_BUF_KL = 13,      /* fp32 [B*N] SureLock divergences of the LM rows (NaN: no previous p) */
   DLLM_BUF_HCACHE = 14,  /* fp32 [L, B*N, d] dLLM-Cache per-layer outputs */
-  DLLM_BUF_LSE = 15      /* fp32 [B*N] log-sum-exp of the last logits per position */
+  DLLM_BUF_LSE = 15,     /* fp32 [B*N] log-sum-exp of the last logits per position */
+  DLLM_BUF_SELROWS = 16, /* int32 [B*N] rows picked by the last selection (ES top-k; dLLM-Cache per layer) */
+  DLLM_BUF_NSEL = 17     /* int32 [1] their number */
 };
 int dllm_get_buffer(dllm_handle* h, int32_t which, void** ptr, size_t* bytes);
 

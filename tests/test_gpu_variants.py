@@ -1,0 +1,170 @@
+"""The SureLock and dLLM-Cache step paths of the engine, and DUS unmasking, against the oracle.
+
+SureLock runs with a seeded lock pattern (the measurement mode) so that locks
+are decided without floating-point thresholds and the active sets can be
+compared bit for bit; dLLM-Cache is compared with every response row selected
+(tau = inf, rho = 1) for the same reason, and its cosine scores are compared
+per layer within tolerance.  Decisions are teacher-forced as in the ES tests.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.policy import dus_schedule
+from oracle.steps import OracleRun
+from synth import get_config, make_tokens, make_weights
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from token_skip_denoising_b200.engine import Engine
+
+DEV = "cuda"
+TINY = get_config("tiny")
+TOL_HIDDEN = 2e-2
+
+
+def _rowrel(a, b):
+    a = np.asarray(a, np.float64).reshape(len(a), -1)
+    b = np.asarray(b, np.float64).reshape(len(b), -1)
+    return float((np.abs(a - b).max(1) / np.maximum(np.abs(b).max(1), 1e-30)).max())
+
+
+@pytest.fixture(scope="module")
+def tiny_w():
+    return make_weights(TINY.model)
+
+
+def _dev(w):
+    return {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in w.items()}
+
+
+def _force(eng, orc):
+    eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
+    eng.buffer("conf").copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
+    eng.buffer("argmax").copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
+
+
+# ------------------------------------------------------------------ SureLock
+
+def test_surelock_steps_match_oracle_with_lock_pattern(tiny_w):
+    cfg = TINY.replace(policy="surelock", tokens_per_step=2, batch=2)
+    N = cfg.seq_len
+    tok0 = make_tokens(cfg)
+    pattern = np.zeros((cfg.batch, N), bool)
+    pattern[:, ::3] = True
+    pattern[1, 1::5] = True
+    orc = OracleRun(cfg, tiny_w, tok0.numpy(), lock_pattern=pattern)
+    eng = Engine(cfg, _dev(tiny_w), tok0.to(DEV).contiguous())
+    pat_dev = torch.tensor(pattern.astype(np.uint8), device=DEV)
+    eng.set_lock_pattern(pat_dev)
+    hid = eng.buffer("hidden")
+    locked_max = 0
+    while not orc.done:
+        rec = orc.step()
+        info = eng.step(info=True)
+        assert info["kind_name"] == "locked"
+        flat = rec["rows"][0] * N + rec["rows"][1]
+        nrows = int(eng.buffer("nrows")[0])
+        np.testing.assert_array_equal(eng.buffer("rows")[:nrows].cpu().numpy(), flat)   # same active set
+        assert _rowrel(hid[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
+        np.testing.assert_array_equal(eng.buffer("lock").cpu().numpy().reshape(cfg.batch, N),
+                                      orc.lock.astype(np.uint8))
+        # KL of the eligible rows that had a previous distribution
+        n_lm = int(eng.buffer("nlmrows")[0])
+        assert n_lm == len(rec["lm_rows"])
+        kl_g = eng.buffer("kl")[:n_lm].cpu().numpy()
+        ok = ~np.isnan(rec["kl"])
+        if ok.any():
+            np.testing.assert_allclose(kl_g[ok], rec["kl"][ok], rtol=0.1, atol=2e-3)
+        lm = flat[rec["lm_rows"]]
+        np.testing.assert_allclose(eng.buffer("conf")[torch.tensor(lm, device=DEV)].cpu().numpy(),
+                                   orc.conf.reshape(-1)[lm], rtol=5e-2, atol=1e-5)
+        locked_max = max(locked_max, int(orc.lock.sum()))
+        _force(eng, orc)
+    assert locked_max > 10 and eng.done
+
+
+def test_surelock_eps_zero_never_locks(tiny_w):
+    cfg = TINY.replace(policy="surelock", kl_eps=0.0, conf_tau=-1.0)
+    eng = Engine(cfg, _dev(tiny_w), make_tokens(cfg).to(DEV).contiguous())
+    while not eng.done:
+        info = eng.step(info=True)
+        assert info["rows_last"] == cfg.seq_len            # every row recomputed every step
+    assert int(eng.buffer("lock").sum()) == 0
+    assert not bool((eng.tokens == cfg.model.mask_id).any())
+
+
+# ------------------------------------------------------------------ dLLM-Cache + DUS
+
+def test_dllm_cache_full_selection_matches_oracle(tiny_w):
+    cfg = TINY.replace(policy="dllm_cache", unmask="dus", block_len=8, prompt_interval=5,
+                       sim_tau=float("inf"), rho_cap=1.0)
+    N, L = cfg.seq_len, cfg.model.n_layers
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, tiny_w, tok0.numpy())
+    eng = Engine(cfg, _dev(tiny_w), tok0.to(DEV).contiguous())
+    hcache = eng.buffer("hcache")
+    n_partial = 0
+    while not orc.done:
+        rec = orc.step()
+        kind = eng.begin_step()
+        assert kind == ("full" if rec["kind"] == "refresh" else "partial")
+        for l in range(L):
+            eng.layer_forward(l)
+            if kind == "partial":
+                sims = eng.buffer("scores")[:cfg.batch * cfg.gen_len].cpu().numpy()
+                ref = rec["layers"][l]["sims"]
+                assert np.abs(sims - ref).max() < 2e-2
+        eng.unmask()
+        torch.cuda.synchronize()
+        b_idx, pos = rec["rows"]
+        flat = b_idx * N + pos
+        got = hcache[L - 1][torch.tensor(flat, device=DEV)].cpu().numpy()
+        assert _rowrel(got, rec["h_out"]) < TOL_HIDDEN
+        n_partial += kind == "partial"
+        _force(eng, orc)
+    assert n_partial > 0 and eng.done
+
+
+def test_dllm_cache_dus_generation(tiny_w):
+    cfg = TINY.replace(policy="dllm_cache", unmask="dus", block_len=8, prompt_interval=5,
+                       sim_tau=0.95, rho_cap=0.25)
+    N = cfg.seq_len
+    eng = Engine(cfg, _dev(tiny_w), make_tokens(cfg).to(DEV).contiguous())
+    rounds = dus_schedule(cfg.block_len)
+    pos = torch.full((1, cfg.block_len), -1, dtype=torch.int32, device=DEV)
+    tk = torch.full_like(pos, -1)
+    cnt = torch.zeros(1, dtype=torch.int32, device=DEV)
+    steps, seen = 0, np.zeros(N, int)
+    cap = math.ceil(cfg.rho_cap * cfg.gen_len)
+    while not eng.done:
+        block, r = divmod(steps, len(rounds))
+        kind = eng.begin_step()
+        for l in range(cfg.model.n_layers):
+            eng.layer_forward(l)
+            if kind == "partial":
+                assert int(eng.buffer("nsel")[0]) <= cap
+        eng.unmask(pos, tk, cnt)
+        committed = sorted(pos[0, :int(cnt[0])].tolist())
+        expect = sorted((cfg.prompt_len + block * cfg.block_len + rounds[r]).tolist())
+        assert committed == expect                           # exactly this round's dilated group
+        for p in committed:
+            seen[p] += 1
+        steps += 1
+    assert steps == (cfg.gen_len // cfg.block_len) * len(rounds)
+    assert np.all(seen[cfg.prompt_len:] == 1) and np.all(seen[:cfg.prompt_len] == 0)
+    assert not bool((eng.tokens == cfg.model.mask_id).any())
+
+
+def test_dllm_cache_forced_ratio_selects_exactly_the_cap(tiny_w):
+    cfg = TINY.replace(policy="dllm_cache", unmask="dus", block_len=8, prompt_interval=100, rho_cap=0.25)
+    eng = Engine(cfg, _dev(tiny_w), make_tokens(cfg).to(DEV).contiguous(), forced_rho=1)
+    eng.step()                                               # refresh
+    eng.begin_step()
+    for l in range(cfg.model.n_layers):
+        eng.layer_forward(l)
+        assert int(eng.buffer("nsel")[0]) == math.ceil(0.25 * cfg.gen_len)
+    eng.unmask()

@@ -29,7 +29,8 @@ UNMASK = {"topconf": 0, "dus": 1}
 SCOPE = {"block": 0, "all": 1}
 STEP_KIND = {0: "full", 1: "skip", 2: "locked", 3: "partial"}
 BUF = {"kcache": 0, "vcache": 1, "hidden": 2, "hprev": 3, "conf": 4, "argmax": 5, "rows": 6, "nrows": 7,
-       "scores": 8, "lock": 9, "masked_prev": 10, "lmrows": 11, "nlmrows": 12, "kl": 13, "hcache": 14, "lse": 15}
+       "scores": 8, "lock": 9, "masked_prev": 10, "lmrows": 11, "nlmrows": 12, "kl": 13, "hcache": 14, "lse": 15,
+       "selrows": 16, "nsel": 17}
 
 
 class DllmConfig(ctypes.Structure):
@@ -74,6 +75,7 @@ _SIGS = {
     "dllm_step": (ctypes.c_int, [c_vp, P(DllmStepInfo), c_vp]),
     "dllm_done": (ctypes.c_int, [c_vp]),
     "dllm_reset": (ctypes.c_int, [c_vp, c_vp]),
+    "dllm_set_lock_pattern": (ctypes.c_int, [c_vp, c_vp]),
     "dllm_profile_enable": (ctypes.c_int, [c_vp, c_i32, c_f64, c_f64]),
     "dllm_profile_read": (ctypes.c_int, [c_vp, P(DllmProfile)]),
     "dllm_kernel_launches": (ctypes.c_int64, []),

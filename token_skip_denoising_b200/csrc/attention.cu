@@ -319,9 +319,17 @@ int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N) {
   return std::max(1, s);
 }
 
+int attn_counters_needed(int B, int Hkv, int G, int rows_per_seq) {
+  (void)B; (void)Hkv; (void)G; (void)rows_per_seq;
+  return 0;
+}
+
 int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, __nv_bfloat16* out,
                 const int* seq_off, int B, int rows_cap, int rows_per_seq_cap, int N, int Hq, int Hkv, int hd,
-                int splits, float* opart, float2* ml, size_t partial_floats, cudaStream_t st) {
+                int splits, float* opart, float2* ml, size_t partial_floats, int* counters, int n_counters,
+                cudaStream_t st) {
+  (void)counters;
+  (void)n_counters;
   if (B <= 0 || N <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return DLLM_ERR_SHAPE;
   if (hd != 64 && hd != 128) return DLLM_ERR_UNSUPPORTED;
   if (rows_cap <= 0 || rows_per_seq_cap <= 0) return DLLM_OK;
@@ -341,12 +349,18 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
   const int qtiles = (rows_per_seq_cap * G + kUnitsPerCta - 1) / kUnitsPerCta;
   dim3 grid(qtiles, B * Hkv, splits);
   const size_t smem = 4 * kKeysPerBlock * hd * 2;
+  static bool attr_done = false;
+  if (!attr_done) {
+    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(4 * kKeysPerBlock * 128 * 2)));
+    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(4 * kKeysPerBlock * 64 * 2)));
+    attr_done = true;
+  }
   if (hd == 128) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     const int rc = launch_pdl(attn_kernel<128>, grid, dim3(128), smem, st, p);
     if (rc) return rc;
   } else {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     const int rc = launch_pdl(attn_kernel<64>, grid, dim3(128), smem, st, p);
     if (rc) return rc;
   }

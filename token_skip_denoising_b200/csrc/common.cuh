@@ -68,7 +68,7 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // (rows of X) tile with tcgen05 into TMEM; the epilogue is fused.
 enum EpiKind : int {
   EPI_STORE_F32 = 0,   // out_f32[j * ldo + n]
-  EPI_STORE_BF16 = 1,  // out_bf16[j * ldo + n]
+  EPI_STORE_BF16 = 1,  // out_bf16[r * ldo + n], r = row_map ? row_map[j] : j
   EPI_QKV_ROPE = 2,    // RoPE on q/k, q -> q_out, k/v -> cache rows of row_map[j]
   EPI_RESID_ADD = 3,   // h[row_map[j] * ldh + n] += C
   EPI_SWIGLU = 4,      // act[j * F + f] = silu(gate) * up   (W tile = 64 gate + 64 up rows)

@@ -180,6 +180,7 @@ struct dllm_handle {
   __nv_bfloat16* zstore;   // SureLock: position-indexed bf16 logits, 2 buffers
   float* lse_store;        // 2 x [B*N]
   int* has_prev;           // [B*N] step + 1 at which the stored logits were written
+  const uint8_t* lock_pattern = nullptr;   // SureLock forced-lock mode (measurement), caller-owned
   // workspace
   int *rows, *rows2, *nrows, *nrows2, *seq_off, *seq_off2, *lm_rows, *n_lm, *act_idx, *act_count;
   float *scores, *kl;
@@ -193,6 +194,8 @@ struct dllm_handle {
   float* attn_opart;
   float2* attn_ml;
   size_t attn_floats;
+  int* attn_ctr;
+  int n_attn_ctr;
   // schedule
   int block = 0, step_in_block = 0, n_steps = 0;
   // current step
@@ -266,7 +269,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->act = w.take<__nv_bfloat16>(R * x->F);
   x->vnew = c.policy == DLLM_POLICY_DLLM_CACHE ? w.take<float>(static_cast<size_t>(x->B) * x->n_resp * x->kvd) : nullptr;
   const int lm_cap = lm_cap_of(x);
-  x->lm_part = w.take<float4>(static_cast<size_t>(lm_cap) * (x->V / 128));
+  x->lm_part = w.take<float4>(c.policy == DLLM_POLICY_SURELOCK ? 0 : static_cast<size_t>(lm_cap) * (x->V / 128));
   // split-K scratch: the largest need over the row counts a step can use
   std::vector<int> caps = {static_cast<int>(BN), x->B * x->n_cand, x->B * x->k_keep, x->B * x->n_resp, lm_cap};
   size_t pf = 0;
@@ -296,6 +299,11 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->attn_floats = af;
   size_t ml = af / std::max(1, x->hd);
   x->attn_ml = w.take<float2>(ml);
+  int actr = 0;
+  for (int cap_seq : {x->N, x->n_cand, x->k_keep, x->n_resp})
+    if (cap_seq > 0) actr = std::max(actr, attn_counters_needed(x->B, c.n_kv_heads, G, cap_seq));
+  x->attn_ctr = w.take<int>(actr);
+  x->n_attn_ctr = actr;
   if (ws_bytes) *ws_bytes = (w.off + 255) & ~size_t(255);
 }
 
@@ -340,6 +348,8 @@ struct LayerCtx {
   float* attn_opart;
   float2* attn_ml;
   size_t attn_floats;
+  int* attn_ctr = nullptr;
+  int n_attn_ctr = 0;
   Prof* prof = nullptr;
 };
 
@@ -374,7 +384,7 @@ int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, con
     cudaEvent_t a = nullptr;
     if (x.prof) x.prof->begin(st, &a, 1);
     DLLM_TRY(attn_launch(x.q, x.kc, x.vc, x.attn, seq_off, x.B, rows_cap, rows_per_seq, x.N, x.Hq, x.Hkv, x.hd, 0,
-                         x.attn_opart, x.attn_ml, x.attn_floats, st));
+                         x.attn_opart, x.attn_ml, x.attn_floats, x.attn_ctr, x.n_attn_ctr, st));
     if (x.prof && a) {
       const double kvb = 2.0 * x.B * x.Hkv * static_cast<double>(x.N) * x.hd * 2.0;
       x.prof->end(st, a, 1, kvb + 4.0 * rows_cap * x.qd, 4.0 * rows_cap * x.Hq * static_cast<double>(x.N) * x.hd);
@@ -417,6 +427,7 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.z = x->z; L.q = x->q; L.attn = x->attn; L.act = x->act;
   L.gs = x->gs;
   L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
+  L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
 }
@@ -554,7 +565,27 @@ int dllm_layer_forward(dllm_handle* x, int32_t layer, void* stream) {
       DLLM_CUDA_TRY(cudaMemcpyAsync(out_l, x->h, BNd * sizeof(float), cudaMemcpyDeviceToDevice, st));
       return DLLM_OK;
     }
-    return DLLM_ERR_UNSUPPORTED;   // partial response updates: see dllm_cache_layer below
+    // partial step (dLLM-Cache explainer sec. 3): score the response rows by the cosine of their new
+    // value vectors to the cached ones, recompute only the selected rows, keep the rest cached
+    const float* in_l = layer == 0 ? x->h : x->hcache + (layer - 1) * BNd;
+    const LayerCtx L = layer_ctx(x, layer);
+    const int cap = x->B * x->n_resp;
+    DLLM_TRY(rmsnorm_rows_launch(in_l, x->rows, x->nrows, cap, x->d, L.g_attn, c.rms_eps, x->z, x->d, st));
+    GemmArgs v;
+    v.W = L.Wqkv + static_cast<size_t>(x->qd + x->kvd) * x->d; v.w_rows_total = x->kvd; v.X = x->z;
+    v.rows_cap = cap; v.rows_dev = x->nrows; v.K = x->d; v.n_tiles_w = x->kvd / 128;
+    v.epi.kind = EPI_STORE_F32; v.epi.out = x->vnew; v.epi.ldo = x->kvd;
+    DLLM_TRY(timed_gemm(&x->prof, v, x->gs, st, 4.0 * x->kvd));
+    DLLM_TRY(score_cos_launch(x->vnew, x->kvd, L.vc, x->rows, x->nrows, cap, x->N, c.n_kv_heads, x->hd, x->scores, st));
+    SelectParams sp;
+    sp.scores = x->scores; sp.B = x->B; sp.n = x->n_resp; sp.mode = c.forced_rho ? SEL_FORCED_ASC : SEL_BELOW_CAP_ASC;
+    sp.k = x->resp_cap; sp.tau = c.sim_tau; sp.cand_start = x->resp_start; sp.seq_n = x->N;
+    sp.act_pos = x->act_idx; sp.k_max = std::max(1, x->resp_cap); sp.count = x->act_count;
+    sp.row_map = x->rows2; sp.seq_off = x->seq_off2; sp.total = x->nrows2;
+    DLLM_TRY(select_launch(sp, st));
+    const int cap2 = x->B * std::max(1, x->resp_cap);
+    DLLM_TRY(copy_rows_launch(in_l, out_l, x->rows2, x->nrows2, cap2, x->d, st));
+    return run_layer(L, out_l, x->rows2, x->nrows2, x->seq_off2, cap2, std::max(1, x->resp_cap), st);
   }
   return run_layer(layer_ctx(x, layer), x->h, x->cur_rows, x->cur_n, x->cur_seq_off, x->cur_rows_cap,
                    x->cur_rows_per_seq, st);
@@ -605,15 +636,34 @@ int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_o
   const float* hsrc = (c.policy == DLLM_POLICY_DLLM_CACHE) ? x->hcache + static_cast<int64_t>(x->L - 1) * x->B * x->N * x->d
                                                           : x->h;
   const int lm_cap = std::min(lm_cap_of(x), x->cur_rows_cap);
+  const bool surelock = c.policy == DLLM_POLICY_SURELOCK;
   DLLM_TRY(lm_rows_launch(x->cur_rows, x->cur_n, x->cur_rows_cap, x->tokens, c.mask_id, x->N, bs, bs + c.block_len,
-                          rmask, x->lm_rows, x->n_lm, st));
+                          rmask, surelock ? 1 : 0, x->lm_rows, x->n_lm, st));
   DLLM_TRY(rmsnorm_rows_launch(hsrc, x->lm_rows, x->n_lm, lm_cap, x->d, x->w.g_final, c.rms_eps, x->z, x->d, st));
   GemmArgs g;
   g.W = x->w.lm_head; g.w_rows_total = x->V; g.X = x->z; g.rows_cap = lm_cap; g.rows_dev = x->n_lm; g.K = x->d;
   g.n_tiles_w = x->V / 128;
-  g.epi.kind = EPI_LMHEAD; g.epi.lm_part = x->lm_part; g.epi.n_vtiles = x->V / 128; g.epi.mask_id = c.mask_id;
-  DLLM_TRY(timed_gemm(&x->prof, g, x->gs, st, 16.0 * (x->V / 128)));
-  DLLM_TRY(lmhead_combine_launch(x->lm_part, x->V / 128, lm_cap, x->n_lm, x->lm_rows, x->conf, x->amax, x->lse, st));
+  if (surelock) {
+    // SureLock: every recomputed unmasked row needs its full distribution (stored, position-indexed,
+    // in the buffer of this step's parity) to compare with the previous step's
+    const int64_t BN = static_cast<int64_t>(x->B) * x->N;
+    __nv_bfloat16* zcur = x->zstore + (x->n_steps & 1) * BN * x->V;
+    __nv_bfloat16* zprev = x->zstore + ((x->n_steps + 1) & 1) * BN * x->V;
+    float* lcur = x->lse_store + (x->n_steps & 1) * BN;
+    float* lprev = x->lse_store + ((x->n_steps + 1) & 1) * BN;
+    g.epi.kind = EPI_STORE_BF16; g.epi.out = zcur; g.epi.ldo = x->V; g.epi.row_map = x->lm_rows;
+    DLLM_TRY(timed_gemm(&x->prof, g, x->gs, st, 2.0 * x->V));
+    KlStep k;
+    k.z_cur = zcur; k.z_prev = zprev; k.lse_prev = lprev; k.lse_cur = lcur; k.stamp = x->has_prev;
+    k.step = x->n_steps; k.rows = x->lm_rows; k.count = x->n_lm; k.rows_cap = lm_cap; k.V = x->V;
+    k.mask_id = c.mask_id; k.tokens = x->tokens; k.lock = x->lock; k.pattern = x->lock_pattern;
+    k.kl_eps = c.kl_eps; k.conf_tau = c.conf_tau; k.conf = x->conf; k.amax = x->amax; k.kl_out = x->kl;
+    DLLM_TRY(kl_step_launch(k, st));
+  } else {
+    g.epi.kind = EPI_LMHEAD; g.epi.lm_part = x->lm_part; g.epi.n_vtiles = x->V / 128; g.epi.mask_id = c.mask_id;
+    DLLM_TRY(timed_gemm(&x->prof, g, x->gs, st, 16.0 * (x->V / 128)));
+    DLLM_TRY(lmhead_combine_launch(x->lm_part, x->V / 128, lm_cap, x->n_lm, x->lm_rows, x->conf, x->amax, x->lse, st));
+  }
   const int max_out = c.unmask == DLLM_UNMASK_DUS ? c.block_len : c.tokens_per_step;
   DLLM_TRY(unmask_launch(x->tokens, x->conf, x->amax, x->B, x->N, bs, c.block_len, c.mask_id, c.tokens_per_step, rmask,
                          pos_out, tok_out, n_out, max_out, st));
@@ -683,6 +733,8 @@ int dllm_get_buffer(dllm_handle* x, int32_t which, void** ptr, size_t* bytes) {
     case DLLM_BUF_KL: p = x->kl; b = BN * 4; break;
     case DLLM_BUF_HCACHE: p = x->hcache; b = x->hcache ? static_cast<size_t>(x->L) * BN * x->d * 4 : 0; break;
     case DLLM_BUF_LSE: p = x->lse; b = BN * 4; break;
+    case DLLM_BUF_SELROWS: p = x->rows2; b = BN * 4; break;
+    case DLLM_BUF_NSEL: p = x->nrows2; b = 4; break;
     default: DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown buffer");
   }
   *ptr = p;
@@ -691,6 +743,13 @@ int dllm_get_buffer(dllm_handle* x, int32_t which, void** ptr, size_t* bytes) {
 }
 
 void dllm_destroy(dllm_handle* x) { delete x; }
+
+int dllm_set_lock_pattern(dllm_handle* x, const uint8_t* pattern) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (x->c.policy != DLLM_POLICY_SURELOCK) DLLM_FAIL(DLLM_ERR_STATE, "lock patterns apply to the SureLock policy");
+  x->lock_pattern = pattern;
+  return DLLM_OK;
+}
 
 int dllm_reset(dllm_handle* x, void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
@@ -751,6 +810,9 @@ int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t ro
   int ctr = std::max({gemm_counters_needed(rows_cap, qkvd / 128), gemm_counters_needed(rows_cap, d / 128),
                       gemm_counters_needed(rows_cap, F / 64)});
   w.take<int>(ctr);
+  const int N0 = cfg->prompt_len + cfg->gen_len;
+  w.take<int>(attn_counters_needed(cfg->batch, cfg->n_kv_heads, cfg->n_heads / cfg->n_kv_heads, rows_per_seq_cap));
+  (void)N0;
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * d);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
@@ -793,6 +855,8 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
                       gemm_counters_needed(rows_cap, L.F / 64)});
   L.gs.counters = w.take<int>(ctr);
   L.gs.n_counters = ctr;
+  L.n_attn_ctr = attn_counters_needed(L.B, L.Hkv, L.Hq / L.Hkv, rows_per_seq_cap);
+  L.attn_ctr = w.take<int>(L.n_attn_ctr);
   L.z = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.d);
   L.q = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
   L.attn = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);

@@ -19,6 +19,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -38,11 +39,11 @@ constexpr uint32_t kABytes = kTileM * kBK * 2;
 // streaming its weights during this kernel's tail (programmatic dependent launch);
 // compute-bound widths take ~200 KB for a deeper ring.  Two TMEM accumulators let the
 // epilogue of one work segment overlap the MMAs of the next.
-template <int BN, int KSUB>
+template <int BN, int KSUB, bool BIG = false>
 struct Cfg {
   static constexpr uint32_t kBBytes = BN * kBK * 2;                // one 64-wide k block of X
   static constexpr uint32_t kStageBytes = KSUB * (kABytes + kBBytes);
-  static constexpr uint32_t kBudget = (BN <= 64 ? 100u : 200u) * 1024u;
+  static constexpr uint32_t kBudget = (BN <= 64 && !BIG ? 100u : 200u) * 1024u;
   static constexpr int kStagesFit = static_cast<int>(kBudget / kStageBytes);
   static constexpr int kStages = kStagesFit > 12 ? 12 : (kStagesFit < 2 ? 2 : kStagesFit);
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // TMEM columns per accumulator
@@ -112,10 +113,15 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
       break;
     }
     case EPI_STORE_BF16: {
+      // row j lands at row row_map[j] of the output when a map is given (scatter)
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(e.out);
+      int rr[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        if (jbase + i < m_rows) o[static_cast<int64_t>(jbase + i) * e.ldo + n] = __float2bfloat16(v[i]);
+        rr[i] = (jbase + i < m_rows) ? (e.row_map ? __ldg(e.row_map + jbase + i) : jbase + i) : -1;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (rr[i] >= 0) o[static_cast<int64_t>(rr[i]) * e.ldo + n] = __float2bfloat16(v[i]);
       break;
     }
     case EPI_RESID_ADD: {
@@ -246,10 +252,10 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
 // Persistent stream-K GEMM: grid = one CTA per SM (or fewer), each CTA walks its
 // contiguous share of the (tile, k-block) iterations; a tile split across CTAs is
 // summed by the last CTA to finish its piece, in k order.
-template <int BN, int KSUB>
+template <int BN, int KSUB, bool BIG>
 __global__ void __launch_bounds__(kThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams p) {
-  using C = Cfg<BN, KSUB>;
+  using C = Cfg<BN, KSUB, BIG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -560,7 +566,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // 2D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128 B swizzle.
-int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+int encode_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   auto enc = get_encode();
   if (!enc) { set_last_error("cuTensorMapEncodeTiled unavailable", __FILE__, __LINE__); return DLLM_ERR_CUDA; }
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -580,6 +586,46 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
   return DLLM_OK;
 }
 
+// Tensor maps are pure functions of (address, shape, box); the step issues the same few
+// hundred of them every denoising step, so they are encoded once and reused.
+struct TmapKey {
+  const void* base;
+  int64_t rows, cols;
+  int box;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && box == o.box;
+  }
+};
+struct TmapKeyHash {
+  size_t operator()(const TmapKey& k) const {
+    size_t h = reinterpret_cast<size_t>(k.base);
+    h ^= static_cast<size_t>(k.rows) * 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    h ^= static_cast<size_t>(k.cols) * 0xc2b2ae3d27d4eb4full + (h << 6) + (h >> 2);
+    h ^= static_cast<size_t>(k.box) + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+
+int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  static std::mutex mu;
+  static std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> cache;
+  const TmapKey key{base, rows, cols, box_rows};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *m = it->second;
+      return DLLM_OK;
+    }
+  }
+  const int rc = encode_tmap(m, base, rows, cols, box_rows);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() > 8192) cache.clear();
+  cache.emplace(key, *m);
+  return DLLM_OK;
+}
+
 int pick_bn(int rows) {
   if (rows <= 16) return 16;
   if (rows <= 32) return 32;
@@ -594,20 +640,29 @@ int pick_grid(int tiles, int KB) {
   return static_cast<int>(std::min<int64_t>(kNumSMs, T));
 }
 
-template <int BN, int KSUB>
-int launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, cudaStream_t st) {
-  using C = Cfg<BN, KSUB>;
+template <int BN, int KSUB, bool BIG>
+int launch_cfg2(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, cudaStream_t st) {
+  using C = Cfg<BN, KSUB, BIG>;
   static bool attr_done = false;
   if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    DLLM_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, KSUB, BIG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem)));
     attr_done = true;
   }
 {
-    const int rc_ = launch_pdl(  gemm_tc_kernel<BN, KSUB>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
+    const int rc_ = launch_pdl(gemm_tc_kernel<BN, KSUB, BIG>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
     if (rc_) return rc_;
   }
   return DLLM_OK;
+}
+
+template <int BN, int KSUB>
+int launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, cudaStream_t st) {
+  static const bool big = getenv("DLLM_GEMM_BIGRING") != nullptr;   // A/B switch for measurements
+  if constexpr (BN <= 64) {
+    if (big) return launch_cfg2<BN, KSUB, true>(tmW, tmX, kp, grid, st);
+  }
+  return launch_cfg2<BN, KSUB, false>(tmW, tmX, kp, grid, st);
 }
 
 // Widest KSUB whose two-stage ring still fits shared memory for this tile width.

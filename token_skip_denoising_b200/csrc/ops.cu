@@ -142,14 +142,20 @@ int dllm_op_attention(const void* q, const void* kcache, const void* vcache, voi
                       int32_t n_kv_heads, int32_t head_dim, int32_t splits, void* workspace, size_t workspace_bytes,
                       void* stream) {
   if (!q || !kcache || !vcache || !out || !seq_off) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad attention args");
+  if (n_kv_heads <= 0 || n_heads % n_kv_heads) OP_FAIL(DLLM_ERR_SHAPE, "n_heads must be a multiple of n_kv_heads");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int G = n_kv_heads > 0 ? n_heads / n_kv_heads : 1;
+  const int G = n_heads / n_kv_heads;
   int sp = splits > 0 ? splits : attn_pick_splits(B, n_kv_heads, G, rows_per_seq_cap, N);
   float* opart = nullptr;
   float2* ml = nullptr;
+  int* ctr = nullptr;
+  int nctr = 0;
   size_t pf = 0;
   if (sp > 1) {
     OpCarver cv(workspace, workspace_bytes);
+    nctr = attn_counters_needed(B, n_kv_heads, G, rows_per_seq_cap);
+    ctr = cv.take<int>(kOpCounters);        // the zeroed counter region at the workspace start
+    if (nctr > kOpCounters) OP_FAIL(DLLM_ERR_SHAPE, "too many attention groups for the op workspace");
     pf = attn_partial_floats(rows_cap, n_heads, head_dim, sp);
     opart = cv.take<float>(pf);
     ml = cv.take<float2>(pf / head_dim);
@@ -157,7 +163,7 @@ int dllm_op_attention(const void* q, const void* kcache, const void* vcache, voi
   }
   return attn_launch(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kcache),
                      static_cast<const __nv_bfloat16*>(vcache), static_cast<__nv_bfloat16*>(out), seq_off, B, rows_cap,
-                     rows_per_seq_cap, N, n_heads, n_kv_heads, head_dim, sp, opart, ml, pf, st);
+                     rows_per_seq_cap, N, n_heads, n_kv_heads, head_dim, sp, opart, ml, pf, ctr, nctr, st);
 }
 
 int dllm_op_lm_head(const void* W, int32_t V, const void* X, int32_t rows_cap, const int32_t* count, int32_t d,

@@ -424,7 +424,8 @@ __global__ void __launch_bounds__(kSelThreads) lm_rows_kernel(const int* __restr
                                                               int rows_cap, const int* __restrict__ tokens, int mask_id,
                                                               int N, int blk_s, int blk_e,
                                                               const uint8_t* __restrict__ round_mask,
-                                                              int* __restrict__ lm_rows, int* lm_count) {
+                                                              int include_unmasked, int* __restrict__ lm_rows,
+                                                              int* lm_count) {
   pdl_trigger();
   pdl_wait();
   __shared__ int s_warp[32];
@@ -437,8 +438,9 @@ __global__ void __launch_bounds__(kSelThreads) lm_rows_kernel(const int* __restr
     if (j < m) {
       flat = rows[j];
       const int pos = flat % N;
-      keep = tokens[flat] == mask_id && pos >= blk_s && pos < blk_e &&
-             (!round_mask || round_mask[pos - blk_s]);
+      const bool masked = tokens[flat] == mask_id;
+      keep = (masked && pos >= blk_s && pos < blk_e && (!round_mask || round_mask[pos - blk_s])) ||
+             (include_unmasked && !masked);
     }
     int tot;
     const int o = block_scan_excl(keep ? 1 : 0, s_warp, tot) + carry;
@@ -513,6 +515,124 @@ __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict_
   }
   __syncthreads();
   if (threadIdx.x == 0 && n_out) n_out[b] = min(s_cnt, max_out);
+}
+
+// SureLock per LM row (one CTA): lse, argmax (mask id excluded), conf = p(argmax) of this
+// step's stored logits; when the position's logits were also stored at the previous step,
+// D = KL(p_t || p_t-1) clamped at 0; the lock rule for rows unmasked at the start of the
+// step: D < eps and conf > tau (or a forced pattern); finally the position's stamp is set.
+__global__ void kl_step_kernel(KlStep k) {
+  pdl_trigger();
+  pdl_wait();
+  const int m = k.count ? min(*k.count, k.rows_cap) : k.rows_cap;
+  const int j = blockIdx.x;
+  if (j >= m) return;
+  const int flat = k.rows[j];
+  const int V = k.V;
+  const __nv_bfloat16* zr = k.z_cur + static_cast<int64_t>(flat) * V;
+  __shared__ float sf[32];
+  __shared__ int si[32];
+  __shared__ float s_res[4];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  float mx = -INFINITY, bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float x = __bfloat162float(zr[v]);
+    mx = fmaxf(mx, x);
+    if (v != k.mask_id && (x > bv || (x == bv && v < bi))) { bv = x; bi = v; }
+  }
+  for (int o = 16; o; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  if (l == 0) { sf[w] = mx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int i = 0; i < nw; ++i) M = fmaxf(M, sf[i]);
+    s_res[0] = M;
+  }
+  __syncthreads();
+  const float M = s_res[0];
+  __syncthreads();
+  if (l == 0) { sf[w] = bv; si[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float B = -INFINITY;
+    int I = 0x7fffffff;
+    for (int i = 0; i < nw; ++i)
+      if (sf[i] > B || (sf[i] == B && si[i] < I)) { B = sf[i]; I = si[i]; }
+    s_res[1] = B;
+    si[31] = I;
+  }
+  __syncthreads();
+  const float BV = s_res[1];
+  const int BI = si[31];
+  __syncthreads();
+  float se = 0.f;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) se += __expf(__bfloat162float(zr[v]) - M);
+  se = warp_sum_f(se);
+  if (l == 0) sf[w] = se;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float S = 0.f;
+    for (int i = 0; i < nw; ++i) S += sf[i];
+    s_res[2] = M + logf(S);
+  }
+  __syncthreads();
+  const float L = s_res[2];
+  // stamps hold step + 1 of the last store, so a store at the previous step reads k.step
+  const bool has_prev = k.stamp && k.z_prev && k.step > 0 && k.stamp[flat] == k.step;
+  float kl = NAN;
+  if (has_prev) {
+    const __nv_bfloat16* pr = k.z_prev + static_cast<int64_t>(flat) * V;
+    const float Lp = k.lse_prev[flat];
+    float acc = 0.f;
+    for (int v = threadIdx.x; v < V; v += blockDim.x) {
+      const float zt = __bfloat162float(zr[v]) - L;
+      const float zq = __bfloat162float(pr[v]) - Lp;
+      acc += __expf(zt) * (zt - zq);
+    }
+    acc = warp_sum_f(acc);
+    __syncthreads();
+    if (l == 0) sf[w] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float K = 0.f;
+      for (int i = 0; i < nw; ++i) K += sf[i];
+      s_res[3] = fmaxf(K, 0.f);
+    }
+    __syncthreads();
+    kl = s_res[3];
+  }
+  if (threadIdx.x == 0) {
+    const float conf = __expf(BV - L);
+    k.conf[flat] = conf;
+    k.amax[flat] = BI;
+    k.lse_cur[flat] = L;
+    if (k.kl_out) k.kl_out[j] = kl;
+    const bool eligible = k.tokens[flat] != k.mask_id;
+    if (k.lock && eligible && has_prev) {
+      const bool lock_now = k.pattern ? (k.pattern[flat] != 0) : (kl < k.kl_eps && conf > k.conf_tau);
+      if (lock_now) k.lock[flat] = 1;
+    }
+    if (k.stamp) k.stamp[flat] = k.step + 1;
+  }
+}
+
+// dst[rows[j]] = src[rows[j]] (d floats) for j < *count.
+__global__ void copy_rows_kernel(const float* __restrict__ src, float* __restrict__ dst, const int* __restrict__ rows,
+                                 const int* count_dev, int rows_cap, int d) {
+  pdl_trigger();
+  pdl_wait();
+  const int m = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int j = blockIdx.x;
+  if (j >= m) return;
+  const int64_t off = static_cast<int64_t>(rows[j]) * d;
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4)
+    *reinterpret_cast<float4*>(dst + off + i) = *reinterpret_cast<const float4*>(src + off + i);
 }
 
 }  // namespace
@@ -607,9 +727,10 @@ int range_rows_launch(int B, int N, int start, int len, int* row_map, int* seq_o
 }
 
 int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const int* tokens, int mask_id, int N,
-                   int blk_s, int blk_e, const uint8_t* round_mask, int* lm_rows, int* lm_count, cudaStream_t st) {
+                   int blk_s, int blk_e, const uint8_t* round_mask, int include_unmasked, int* lm_rows, int* lm_count,
+                   cudaStream_t st) {
 {
-    const int rc_ = launch_pdl(  lm_rows_kernel, dim3(1), dim3(kSelThreads), 0, st, rows, count_dev, rows_cap, tokens, mask_id, N, blk_s, blk_e, round_mask,
+    const int rc_ = launch_pdl(  lm_rows_kernel, dim3(1), dim3(kSelThreads), 0, st, rows, count_dev, rows_cap, tokens, mask_id, N, blk_s, blk_e, round_mask, include_unmasked,
                                             lm_rows, lm_count);
     if (rc_) return rc_;
   }
@@ -638,6 +759,22 @@ int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N,
     if (rc_) return rc_;
   }
   return DLLM_OK;
+}
+
+}  // namespace dllm
+
+namespace dllm {
+
+int kl_step_launch(const KlStep& k, cudaStream_t st) {
+  if (k.rows_cap <= 0) return DLLM_OK;
+  return launch_pdl(kl_step_kernel, dim3(k.rows_cap), dim3(256), 0, st, k);
+}
+
+int copy_rows_launch(const float* src, float* dst, const int* rows, const int* count_dev, int rows_cap, int d,
+                     cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  if (d % 4) return DLLM_ERR_SHAPE;
+  return launch_pdl(copy_rows_kernel, dim3(rows_cap), dim3(256), 0, st, src, dst, rows, count_dev, rows_cap, d);
 }
 
 }  // namespace dllm

@@ -38,13 +38,41 @@ int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* m
                     cudaStream_t st);
 int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, const int* rows, const int* count_dev,
                      int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st);
+// SureLock: statistics of the stored logits of each LM row, its divergence from the
+// previous step's distribution and the lock decision (see KlStep in rowops.cu).
+struct KlStep {
+  const __nv_bfloat16* z_cur = nullptr;   // logits of this step, position-indexed [B*N, V]
+  const __nv_bfloat16* z_prev = nullptr;  // previous step's logits, same layout
+  const float* lse_prev = nullptr;        // [B*N]
+  float* lse_cur = nullptr;               // [B*N]
+  int* stamp = nullptr;                   // [B*N]: step + 1 at which a position's logits were stored
+  int step = 0;
+  const int* rows = nullptr;              // LM rows (flat) and their device count
+  const int* count = nullptr;
+  int rows_cap = 0;
+  int V = 0, mask_id = 0;
+  const int* tokens = nullptr;            // eligibility: token != mask at the start of the step
+  uint8_t* lock = nullptr;
+  const uint8_t* pattern = nullptr;       // forced locks (measurement mode) instead of the KL rule
+  float kl_eps = 0.f, conf_tau = 0.f;
+  float* conf = nullptr;
+  int* amax = nullptr;
+  float* kl_out = nullptr;                // [rows]: divergence, NaN without a previous distribution
+};
+int kl_step_launch(const KlStep& k, cudaStream_t st);
+int copy_rows_launch(const float* src, float* dst, const int* rows, const int* count_dev, int rows_cap, int d,
+                     cudaStream_t st);
+
 int kl_conf_launch(const __nv_bfloat16* z, int64_t ldz, const __nv_bfloat16* zp_store, int64_t ldp,
                    const float* lse_prev, const int* has_prev, const int* rows, const int* count_dev, int rows_cap,
                    int V, int mask_id, float* conf, int* amax, float* lse_out, float* kl_out, cudaStream_t st);
 int select_launch(const SelectParams& p, cudaStream_t st);
 int range_rows_launch(int B, int N, int start, int len, int* row_map, int* seq_off, int* total, cudaStream_t st);
+// include_unmasked: also keep every recomputed row that is already unmasked (SureLock's
+// lock-eligible rows need their distribution every step).
 int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const int* tokens, int mask_id, int N,
-                   int blk_s, int blk_e, const uint8_t* round_mask, int* lm_rows, int* lm_count, cudaStream_t st);
+                   int blk_s, int blk_e, const uint8_t* round_mask, int include_unmasked, int* lm_rows, int* lm_count,
+                   cudaStream_t st);
 int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8_t* masked_prev, int mask_id,
                          const int* rows, int n_rows, int d, cudaStream_t st);
 int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N, int blk_s, int blk_len, int mask_id,
@@ -53,8 +81,11 @@ int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N,
 
 size_t attn_partial_floats(int rows_cap, int Hq, int hd, int splits);
 int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N);
+int attn_counters_needed(int B, int Hkv, int G, int rows_per_seq);
+// counters: zero on entry, left at zero.
 int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, __nv_bfloat16* out,
                 const int* seq_off, int B, int rows_cap, int rows_per_seq_cap, int N, int Hq, int Hkv, int hd,
-                int splits, float* opart, float2* ml, size_t partial_floats, cudaStream_t st);
+                int splits, float* opart, float2* ml, size_t partial_floats, int* counters, int n_counters,
+                cudaStream_t st);
 
 }  // namespace dllm

@@ -96,6 +96,11 @@ class Engine:
             self.tokens.copy_(tokens, non_blocking=True)
         check(self.lib.dllm_reset(self.handle, stream_ptr(self.stream)), "dllm_reset")
 
+    def set_lock_pattern(self, pattern: torch.Tensor | None):
+        """SureLock measurement mode: lock rows by a seeded pattern (uint8 [B, N] on the device)."""
+        self._lock_pattern = pattern
+        check(self.lib.dllm_set_lock_pattern(self.handle, ptr(pattern)), "dllm_set_lock_pattern")
+
     def profile(self, every: int, hbm_gbs: float = 0.0, tensor_tflops: float = 0.0):
         """Bracket every `every`-th GEMM / attention launch with CUDA events (0: off)."""
         check(self.lib.dllm_profile_enable(self.handle, int(every), hbm_gbs, tensor_tflops),
@@ -129,6 +134,7 @@ class Engine:
             "masked_prev": (torch.uint8, (B * N,)), "lmrows": (torch.int32, (B * N,)),
             "nlmrows": (torch.int32, (1,)), "kl": (torch.float32, (B * N,)),
             "hcache": (torch.float32, (c.n_layers, B * N, c.d_model)), "lse": (torch.float32, (B * N,)),
+            "selrows": (torch.int32, (B * N,)), "nsel": (torch.int32, (1,)),
         }
         dt, shp = defaults[name]
         return _lib.view(p.value, shape or shp, dtype or dt)
