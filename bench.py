@@ -102,6 +102,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- replicas
+def reduce_over_ranks(values, world: int, device="cpu"):
+    """Max over ranks of each per-rank value (device times, wall times); with one rank the
+    values are returned unchanged.  Replicas exchange nothing else: each rank generates its
+    own batch, so whole-job throughput = tokens of all ranks / the slowest rank's time."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tokens_per_s(batch: int, gen_len: int, steps: int, world: int, seconds: float) -> float:
+    return batch * gen_len * steps * world / seconds
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -159,12 +177,8 @@ def run_ours(args, rank, world, local_rank):
     ms = t0.elapsed_time(t1)
     prof = eng.profile_read()
     eng.profile(0)
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    tokens_total = cfg.batch * cfg.gen_len * args.steps * world
-    value = tokens_total / (ms_max / 1e3)
+    ms_max = reduce_over_ranks([ms], world, dev)[0]
+    value = whole_job_tokens_per_s(cfg.batch, cfg.gen_len, args.steps, world, ms_max / 1e3)
     assert not bool((tok == cfg.model.mask_id).any()), "generation left mask ids"
 
     # ---- end to end through the public API, host buffers, copies inside the region
@@ -178,11 +192,8 @@ def run_ours(args, rank, world, local_rank):
         eng.generate()
         out_host.copy_(tok, non_blocking=True)       # D2H of the result
     torch.cuda.synchronize()
-    e2e_s = time.perf_counter() - w0
-    e2e_t = torch.tensor([e2e_s], device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_total / float(e2e_t.item())
+    e2e_s = reduce_over_ranks([time.perf_counter() - w0], world, dev)[0]
+    e2e_value = whole_job_tokens_per_s(cfg.batch, cfg.gen_len, args.steps, world, e2e_s)
 
     # ---- roofline of the dominant kernel (the fused tcgen05 GEMM)
     gemm_gbs = prof["gemm_bytes"] / (prof["gemm_ms"] / 1e3) / 1e9 if prof["gemm_ms"] > 0 else 0.0

@@ -196,6 +196,15 @@ struct dllm_handle {
   size_t attn_floats;
   int* attn_ctr;
   int n_attn_ctr;
+  __nv_bfloat16* z2;
+  float* fused_partial;
+  int* fused_ctr;
+  int fused_max_tiles;
+  int* fused_sync;         // state: 8 phase counters of the fused layer kernel
+  int fused_epoch = 0;
+  float* fused_opart;
+  float2* fused_ml;
+  size_t fused_attn_floats;
   // schedule
   int block = 0, step_in_block = 0, n_steps = 0;
   // current step
@@ -238,6 +247,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->masked_prev = s.take<uint8_t>(BN);
   x->lock = s.take<uint8_t>(BN);
   x->has_prev = s.take<int>(BN);
+  x->fused_sync = s.take<int>(8);
   if (c.policy == DLLM_POLICY_SURELOCK) {
     x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
     x->lse_store = s.take<float>(2 * BN);
@@ -299,6 +309,14 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->attn_floats = af;
   size_t ml = af / std::max(1, x->hd);
   x->attn_ml = w.take<float2>(ml);
+  // fused small-row layer scratch
+  x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(32) * x->d);
+  x->fused_partial = w.take<float>(fused_partial_floats(32));
+  x->fused_max_tiles = std::max({x->qkvd / 128, x->d / 128, x->F / 64});
+  x->fused_ctr = w.take<int>(4 * x->fused_max_tiles);
+  x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * 32 * c.n_heads * x->hd;
+  x->fused_opart = w.take<float>(x->fused_attn_floats);
+  x->fused_ml = w.take<float2>(x->fused_attn_floats / x->hd);
   int actr = 0;
   for (int cap_seq : {x->N, x->n_cand, x->k_keep, x->n_resp})
     if (cap_seq > 0) actr = std::max(actr, attn_counters_needed(x->B, c.n_kv_heads, G, cap_seq));
@@ -351,6 +369,16 @@ struct LayerCtx {
   int* attn_ctr = nullptr;
   int n_attn_ctr = 0;
   Prof* prof = nullptr;
+  // fused small-row layer (null: always the kernel-per-step path)
+  __nv_bfloat16* z2 = nullptr;
+  float* fused_partial = nullptr;
+  int* fused_ctr = nullptr;
+  int fused_max_tiles = 0;
+  int* fused_sync = nullptr;
+  int* fused_epoch = nullptr;
+  float* fused_opart = nullptr;
+  float2* fused_ml = nullptr;
+  size_t fused_attn_floats = 0;
 };
 
 // GEMM launch with optional event bracketing; bytes / flops are the algorithmic figures
@@ -372,6 +400,24 @@ int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_
 // O (+residual) -> RMSNorm -> gate/up (+SwiGLU) -> down (+residual).
 int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, const int* seq_off, int rows_cap,
               int rows_per_seq, cudaStream_t st) {
+  static const bool fused_on = getenv("DLLM_FUSED") != nullptr;   // opt-in while the fused layer is validated
+  if (fused_on && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on)) {
+    FusedLayerArgs a;
+    a.B = x.B; a.N = x.N; a.d = x.d; a.qd = x.qd; a.kvd = x.kvd; a.qkvd = x.qkvd; a.F = x.F; a.hd = x.hd;
+    a.Hq = x.Hq; a.Hkv = x.Hkv; a.eps = x.eps;
+    a.Wqkv = x.Wqkv; a.Wo = x.Wo; a.Wgu = x.Wgu; a.Wdn = x.Wdn; a.g_attn = x.g_attn; a.g_ffn = x.g_ffn;
+    a.kc = x.kc; a.vc = x.vc; a.rope_cos = x.rope_cos; a.rope_sin = x.rope_sin;
+    a.h = hbuf; a.rows = rows; a.n_rows = n; a.seq_off = seq_off; a.rows_cap = rows_cap; a.rows_per_seq = rows_per_seq;
+    a.z1 = x.z; a.z2 = x.z2; a.q = x.q; a.attn = x.attn; a.act = x.act;
+    a.attn_opart = x.fused_opart; a.attn_ml = x.fused_ml; a.attn_floats = x.fused_attn_floats;
+    a.partial = x.fused_partial; a.tile_counters = x.fused_ctr; a.max_tiles = x.fused_max_tiles;
+    a.sync = x.fused_sync; a.epoch = *x.fused_epoch;
+    const int rc = fused_layer_launch(a, st);
+    if (rc != DLLM_ERR_UNSUPPORTED) {
+      if (rc == DLLM_OK) *x.fused_epoch += 1;
+      return rc;
+    }
+  }
   DLLM_TRY(rmsnorm_rows_launch(hbuf, rows, n, rows_cap, x.d, x.g_attn, x.eps, x.z, x.d, st));
   GemmArgs g;
   g.W = x.Wqkv; g.w_rows_total = x.qkvd; g.X = x.z; g.rows_cap = rows_cap; g.rows_dev = n; g.K = x.d;
@@ -428,6 +474,10 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.gs = x->gs;
   L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
   L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
+  L.z2 = x->z2; L.fused_partial = x->fused_partial; L.fused_ctr = x->fused_ctr;
+  L.fused_max_tiles = x->fused_max_tiles; L.fused_sync = x->fused_sync;
+  L.fused_epoch = const_cast<int*>(&x->fused_epoch);
+  L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
 }
@@ -759,6 +809,7 @@ int dllm_reset(dllm_handle* x, void* stream) {
   x->block = 0;
   x->step_in_block = 0;
   x->n_steps = 0;
+  x->fused_epoch = 0;
   x->began = false;
   return DLLM_OK;
 }

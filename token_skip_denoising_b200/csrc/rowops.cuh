@@ -88,4 +88,30 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
                 int splits, float* opart, float2* ml, size_t partial_floats, int* counters, int n_counters,
                 cudaStream_t st);
 
+// One transformer layer for at most 32 rows as a single persistent kernel (fused_layer.cu).
+struct FusedLayerArgs {
+  int B, N, d, qd, kvd, qkvd, F, hd, Hq, Hkv;
+  float eps;
+  const __nv_bfloat16 *Wqkv, *Wo, *Wgu, *Wdn;
+  const float *g_attn, *g_ffn;
+  __nv_bfloat16 *kc, *vc;
+  const float *rope_cos, *rope_sin;
+  float* h;
+  const int* rows;
+  const int* n_rows;
+  const int* seq_off;
+  int rows_cap, rows_per_seq;
+  __nv_bfloat16 *z1, *z2, *q, *attn, *act;
+  float* attn_opart;
+  float2* attn_ml;
+  size_t attn_floats;
+  float* partial;          // fused_partial_floats(rows_cap)
+  int* tile_counters;      // 4 * max_tiles, zero between launches
+  int max_tiles;
+  int* sync;               // 8 phase counters, zero at epoch 0
+  int epoch;
+};
+size_t fused_partial_floats(int rows_cap);
+int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st);
+
 }  // namespace dllm
