@@ -471,6 +471,8 @@ size_t fused_partial_floats(int rows_cap) {
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.rows_cap <= 0 || a.rows_cap > 32) return DLLM_ERR_UNSUPPORTED;
   const int bn = a.rows_cap <= 16 ? 16 : 32;
+  const int ksub = bn == 16 ? 4 : 2;
+  if (a.d % (64 * ksub) || a.qd % (64 * ksub) || a.F % (64 * ksub) || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   const int grid = kNumSMs;
   CUtensorMap tw[4], tx[4];
   const void* W[4] = {a.Wqkv, a.Wo, a.Wgu, a.Wdn};

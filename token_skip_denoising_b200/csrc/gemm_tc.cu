@@ -430,6 +430,9 @@ struct TmapKeyHash {
   }
 };
 
+}  // namespace
+
+// Cached tensor-map encoding (also used by the fused layer kernel).
 int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   static std::mutex mu;
   static std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> cache;
@@ -449,6 +452,8 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
   cache.emplace(key, *m);
   return DLLM_OK;
 }
+
+namespace {
 
 int pick_bn(int rows) {
   if (rows <= 16) return 16;
