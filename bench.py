@@ -286,6 +286,129 @@ def micro_sweep(peaks, reps=20):
     return out
 
 
+# ---------------------------------------------------------------- SureLock / dLLM-Cache steps
+def _timed_steps(eng, n, stream):
+    """Device time (ms) of each of the next n denoising steps, one event pair per step."""
+    import torch
+    out = []
+    for _ in range(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        eng.step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def _step_roofline_ms(peaks, m, n_layers_rows, lm_rows, N, batch, extra_bytes=0.0):
+    """max(weight + K/V + extra bytes at HBM bandwidth, active-row FLOPs at the sustained
+    bf16 peak) for one step; n_layers_rows = the active row count of each layer."""
+    P = m.params_per_layer
+    flops = sum(2.0 * r * P + 4.0 * r * N * m.n_heads * m.head_dim for r in n_layers_rows)
+    flops += 2.0 * lm_rows * m.vocab * m.d_model
+    byts = len(n_layers_rows) * (2.0 * P + 2.0 * batch * N * m.kv_dim * 2) + 2.0 * m.vocab * m.d_model
+    byts += extra_bytes
+    t_b = byts / (peaks["hbm_gbs"] * 1e6)
+    t_f = flops / (peaks["bf16_tflops_sustained"] * 1e9)
+    return max(t_b, t_f), ("hbm" if t_b >= t_f else "tensor")
+
+
+def variant_steps(peaks, steps=3, warm=2):
+    """Per-step device latency of the SureLock (Dream-7B shape, batch 8) and dLLM-Cache + DUS
+    (long-context LLaDA-8B shape, batch 4) generations, at the measured selection and at
+    forced lock fractions / a forced cap, with tokens/s extrapolated to a whole run."""
+    import numpy as np
+    import torch
+
+    from synth import get_config, lock_pattern, make_tokens, make_weights
+    from token_skip_denoising_b200.engine import Engine
+
+    stream = torch.cuda.current_stream()
+    res = {}
+    # ---- SureLock, Dream-7B shape
+    cfg = get_config("dream_surelock")
+    m, B, N = cfg.model, cfg.batch, cfg.seq_len
+    w = make_weights(m, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    eng = Engine(cfg, w, tok0.clone(), stream=stream)
+    rows = []
+    for frac in (None, 0.25, 0.5, 0.75):
+        eng.reset(tok0)
+        pat = lock_pattern(B, N, frac).cuda() if frac is not None else None
+        eng.set_lock_pattern(pat)
+        _timed_steps(eng, warm, stream)                # step 0 computes every row; step 1 locks
+        t = statistics.median(_timed_steps(eng, steps, stream))
+        locked = int(eng.buffer("lock").sum())
+        active = int(eng.buffer("nrows")[0])
+        n_lm = int(eng.buffer("nlmrows")[0])
+        # logits of the recomputed rows: one store, three reads of this step's, one of the previous
+        logit_bytes = 5.0 * n_lm * m.vocab * 2
+        roof, bound = _step_roofline_ms(peaks, m, [active] * m.n_layers, n_lm, N, B, logit_bytes)
+        rows.append({"lock": "rule (KL < eps and conf > tau)" if frac is None else f"forced {frac:.2f} of positions",
+                     "locked_frac": round(locked / (B * N), 4), "active_rows": active, "lm_rows": n_lm,
+                     "ms_per_step": round(t, 3), "tokens_per_s": round(B * cfg.tokens_per_step / (t / 1e3), 2),
+                     "roofline_ms": round(roof, 3), "roofline_frac": round(roof / t, 4), "bound": bound})
+    eng.set_lock_pattern(None)
+    res["surelock_dream7b_b8"] = {
+        "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "
+                    f"{cfg.block_len}, 1 token/step; lock when KL < {cfg.kl_eps} and conf > {cfg.conf_tau}",
+        "tokens_per_s": "per step: batch x tokens per step / step time (the lock fraction of that step)",
+        "cases": rows}
+    del eng
+    w.clear()
+    torch.cuda.empty_cache()
+
+    # ---- dLLM-Cache + DUS, long-context LLaDA-8B shape
+    cfg = get_config("llada_cache_dus")
+    m, B, N = cfg.model, cfg.batch, cfg.seq_len
+    w = make_weights(m, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    n_resp = B * cfg.gen_len
+    R = max(1, math.ceil(math.log2(cfg.block_len)))
+    n_steps = cfg.n_blocks * R
+    n_ref = math.ceil(n_steps / cfg.prompt_interval)
+    rows = []
+    for forced in (0, 1):
+        eng = Engine(cfg, w, tok0.clone(), stream=stream, forced_rho=forced)
+        t_full = _timed_steps(eng, 1, stream)[0]               # step 0: full refresh
+        _timed_steps(eng, warm, stream)
+        t_part = statistics.median(_timed_steps(eng, steps, stream))
+        # selected rows of every layer, from one more (untimed) step taken layer by layer
+        eng.begin_step()
+        sel = []
+        for layer in range(m.n_layers):
+            eng.layer_forward(layer)
+            sel.append(int(eng.buffer("nsel")[0]))
+        eng.unmask()
+        torch.cuda.synchronize()
+        lm_rows = int(eng.buffer("nlmrows")[0])
+        hid_bytes = m.n_layers * 2.0 * n_resp * m.d_model * 4          # cached layer inputs and outputs
+        roof_p, bound_p = _step_roofline_ms(peaks, m, sel, lm_rows, N, B, hid_bytes)
+        vproj = m.n_layers * 2.0 * n_resp * m.d_model * m.kv_dim / (peaks["bf16_tflops_sustained"] * 1e9)
+        roof_p = max(roof_p, vproj)
+        roof_f, _ = _step_roofline_ms(peaks, m, [B * N] * m.n_layers, lm_rows, N, B)
+        gen_s = (n_ref * t_full + (n_steps - n_ref) * t_part) / 1e3
+        rows.append({"selection": "forced: exactly the cap" if forced else f"cos < {cfg.sim_tau}, capped",
+                     "rho_mean": round(float(np.mean(sel)) / n_resp, 4), "sel_rows_per_layer_max": max(sel),
+                     "refresh_ms": round(t_full, 3), "partial_ms": round(t_part, 3),
+                     "partial_roofline_ms": round(roof_p, 3), "partial_roofline_frac": round(roof_p / t_part, 4),
+                     "partial_bound": bound_p,
+                     "refresh_roofline_ms": round(roof_f, 3), "refresh_roofline_frac": round(roof_f / t_full, 4),
+                     "tokens_per_s": round(B * cfg.gen_len / gen_s, 2)})
+        del eng
+        torch.cuda.empty_cache()
+    res["dllm_cache_dus_llada8b_b4"] = {
+        "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "
+                    f"{cfg.block_len}, DUS {R} rounds/block; prompt refresh every {cfg.prompt_interval} steps; "
+                    f"cos < {cfg.sim_tau} capped at rho {cfg.rho_cap}",
+        "tokens_per_s": f"{n_ref} refresh + {n_steps - n_ref} partial steps at the measured step times",
+        "cases": rows}
+    w.clear()
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- oracle timing (CPU)
 def oracle_sample_timing(cfg, w_dev, seconds_cap=40.0):
     """Time the oracle on a bounded sample of the workload on the host cores and
@@ -413,6 +536,7 @@ def main():
     ap.add_argument("--workload", default="llada_es")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3          # timing rule: at least three untimed warm-up steps
@@ -442,6 +566,10 @@ def main():
             w.clear()
             torch.cuda.empty_cache()
             line["active_ratio_sweep"] = micro_sweep(peaks)
+        if not args.no_variants:
+            w.clear()
+            torch.cuda.empty_cache()
+            line["variant_steps"] = variant_steps(peaks)
     elif rank == 0:
         line["cpu_baseline"] = None
     if world > 1:

@@ -7,5 +7,5 @@ read their inputs from it, and neither imports the other.
 from .configs import ModelDims, RunConfig, CONFIGS, get_config  # noqa: F401
 from .gen import (  # noqa: F401
     make_weights, make_prompt, make_tokens, microbench_hidden,
-    microbench_active, WEIGHT_SEED, PROMPT_SEED,
+    microbench_active, lock_pattern, WEIGHT_SEED, PROMPT_SEED,
 )

@@ -123,3 +123,15 @@ def kv_cache_fill(n_layers: int, batch: int, n_kv: int, n: int, hd: int,
     g = _gen(device, seed + 31)
     x = torch.randn((n_layers, 2, batch, n_kv, n, hd), generator=g, device=device)
     return x.to(torch.bfloat16)
+
+
+def lock_pattern(batch: int, n: int, frac: float, seed: int = MICRO_SEED) -> torch.Tensor:
+    """A seeded lock pattern [B, N] uint8: exactly round(frac * N) positions of each
+    sequence marked, drawn uniformly without replacement (the forced lock fraction of
+    the SureLock measurement mode)."""
+    g = _gen("cpu", seed + 53)
+    out = torch.zeros((batch, n), dtype=torch.uint8)
+    m = int(round(frac * n))
+    for b in range(batch):
+        out[b, torch.randperm(n, generator=g)[:m]] = 1
+    return out

@@ -200,8 +200,7 @@ struct dllm_handle {
   float* fused_partial;
   int* fused_ctr;
   int fused_max_tiles;
-  int* fused_sync;         // state: 8 phase counters of the fused layer kernel
-  int fused_epoch = 0;
+  int* fused_sync;         // state: phase counters of the fused layer kernel (zero between launches)
   float* fused_opart;
   float2* fused_ml;
   size_t fused_attn_floats;
@@ -247,7 +246,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->masked_prev = s.take<uint8_t>(BN);
   x->lock = s.take<uint8_t>(BN);
   x->has_prev = s.take<int>(BN);
-  x->fused_sync = s.take<int>(8);
+  x->fused_sync = s.take<int>(16);
   if (c.policy == DLLM_POLICY_SURELOCK) {
     x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
     x->lse_store = s.take<float>(2 * BN);
@@ -375,7 +374,6 @@ struct LayerCtx {
   int* fused_ctr = nullptr;
   int fused_max_tiles = 0;
   int* fused_sync = nullptr;
-  int* fused_epoch = nullptr;
   float* fused_opart = nullptr;
   float2* fused_ml = nullptr;
   size_t fused_attn_floats = 0;
@@ -411,12 +409,9 @@ int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, con
     a.z1 = x.z; a.z2 = x.z2; a.q = x.q; a.attn = x.attn; a.act = x.act;
     a.attn_opart = x.fused_opart; a.attn_ml = x.fused_ml; a.attn_floats = x.fused_attn_floats;
     a.partial = x.fused_partial; a.tile_counters = x.fused_ctr; a.max_tiles = x.fused_max_tiles;
-    a.sync = x.fused_sync; a.epoch = *x.fused_epoch;
+    a.sync = x.fused_sync;
     const int rc = fused_layer_launch(a, st);
-    if (rc != DLLM_ERR_UNSUPPORTED) {
-      if (rc == DLLM_OK) *x.fused_epoch += 1;
-      return rc;
-    }
+    if (rc != DLLM_ERR_UNSUPPORTED) return rc;
   }
   DLLM_TRY(rmsnorm_rows_launch(hbuf, rows, n, rows_cap, x.d, x.g_attn, x.eps, x.z, x.d, st));
   GemmArgs g;
@@ -476,7 +471,6 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
   L.z2 = x->z2; L.fused_partial = x->fused_partial; L.fused_ctr = x->fused_ctr;
   L.fused_max_tiles = x->fused_max_tiles; L.fused_sync = x->fused_sync;
-  L.fused_epoch = const_cast<int*>(&x->fused_epoch);
   L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
@@ -809,7 +803,6 @@ int dllm_reset(dllm_handle* x, void* stream) {
   x->block = 0;
   x->step_in_block = 0;
   x->n_steps = 0;
-  x->fused_epoch = 0;
   x->began = false;
   return DLLM_OK;
 }

@@ -76,8 +76,8 @@ struct FParams {
   attn::AttnParams ap;    // q, caches, out (O operand), seq_off, split partials
   int attn_qtiles;
   int attn_items;
-  int* sync;              // [S_COUNT] monotonic phase counters
-  int target;             // (launch epoch + 1) * gridDim.x
+  int* sync;              // [S_COUNT] phase counters + [S_COUNT] exit counter, zero at launch
+  int target;             // gridDim.x: every CTA signals each phase once
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -430,6 +430,14 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 5) tmem_dealloc(tmem, C::kTmemCols);
+  // the last CTA out clears the counters, so every launch (a graph replay too) starts from zero
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sync + S_COUNT, 1) == G - 1) {
+      for (int q = 0; q <= S_COUNT; ++q) atomicExch(p.sync + q, 0);
+      __threadfence();
+    }
+  }
 }
 
 template <int BN, int KSUB>
@@ -538,7 +546,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.attn_qtiles = qtiles;
   p.attn_items = a.B * a.Hkv * qtiles * splits;
   p.sync = a.sync;
-  p.target = (a.epoch + 1) * grid;
+  p.target = grid;
   if (bn == 16) return launch_fused<16, 4>(tw, tx, p, grid, st);
   return launch_fused<32, 2>(tw, tx, p, grid, st);
 }

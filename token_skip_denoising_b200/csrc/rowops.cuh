@@ -108,8 +108,7 @@ struct FusedLayerArgs {
   float* partial;          // fused_partial_floats(rows_cap)
   int* tile_counters;      // 4 * max_tiles, zero between launches
   int max_tiles;
-  int* sync;               // 8 phase counters, zero at epoch 0
-  int epoch;
+  int* sync;               // 9 counters, zero before the launch; the kernel leaves them zero
 };
 size_t fused_partial_floats(int rows_cap);
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st);
