@@ -57,6 +57,10 @@ enum {
 enum { DLLM_POLICY_VANILLA = 0, DLLM_POLICY_ES = 1, DLLM_POLICY_SURELOCK = 2, DLLM_POLICY_DLLM_CACHE = 3 };
 enum { DLLM_UNMASK_TOPCONF = 0, DLLM_UNMASK_DUS = 1 };
 enum { DLLM_SCOPE_BLOCK = 0, DLLM_SCOPE_ALL = 1 };
+/* How a layer over a small row set runs: AUTO lets the library choose, SPLIT launches one
+   kernel per step of the layer, FUSED runs the whole layer as one persistent kernel whenever
+   at most 32 rows are recomputed (larger row sets always take SPLIT). */
+enum { DLLM_LAYER_AUTO = 0, DLLM_LAYER_SPLIT = 1, DLLM_LAYER_FUSED = 2 };
 enum { DLLM_STEP_FULL = 0, DLLM_STEP_SKIP = 1, DLLM_STEP_LOCKED = 2, DLLM_STEP_PARTIAL = 3 };
 
 /* Model shape, generation schedule and row-selection policy. */
@@ -83,6 +87,7 @@ typedef struct dllm_config {
   /* unmasking */
   int32_t unmask;          /* DLLM_UNMASK_* */
   int32_t tokens_per_step; /* TOPCONF: n committed per step and sequence */
+  int32_t layer_kernel;    /* DLLM_LAYER_* */
 } dllm_config;
 
 /* Device pointers to the weights (bf16 unless noted), all row-major [out, in]. */
@@ -214,7 +219,13 @@ enum {
   DLLM_BUF_HCACHE = 14,  /* fp32 [L, B*N, d] dLLM-Cache per-layer outputs */
   DLLM_BUF_LSE = 15,     /* fp32 [B*N] log-sum-exp of the last logits per position */
   DLLM_BUF_SELROWS = 16, /* int32 [B*N] rows picked by the last selection (ES top-k; dLLM-Cache per layer) */
-  DLLM_BUF_NSEL = 17     /* int32 [1] their number */
+  DLLM_BUF_NSEL = 17,    /* int32 [1] their number */
+  /* workspace views of the last layer's intermediates (row j = j-th recomputed row; valid
+     until the next call that runs a layer) */
+  DLLM_BUF_LAYER_Z = 18,    /* bf16 [rows, d] RMSNorm before the FFN */
+  DLLM_BUF_LAYER_Q = 19,    /* bf16 [rows, Hq*hd] rotated queries */
+  DLLM_BUF_LAYER_ATTN = 20, /* bf16 [rows, Hq*hd] attention output */
+  DLLM_BUF_LAYER_ACT = 21   /* bf16 [rows, F] SwiGLU activation */
 };
 int dllm_get_buffer(dllm_handle* h, int32_t which, void** ptr, size_t* bytes);
 

@@ -1,0 +1,96 @@
+"""The persistent one-kernel layer (DLLM_LAYER_FUSED) against the kernel-per-step layer.
+
+Both paths compute the same layer; they differ only in the order of the split-K
+partial sums and so in bf16 rounding of the intermediates.  Every intermediate of
+every layer of a skip step is compared, for row counts on both sides of the
+16-row MMA tile, for GEMMs with fewer (tile, k-block) items than SMs and with
+more, for head dims 64 and 128 and for grouped-query attention.  The oracle
+comparison of whole steps runs on the default path in the step tests.
+"""
+import pytest
+import torch
+
+from synth import get_config, make_tokens, make_weights
+from synth.configs import scaled
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from token_skip_denoising_b200.engine import Engine, device_status
+
+TOL = 2e-2
+
+
+def _rel(a, b):
+    a, b = a.float(), b.float()
+    return float((a - b).abs().max() / b.abs().max().clamp_min(1e-30))
+
+
+CASES = {
+    # tiny: d 256, hd 64; every GEMM has fewer items than SMs; 32 candidates, 8 kept rows
+    "tiny": get_config("tiny"),
+    # GQA with hd 128 (Dream-like head layout), 7 kept rows of 32
+    "gqa": scaled(get_config("llada_es"), n_layers=3, d_model=1024, n_heads=8, n_kv_heads=2, head_dim=128,
+                  ffn_dim=2816, vocab=2048, mask_id=2047).replace(skip_layer=1, prompt_len=96, gen_len=64),
+    # LLaDA-8B layer shape, 3 layers: every GEMM has more items than SMs
+    "llada": scaled(get_config("llada_es"), n_layers=3, vocab=2048, mask_id=2047).replace(skip_layer=1),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_layer_matches_split_layer(name):
+    cfg = CASES[name]
+    w = make_weights(cfg.model, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    A = Engine(cfg, w, tok0.clone(), layer_kernel="split")
+    B = Engine(cfg, w, tok0.clone(), layer_kernel="fused")
+    for e in (A, B):
+        e.step()                                   # refresh: all rows (split path in both)
+        assert e.begin_step() == "skip"
+    hd = cfg.model.head_dim
+    seen = set()
+    for layer in range(cfg.model.n_layers):
+        if layer == cfg.skip_layer:
+            A.select_active()
+            B.select_active(A.buffer("scores")[:cfg.batch * cfg.block_len].clone())   # same active set
+        for e in (A, B):
+            e.layer_forward(layer)
+        torch.cuda.synchronize()
+        assert device_status() == 0
+        n = int(A.buffer("nrows")[0])
+        assert int(B.buffer("nrows")[0]) == n
+        seen.add(n)
+        rows = A.buffer("rows")[:n].long()
+        assert torch.equal(B.buffer("rows")[:n].long(), rows)
+        for buf in ("layer_q", "layer_attn", "layer_z", "layer_act"):
+            assert _rel(B.buffer(buf)[:n], A.buffer(buf)[:n]) < TOL, (layer, buf)
+        assert _rel(B.buffer("hidden")[rows], A.buffer("hidden")[rows]) < TOL, layer
+        for cache in ("kcache", "vcache"):
+            assert _rel(B.buffer(cache)[layer].reshape(-1, hd), A.buffer(cache)[layer].reshape(-1, hd)) < TOL
+    assert max(seen) == cfg.block_len and min(seen) == cfg.keep_count(cfg.block_len)
+    for e in (A, B):
+        e.unmask()
+    torch.cuda.synchronize()
+    assert torch.equal(A.tokens, B.tokens) or _rel(B.buffer("conf"), A.buffer("conf")) < TOL
+    assert device_status() == 0
+
+
+def test_fused_layer_repeats_without_reset():
+    """The phase counters clear themselves: many fused launches in a row stay correct."""
+    cfg = CASES["tiny"]
+    w = make_weights(cfg.model, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    A = Engine(cfg, w, tok0.clone(), layer_kernel="split")
+    B = Engine(cfg, w, tok0.clone(), layer_kernel="fused")
+    for _ in range(5):
+        A.step()
+        B.step()
+        torch.cuda.synchronize()
+        assert device_status() == 0
+        # teacher-force B onto A's decisions so the two stay on the same trajectory
+        B.tokens.copy_(A.tokens)
+        for buf in ("conf", "argmax", "hidden", "hprev", "masked_prev"):
+            B.buffer(buf).copy_(A.buffer(buf))
+        for buf in ("kcache", "vcache"):
+            assert _rel(B.buffer(buf), A.buffer(buf)) < TOL
+            B.buffer(buf).copy_(A.buffer(buf))

@@ -30,7 +30,8 @@ SCOPE = {"block": 0, "all": 1}
 STEP_KIND = {0: "full", 1: "skip", 2: "locked", 3: "partial"}
 BUF = {"kcache": 0, "vcache": 1, "hidden": 2, "hprev": 3, "conf": 4, "argmax": 5, "rows": 6, "nrows": 7,
        "scores": 8, "lock": 9, "masked_prev": 10, "lmrows": 11, "nlmrows": 12, "kl": 13, "hcache": 14, "lse": 15,
-       "selrows": 16, "nsel": 17}
+       "selrows": 16, "nsel": 17, "layer_z": 18, "layer_q": 19, "layer_attn": 20, "layer_act": 21}
+LAYER_KERNEL = {"auto": 0, "split": 1, "fused": 2}
 
 
 class DllmConfig(ctypes.Structure):
@@ -42,7 +43,7 @@ class DllmConfig(ctypes.Structure):
                 ("skip_layer", c_i32), ("keep_ratio", c_f32), ("alpha", c_f32), ("refresh_period", c_i32),
                 ("kl_eps", c_f32), ("conf_tau", c_f32),
                 ("sim_tau", c_f32), ("rho_cap", c_f32), ("prompt_interval", c_i32), ("forced_rho", c_i32),
-                ("unmask", c_i32), ("tokens_per_step", c_i32)]
+                ("unmask", c_i32), ("tokens_per_step", c_i32), ("layer_kernel", c_i32)]
 
 
 class DllmWeights(ctypes.Structure):
@@ -174,7 +175,10 @@ def make_config(run, **over) -> DllmConfig:
     c.forced_rho = 0
     c.unmask = UNMASK[run.unmask]
     c.tokens_per_step = run.tokens_per_step
+    c.layer_kernel = 0
     for k, v in over.items():
+        if k == "layer_kernel" and isinstance(v, str):
+            v = LAYER_KERNEL[v]
         setattr(c, k, v)
     return c
 

@@ -113,10 +113,11 @@ __device__ __forceinline__ void attn_item(const AttnParams& p, int qt, int b, in
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const int d0 = kk * 16 + 2 * c;
-      qa[kk][0] = va ? *reinterpret_cast<const uint32_t*>(qa_row + d0) : 0u;
-      qa[kk][1] = vb ? *reinterpret_cast<const uint32_t*>(qb_row + d0) : 0u;
-      qa[kk][2] = va ? *reinterpret_cast<const uint32_t*>(qa_row + d0 + 8) : 0u;
-      qa[kk][3] = vb ? *reinterpret_cast<const uint32_t*>(qb_row + d0 + 8) : 0u;
+      // read through L2: in the fused layer other SMs wrote q earlier in the same launch
+      qa[kk][0] = va ? __ldcg(reinterpret_cast<const unsigned int*>(qa_row + d0)) : 0u;
+      qa[kk][1] = vb ? __ldcg(reinterpret_cast<const unsigned int*>(qb_row + d0)) : 0u;
+      qa[kk][2] = va ? __ldcg(reinterpret_cast<const unsigned int*>(qa_row + d0 + 8)) : 0u;
+      qa[kk][3] = vb ? __ldcg(reinterpret_cast<const unsigned int*>(qb_row + d0 + 8)) : 0u;
     }
   }
 

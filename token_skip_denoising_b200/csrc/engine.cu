@@ -110,6 +110,8 @@ int validate(const dllm_config* c) {
   if (c->unmask == DLLM_UNMASK_DUS && c->block_len == 2)
     DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "DUS: a block of 2 has no single-round non-adjacent schedule");
   if (c->block_len > 8192) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "block_len above 8192");
+  if (c->layer_kernel < DLLM_LAYER_AUTO || c->layer_kernel > DLLM_LAYER_FUSED)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown layer_kernel");
   if (c->policy == DLLM_POLICY_ES && (c->skip_layer < 0 || c->skip_layer > c->n_layers))
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "skip_layer outside [0, n_layers]");
   if (c->policy == DLLM_POLICY_ES && !(c->keep_ratio > 0.f && c->keep_ratio <= 1.f))
@@ -197,9 +199,7 @@ struct dllm_handle {
   int* attn_ctr;
   int n_attn_ctr;
   __nv_bfloat16* z2;
-  float* fused_partial;
-  int* fused_ctr;
-  int fused_max_tiles;
+  float* fused_scratch;
   int* fused_sync;         // state: phase counters of the fused layer kernel (zero between launches)
   float* fused_opart;
   float2* fused_ml;
@@ -246,7 +246,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->masked_prev = s.take<uint8_t>(BN);
   x->lock = s.take<uint8_t>(BN);
   x->has_prev = s.take<int>(BN);
-  x->fused_sync = s.take<int>(16);
+  x->fused_sync = s.take<int>(kFusedSyncInts);
   if (c.policy == DLLM_POLICY_SURELOCK) {
     x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
     x->lse_store = s.take<float>(2 * BN);
@@ -310,9 +310,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->attn_ml = w.take<float2>(ml);
   // fused small-row layer scratch
   x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(32) * x->d);
-  x->fused_partial = w.take<float>(fused_partial_floats(32));
-  x->fused_max_tiles = std::max({x->qkvd / 128, x->d / 128, x->F / 64});
-  x->fused_ctr = w.take<int>(4 * x->fused_max_tiles);
+  x->fused_scratch = w.take<float>(fused_scratch_floats(32, x->qkvd, x->F));
   x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * 32 * c.n_heads * x->hd;
   x->fused_opart = w.take<float>(x->fused_attn_floats);
   x->fused_ml = w.take<float2>(x->fused_attn_floats / x->hd);
@@ -368,11 +366,11 @@ struct LayerCtx {
   int* attn_ctr = nullptr;
   int n_attn_ctr = 0;
   Prof* prof = nullptr;
-  // fused small-row layer (null: always the kernel-per-step path)
+  // fused small-row layer (used when `fused` is set and the scratch below is present)
+  bool fused = false;
   __nv_bfloat16* z2 = nullptr;
-  float* fused_partial = nullptr;
-  int* fused_ctr = nullptr;
-  int fused_max_tiles = 0;
+  const __nv_bfloat16* Wqkv_next = nullptr;   // the next layer's QKV weights (L2 prefetch), or null
+  float* fused_scratch = nullptr;
   int* fused_sync = nullptr;
   float* fused_opart = nullptr;
   float2* fused_ml = nullptr;
@@ -398,17 +396,17 @@ int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_
 // O (+residual) -> RMSNorm -> gate/up (+SwiGLU) -> down (+residual).
 int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, const int* seq_off, int rows_cap,
               int rows_per_seq, cudaStream_t st) {
-  static const bool fused_on = getenv("DLLM_FUSED") != nullptr;   // opt-in while the fused layer is validated
-  if (fused_on && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on)) {
+  if (x.fused && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on)) {
     FusedLayerArgs a;
     a.B = x.B; a.N = x.N; a.d = x.d; a.qd = x.qd; a.kvd = x.kvd; a.qkvd = x.qkvd; a.F = x.F; a.hd = x.hd;
     a.Hq = x.Hq; a.Hkv = x.Hkv; a.eps = x.eps;
     a.Wqkv = x.Wqkv; a.Wo = x.Wo; a.Wgu = x.Wgu; a.Wdn = x.Wdn; a.g_attn = x.g_attn; a.g_ffn = x.g_ffn;
+    a.Wqkv_next = x.Wqkv_next;
     a.kc = x.kc; a.vc = x.vc; a.rope_cos = x.rope_cos; a.rope_sin = x.rope_sin;
     a.h = hbuf; a.rows = rows; a.n_rows = n; a.seq_off = seq_off; a.rows_cap = rows_cap; a.rows_per_seq = rows_per_seq;
-    a.z1 = x.z; a.z2 = x.z2; a.q = x.q; a.attn = x.attn; a.act = x.act;
+    a.z1 = x.z2; a.z2 = x.z; a.q = x.q; a.attn = x.attn; a.act = x.act;   // x.z ends with the FFN RMSNorm, as below
     a.attn_opart = x.fused_opart; a.attn_ml = x.fused_ml; a.attn_floats = x.fused_attn_floats;
-    a.partial = x.fused_partial; a.tile_counters = x.fused_ctr; a.max_tiles = x.fused_max_tiles;
+    a.scratch = x.fused_scratch;
     a.sync = x.fused_sync;
     const int rc = fused_layer_launch(a, st);
     if (rc != DLLM_ERR_UNSUPPORTED) return rc;
@@ -469,8 +467,9 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.gs = x->gs;
   L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
   L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
-  L.z2 = x->z2; L.fused_partial = x->fused_partial; L.fused_ctr = x->fused_ctr;
-  L.fused_max_tiles = x->fused_max_tiles; L.fused_sync = x->fused_sync;
+  L.fused = c.layer_kernel != DLLM_LAYER_SPLIT;   // AUTO: the fused layer whenever it applies
+  if (l + 1 < x->L) L.Wqkv_next = L.Wqkv + static_cast<size_t>(x->qkvd) * x->d;
+  L.z2 = x->z2; L.fused_scratch = x->fused_scratch; L.fused_sync = x->fused_sync;
   L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
@@ -779,6 +778,10 @@ int dllm_get_buffer(dllm_handle* x, int32_t which, void** ptr, size_t* bytes) {
     case DLLM_BUF_LSE: p = x->lse; b = BN * 4; break;
     case DLLM_BUF_SELROWS: p = x->rows2; b = BN * 4; break;
     case DLLM_BUF_NSEL: p = x->nrows2; b = 4; break;
+    case DLLM_BUF_LAYER_Z: p = x->z; b = BN * x->d * 2; break;
+    case DLLM_BUF_LAYER_Q: p = x->q; b = BN * x->qd * 2; break;
+    case DLLM_BUF_LAYER_ATTN: p = x->attn; b = BN * x->qd * 2; break;
+    case DLLM_BUF_LAYER_ACT: p = x->act; b = BN * x->F * 2; break;
     default: DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown buffer");
   }
   *ptr = p;

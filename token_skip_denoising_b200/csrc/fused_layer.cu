@@ -3,15 +3,22 @@
 // With at most 32 active rows (the ES-dLLM skip step: the block's rows below the
 // skip layer, the kept rows above it) a layer is four weight streams (QKV, O,
 // gate/up, down: 436 MB for the LLaDA-8B shape) separated by small dependent
-// steps (RMSNorm, attention over the cached K/V, the merge of split attention
-// partials).  As separate kernels each weight stream pays a pipeline fill and
-// drain.  Here one CTA per SM runs the whole layer:
+// steps (RMSNorm, RoPE, attention over the cached K/V, the split merge, SwiGLU).
+// One CTA per SM runs the whole layer:
 //   warp 4 (TMA producer) streams the weight tiles of all four GEMMs through one
-//     ring without draining between them; the activation tiles of a GEMM are
-//     requested only once its input is complete (grid-wide counters);
-//   warp 5 (MMA issuer) accumulates into two TMEM buffers;
-//   warps 0-3 run the GEMM epilogues and, between GEMMs, the RMSNorm rows, the
-//     attention items and the split merge, signalling each phase on a counter.
+//     ring; the activation tiles of a GEMM are requested once its input is
+//     complete (grid-wide phase counters).  While it waits for an input it
+//     prefetches its next weight tiles into L2, and after its last load it
+//     prefetches the start of the next layer's QKV weights, so that HBM keeps
+//     streaming across the dependent steps and the launch boundary.  At the start
+//     it prefetches this layer's K/V cache into L2 for the attention step;
+//   warp 5 (MMA issuer) accumulates each (weight tile, k range) piece into one of
+//     two TMEM buffers;
+//   warps 0-3 add every piece into an fp32 target with global reductions (the
+//     residual stream h for O and down, row-major sums for QKV and gate/up), so no
+//     piece waits for another, and between GEMMs run RMSNorm, RoPE with the K/V
+//     scatter, the attention items, the split merge and SwiGLU, signalling each
+//     phase on a counter.
 // Every cross-CTA wait is bounded; on expiry the kernel records a timeout in the
 // device status word and every role stops.
 #include <algorithm>
@@ -31,38 +38,40 @@ namespace {
 using namespace gemm;
 
 constexpr int kThreads = 192;
+constexpr int kKsub = 2;                          // 64-column k-blocks per ring stage
 constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kPrefetchAhead = 256u * 1024u;  // weight bytes a CTA may prefetch ahead of its loads
+constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
-enum Phase : int { S_NORM1 = 0, S_QKV, S_ATTN, S_COMB, S_O, S_NORM2, S_GU, S_DOWN, S_COUNT };
+enum Phase : int { S_NORM1 = 0, S_QKV, S_ROPE, S_ATTN, S_COMB, S_O, S_NORM2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
+static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
 
-template <int BN, int KSUB>
+template <int BN>
 struct FCfg {
   static constexpr uint32_t kBBytes = BN * kBK * 2;
-  static constexpr uint32_t kStageBytes = KSUB * (kABytes + kBBytes);
+  static constexpr uint32_t kStageBytes = kKsub * (kABytes + kBBytes);
   static constexpr int kFit = static_cast<int>((144u * 1024u) / kStageBytes);
-  static constexpr int kStages = kFit > 12 ? 12 : (kFit < 2 ? 2 : kFit);
+  static constexpr int kStages = kFit > 8 ? 8 : (kFit < 2 ? 2 : kFit);
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
-  static constexpr int kXPitch = 17;
   static constexpr size_t kAttnBytes = 4 * 64 * 128 * 2;   // K/V double buffer for hd <= 128
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + 128 * kXPitch * 4 +
-                                  (2 * kStages + 4) * 8 + 64;
+  static constexpr size_t kMiscBytes = 256;                 // row map + reduction slots
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + kMiscBytes + (2 * kStages + 4) * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "fused layer does not fit shared memory");
 };
 
 struct FGemm {
   int K;
-  int n_tiles;            // output tiles (SwiGLU: F / 64)
-  int swiglu, ffn;
+  int n_tiles;            // 128-row weight tiles
   int wait_slot;          // phase whose completion the activation operand needs
-  int done_slot;          // phase signalled when this GEMM's tiles are final
-  EpiParams epi;
-  float* partial;         // [gridDim.x][2][BN * 128]
-  int* counters;          // [n_tiles], zero between launches
+  float* out;             // out[row(j) * ldo + n] += (W X^T)[n][j]
+  int ldo;
+  int use_rows;           // row(j) = rows[j] (position-indexed h) or j
 };
 
 struct FParams {
   FGemm gm[4];
+  int next_tiles, next_K; // the next layer's QKV weights (L2 prefetch after the last load; 0: none)
   int rows_cap;
   const int* n_rows;      // device count of the rows
   const int* rows;        // row j -> flat b * N + pos
@@ -73,10 +82,20 @@ struct FParams {
   float* h;               // position-indexed fp32 hidden
   __nv_bfloat16* z1;      // [rows_cap, d]  RMSNorm before attention (QKV operand)
   __nv_bfloat16* z2;      // [rows_cap, d]  RMSNorm before the FFN (gate/up operand)
+  float* s_qkv;           // [rows_cap, qkvd] fp32 QKV sums
+  float* s_gu;            // [rows_cap, 2F]   fp32 gate/up sums
+  int qkvd, qd, kvd, hd, Hkv, N, F;
+  const float* rope_cos;
+  const float* rope_sin;
+  __nv_bfloat16* q;       // [rows_cap, qd] rotated queries (attention operand)
+  __nv_bfloat16* kc;      // this layer's caches [B, Hkv, N, hd]
+  __nv_bfloat16* vc;
+  __nv_bfloat16* act;     // [rows_cap, F] SwiGLU output (down operand)
+  size_t kv_bytes;        // bytes of each cache prefetched into L2 at the start (0: none)
   attn::AttnParams ap;    // q, caches, out (O operand), seq_off, split partials
   int attn_qtiles;
   int attn_items;
-  int* sync;              // [S_COUNT] phase counters + [S_COUNT] exit counter, zero at launch
+  int* sync;              // [S_COUNT] phase counters + exit counter, zero at launch
   int target;             // gridDim.x: every CTA signals each phase once
 };
 
@@ -86,6 +105,32 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void prefetch_tile_l2(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+// The (tile, k-block) items of a GEMM that CTA c owns: a contiguous range of the
+// tile-major item order, split evenly over min(items, grid) CTAs.
+struct Items {
+  int64_t lo, hi;
+  int KB;
+};
+__device__ __forceinline__ Items items_of(int K, int n_tiles, int G, int c) {
+  Items r;
+  r.KB = K / (kBK * kKsub);
+  const int64_t T = static_cast<int64_t>(n_tiles) * r.KB;
+  const int Gg = static_cast<int>(T < G ? T : G);
+  r.lo = c < Gg ? T * c / Gg : 0;
+  r.hi = c < Gg ? T * (c + 1) / Gg : 0;
+  return r;
+}
 
 // Bounded wait until counter >= target.
 __device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile int* abort) {
@@ -108,8 +153,8 @@ __device__ __forceinline__ bool epi_wait_phase(const int* ctr, int target, volat
   return !stop;
 }
 
-// The 128 epilogue threads publish a finished phase: every thread's writes are made
-// visible, then one thread bumps the counter.
+// The 128 epilogue threads publish a finished phase: every thread's writes and
+// reductions are made visible, then one thread bumps the counter.
 __device__ __forceinline__ void signal_phase(int* ctr, int tid) {
   __threadfence();
   fence_proxy_async();
@@ -117,12 +162,12 @@ __device__ __forceinline__ void signal_phase(int* ctr, int tid) {
   if (tid == 0) atomicAdd(ctr, 1);
 }
 
-// RMSNorm of one row by the 128 epilogue threads.
+// RMSNorm of one row by the 128 epilogue threads (h is read from L2: other SMs wrote it).
 __device__ __forceinline__ void norm_row(const float* __restrict__ x, const float* __restrict__ g, float eps, int d,
                                          __nv_bfloat16* __restrict__ out, int tid, float* red) {
   float ss = 0.f;
   for (int i = tid * 4; i < d; i += 512) {
-    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
   ss = warp_sum(ss);
@@ -130,7 +175,7 @@ __device__ __forceinline__ void norm_row(const float* __restrict__ x, const floa
   epi_bar();
   const float r = rsqrtf((red[0] + red[1] + red[2] + red[3]) / static_cast<float>(d) + eps);
   for (int i = tid * 4; i < d; i += 512) {
-    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
     const float4 gg = *reinterpret_cast<const float4*>(g + i);
     __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r * gg.x, v.y * r * gg.y);
     __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r * gg.z, v.w * r * gg.w);
@@ -146,24 +191,26 @@ struct NamedBar {
   __device__ __forceinline__ void operator()() const { epi_bar(); }
 };
 
-template <int BN, int KSUB>
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                    const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmW3,
                    const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmX1,
-                   const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3, FParams p) {
-  using C = FCfg<BN, KSUB>;
+                   const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3,
+                   const __grid_constant__ CUtensorMap tmNext, FParams p) {
+  using C = FCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* attn_smem = smem + C::kStages * C::kStageBytes;
-  float* xbuf = reinterpret_cast<float*>(attn_smem + C::kAttnBytes);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(xbuf + 128 * C::kXPitch);
+  int* s_rows = reinterpret_cast<int*>(attn_smem + C::kAttnBytes);   // [32]
+  float* red = reinterpret_cast<float*>(s_rows + 32);                 // [4]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(attn_smem + C::kAttnBytes + C::kMiscBytes);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* acc_full = empty_bar + C::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last piece
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
 
   const CUtensorMap* tmW[4] = {&tmW0, &tmW1, &tmW2, &tmW3};
   const CUtensorMap* tmX[4] = {&tmX0, &tmX1, &tmX2, &tmX3};
@@ -177,6 +224,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       tma_prefetch_desc(tmW[q]);
       tma_prefetch_desc(tmX[q]);
     }
+    tma_prefetch_desc(&tmNext);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -186,7 +234,6 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       mbar_init(&acc_empty[b], 128);
     }
     s_flag[0] = 0;
-    s_flag[1] = 0;
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(tmem_slot, C::kTmemCols);
@@ -200,67 +247,121 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       // ---------------- producer: every GEMM's weight tiles through one ring
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
+      // this layer's K/V cache into L2: the attention step reads all of it
+      if (p.kv_bytes) {
+        const size_t slice = ((p.kv_bytes + G - 1) / G + 15) & ~size_t(15);
+        const size_t a0 = slice * c;
+        const size_t a1 = a0 + slice < p.kv_bytes ? a0 + slice : p.kv_bytes;
+        for (size_t o = a0; o < a1; o += 32768) {
+          const uint32_t n = static_cast<uint32_t>(a1 - o < 32768 ? a1 - o : 32768);
+          prefetch_l2(reinterpret_cast<const uint8_t*>(p.kc) + o, n);
+          prefetch_l2(reinterpret_cast<const uint8_t*>(p.vc) + o, n);
+        }
+      }
+      Items R[5];
+      for (int g = 0; g < 4; ++g) R[g] = items_of(p.gm[g].K, p.gm[g].n_tiles, G, c);
+      R[4] = p.next_tiles ? items_of(p.next_K, p.next_tiles, G, c) : Items{0, 0, 1};
+      // flat positions over the items of all GEMMs (and the next layer's QKV)
+      int64_t ld_f = 0, pf_f = 0;
+      constexpr int64_t kAhead = kPrefetchAhead / (kKsub * kABytes);
+      auto prefetch_some = [&](int max_items) -> int {
+        if (pf_f < ld_f) pf_f = ld_f;
+        int done = 0;
+        while (done < max_items && pf_f - ld_f < kAhead) {
+          int64_t f = pf_f;
+          int g = 0;
+          while (g < 5 && f >= R[g].hi - R[g].lo) {
+            f -= R[g].hi - R[g].lo;
+            ++g;
+          }
+          if (g >= 5) break;
+          const int64_t item = R[g].lo + f;
+          const int tile = static_cast<int>(item / R[g].KB);
+          const int kb = static_cast<int>(item % R[g].KB);
+          const CUtensorMap* m = g < 4 ? tmW[g] : &tmNext;
+#pragma unroll
+          for (int sub = 0; sub < kKsub; ++sub) {
+            prefetch_tile_l2(m, (kb * kKsub + sub) * kBK, tile * kTileM);
+            prefetch_tile_l2(m, (kb * kKsub + sub) * kBK, tile * kTileM + 64);
+          }
+          ++pf_f;
+          ++done;
+        }
+        return done;
+      };
+      // bounded wait for an activation operand, prefetching weights meanwhile
+      auto wait_x = [&](int slot) -> bool {
+        for (uint32_t k = 0; k < kSpinLimit; ++k) {
+          if (ld_acquire(p.sync + slot) >= p.target) return true;
+          if (s_flag[0]) return false;
+          if (prefetch_some(1) == 0) __nanosleep(64);
+        }
+        set_dev_status(DLLM_DEV_TIMEOUT);
+        s_flag[0] = 1;
+        return false;
+      };
       int i = 0;
       for (int g = 0; g < 4 && !s_flag[0]; ++g) {
         const FGemm& gm = p.gm[g];
-        const int KB = gm.K / (kBK * KSUB);
-        const int64_t T = static_cast<int64_t>(gm.n_tiles) * KB;
-        const int64_t lo = sk_lo(T, G, c), hi = sk_lo(T, G, c + 1);
+        const int KB = R[g].KB;
         bool ready = false;
         int pend_s[C::kStages], pend_x[C::kStages], n_pend = 0, pend_first = 0;
         auto flush = [&]() {
           fence_proxy_async();
           for (int q = 0; q < n_pend; ++q) {
-            uint8_t* bx = stage_base + pend_s[q] * C::kStageBytes + KSUB * kABytes;
+            uint8_t* bx = stage_base + pend_s[q] * C::kStageBytes + kKsub * kABytes;
 #pragma unroll
-            for (int sub = 0; sub < KSUB; ++sub)
+            for (int sub = 0; sub < kKsub; ++sub)
               tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[pend_s[q]], pend_x[q] + sub * kBK, 0, pol_x);
           }
           n_pend = 0;
           ready = true;
         };
-        for (int64_t it = lo; it < hi && !s_flag[0];) {
+        for (int64_t it = R[g].lo; it < R[g].hi && !s_flag[0];) {
           const int tile = static_cast<int>(it / KB);
           const int kb0 = static_cast<int>(it % KB);
-          const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+          const int kb1 = (R[g].hi - it < KB - kb0) ? kb0 + static_cast<int>(R[g].hi - it) : KB;
           it += kb1 - kb0;
-          const int row0 = gm.swiglu ? tile * 64 : tile * kTileM;
-          const int row1 = gm.swiglu ? gm.ffn + tile * 64 : tile * kTileM + 64;
           for (int kb = kb0; kb < kb1; ++kb, ++i) {
             const int s = i % C::kStages;
             const uint32_t ph = (i / C::kStages) & 1;
             if (!ready && n_pend > 0 && i - C::kStages >= pend_first) {
               // the stage to reuse still waits for its activation tile
-              if (!wait_count(p.sync + gm.wait_slot, p.target, s_flag)) break;
+              if (!wait_x(gm.wait_slot)) break;
               flush();
             }
             if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
             uint8_t* a = stage_base + s * C::kStageBytes;
             mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
 #pragma unroll
-            for (int sub = 0; sub < KSUB; ++sub) {
-              const int x = (kb * KSUB + sub) * kBK;
-              tma_load_2d(a + sub * kABytes, tmW[g], &full_bar[s], x, row0, pol_w);
-              tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, row1, pol_w);
+            for (int sub = 0; sub < kKsub; ++sub) {
+              const int x = (kb * kKsub + sub) * kBK;
+              tma_load_2d(a + sub * kABytes, tmW[g], &full_bar[s], x, tile * kTileM, pol_w);
+              tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, tile * kTileM + 64, pol_w);
             }
+            ++ld_f;
             if (!ready && ld_acquire(p.sync + gm.wait_slot) >= p.target) flush();
             if (ready) {
-              uint8_t* bx = a + KSUB * kABytes;
+              uint8_t* bx = a + kKsub * kABytes;
 #pragma unroll
-              for (int sub = 0; sub < KSUB; ++sub)
-                tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[s], (kb * KSUB + sub) * kBK, 0, pol_x);
+              for (int sub = 0; sub < kKsub; ++sub)
+                tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[s], (kb * kKsub + sub) * kBK, 0, pol_x);
             } else {
               if (n_pend == 0) pend_first = i;
               pend_s[n_pend] = s;
-              pend_x[n_pend] = kb * KSUB * kBK;
+              pend_x[n_pend] = kb * kKsub * kBK;
               ++n_pend;
             }
           }
         }
         if (!ready && n_pend > 0 && !s_flag[0]) {
-          if (wait_count(p.sync + gm.wait_slot, p.target, s_flag)) flush();
+          if (wait_x(gm.wait_slot)) flush();
         }
       }
+      // the start of the next layer's weight stream, while this layer drains
+      if (!s_flag[0])
+        while (prefetch_some(8) > 0) {
+        }
     }
   } else if (warp == 5) {
     if (lane == 0) {
@@ -268,13 +369,11 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       constexpr uint32_t idesc = make_idesc_bf16(kTileM, BN);
       int i = 0, j = 0;
       for (int g = 0; g < 4 && !s_flag[0]; ++g) {
-        const FGemm& gm = p.gm[g];
-        const int KB = gm.K / (kBK * KSUB);
-        const int64_t T = static_cast<int64_t>(gm.n_tiles) * KB;
-        const int64_t lo = sk_lo(T, G, c), hi = sk_lo(T, G, c + 1);
-        for (int64_t it = lo; it < hi && !s_flag[0];) {
+        const Items r = items_of(p.gm[g].K, p.gm[g].n_tiles, G, c);
+        const int KB = r.KB;
+        for (int64_t it = r.lo; it < r.hi && !s_flag[0];) {
           const int kb0 = static_cast<int>(it % KB);
-          const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+          const int kb1 = (r.hi - it < KB - kb0) ? kb0 + static_cast<int>(r.hi - it) : KB;
           it += kb1 - kb0;
           const int b = j & 1;
           const uint32_t u = static_cast<uint32_t>(j >> 1);
@@ -288,9 +387,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
             if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; break; }
             tc_fence_after();
             const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
-            const uint32_t bb = a + KSUB * kABytes;
+            const uint32_t bb = a + kKsub * kABytes;
 #pragma unroll
-            for (int sub = 0; sub < KSUB; ++sub)
+            for (int sub = 0; sub < kKsub; ++sub)
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k)
                 tc_mma_f16(d, make_desc_k_sw128(a + sub * kABytes + k * 32),
@@ -303,22 +402,22 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       }
     }
   } else {
-    // ---------------- warps 0-3: epilogues and the steps between GEMMs
+    // ---------------- warps 0-3: reductions of the GEMM pieces and the steps between GEMMs
     const int t = threadIdx.x;
     const int m_rows = min(*p.n_rows, p.rows_cap);
-    float* red = xbuf;
+    if (t < 32) s_rows[t] = t < m_rows ? p.rows[t] : 0;
+    epi_bar();
+    const int64_t gt = static_cast<int64_t>(c) * 128 + t;   // grid-wide epilogue thread index
+    const int64_t gstride = static_cast<int64_t>(G) * 128;
     int j = 0;
     auto gemm_epilogues = [&](int g) {
       const FGemm& gm = p.gm[g];
-      const EpiParams& e = gm.epi;
-      const int KB = gm.K / (kBK * KSUB);
-      const int64_t T = static_cast<int64_t>(gm.n_tiles) * KB;
-      const int64_t lo = sk_lo(T, G, c), hi = sk_lo(T, G, c + 1);
-      const int first_tile = static_cast<int>(lo / KB);
-      for (int64_t it = lo; it < hi;) {
+      const Items r = items_of(gm.K, gm.n_tiles, G, c);
+      const int KB = r.KB;
+      for (int64_t it = r.lo; it < r.hi;) {
         const int tile = static_cast<int>(it / KB);
         const int kb0 = static_cast<int>(it % KB);
-        const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
+        const int kb1 = (r.hi - it < KB - kb0) ? kb0 + static_cast<int>(r.hi - it) : KB;
         it += kb1 - kb0;
         const int b = j & 1;
         const uint32_t u = static_cast<uint32_t>(j >> 1);
@@ -330,66 +429,81 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         }
         tc_fence_after();
         const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * C::kAccCols;
-        const int row0 = gm.swiglu ? tile * 64 : tile * kTileM;
-        const int row1 = gm.swiglu ? gm.ffn + tile * 64 : tile * kTileM + 64;
-        const int n = t < 64 ? row0 + t : row1 + (t - 64);
-        if (kb0 == 0 && kb1 == KB) {
-          for (int cc = 0; cc < BN; cc += 16) {
-            float v[16];
-            tmem_ld16(tb + cc, v);
-            if (cc + 16 >= BN) {
-              tc_fence_before();
-              mbar_arrive(&acc_empty[b]);
-            }
-            epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, cc, m_rows, tile, xbuf);
-          }
-        } else {
-          const int which = (tile == first_tile) ? 0 : 1;
-          float* mine = gm.partial + (static_cast<size_t>(c) * 2 + which) * (BN * 128);
-          for (int cc = 0; cc < BN; cc += 16) {
-            float v[16];
-            tmem_ld16(tb + cc, v);
+        float* col = gm.out + tile * kTileM + t;        // output feature n = tile * 128 + t
 #pragma unroll
-            for (int q = 0; q < 16; ++q) mine[(cc + q) * 128 + t] = v[q];
+        for (int cc = 0; cc < BN; cc += 16) {
+          float v[16];
+          tmem_ld16(tb + cc, v);
+          if (cc + 16 >= BN) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[b]);
           }
-          tc_fence_before();
-          mbar_arrive(&acc_empty[b]);
-          __threadfence();
-          epi_bar();
-          const int64_t x0 = static_cast<int64_t>(tile) * KB;
-          const int c_first = sk_first_cta(x0, T, G);
-          const int c_last = sk_first_cta(x0 + KB - 1, T, G);
-          if (t == 0) s_flag[1] = (atomicAdd(&gm.counters[tile], 1) == c_last - c_first) ? 1 : 0;
-          epi_bar();
-          if (s_flag[1]) {
-            __threadfence();
-            for (int cc = 0; cc < BN; cc += 16) {
-              float v[16];
 #pragma unroll
-              for (int q = 0; q < 16; ++q) v[q] = 0.f;
-              for (int cp = c_first; cp <= c_last; ++cp) {
-                const int wp = (tile == static_cast<int>(sk_lo(T, G, cp) / KB)) ? 0 : 1;
-                const float* src = gm.partial + (static_cast<size_t>(cp) * 2 + wp) * (BN * 128);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) v[q] += __ldcg(src + (cc + q) * 128 + t);
-              }
-              epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, cc, m_rows, tile, xbuf);
-            }
-            if (t == 0) gm.counters[tile] = 0;
+          for (int q = 0; q < 16; ++q) {
+            const int jj = cc + q;
+            if (jj < m_rows) atomicAdd(col + static_cast<int64_t>(gm.use_rows ? s_rows[jj] : jj) * gm.ldo, v[q]);
           }
-          epi_bar();
         }
       }
     };
 
-    // RMSNorm before attention
-    for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(p.rows[r]) * p.d, p.g_attn, p.eps, p.d,
+    // zero the fp32 sums of this launch's rows, RMSNorm before attention
+    {
+      const int64_t nq = static_cast<int64_t>(m_rows) * p.qkvd / 4;
+      const int64_t ng = static_cast<int64_t>(m_rows) * 2 * p.F / 4;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t x = gt; x < nq; x += gstride) reinterpret_cast<float4*>(p.s_qkv)[x] = z;
+      for (int64_t x = gt; x < ng; x += gstride) reinterpret_cast<float4*>(p.s_gu)[x] = z;
+    }
+    for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_attn, p.eps, p.d,
                                                  p.z1 + static_cast<int64_t>(r) * p.d, t, red);
     signal_phase(p.sync + S_NORM1, t);
-    gemm_epilogues(0);                                             // QKV (+RoPE, K/V scatter)
+    gemm_epilogues(0);                                             // QKV sums
     signal_phase(p.sync + S_QKV, t);
-    // attention items over the cached K/V (the new rows are in the cache now)
+    // RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention operand, k and v
+    // scattered into the cache rows of their positions
     if (epi_wait_phase(p.sync + S_QKV, p.target, s_flag, t)) {
+      const int half = p.hd >> 1;
+      const int pairs = p.qkvd >> 1;
+      const int64_t total = static_cast<int64_t>(m_rows) * pairs;
+      for (int64_t uu = gt; uu < total; uu += gstride) {
+        const int jr = static_cast<int>(uu / pairs);
+        const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
+        const int pi = rr % half;
+        const int n_lo = (rr / half) * p.hd + pi;
+        const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
+        const float xl = __ldcg(srow + n_lo), xh = __ldcg(srow + n_lo + half);
+        const int flat = s_rows[jr];
+        const int b = flat / p.N;
+        const int pos = flat - b * p.N;
+        float yl = xl, yh = xh;
+        if (n_lo < p.qd + p.kvd) {
+          const float cs = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi);
+          const float sn = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi);
+          yl = xl * cs - xh * sn;
+          yh = xh * cs + xl * sn;
+        }
+        if (n_lo < p.qd) {
+          __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
+          dst[0] = __float2bfloat16(yl);
+          dst[half] = __float2bfloat16(yh);
+        } else {
+          int nn = n_lo - p.qd;
+          __nv_bfloat16* cache = p.kc;
+          if (nn >= p.kvd) {
+            nn -= p.kvd;
+            cache = p.vc;
+          }
+          const int kvh = nn / p.hd;
+          __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
+          dst[0] = __float2bfloat16(yl);
+          dst[half] = __float2bfloat16(yh);
+        }
+      }
+    }
+    signal_phase(p.sync + S_ROPE, t);
+    // attention items over the cached K/V (the new rows are in the cache now)
+    if (epi_wait_phase(p.sync + S_ROPE, p.target, s_flag, t)) {
       for (int it = c; it < p.attn_items; it += G) {
         int rem = it;
         const int split = rem % p.ap.splits;
@@ -398,7 +512,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         rem /= p.attn_qtiles;
         const int kvh = rem % p.ap.Hkv;
         const int b = rem / p.ap.Hkv;
-        if (p.gm[0].epi.head_dim == 128) attn::attn_item<128>(p.ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+        if (p.hd == 128) attn::attn_item<128>(p.ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
         else attn::attn_item<64>(p.ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
         epi_bar();
       }
@@ -408,22 +522,34 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     if (p.ap.splits > 1 && epi_wait_phase(p.sync + S_ATTN, p.target, s_flag, t)) {
       const int units = m_rows * p.ap.Hq;
       for (int uu = c * 4 + warp; uu < units; uu += G * 4) {
-        if (p.gm[0].epi.head_dim == 128) attn::attn_merge<128>(p.ap, uu / p.ap.Hq, uu % p.ap.Hq, lane);
+        if (p.hd == 128) attn::attn_merge<128>(p.ap, uu / p.ap.Hq, uu % p.ap.Hq, lane);
         else attn::attn_merge<64>(p.ap, uu / p.ap.Hq, uu % p.ap.Hq, lane);
       }
     }
     signal_phase(p.sync + S_COMB, t);
-    gemm_epilogues(1);                                             // O (+residual)
+    gemm_epilogues(1);                                             // O, added into h
     signal_phase(p.sync + S_O, t);
     // RMSNorm before the FFN
     if (epi_wait_phase(p.sync + S_O, p.target, s_flag, t)) {
-      for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(p.rows[r]) * p.d, p.g_ffn, p.eps, p.d,
+      for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_ffn, p.eps, p.d,
                                                    p.z2 + static_cast<int64_t>(r) * p.d, t, red);
     }
     signal_phase(p.sync + S_NORM2, t);
-    gemm_epilogues(2);                                             // gate/up (+SwiGLU)
+    gemm_epilogues(2);                                             // gate/up sums
     signal_phase(p.sync + S_GU, t);
-    gemm_epilogues(3);                                             // down (+residual)
+    // SwiGLU: act = silu(gate) * up
+    if (epi_wait_phase(p.sync + S_GU, p.target, s_flag, t)) {
+      const int64_t total = static_cast<int64_t>(m_rows) * p.F;
+      for (int64_t uu = gt; uu < total; uu += gstride) {
+        const int jr = static_cast<int>(uu / p.F);
+        const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * p.F);
+        const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
+        const float g = __ldcg(srow + f), up = __ldcg(srow + p.F + f);
+        p.act[static_cast<int64_t>(jr) * p.F + f] = __float2bfloat16(g / (1.f + __expf(-g)) * up);
+      }
+    }
+    signal_phase(p.sync + S_SWIGLU, t);
+    gemm_epilogues(3);                                             // down, added into h
     signal_phase(p.sync + S_DOWN, t);
   }
 
@@ -440,12 +566,13 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   }
 }
 
-template <int BN, int KSUB>
-int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const FParams& p, int grid, cudaStream_t st) {
-  using C = FCfg<BN, KSUB>;
+template <int BN>
+int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const CUtensorMap& tn, const FParams& p,
+                 int grid, cudaStream_t st) {
+  using C = FCfg<BN>;
   static bool attr_done = false;
   if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(fused_layer_kernel<BN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    DLLM_CUDA_TRY(cudaFuncSetAttribute(fused_layer_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem)));
     attr_done = true;
   }
@@ -459,8 +586,8 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const F
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_layer_kernel<BN, KSUB>, tw[0], tw[1], tw[2], tw[3], tx[0],
-                                           tx[1], tx[2], tx[3], p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_layer_kernel<BN>, tw[0], tw[1], tw[2], tw[3], tx[0], tx[1],
+                                           tx[2], tx[3], tn, p);
   count_launch();
   if (e != cudaSuccess) {
     set_last_error(cudaGetErrorString(e), __FILE__, __LINE__);
@@ -471,18 +598,16 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const F
 
 }  // namespace
 
-size_t fused_partial_floats(int rows_cap) {
-  const int bn = rows_cap <= 16 ? 16 : 32;
-  return static_cast<size_t>(4) * kNumSMs * 2 * bn * 128;
+size_t fused_scratch_floats(int rows_cap, int qkvd, int F) {
+  return static_cast<size_t>(rows_cap) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F));
 }
 
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.rows_cap <= 0 || a.rows_cap > 32) return DLLM_ERR_UNSUPPORTED;
+  if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   const int bn = a.rows_cap <= 16 ? 16 : 32;
-  const int ksub = bn == 16 ? 4 : 2;
-  if (a.d % (64 * ksub) || a.qd % (64 * ksub) || a.F % (64 * ksub) || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   const int grid = kNumSMs;
-  CUtensorMap tw[4], tx[4];
+  CUtensorMap tw[4], tx[4], tn;
   const void* W[4] = {a.Wqkv, a.Wo, a.Wgu, a.Wdn};
   const int64_t wrows[4] = {a.qkvd, a.d, 2LL * a.F, a.d};
   const int K[4] = {a.d, a.qd, a.d, a.F};
@@ -494,30 +619,30 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
     if (rc) return rc;
   }
   FParams p;
-  const int n_tiles[4] = {a.qkvd / 128, a.d / 128, a.F / 64, a.d / 128};
-  const int waits[4] = {S_NORM1, S_COMB, S_NORM2, S_GU};
-  const int dones[4] = {S_QKV, S_O, S_GU, S_DOWN};
+  if (a.Wqkv_next) {
+    const int rc = make_tmap(&tn, a.Wqkv_next, a.qkvd, a.d, 64);
+    if (rc) return rc;
+    p.next_tiles = a.qkvd / 128;
+    p.next_K = a.d;
+  } else {
+    tn = tw[0];
+    p.next_tiles = 0;
+    p.next_K = a.d;
+  }
+  float* s_qkv = a.scratch;
+  float* s_gu = a.scratch + static_cast<size_t>(a.rows_cap) * a.qkvd;
+  const int waits[4] = {S_NORM1, S_COMB, S_NORM2, S_SWIGLU};
+  float* outs[4] = {s_qkv, a.h, s_gu, a.h};
+  const int ldos[4] = {a.qkvd, a.d, 2 * a.F, a.d};
   for (int q = 0; q < 4; ++q) {
     FGemm& g = p.gm[q];
     g.K = K[q];
-    g.n_tiles = n_tiles[q];
-    g.swiglu = q == 2;
-    g.ffn = a.F;
+    g.n_tiles = static_cast<int>(wrows[q] / 128);
     g.wait_slot = waits[q];
-    g.done_slot = dones[q];
-    g.partial = a.partial + static_cast<size_t>(q) * kNumSMs * 2 * bn * 128;
-    g.counters = a.tile_counters + q * a.max_tiles;
+    g.out = outs[q];
+    g.ldo = ldos[q];
+    g.use_rows = (q == 1 || q == 3) ? 1 : 0;
   }
-  EpiParams& e0 = p.gm[0].epi;
-  e0.kind = EPI_QKV_ROPE; e0.q_out = a.q; e0.kcache = a.kc; e0.vcache = a.vc; e0.row_map = a.rows;
-  e0.seq_n = a.N; e0.n_kv = a.Hkv; e0.head_dim = a.hd; e0.q_dim = a.qd; e0.kv_dim = a.kvd;
-  e0.rope_cos = a.rope_cos; e0.rope_sin = a.rope_sin;
-  EpiParams& e1 = p.gm[1].epi;
-  e1.kind = EPI_RESID_ADD; e1.h = a.h; e1.ldh = a.d; e1.row_map = a.rows; e1.head_dim = a.hd;
-  EpiParams& e2 = p.gm[2].epi;
-  e2.kind = EPI_SWIGLU; e2.act = a.act; e2.ffn = a.F; e2.head_dim = a.hd;
-  EpiParams& e3 = p.gm[3].epi;
-  e3.kind = EPI_RESID_ADD; e3.h = a.h; e3.ldh = a.d; e3.row_map = a.rows; e3.head_dim = a.hd;
   p.rows_cap = a.rows_cap;
   p.n_rows = a.n_rows;
   p.rows = a.rows;
@@ -528,6 +653,17 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.h = a.h;
   p.z1 = a.z1;
   p.z2 = a.z2;
+  p.s_qkv = s_qkv;
+  p.s_gu = s_gu;
+  p.qkvd = a.qkvd; p.qd = a.qd; p.kvd = a.kvd; p.hd = a.hd; p.Hkv = a.Hkv; p.N = a.N; p.F = a.F;
+  p.rope_cos = a.rope_cos;
+  p.rope_sin = a.rope_sin;
+  p.q = a.q;
+  p.kc = a.kc;
+  p.vc = a.vc;
+  p.act = a.act;
+  const size_t kv_bytes = static_cast<size_t>(a.B) * a.Hkv * a.N * a.hd * 2;
+  p.kv_bytes = kv_bytes <= kMaxKvPrefetch ? kv_bytes : 0;
   // attention work: every (sequence, KV head, query tile, key split) item
   const int Gq = a.Hq / a.Hkv;
   const int units = a.rows_per_seq * Gq;
@@ -547,8 +683,8 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.attn_items = a.B * a.Hkv * qtiles * splits;
   p.sync = a.sync;
   p.target = grid;
-  if (bn == 16) return launch_fused<16, 4>(tw, tx, p, grid, st);
-  return launch_fused<32, 2>(tw, tx, p, grid, st);
+  if (bn == 16) return launch_fused<16>(tw, tx, tn, p, grid, st);
+  return launch_fused<32>(tw, tx, tn, p, grid, st);
 }
 
 }  // namespace dllm

@@ -135,8 +135,13 @@ class Engine:
             "nlmrows": (torch.int32, (1,)), "kl": (torch.float32, (B * N,)),
             "hcache": (torch.float32, (c.n_layers, B * N, c.d_model)), "lse": (torch.float32, (B * N,)),
             "selrows": (torch.int32, (B * N,)), "nsel": (torch.int32, (1,)),
+            "layer_z": (torch.bfloat16, (-1, c.d_model)), "layer_q": (torch.bfloat16, (-1, c.n_heads * c.head_dim)),
+            "layer_attn": (torch.bfloat16, (-1, c.n_heads * c.head_dim)),
+            "layer_act": (torch.bfloat16, (-1, c.ffn_dim)),
         }
         dt, shp = defaults[name]
+        if shape is None and shp[0] == -1:
+            shp = (nb.value // (shp[1] * torch.empty(0, dtype=dt).element_size()), shp[1])
         return _lib.view(p.value, shape or shp, dtype or dt)
 
 
