@@ -147,6 +147,14 @@ int dllm_begin_step(dllm_handle* h, int32_t* kind_out, void* stream);
  * rows by value-vector cosine and recomputes only the selected ones. */
 int dllm_layer_forward(dllm_handle* h, int32_t layer, void* stream);
 
+/* Runs layers l0 .. l1-1 for the current row set, with the same result as
+ * dllm_layer_forward on each in turn.  When at most 32 rows are recomputed (and
+ * layer_kernel allows it) the whole run is one persistent kernel whose weight
+ * stream continues across the layer boundaries.  Same algorithm and page
+ * passages as dllm_layer_forward; l0 == l1 is a no-op; DLLM_ERR_INVALID_ARG when
+ * the range is outside [0, n_layers]. */
+int dllm_layers_forward(dllm_handle* h, int32_t l0, int32_t l1, void* stream);
+
 /* ES-dLLM early skip at the skip layer: scores the candidates by Eq. 1 (or
  * uses `scores_or_null`, fp32 [B, n_cand] device, for teacher forcing), keeps
  * the top k per sequence (ties to the lower position) and makes them the row

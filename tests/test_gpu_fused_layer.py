@@ -94,3 +94,72 @@ def test_fused_layer_repeats_without_reset():
         for buf in ("kcache", "vcache"):
             assert _rel(B.buffer(buf), A.buffer(buf)) < TOL
             B.buffer(buf).copy_(A.buffer(buf))
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa", "llada"])
+def test_layer_runs_match_single_layers(name):
+    """dllm_layers_forward (one persistent kernel per run of layers) against the split path
+    layer by layer: hidden rows, every layer's K/V cache and the unmasked tokens."""
+    cfg = CASES[name]
+    w = make_weights(cfg.model, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    A = Engine(cfg, w, tok0.clone(), layer_kernel="split")
+    B = Engine(cfg, w, tok0.clone(), layer_kernel="fused")
+    L, ls = cfg.model.n_layers, cfg.skip_layer
+    for e in (A, B):
+        e.step()
+        assert e.begin_step() == "skip"
+    for layer in range(ls):
+        A.layer_forward(layer)
+    B.layers_forward(0, ls)
+    A.select_active()
+    B.select_active(A.buffer("scores")[:cfg.batch * cfg.block_len].clone())
+    for layer in range(ls, L):
+        A.layer_forward(layer)
+    B.layers_forward(ls, L)
+    torch.cuda.synchronize()
+    assert device_status() == 0
+    n = int(A.buffer("nrows")[0])
+    rows = A.buffer("rows")[:n].long()
+    assert torch.equal(B.buffer("rows")[:n].long(), rows)
+    assert _rel(B.buffer("hidden")[rows], A.buffer("hidden")[rows]) < TOL
+    for cache in ("kcache", "vcache"):
+        for layer in range(L):
+            assert _rel(B.buffer(cache)[layer], A.buffer(cache)[layer]) < TOL, (cache, layer)
+    B.layers_forward(0, 0)                                    # empty run
+    with pytest.raises(RuntimeError):
+        B.layers_forward(1, L + 1)
+
+
+def test_layer_run_in_a_cuda_graph():
+    """A fused run of layers captured once and replayed gives the eager result each time."""
+    cfg = CASES["llada"]
+    w = make_weights(cfg.model, device="cuda")
+    tok0 = make_tokens(cfg).cuda()
+    E = Engine(cfg, w, tok0.clone(), layer_kernel="fused")
+    E.step()
+    E.begin_step()
+    ls, L = cfg.skip_layer, cfg.model.n_layers
+    h0 = E.buffer("hidden").clone()
+    kc0, vc0 = E.buffer("kcache").clone(), E.buffer("vcache").clone()
+    E.layers_forward(0, L)
+    torch.cuda.synchronize()
+    ref = E.buffer("hidden").clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    E.stream = s
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            E.layers_forward(0, L)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        E.buffer("hidden").copy_(h0)
+        E.buffer("kcache").copy_(kc0)
+        E.buffer("vcache").copy_(vc0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert device_status() == 0
+        assert _rel(E.buffer("hidden"), ref) < 1e-2   # fp32 reduction order differs run to run
+    E.stream = None
+    del g

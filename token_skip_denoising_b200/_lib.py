@@ -71,6 +71,7 @@ _SIGS = {
     "dllm_step_init": (ctypes.c_int, [P(c_vp), P(DllmConfig), P(DllmWeights), c_vp, c_vp, c_vp, c_vp]),
     "dllm_begin_step": (ctypes.c_int, [c_vp, P(c_i32), c_vp]),
     "dllm_layer_forward": (ctypes.c_int, [c_vp, c_i32, c_vp]),
+    "dllm_layers_forward": (ctypes.c_int, [c_vp, c_i32, c_i32, c_vp]),
     "dllm_select_active": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     "dllm_unmask": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     "dllm_step": (ctypes.c_int, [c_vp, P(DllmStepInfo), c_vp]),

@@ -201,6 +201,8 @@ struct dllm_handle {
   __nv_bfloat16* z2;
   float* fused_scratch;
   int* fused_sync;         // state: phase counters of the fused layer kernel (zero between launches)
+  int* fused_attn_ctr;     // state: split arrival counters of its attention step (zero between uses)
+  int n_fused_attn_ctr;
   float* fused_opart;
   float2* fused_ml;
   size_t fused_attn_floats;
@@ -247,6 +249,8 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->lock = s.take<uint8_t>(BN);
   x->has_prev = s.take<int>(BN);
   x->fused_sync = s.take<int>(kFusedSyncInts);
+  x->n_fused_attn_ctr = fused_attn_counters(x->B, c.n_heads, c.n_kv_heads, 32);
+  x->fused_attn_ctr = s.take<int>(x->n_fused_attn_ctr);
   if (c.policy == DLLM_POLICY_SURELOCK) {
     x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
     x->lse_store = s.take<float>(2 * BN);
@@ -366,12 +370,18 @@ struct LayerCtx {
   int* attn_ctr = nullptr;
   int n_attn_ctr = 0;
   Prof* prof = nullptr;
-  // fused small-row layer (used when `fused` is set and the scratch below is present)
+  // fused small-row layers (used when `fused` is set and the scratch below is present): the
+  // kernel addresses whole weight stacks and caches, so the context also holds layer 0's pointers
   bool fused = false;
+  int layer = 0, n_layers_total = 1;
+  const __nv_bfloat16 *Wqkv0 = nullptr, *Wo0 = nullptr, *Wgu0 = nullptr, *Wdn0 = nullptr;
+  const float *g_attn0 = nullptr, *g_ffn0 = nullptr;
+  __nv_bfloat16 *kc0 = nullptr, *vc0 = nullptr;
   __nv_bfloat16* z2 = nullptr;
-  const __nv_bfloat16* Wqkv_next = nullptr;   // the next layer's QKV weights (L2 prefetch), or null
   float* fused_scratch = nullptr;
   int* fused_sync = nullptr;
+  int* fused_attn_ctr = nullptr;
+  int n_fused_attn_ctr = 0;
   float* fused_opart = nullptr;
   float2* fused_ml = nullptr;
   size_t fused_attn_floats = 0;
@@ -391,24 +401,37 @@ int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_
   return rc;
 }
 
+// The fused persistent kernel serves row sets of at most 32 rows (not while GEMMs are timed).
+bool fused_applies(const LayerCtx& x, int rows_cap) {
+  return x.fused && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on);
+}
+
+// Layers x.layer .. x.layer + n_layers - 1 as one fused persistent kernel (DLLM_ERR_UNSUPPORTED
+// when the shapes do not allow it).
+int run_fused_layers(const LayerCtx& x, int n_layers, float* hbuf, const int* rows, const int* n, const int* seq_off,
+                     int rows_cap, int rows_per_seq, cudaStream_t st) {
+  FusedLayerArgs a;
+  a.B = x.B; a.N = x.N; a.d = x.d; a.qd = x.qd; a.kvd = x.kvd; a.qkvd = x.qkvd; a.F = x.F; a.hd = x.hd;
+  a.Hq = x.Hq; a.Hkv = x.Hkv; a.eps = x.eps;
+  a.L = x.n_layers_total; a.l0 = x.layer; a.n_layers = n_layers;
+  a.Wqkv = x.Wqkv0; a.Wo = x.Wo0; a.Wgu = x.Wgu0; a.Wdn = x.Wdn0; a.g_attn = x.g_attn0; a.g_ffn = x.g_ffn0;
+  a.kc = x.kc0; a.vc = x.vc0; a.rope_cos = x.rope_cos; a.rope_sin = x.rope_sin;
+  a.h = hbuf; a.rows = rows; a.n_rows = n; a.seq_off = seq_off; a.rows_cap = rows_cap; a.rows_per_seq = rows_per_seq;
+  a.z1 = x.z2; a.z2 = x.z; a.q = x.q; a.attn = x.attn; a.act = x.act;   // x.z ends with the FFN RMSNorm, as below
+  a.attn_opart = x.fused_opart; a.attn_ml = x.fused_ml; a.attn_floats = x.fused_attn_floats;
+  a.attn_ctr = x.fused_attn_ctr; a.n_attn_ctr = x.n_fused_attn_ctr;
+  a.scratch = x.fused_scratch;
+  a.sync = x.fused_sync;
+  return fused_layer_launch(a, st);
+}
+
 // One transformer layer on rows[j] (j < *n) of the position-indexed hidden buffer hbuf:
 // RMSNorm gather -> QKV (+RoPE, K/V scatter) -> attention over all cached keys ->
 // O (+residual) -> RMSNorm -> gate/up (+SwiGLU) -> down (+residual).
 int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, const int* seq_off, int rows_cap,
               int rows_per_seq, cudaStream_t st) {
-  if (x.fused && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on)) {
-    FusedLayerArgs a;
-    a.B = x.B; a.N = x.N; a.d = x.d; a.qd = x.qd; a.kvd = x.kvd; a.qkvd = x.qkvd; a.F = x.F; a.hd = x.hd;
-    a.Hq = x.Hq; a.Hkv = x.Hkv; a.eps = x.eps;
-    a.Wqkv = x.Wqkv; a.Wo = x.Wo; a.Wgu = x.Wgu; a.Wdn = x.Wdn; a.g_attn = x.g_attn; a.g_ffn = x.g_ffn;
-    a.Wqkv_next = x.Wqkv_next;
-    a.kc = x.kc; a.vc = x.vc; a.rope_cos = x.rope_cos; a.rope_sin = x.rope_sin;
-    a.h = hbuf; a.rows = rows; a.n_rows = n; a.seq_off = seq_off; a.rows_cap = rows_cap; a.rows_per_seq = rows_per_seq;
-    a.z1 = x.z2; a.z2 = x.z; a.q = x.q; a.attn = x.attn; a.act = x.act;   // x.z ends with the FFN RMSNorm, as below
-    a.attn_opart = x.fused_opart; a.attn_ml = x.fused_ml; a.attn_floats = x.fused_attn_floats;
-    a.scratch = x.fused_scratch;
-    a.sync = x.fused_sync;
-    const int rc = fused_layer_launch(a, st);
+  if (fused_applies(x, rows_cap)) {
+    const int rc = run_fused_layers(x, 1, hbuf, rows, n, seq_off, rows_cap, rows_per_seq, st);
     if (rc != DLLM_ERR_UNSUPPORTED) return rc;
   }
   DLLM_TRY(rmsnorm_rows_launch(hbuf, rows, n, rows_cap, x.d, x.g_attn, x.eps, x.z, x.d, st));
@@ -468,8 +491,18 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
   L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
   L.fused = c.layer_kernel != DLLM_LAYER_SPLIT;   // AUTO: the fused layer whenever it applies
-  if (l + 1 < x->L) L.Wqkv_next = L.Wqkv + static_cast<size_t>(x->qkvd) * x->d;
+  L.layer = l;
+  L.n_layers_total = x->L;
+  L.Wqkv0 = static_cast<const __nv_bfloat16*>(x->w.w_qkv);
+  L.Wo0 = static_cast<const __nv_bfloat16*>(x->w.w_o);
+  L.Wgu0 = static_cast<const __nv_bfloat16*>(x->w.w_gu);
+  L.Wdn0 = static_cast<const __nv_bfloat16*>(x->w.w_down);
+  L.g_attn0 = x->w.g_attn;
+  L.g_ffn0 = x->w.g_ffn;
+  L.kc0 = x->kcache;
+  L.vc0 = x->vcache;
   L.z2 = x->z2; L.fused_scratch = x->fused_scratch; L.fused_sync = x->fused_sync;
+  L.fused_attn_ctr = x->fused_attn_ctr; L.n_fused_attn_ctr = x->n_fused_attn_ctr;
   L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
@@ -634,6 +667,24 @@ int dllm_layer_forward(dllm_handle* x, int32_t layer, void* stream) {
                    x->cur_rows_per_seq, st);
 }
 
+int dllm_layers_forward(dllm_handle* x, int32_t l0, int32_t l1, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "layers_forward before begin_step");
+  if (l0 < 0 || l1 > x->L || l0 > l1) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "layer range out of bounds");
+  if (l0 == l1) return DLLM_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (x->c.policy != DLLM_POLICY_DLLM_CACHE) {   // dLLM-Cache picks its rows per layer
+    const LayerCtx L0 = layer_ctx(x, l0);
+    if (fused_applies(L0, x->cur_rows_cap)) {
+      const int rc = run_fused_layers(L0, l1 - l0, x->h, x->cur_rows, x->cur_n, x->cur_seq_off, x->cur_rows_cap,
+                                      x->cur_rows_per_seq, st);
+      if (rc != DLLM_ERR_UNSUPPORTED) return rc;
+    }
+  }
+  for (int l = l0; l < l1; ++l) DLLM_TRY(dllm_layer_forward(x, l, stream));
+  return DLLM_OK;
+}
+
 int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* active_idx, int32_t* active_count,
                        void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
@@ -728,11 +779,9 @@ int dllm_step(dllm_handle* x, dllm_step_info* info, void* stream) {
   DLLM_TRY(dllm_begin_step(x, &kind, stream));
   const auto& c = x->c;
   const int ls = c.policy == DLLM_POLICY_ES ? c.skip_layer : x->L;
-  for (int l = 0; l < x->L; ++l) {
-    if (l == ls) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
-    DLLM_TRY(dllm_layer_forward(x, l, stream));
-  }
-  if (ls == x->L && c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+  DLLM_TRY(dllm_layers_forward(x, 0, ls, stream));
+  if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+  DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));
   DLLM_TRY(dllm_unmask(x, nullptr, nullptr, nullptr, stream));
   if (info) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);

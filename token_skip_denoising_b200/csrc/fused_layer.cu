@@ -1,27 +1,27 @@
-// One transformer layer for a few recomputed rows as a single persistent kernel.
+// A run of transformer layers for a few recomputed rows as a single persistent kernel.
 //
 // With at most 32 active rows (the ES-dLLM skip step: the block's rows below the
 // skip layer, the kept rows above it) a layer is four weight streams (QKV, O,
 // gate/up, down: 436 MB for the LLaDA-8B shape) separated by small dependent
 // steps (RMSNorm, RoPE, attention over the cached K/V, the split merge, SwiGLU).
-// One CTA per SM runs the whole layer:
+// One CTA per SM runs every layer of the run, so the weight stream never stops at
+// a layer boundary:
 //   warp 4 (TMA producer) streams the weight tiles of all four GEMMs through one
 //     ring; the activation tiles of a GEMM are requested once its input is
-//     complete (grid-wide phase counters).  While it waits for an input it
-//     prefetches its next weight tiles into L2, and after its last load it
-//     prefetches the start of the next layer's QKV weights, so that HBM keeps
-//     streaming across the dependent steps and the launch boundary.  At the start
-//     it prefetches this layer's K/V cache into L2 for the attention step;
+//     complete (grid-wide phase counters).  At the start of each layer it
+//     prefetches that layer's K/V cache into L2 for the attention step;
 //   warp 5 (MMA issuer) accumulates each (weight tile, k range) piece into one of
 //     two TMEM buffers;
 //   warps 0-3 add every piece into an fp32 target with global reductions (the
 //     residual stream h for O and down, row-major sums for QKV and gate/up), so no
 //     piece waits for another, and between GEMMs run RMSNorm, RoPE with the K/V
-//     scatter, the attention items, the split merge and SwiGLU, signalling each
-//     phase on a counter.
+//     scatter, the attention items (the last split of a query tile merges the
+//     partials) and SwiGLU, signalling each phase on a counter that grows by the
+//     grid size per layer.
 // Every cross-CTA wait is bounded; on expiry the kernel records a timeout in the
 // device status word and every role stops.
 #include <algorithm>
+#include <cstdlib>
 
 #include "attn_dev.cuh"
 #include "common.cuh"
@@ -40,10 +40,9 @@ using namespace gemm;
 constexpr int kThreads = 192;
 constexpr int kKsub = 2;                          // 64-column k-blocks per ring stage
 constexpr uint32_t kSpinLimit = 1u << 22;
-constexpr uint32_t kPrefetchAhead = 256u * 1024u;  // weight bytes a CTA may prefetch ahead of its loads
 constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
-enum Phase : int { S_NORM1 = 0, S_QKV, S_ROPE, S_ATTN, S_COMB, S_O, S_NORM2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
+enum Phase : int { S_NORM1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_NORM2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
 static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
 
 template <int BN>
@@ -62,7 +61,7 @@ struct FCfg {
 
 struct FGemm {
   int K;
-  int n_tiles;            // 128-row weight tiles
+  int n_tiles;            // 128-row weight tiles of one layer (the tensor map stacks every layer)
   int wait_slot;          // phase whose completion the activation operand needs
   float* out;             // out[row(j) * ldo + n] += (W X^T)[n][j]
   int ldo;
@@ -71,13 +70,13 @@ struct FGemm {
 
 struct FParams {
   FGemm gm[4];
-  int next_tiles, next_K; // the next layer's QKV weights (L2 prefetch after the last load; 0: none)
+  int l0, n_layers;       // layers l0 .. l0 + n_layers - 1 of the stacks
   int rows_cap;
   const int* n_rows;      // device count of the rows
   const int* rows;        // row j -> flat b * N + pos
   int d;
   float eps;
-  const float* g_attn;
+  const float* g_attn;     // [L, d] (layer 0 of the stack)
   const float* g_ffn;
   float* h;               // position-indexed fp32 hidden
   __nv_bfloat16* z1;      // [rows_cap, d]  RMSNorm before attention (QKV operand)
@@ -88,15 +87,16 @@ struct FParams {
   const float* rope_cos;
   const float* rope_sin;
   __nv_bfloat16* q;       // [rows_cap, qd] rotated queries (attention operand)
-  __nv_bfloat16* kc;      // this layer's caches [B, Hkv, N, hd]
+  __nv_bfloat16* kc;      // caches [L, B, Hkv, N, hd] (layer 0 of the stack)
   __nv_bfloat16* vc;
+  int64_t kv_layer;       // elements of one layer's cache
   __nv_bfloat16* act;     // [rows_cap, F] SwiGLU output (down operand)
-  size_t kv_bytes;        // bytes of each cache prefetched into L2 at the start (0: none)
-  attn::AttnParams ap;    // q, caches, out (O operand), seq_off, split partials
+  size_t kv_bytes;        // bytes of each cache prefetched into L2 at a layer's start (0: none)
+  attn::AttnParams ap;    // q, out (O operand), seq_off, split partials (caches set per layer)
   int attn_qtiles;
   int attn_items;
+  int* attn_ctr;          // [B * Hkv * attn_qtiles] split arrivals, zero between uses
   int* sync;              // [S_COUNT] phase counters + exit counter, zero at launch
-  int target;             // gridDim.x: every CTA signals each phase once
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -107,12 +107,6 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void prefetch_tile_l2(const void* tmap, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(x), "r"(y)
                : "memory");
 }
 
@@ -147,19 +141,24 @@ __device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile 
 // The 128 epilogue threads wait for a phase of every CTA: thread 0 polls, the barrier
 // vote hands the outcome to all of them (true: go on).
 __device__ __forceinline__ bool epi_wait_phase(const int* ctr, int target, volatile int* abort, int tid) {
-  const bool ok = tid == 0 ? wait_count(ctr, target, abort) : true;
-  const bool stop = epi_any(!ok || *abort);
-  if (!stop) __threadfence();
-  return !stop;
+  bool ok = true;
+  if (tid == 0) {
+    ok = wait_count(ctr, target, abort);
+    __threadfence();
+  }
+  return !epi_any(!ok || *abort);   // the barrier orders the other threads' reads after the acquire
 }
 
-// The 128 epilogue threads publish a finished phase: every thread's writes and
-// reductions are made visible, then one thread bumps the counter.
+// The 128 epilogue threads publish a finished phase: their writes (for the TMA loads
+// of other CTAs, through the async proxy too) are ordered before the barrier, and one
+// thread's fence after it makes all of them visible before the counter moves.
 __device__ __forceinline__ void signal_phase(int* ctr, int tid) {
-  __threadfence();
   fence_proxy_async();
   epi_bar();
-  if (tid == 0) atomicAdd(ctr, 1);
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1);
+  }
 }
 
 // RMSNorm of one row by the 128 epilogue threads (h is read from L2: other SMs wrote it).
@@ -196,8 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                    const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmW3,
                    const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmX1,
-                   const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3,
-                   const __grid_constant__ CUtensorMap tmNext, FParams p) {
+                   const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3, FParams p) {
   using C = FCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -210,7 +208,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   uint64_t* acc_full = empty_bar + C::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last split
 
   const CUtensorMap* tmW[4] = {&tmW0, &tmW1, &tmW2, &tmW3};
   const CUtensorMap* tmX[4] = {&tmX0, &tmX1, &tmX2, &tmX3};
@@ -224,7 +222,6 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       tma_prefetch_desc(tmW[q]);
       tma_prefetch_desc(tmX[q]);
     }
-    tma_prefetch_desc(&tmNext);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -234,6 +231,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       mbar_init(&acc_empty[b], 128);
     }
     s_flag[0] = 0;
+    s_flag[1] = 0;
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(tmem_slot, C::kTmemCols);
@@ -244,160 +242,125 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
 
   if (warp == 4) {
     if (lane == 0) {
-      // ---------------- producer: every GEMM's weight tiles through one ring
+      // ---------------- producer: every GEMM's weight tiles of every layer through one ring
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      // this layer's K/V cache into L2: the attention step reads all of it
-      if (p.kv_bytes) {
-        const size_t slice = ((p.kv_bytes + G - 1) / G + 15) & ~size_t(15);
-        const size_t a0 = slice * c;
-        const size_t a1 = a0 + slice < p.kv_bytes ? a0 + slice : p.kv_bytes;
-        for (size_t o = a0; o < a1; o += 32768) {
-          const uint32_t n = static_cast<uint32_t>(a1 - o < 32768 ? a1 - o : 32768);
-          prefetch_l2(reinterpret_cast<const uint8_t*>(p.kc) + o, n);
-          prefetch_l2(reinterpret_cast<const uint8_t*>(p.vc) + o, n);
-        }
-      }
-      Items R[5];
+      Items R[4];
       for (int g = 0; g < 4; ++g) R[g] = items_of(p.gm[g].K, p.gm[g].n_tiles, G, c);
-      R[4] = p.next_tiles ? items_of(p.next_K, p.next_tiles, G, c) : Items{0, 0, 1};
-      // flat positions over the items of all GEMMs (and the next layer's QKV)
-      int64_t ld_f = 0, pf_f = 0;
-      constexpr int64_t kAhead = kPrefetchAhead / (kKsub * kABytes);
-      auto prefetch_some = [&](int max_items) -> int {
-        if (pf_f < ld_f) pf_f = ld_f;
-        int done = 0;
-        while (done < max_items && pf_f - ld_f < kAhead) {
-          int64_t f = pf_f;
-          int g = 0;
-          while (g < 5 && f >= R[g].hi - R[g].lo) {
-            f -= R[g].hi - R[g].lo;
-            ++g;
-          }
-          if (g >= 5) break;
-          const int64_t item = R[g].lo + f;
-          const int tile = static_cast<int>(item / R[g].KB);
-          const int kb = static_cast<int>(item % R[g].KB);
-          const CUtensorMap* m = g < 4 ? tmW[g] : &tmNext;
-#pragma unroll
-          for (int sub = 0; sub < kKsub; ++sub) {
-            prefetch_tile_l2(m, (kb * kKsub + sub) * kBK, tile * kTileM);
-            prefetch_tile_l2(m, (kb * kKsub + sub) * kBK, tile * kTileM + 64);
-          }
-          ++pf_f;
-          ++done;
-        }
-        return done;
-      };
-      // bounded wait for an activation operand, prefetching weights meanwhile
-      auto wait_x = [&](int slot) -> bool {
-        for (uint32_t k = 0; k < kSpinLimit; ++k) {
-          if (ld_acquire(p.sync + slot) >= p.target) return true;
-          if (s_flag[0]) return false;
-          if (prefetch_some(1) == 0) __nanosleep(64);
-        }
-        set_dev_status(DLLM_DEV_TIMEOUT);
-        s_flag[0] = 1;
-        return false;
-      };
       int i = 0;
-      for (int g = 0; g < 4 && !s_flag[0]; ++g) {
-        const FGemm& gm = p.gm[g];
-        const int KB = R[g].KB;
-        bool ready = false;
-        int pend_s[C::kStages], pend_x[C::kStages], n_pend = 0, pend_first = 0;
-        auto flush = [&]() {
-          fence_proxy_async();
-          for (int q = 0; q < n_pend; ++q) {
-            uint8_t* bx = stage_base + pend_s[q] * C::kStageBytes + kKsub * kABytes;
-#pragma unroll
-            for (int sub = 0; sub < kKsub; ++sub)
-              tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[pend_s[q]], pend_x[q] + sub * kBK, 0, pol_x);
+      for (int li = 0; li < p.n_layers && !s_flag[0]; ++li) {
+        const int target = (li + 1) * G;
+        // this layer's K/V cache into L2: its attention step reads all of it
+        if (p.kv_bytes) {
+          const size_t slice = ((p.kv_bytes + G - 1) / G + 15) & ~size_t(15);
+          const size_t a0 = slice * c;
+          const size_t a1 = a0 + slice < p.kv_bytes ? a0 + slice : p.kv_bytes;
+          const size_t lo = static_cast<size_t>(p.l0 + li) * p.kv_layer * 2;
+          for (size_t o = a0; o < a1; o += 32768) {
+            const uint32_t n = static_cast<uint32_t>(a1 - o < 32768 ? a1 - o : 32768);
+            prefetch_l2(reinterpret_cast<const uint8_t*>(p.kc) + lo + o, n);
+            prefetch_l2(reinterpret_cast<const uint8_t*>(p.vc) + lo + o, n);
           }
-          n_pend = 0;
-          ready = true;
-        };
-        for (int64_t it = R[g].lo; it < R[g].hi && !s_flag[0];) {
-          const int tile = static_cast<int>(it / KB);
-          const int kb0 = static_cast<int>(it % KB);
-          const int kb1 = (R[g].hi - it < KB - kb0) ? kb0 + static_cast<int>(R[g].hi - it) : KB;
-          it += kb1 - kb0;
-          for (int kb = kb0; kb < kb1; ++kb, ++i) {
-            const int s = i % C::kStages;
-            const uint32_t ph = (i / C::kStages) & 1;
-            if (!ready && n_pend > 0 && i - C::kStages >= pend_first) {
-              // the stage to reuse still waits for its activation tile
-              if (!wait_x(gm.wait_slot)) break;
-              flush();
-            }
-            if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
-            uint8_t* a = stage_base + s * C::kStageBytes;
-            mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
-#pragma unroll
-            for (int sub = 0; sub < kKsub; ++sub) {
-              const int x = (kb * kKsub + sub) * kBK;
-              tma_load_2d(a + sub * kABytes, tmW[g], &full_bar[s], x, tile * kTileM, pol_w);
-              tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, tile * kTileM + 64, pol_w);
-            }
-            ++ld_f;
-            if (!ready && ld_acquire(p.sync + gm.wait_slot) >= p.target) flush();
-            if (ready) {
-              uint8_t* bx = a + kKsub * kABytes;
+        }
+        // bounded wait for an activation operand of this layer
+        auto wait_x = [&](int slot) -> bool { return wait_count(p.sync + slot, target, s_flag); };
+        for (int g = 0; g < 4 && !s_flag[0]; ++g) {
+          const FGemm& gm = p.gm[g];
+          const int KB = R[g].KB;
+          const int wrow0 = (p.l0 + li) * gm.n_tiles * kTileM;
+          bool ready = false;
+          int pend_s[C::kStages], pend_x[C::kStages], n_pend = 0, pend_first = 0;
+          auto flush = [&]() {
+            fence_proxy_async();
+            for (int q = 0; q < n_pend; ++q) {
+              uint8_t* bx = stage_base + pend_s[q] * C::kStageBytes + kKsub * kABytes;
 #pragma unroll
               for (int sub = 0; sub < kKsub; ++sub)
-                tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[s], (kb * kKsub + sub) * kBK, 0, pol_x);
-            } else {
-              if (n_pend == 0) pend_first = i;
-              pend_s[n_pend] = s;
-              pend_x[n_pend] = kb * kKsub * kBK;
-              ++n_pend;
+                tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[pend_s[q]], pend_x[q] + sub * kBK, 0, pol_x);
+            }
+            n_pend = 0;
+            ready = true;
+          };
+          for (int64_t it = R[g].lo; it < R[g].hi && !s_flag[0];) {
+            const int tile = static_cast<int>(it / KB);
+            const int kb0 = static_cast<int>(it % KB);
+            const int kb1 = (R[g].hi - it < KB - kb0) ? kb0 + static_cast<int>(R[g].hi - it) : KB;
+            it += kb1 - kb0;
+            for (int kb = kb0; kb < kb1; ++kb, ++i) {
+              const int s = i % C::kStages;
+              const uint32_t ph = (i / C::kStages) & 1;
+              if (!ready && n_pend > 0 && i - C::kStages >= pend_first) {
+                // the stage to reuse still waits for its activation tile
+                if (!wait_x(gm.wait_slot)) break;
+                flush();
+              }
+              if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
+              uint8_t* a = stage_base + s * C::kStageBytes;
+              mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
+#pragma unroll
+              for (int sub = 0; sub < kKsub; ++sub) {
+                const int x = (kb * kKsub + sub) * kBK;
+                tma_load_2d(a + sub * kABytes, tmW[g], &full_bar[s], x, wrow0 + tile * kTileM, pol_w);
+                tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, wrow0 + tile * kTileM + 64,
+                            pol_w);
+              }
+              if (!ready && ld_acquire(p.sync + gm.wait_slot) >= target) flush();
+              if (ready) {
+                uint8_t* bx = a + kKsub * kABytes;
+#pragma unroll
+                for (int sub = 0; sub < kKsub; ++sub)
+                  tma_load_2d(bx + sub * C::kBBytes, tmX[g], &full_bar[s], (kb * kKsub + sub) * kBK, 0, pol_x);
+              } else {
+                if (n_pend == 0) pend_first = i;
+                pend_s[n_pend] = s;
+                pend_x[n_pend] = kb * kKsub * kBK;
+                ++n_pend;
+              }
             }
           }
-        }
-        if (!ready && n_pend > 0 && !s_flag[0]) {
-          if (wait_x(gm.wait_slot)) flush();
+          if (!ready && n_pend > 0 && !s_flag[0]) {
+            if (wait_x(gm.wait_slot)) flush();
+          }
         }
       }
-      // the start of the next layer's weight stream, while this layer drains
-      if (!s_flag[0])
-        while (prefetch_some(8) > 0) {
-        }
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ---------------- MMA issuer
       constexpr uint32_t idesc = make_idesc_bf16(kTileM, BN);
       int i = 0, j = 0;
-      for (int g = 0; g < 4 && !s_flag[0]; ++g) {
-        const Items r = items_of(p.gm[g].K, p.gm[g].n_tiles, G, c);
-        const int KB = r.KB;
-        for (int64_t it = r.lo; it < r.hi && !s_flag[0];) {
-          const int kb0 = static_cast<int>(it % KB);
-          const int kb1 = (r.hi - it < KB - kb0) ? kb0 + static_cast<int>(r.hi - it) : KB;
-          it += kb1 - kb0;
-          const int b = j & 1;
-          const uint32_t u = static_cast<uint32_t>(j >> 1);
-          ++j;
-          if (!mbar_wait(&acc_empty[b], (u & 1) ^ 1)) { s_flag[0] = 1; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + b * C::kAccCols;
-          for (int kb = kb0; kb < kb1; ++kb, ++i) {
-            const int s = i % C::kStages;
-            const uint32_t ph = (i / C::kStages) & 1;
-            if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; break; }
+      for (int li = 0; li < p.n_layers && !s_flag[0]; ++li) {
+        for (int g = 0; g < 4 && !s_flag[0]; ++g) {
+          const Items r = items_of(p.gm[g].K, p.gm[g].n_tiles, G, c);
+          const int KB = r.KB;
+          for (int64_t it = r.lo; it < r.hi && !s_flag[0];) {
+            const int kb0 = static_cast<int>(it % KB);
+            const int kb1 = (r.hi - it < KB - kb0) ? kb0 + static_cast<int>(r.hi - it) : KB;
+            it += kb1 - kb0;
+            const int b = j & 1;
+            const uint32_t u = static_cast<uint32_t>(j >> 1);
+            ++j;
+            if (!mbar_wait(&acc_empty[b], (u & 1) ^ 1)) { s_flag[0] = 1; break; }
             tc_fence_after();
-            const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
-            const uint32_t bb = a + kKsub * kABytes;
+            const uint32_t d = tmem + b * C::kAccCols;
+            for (int kb = kb0; kb < kb1; ++kb, ++i) {
+              const int s = i % C::kStages;
+              const uint32_t ph = (i / C::kStages) & 1;
+              if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; break; }
+              tc_fence_after();
+              const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
+              const uint32_t bb = a + kKsub * kABytes;
 #pragma unroll
-            for (int sub = 0; sub < kKsub; ++sub)
+              for (int sub = 0; sub < kKsub; ++sub)
 #pragma unroll
-              for (int k = 0; k < kBK / 16; ++k)
-                tc_mma_f16(d, make_desc_k_sw128(a + sub * kABytes + k * 32),
-                           make_desc_k_sw128(bb + sub * C::kBBytes + k * 32), idesc,
-                           (kb > kb0 || sub > 0 || k > 0) ? 1u : 0u);
-            tc_commit(&empty_bar[s]);
+                for (int k = 0; k < kBK / 16; ++k)
+                  tc_mma_f16(d, make_desc_k_sw128(a + sub * kABytes + k * 32),
+                             make_desc_k_sw128(bb + sub * C::kBBytes + k * 32), idesc,
+                             (kb > kb0 || sub > 0 || k > 0) ? 1u : 0u);
+              tc_commit(&empty_bar[s]);
+            }
+            tc_commit(&acc_full[b]);
           }
-          tc_commit(&acc_full[b]);
         }
       }
     }
@@ -409,6 +372,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     epi_bar();
     const int64_t gt = static_cast<int64_t>(c) * 128 + t;   // grid-wide epilogue thread index
     const int64_t gstride = static_cast<int64_t>(G) * 128;
+    const int half = p.hd >> 1;
     int j = 0;
     auto gemm_epilogues = [&](int g) {
       const FGemm& gm = p.gm[g];
@@ -447,110 +411,134 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       }
     };
 
-    // zero the fp32 sums of this launch's rows, RMSNorm before attention
-    {
-      const int64_t nq = static_cast<int64_t>(m_rows) * p.qkvd / 4;
-      const int64_t ng = static_cast<int64_t>(m_rows) * 2 * p.F / 4;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int64_t x = gt; x < nq; x += gstride) reinterpret_cast<float4*>(p.s_qkv)[x] = z;
-      for (int64_t x = gt; x < ng; x += gstride) reinterpret_cast<float4*>(p.s_gu)[x] = z;
-    }
-    for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_attn, p.eps, p.d,
-                                                 p.z1 + static_cast<int64_t>(r) * p.d, t, red);
-    signal_phase(p.sync + S_NORM1, t);
-    gemm_epilogues(0);                                             // QKV sums
-    signal_phase(p.sync + S_QKV, t);
-    // RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention operand, k and v
-    // scattered into the cache rows of their positions
-    if (epi_wait_phase(p.sync + S_QKV, p.target, s_flag, t)) {
-      const int half = p.hd >> 1;
-      const int pairs = p.qkvd >> 1;
-      const int64_t total = static_cast<int64_t>(m_rows) * pairs;
-      for (int64_t uu = gt; uu < total; uu += gstride) {
-        const int jr = static_cast<int>(uu / pairs);
-        const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
-        const int pi = rr % half;
-        const int n_lo = (rr / half) * p.hd + pi;
-        const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
-        const float xl = __ldcg(srow + n_lo), xh = __ldcg(srow + n_lo + half);
-        const int flat = s_rows[jr];
-        const int b = flat / p.N;
-        const int pos = flat - b * p.N;
-        float yl = xl, yh = xh;
-        if (n_lo < p.qd + p.kvd) {
-          const float cs = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi);
-          const float sn = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi);
-          yl = xl * cs - xh * sn;
-          yh = xh * cs + xl * sn;
-        }
-        if (n_lo < p.qd) {
-          __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
-          dst[0] = __float2bfloat16(yl);
-          dst[half] = __float2bfloat16(yh);
-        } else {
-          int nn = n_lo - p.qd;
-          __nv_bfloat16* cache = p.kc;
-          if (nn >= p.kvd) {
-            nn -= p.kvd;
-            cache = p.vc;
+    for (int li = 0; li < p.n_layers; ++li) {
+      const int l = p.l0 + li;
+      const int target = (li + 1) * G;
+      __nv_bfloat16* kc = p.kc + static_cast<int64_t>(l) * p.kv_layer;
+      __nv_bfloat16* vc = p.vc + static_cast<int64_t>(l) * p.kv_layer;
+      // the previous layer's down sums are complete in h (and its sums have been read)
+      if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t)) s_flag[0] = 1;
+      // zero the fp32 sums of this layer's rows, RMSNorm before attention
+      if (!s_flag[0]) {
+        const int64_t nq = static_cast<int64_t>(m_rows) * p.qkvd / 4;
+        const int64_t ng = static_cast<int64_t>(m_rows) * 2 * p.F / 4;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t x = gt; x < nq; x += gstride) reinterpret_cast<float4*>(p.s_qkv)[x] = z;
+        for (int64_t x = gt; x < ng; x += gstride) reinterpret_cast<float4*>(p.s_gu)[x] = z;
+        for (int r = c; r < m_rows; r += G)
+          norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_attn + static_cast<int64_t>(l) * p.d, p.eps, p.d,
+                   p.z1 + static_cast<int64_t>(r) * p.d, t, red);
+      }
+      signal_phase(p.sync + S_NORM1, t);
+      gemm_epilogues(0);                                           // QKV sums
+      signal_phase(p.sync + S_QKV, t);
+      // RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention operand, k and v
+      // scattered into the cache rows of their positions
+      if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t)) {
+        const int pairs = p.qkvd >> 1;
+        const int64_t total = static_cast<int64_t>(m_rows) * pairs;
+        for (int64_t uu = gt; uu < total; uu += gstride) {
+          const int jr = static_cast<int>(uu / pairs);
+          const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
+          const int pi = rr % half;
+          const int n_lo = (rr / half) * p.hd + pi;
+          const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
+          const float xl = __ldcg(srow + n_lo), xh = __ldcg(srow + n_lo + half);
+          const int flat = s_rows[jr];
+          const int b = flat / p.N;
+          const int pos = flat - b * p.N;
+          float yl = xl, yh = xh;
+          if (n_lo < p.qd + p.kvd) {
+            const float cs = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi);
+            const float sn = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi);
+            yl = xl * cs - xh * sn;
+            yh = xh * cs + xl * sn;
           }
-          const int kvh = nn / p.hd;
-          __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
-          dst[0] = __float2bfloat16(yl);
-          dst[half] = __float2bfloat16(yh);
+          if (n_lo < p.qd) {
+            __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
+            dst[0] = __float2bfloat16(yl);
+            dst[half] = __float2bfloat16(yh);
+          } else {
+            int nn = n_lo - p.qd;
+            __nv_bfloat16* cache = kc;
+            if (nn >= p.kvd) {
+              nn -= p.kvd;
+              cache = vc;
+            }
+            const int kvh = nn / p.hd;
+            __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
+            dst[0] = __float2bfloat16(yl);
+            dst[half] = __float2bfloat16(yh);
+          }
         }
       }
-    }
-    signal_phase(p.sync + S_ROPE, t);
-    // attention items over the cached K/V (the new rows are in the cache now)
-    if (epi_wait_phase(p.sync + S_ROPE, p.target, s_flag, t)) {
-      for (int it = c; it < p.attn_items; it += G) {
-        int rem = it;
-        const int split = rem % p.ap.splits;
-        rem /= p.ap.splits;
-        const int qt = rem % p.attn_qtiles;
-        rem /= p.attn_qtiles;
-        const int kvh = rem % p.ap.Hkv;
-        const int b = rem / p.ap.Hkv;
-        if (p.hd == 128) attn::attn_item<128>(p.ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
-        else attn::attn_item<64>(p.ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
-        epi_bar();
+      signal_phase(p.sync + S_ROPE, t);
+      // attention items over the cached K/V (the new rows are in the cache now); the last
+      // split of a (sequence, KV head, query tile) to finish merges the partials
+      if (epi_wait_phase(p.sync + S_ROPE, target, s_flag, t)) {
+        attn::AttnParams ap = p.ap;
+        ap.kc = kc;
+        ap.vc = vc;
+        const int Gq = ap.Hq / ap.Hkv;
+        for (int it = c; it < p.attn_items; it += G) {
+          int rem = it;
+          const int split = rem % ap.splits;
+          rem /= ap.splits;
+          const int qt = rem % p.attn_qtiles;
+          rem /= p.attn_qtiles;
+          const int kvh = rem % ap.Hkv;
+          const int b = rem / ap.Hkv;
+          if (p.hd == 128) attn::attn_item<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          else attn::attn_item<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          if (ap.splits > 1) {
+            __threadfence();
+            epi_bar();
+            const int grp = (b * ap.Hkv + kvh) * p.attn_qtiles + qt;
+            if (t == 0) s_flag[1] = atomicAdd(p.attn_ctr + grp, 1) == ap.splits - 1 ? 1 : 0;
+            epi_bar();
+            if (s_flag[1]) {
+              __threadfence();
+              const int off = ap.seq_off[b];
+              const int n_units = (ap.seq_off[b + 1] - off) * Gq;
+              const int u1 = min(n_units, (qt + 1) * 64);
+              for (int uu = qt * 64 + warp; uu < u1; uu += 4) {
+                const int row = off + uu / Gq, hh = kvh * Gq + uu % Gq;
+                if (p.hd == 128) attn::attn_merge<128>(ap, row, hh, lane);
+                else attn::attn_merge<64>(ap, row, hh, lane);
+              }
+              if (t == 0) p.attn_ctr[grp] = 0;
+            }
+          }
+          epi_bar();
+        }
       }
-    }
-    signal_phase(p.sync + S_ATTN, t);
-    // merge of the split partials: one warp per (row, head)
-    if (p.ap.splits > 1 && epi_wait_phase(p.sync + S_ATTN, p.target, s_flag, t)) {
-      const int units = m_rows * p.ap.Hq;
-      for (int uu = c * 4 + warp; uu < units; uu += G * 4) {
-        if (p.hd == 128) attn::attn_merge<128>(p.ap, uu / p.ap.Hq, uu % p.ap.Hq, lane);
-        else attn::attn_merge<64>(p.ap, uu / p.ap.Hq, uu % p.ap.Hq, lane);
+      signal_phase(p.sync + S_COMB, t);
+      gemm_epilogues(1);                                           // O, added into h
+      signal_phase(p.sync + S_O, t);
+      // RMSNorm before the FFN
+      if (epi_wait_phase(p.sync + S_O, target, s_flag, t)) {
+        for (int r = c; r < m_rows; r += G)
+          norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_ffn + static_cast<int64_t>(l) * p.d, p.eps, p.d,
+                   p.z2 + static_cast<int64_t>(r) * p.d, t, red);
       }
-    }
-    signal_phase(p.sync + S_COMB, t);
-    gemm_epilogues(1);                                             // O, added into h
-    signal_phase(p.sync + S_O, t);
-    // RMSNorm before the FFN
-    if (epi_wait_phase(p.sync + S_O, p.target, s_flag, t)) {
-      for (int r = c; r < m_rows; r += G) norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_ffn, p.eps, p.d,
-                                                   p.z2 + static_cast<int64_t>(r) * p.d, t, red);
-    }
-    signal_phase(p.sync + S_NORM2, t);
-    gemm_epilogues(2);                                             // gate/up sums
-    signal_phase(p.sync + S_GU, t);
-    // SwiGLU: act = silu(gate) * up
-    if (epi_wait_phase(p.sync + S_GU, p.target, s_flag, t)) {
-      const int64_t total = static_cast<int64_t>(m_rows) * p.F;
-      for (int64_t uu = gt; uu < total; uu += gstride) {
-        const int jr = static_cast<int>(uu / p.F);
-        const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * p.F);
-        const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
-        const float g = __ldcg(srow + f), up = __ldcg(srow + p.F + f);
-        p.act[static_cast<int64_t>(jr) * p.F + f] = __float2bfloat16(g / (1.f + __expf(-g)) * up);
+      signal_phase(p.sync + S_NORM2, t);
+      gemm_epilogues(2);                                           // gate/up sums
+      signal_phase(p.sync + S_GU, t);
+      // SwiGLU: act = silu(gate) * up
+      if (epi_wait_phase(p.sync + S_GU, target, s_flag, t)) {
+        const int64_t total = static_cast<int64_t>(m_rows) * p.F;
+        for (int64_t uu = gt; uu < total; uu += gstride) {
+          const int jr = static_cast<int>(uu / p.F);
+          const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * p.F);
+          const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
+          const float g = __ldcg(srow + f), up = __ldcg(srow + p.F + f);
+          p.act[static_cast<int64_t>(jr) * p.F + f] = __float2bfloat16(g / (1.f + __expf(-g)) * up);
+        }
       }
+      signal_phase(p.sync + S_SWIGLU, t);
+      gemm_epilogues(3);                                           // down, added into h
+      signal_phase(p.sync + S_DOWN, t);
     }
-    signal_phase(p.sync + S_SWIGLU, t);
-    gemm_epilogues(3);                                             // down, added into h
-    signal_phase(p.sync + S_DOWN, t);
   }
 
   tc_fence_before();
@@ -567,8 +555,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
 }
 
 template <int BN>
-int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const CUtensorMap& tn, const FParams& p,
-                 int grid, cudaStream_t st) {
+int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const FParams& p, int grid,
+                 cudaStream_t st) {
   using C = FCfg<BN>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -587,7 +575,7 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const C
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_layer_kernel<BN>, tw[0], tw[1], tw[2], tw[3], tx[0], tx[1],
-                                           tx[2], tx[3], tn, p);
+                                           tx[2], tx[3], p);
   count_launch();
   if (e != cudaSuccess) {
     set_last_error(cudaGetErrorString(e), __FILE__, __LINE__);
@@ -602,33 +590,32 @@ size_t fused_scratch_floats(int rows_cap, int qkvd, int F) {
   return static_cast<size_t>(rows_cap) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F));
 }
 
+int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
+  const int qtiles = (rows_cap * (Hq / Hkv) + 63) / 64;
+  return B * Hkv * qtiles;
+}
+
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.rows_cap <= 0 || a.rows_cap > 32) return DLLM_ERR_UNSUPPORTED;
   if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
+  if (a.n_layers <= 0 || a.l0 < 0 || a.l0 + a.n_layers > a.L) return DLLM_ERR_INVALID_ARG;
   const int bn = a.rows_cap <= 16 ? 16 : 32;
   const int grid = kNumSMs;
-  CUtensorMap tw[4], tx[4], tn;
+  CUtensorMap tw[4], tx[4];
+  // every layer of a weight stack in one map: layer l's tile rows start at l * rows per layer
   const void* W[4] = {a.Wqkv, a.Wo, a.Wgu, a.Wdn};
   const int64_t wrows[4] = {a.qkvd, a.d, 2LL * a.F, a.d};
   const int K[4] = {a.d, a.qd, a.d, a.F};
   const void* X[4] = {a.z1, a.attn, a.z2, a.act};
   for (int q = 0; q < 4; ++q) {
-    int rc = make_tmap(&tw[q], W[q], wrows[q], K[q], 64);
+    int rc = make_tmap(&tw[q], W[q], wrows[q] * a.L, K[q], 64);
     if (rc) return rc;
     rc = make_tmap(&tx[q], X[q], a.rows_cap, K[q], bn);
     if (rc) return rc;
   }
   FParams p;
-  if (a.Wqkv_next) {
-    const int rc = make_tmap(&tn, a.Wqkv_next, a.qkvd, a.d, 64);
-    if (rc) return rc;
-    p.next_tiles = a.qkvd / 128;
-    p.next_K = a.d;
-  } else {
-    tn = tw[0];
-    p.next_tiles = 0;
-    p.next_K = a.d;
-  }
+  p.l0 = a.l0;
+  p.n_layers = a.n_layers;
   float* s_qkv = a.scratch;
   float* s_gu = a.scratch + static_cast<size_t>(a.rows_cap) * a.qkvd;
   const int waits[4] = {S_NORM1, S_COMB, S_NORM2, S_SWIGLU};
@@ -661,18 +648,27 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.q = a.q;
   p.kc = a.kc;
   p.vc = a.vc;
+  p.kv_layer = static_cast<int64_t>(a.B) * a.Hkv * a.N * a.hd;
   p.act = a.act;
-  const size_t kv_bytes = static_cast<size_t>(a.B) * a.Hkv * a.N * a.hd * 2;
+  const size_t kv_bytes = static_cast<size_t>(p.kv_layer) * 2;
   p.kv_bytes = kv_bytes <= kMaxKvPrefetch ? kv_bytes : 0;
   // attention work: every (sequence, KV head, query tile, key split) item
   const int Gq = a.Hq / a.Hkv;
   const int units = a.rows_per_seq * Gq;
   const int qtiles = (units + 63) / 64;
   const int n_blocks = (a.N + 63) / 64;
-  int splits = std::max(1, std::min(n_blocks, (2 * kNumSMs + a.B * a.Hkv * qtiles - 1) / (a.B * a.Hkv * qtiles)));
+  // key splits: enough items for about one round over the grid
+  static const int splits_env = [] {
+    const char* e = getenv("DLLM_FUSED_ATTN_SPLITS");   // tuning knob for measurements
+    return e ? std::max(0, atoi(e)) : 0;
+  }();
+  const int groups = a.B * a.Hkv * qtiles;
+  int splits = splits_env > 0 ? splits_env : std::max(1, kNumSMs / groups);
+  splits = std::max(1, std::min(n_blocks, splits));
   const int bps = (n_blocks + splits - 1) / splits;
   splits = (n_blocks + bps - 1) / bps;
   if (static_cast<size_t>(splits) * a.rows_cap * a.Hq * a.hd > a.attn_floats) return DLLM_ERR_SHAPE;
+  if (a.B * a.Hkv * qtiles > a.n_attn_ctr) return DLLM_ERR_SHAPE;
   attn::AttnParams& ap = p.ap;
   ap.q = a.q; ap.kc = a.kc; ap.vc = a.vc; ap.out = a.attn; ap.seq_off = a.seq_off;
   ap.B = a.B; ap.N = a.N; ap.Hq = a.Hq; ap.Hkv = a.Hkv; ap.rows_cap = a.rows_cap;
@@ -681,10 +677,10 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   ap.opart = a.attn_opart; ap.ml = a.attn_ml;
   p.attn_qtiles = qtiles;
   p.attn_items = a.B * a.Hkv * qtiles * splits;
+  p.attn_ctr = a.attn_ctr;
   p.sync = a.sync;
-  p.target = grid;
-  if (bn == 16) return launch_fused<16>(tw, tx, tn, p, grid, st);
-  return launch_fused<32>(tw, tx, tn, p, grid, st);
+  if (bn == 16) return launch_fused<16>(tw, tx, p, grid, st);
+  return launch_fused<32>(tw, tx, p, grid, st);
 }
 
 }  // namespace dllm

@@ -89,15 +89,15 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
                 cudaStream_t st);
 
 // One transformer layer for at most 32 rows as a single persistent kernel (fused_layer.cu).
-// One layer over at most 32 rows as one persistent kernel (fused_layer.cu).
+// A run of layers over at most 32 rows as one persistent kernel (fused_layer.cu).
 constexpr int kFusedSyncInts = 16;
 struct FusedLayerArgs {
   int B, N, d, qd, kvd, qkvd, F, hd, Hq, Hkv;
+  int L, l0, n_layers;              // layers l0 .. l0 + n_layers - 1 of L
   float eps;
-  const __nv_bfloat16 *Wqkv, *Wo, *Wgu, *Wdn;
-  const __nv_bfloat16* Wqkv_next;   // the next layer's QKV weights (prefetched into L2), or null
-  const float *g_attn, *g_ffn;
-  __nv_bfloat16 *kc, *vc;           // this layer's caches [B, Hkv, N, hd]
+  const __nv_bfloat16 *Wqkv, *Wo, *Wgu, *Wdn;   // weight stacks [L, rows, K] (layer 0)
+  const float *g_attn, *g_ffn;                  // [L, d]
+  __nv_bfloat16 *kc, *vc;                       // caches [L, B, Hkv, N, hd]
   const float *rope_cos, *rope_sin;
   float* h;
   const int* rows;
@@ -108,10 +108,13 @@ struct FusedLayerArgs {
   float* attn_opart;
   float2* attn_ml;
   size_t attn_floats;
+  int* attn_ctr;           // fused_attn_counters(...) ints, zero before the launch; left zero
+  int n_attn_ctr;
   float* scratch;          // fused_scratch_floats(rows_cap, qkvd, F): fp32 QKV and gate/up sums
   int* sync;               // kFusedSyncInts counters, zero before the launch; the kernel leaves them zero
 };
 size_t fused_scratch_floats(int rows_cap, int qkvd, int F);
+int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap);
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st);
 
 }  // namespace dllm

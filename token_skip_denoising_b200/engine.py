@@ -82,6 +82,10 @@ class Engine:
     def layer_forward(self, layer: int):
         check(self.lib.dllm_layer_forward(self.handle, layer, stream_ptr(self.stream)), "dllm_layer_forward")
 
+    def layers_forward(self, l0: int, l1: int):
+        """Layers l0 .. l1-1 for the current row set (one persistent kernel when it applies)."""
+        check(self.lib.dllm_layers_forward(self.handle, l0, l1, stream_ptr(self.stream)), "dllm_layers_forward")
+
     def select_active(self, scores: torch.Tensor | None = None, active_idx=None, active_count=None):
         check(self.lib.dllm_select_active(self.handle, ptr(scores), ptr(active_idx), ptr(active_count),
                                           stream_ptr(self.stream)), "dllm_select_active")
