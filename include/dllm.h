@@ -120,6 +120,12 @@ typedef struct dllm_handle dllm_handle;
 const char* dllm_status_string(int status);
 /* Message of the last failing call on this thread ("" if none). */
 const char* dllm_last_error(void);
+/* Device status word values: the first failure a kernel records is kept until read. */
+enum {
+  DLLM_DEV_OK = 0,
+  DLLM_DEV_TIMEOUT = 1,    /* a bounded wait ran out (the kernel stopped its work and returned) */
+  DLLM_DEV_BAD_INDEX = 2   /* an index outside its table (a token id, an argmax of no finite logit) */
+};
 /* Reads (and with reset != 0 clears) the device status word; synchronises the device. */
 int dllm_device_status(int32_t* status, int32_t reset);
 
@@ -230,7 +236,8 @@ enum {
   DLLM_BUF_NSEL = 17,    /* int32 [1] their number */
   /* workspace views of the last layer's intermediates (row j = j-th recomputed row; valid
      until the next call that runs a layer) */
-  DLLM_BUF_LAYER_Z = 18,    /* bf16 [rows, d] RMSNorm before the FFN */
+  DLLM_BUF_LAYER_Z = 18,    /* bf16 [rows, d] gate/up operand: RMSNorm before the FFN (the fused
+                               layer keeps g * h there and scales the sums by 1/rms instead) */
   DLLM_BUF_LAYER_Q = 19,    /* bf16 [rows, Hq*hd] rotated queries */
   DLLM_BUF_LAYER_ATTN = 20, /* bf16 [rows, Hq*hd] attention output */
   DLLM_BUF_LAYER_ACT = 21   /* bf16 [rows, F] SwiGLU activation */
@@ -249,9 +256,11 @@ void dllm_destroy(dllm_handle* h);
 /* RoPE tables cos/sin fp32 [N, hd/2] with angle pos * theta^(-2i/hd). */
 int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, double theta, void* stream);
 
-/* h[rows[j]] = float(E[tokens[rows[j]]]) for j < *count (count nullable: rows_cap). */
-int dllm_op_embed_rows(const void* embed, const int32_t* tokens, const int32_t* rows, const int32_t* count,
-                       int32_t rows_cap, int32_t d, float* h, void* stream);
+/* h[rows[j]] = float(E[tokens[rows[j]]]) for j < *count (count nullable: rows_cap), E bf16 [vocab, d].
+ * A token id outside [0, vocab) is never read: its row is zeroed and the device status word
+ * records DLLM_DEV_BAD_INDEX (dllm_device_status). */
+int dllm_op_embed_rows(const void* embed, int32_t vocab, const int32_t* tokens, const int32_t* rows,
+                       const int32_t* count, int32_t rows_cap, int32_t d, float* h, void* stream);
 
 /* z[j] = bf16(x / sqrt(mean(x^2) + eps) * g), x = h[rows[j]] (rows nullable: j). */
 int dllm_op_rmsnorm_rows(const float* h, const int32_t* rows, const int32_t* count, int32_t rows_cap, int32_t d,

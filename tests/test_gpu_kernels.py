@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     from token_skip_denoising_b200 import ops
+    from token_skip_denoising_b200.engine import device_status
 
 DEV = "cuda"
 
@@ -113,6 +114,20 @@ def test_embed_rows():
     for r in rows.tolist():
         assert torch.equal(h[r].cpu(), E[flat[r]].float())
     assert torch.all(h[1] == -1.0)
+
+
+def test_embed_rows_rejects_token_ids_outside_the_vocabulary():
+    """The gather checks every id against the vocabulary before reading: an id outside it
+    zeroes its row and sets DLLM_DEV_BAD_INDEX instead of reading past the table."""
+    E = _bf16((64, 256), 10, 0.02)
+    tokens = torch.tensor([[3, -1, 64, 2**31 - 1, 63]], dtype=torch.int32)
+    rows = torch.arange(5, dtype=torch.int32)
+    h = torch.full((5, 256), -1.0, device=DEV)
+    assert device_status() == 0
+    ops.embed_rows(E.to(DEV), tokens.to(DEV), rows.to(DEV), None, 5, h)
+    assert device_status() == 2                     # DLLM_DEV_BAD_INDEX, and cleared
+    assert torch.equal(h[0].cpu(), E[3].float()) and torch.equal(h[4].cpu(), E[63].float())
+    assert torch.all(h[1:4] == 0.0)
 
 
 # ------------------------------------------------------------------ QKV + RoPE, SwiGLU

@@ -84,7 +84,7 @@ _SIGS = {
     "dllm_get_buffer": (ctypes.c_int, [c_vp, c_i32, P(c_vp), P(c_sz)]),
     "dllm_destroy": (None, [c_vp]),
     "dllm_op_rope_table": (ctypes.c_int, [c_vp, c_vp, c_i32, c_i32, c_f64, c_vp]),
-    "dllm_op_embed_rows": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
+    "dllm_op_embed_rows": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
     "dllm_op_rmsnorm_rows": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_f32, c_vp, c_vp]),
     "dllm_op_gemm": (ctypes.c_int, [c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32,
                                     c_vp, c_sz, c_vp]),

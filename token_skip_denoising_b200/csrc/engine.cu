@@ -314,7 +314,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->attn_ml = w.take<float2>(ml);
   // fused small-row layer scratch
   x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(32) * x->d);
-  x->fused_scratch = w.take<float>(fused_scratch_floats(32, x->qkvd, x->F));
+  x->fused_scratch = w.take<float>(fused_scratch_floats(x->qkvd, x->F));
   x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * 32 * c.n_heads * x->hd;
   x->fused_opart = w.take<float>(x->fused_attn_floats);
   x->fused_ml = w.take<float2>(x->fused_attn_floats / x->hd);
@@ -619,7 +619,7 @@ int dllm_begin_step(dllm_handle* x, int32_t* kind_out, void* stream) {
   x->cur_n = x->nrows;
   x->cur_seq_off = x->seq_off;
   x->rows_first = x->cur_rows_cap;
-  DLLM_TRY(embed_rows_launch(static_cast<const __nv_bfloat16*>(x->w.embed), x->tokens, x->rows, x->nrows,
+  DLLM_TRY(embed_rows_launch(static_cast<const __nv_bfloat16*>(x->w.embed), x->V, x->tokens, x->rows, x->nrows,
                              x->cur_rows_cap, x->d, x->h, st));
   x->began = true;
   if (kind_out) *kind_out = kind;

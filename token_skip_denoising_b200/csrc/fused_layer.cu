@@ -14,10 +14,14 @@
 //     two TMEM buffers;
 //   warps 0-3 add every piece into an fp32 target with global reductions (the
 //     residual stream h for O and down, row-major sums for QKV and gate/up), so no
-//     piece waits for another, and between GEMMs run RMSNorm, RoPE with the K/V
-//     scatter, the attention items (the last split of a query tile merges the
-//     partials) and SwiGLU, signalling each phase on a counter that grows by the
-//     grid size per layer.
+//     piece waits for another, and between GEMMs run the elementwise steps spread
+//     over the whole grid.  RMSNorm is a per-row scale, so the QKV and gate/up
+//     operands are bf16(g * h) (each CTA also leaves its partial sums of h^2) and the
+//     GEMM sums are multiplied by 1/rms afterwards, in the RoPE and SwiGLU steps.
+//     Phases per layer, each a counter that grows by the grid size: operand g * h ->
+//     QKV sums -> RoPE and K/V scatter -> attention (the last split of a query tile
+//     merges the partials) -> O in h -> operand g * h -> gate/up sums -> SwiGLU ->
+//     down in h.
 // Every cross-CTA wait is bounded; on expiry the kernel records a timeout in the
 // device status word and every role stops.
 #include <algorithm>
@@ -39,10 +43,11 @@ using namespace gemm;
 
 constexpr int kThreads = 192;
 constexpr int kKsub = 2;                          // 64-column k-blocks per ring stage
+constexpr int kMaxRows = 32;                      // rows of the fp32 sum buffers (any launch's row count)
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
-enum Phase : int { S_NORM1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_NORM2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
+enum Phase : int { S_X1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_X2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
 static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
 
 template <int BN>
@@ -54,7 +59,7 @@ struct FCfg {
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr size_t kAttnBytes = 4 * 64 * 128 * 2;   // K/V double buffer for hd <= 128
-  static constexpr size_t kMiscBytes = 256;                 // row map + reduction slots
+  static constexpr size_t kMiscBytes = 512;                 // row map, 1/rms of the rows, operand flag
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + kMiscBytes + (2 * kStages + 4) * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "fused layer does not fit shared memory");
 };
@@ -79,10 +84,12 @@ struct FParams {
   const float* g_attn;     // [L, d] (layer 0 of the stack)
   const float* g_ffn;
   float* h;               // position-indexed fp32 hidden
-  __nv_bfloat16* z1;      // [rows_cap, d]  RMSNorm before attention (QKV operand)
-  __nv_bfloat16* z2;      // [rows_cap, d]  RMSNorm before the FFN (gate/up operand)
-  float* s_qkv;           // [rows_cap, qkvd] fp32 QKV sums
-  float* s_gu;            // [rows_cap, 2F]   fp32 gate/up sums
+  __nv_bfloat16* z1;      // [rows_cap, d]  g_attn * h (QKV operand; 1/rms applied to the sums)
+  __nv_bfloat16* z2;      // [rows_cap, d]  g_ffn * h (gate/up operand)
+  float* s_qkv;           // [kMaxRows, qkvd] fp32 QKV sums
+  float* s_gu;            // [kMaxRows, 2F]   fp32 gate/up sums
+  float* ssp1;            // [grid, kMaxRows] per-CTA partial sums of h^2 before attention (RMSNorm)
+  float* ssp2;            // [grid, kMaxRows] the same before the FFN
   int qkvd, qd, kvd, hd, Hkv, N, F;
   const float* rope_cos;
   const float* rope_sin;
@@ -161,31 +168,6 @@ __device__ __forceinline__ void signal_phase(int* ctr, int tid) {
   }
 }
 
-// RMSNorm of one row by the 128 epilogue threads (h is read from L2: other SMs wrote it).
-__device__ __forceinline__ void norm_row(const float* __restrict__ x, const float* __restrict__ g, float eps, int d,
-                                         __nv_bfloat16* __restrict__ out, int tid, float* red) {
-  float ss = 0.f;
-  for (int i = tid * 4; i < d; i += 512) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
-  ss = warp_sum(ss);
-  if ((tid & 31) == 0) red[tid >> 5] = ss;
-  epi_bar();
-  const float r = rsqrtf((red[0] + red[1] + red[2] + red[3]) / static_cast<float>(d) + eps);
-  for (int i = tid * 4; i < d; i += 512) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
-    const float4 gg = *reinterpret_cast<const float4*>(g + i);
-    __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r * gg.x, v.y * r * gg.y);
-    __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r * gg.z, v.w * r * gg.w);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&a);
-    pk.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(out + i) = pk;
-  }
-  epi_bar();
-}
-
 struct NamedBar {
   __device__ __forceinline__ void operator()() const { epi_bar(); }
 };
@@ -202,7 +184,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   uint8_t* stage_base = smem;
   uint8_t* attn_smem = smem + C::kStages * C::kStageBytes;
   int* s_rows = reinterpret_cast<int*>(attn_smem + C::kAttnBytes);   // [32]
-  float* red = reinterpret_cast<float*>(s_rows + 32);                 // [4]
+  float* s_rinv1 = reinterpret_cast<float*>(s_rows + 32);             // [32] 1/rms before attention
+  float* s_rinv2 = s_rinv1 + 32;                                      // [32] 1/rms before the FFN
+  float* s_ss = s_rinv2 + 32;                                         // [32] partial sums of squares
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(attn_smem + C::kAttnBytes + C::kMiscBytes);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* acc_full = empty_bar + C::kStages;
@@ -262,8 +246,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
             prefetch_l2(reinterpret_cast<const uint8_t*>(p.vc) + lo + o, n);
           }
         }
-        // bounded wait for an activation operand of this layer
-        auto wait_x = [&](int slot) -> bool { return wait_count(p.sync + slot, target, s_flag); };
+        // bounded wait for the activation operand of GEMM g of this layer (a grid phase)
+        auto x_ready = [&](int g) -> bool { return ld_acquire(p.sync + p.gm[g].wait_slot) >= target; };
+        auto wait_x = [&](int g) -> bool { return wait_count(p.sync + p.gm[g].wait_slot, target, s_flag); };
         for (int g = 0; g < 4 && !s_flag[0]; ++g) {
           const FGemm& gm = p.gm[g];
           const int KB = R[g].KB;
@@ -291,7 +276,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
               const uint32_t ph = (i / C::kStages) & 1;
               if (!ready && n_pend > 0 && i - C::kStages >= pend_first) {
                 // the stage to reuse still waits for its activation tile
-                if (!wait_x(gm.wait_slot)) break;
+                if (!wait_x(g)) break;
                 flush();
               }
               if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
@@ -304,7 +289,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
                 tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, wrow0 + tile * kTileM + 64,
                             pol_w);
               }
-              if (!ready && ld_acquire(p.sync + gm.wait_slot) >= target) flush();
+              if (!ready && x_ready(g)) flush();
               if (ready) {
                 uint8_t* bx = a + kKsub * kABytes;
 #pragma unroll
@@ -319,7 +304,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
             }
           }
           if (!ready && n_pend > 0 && !s_flag[0]) {
-            if (wait_x(gm.wait_slot)) flush();
+            if (wait_x(g)) flush();
           }
         }
       }
@@ -374,8 +359,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     const int64_t gstride = static_cast<int64_t>(G) * 128;
     const int half = p.hd >> 1;
     int j = 0;
-    auto gemm_epilogues = [&](int g) {
+    auto gemm_epilogues = [&](int g, int li) {
       const FGemm& gm = p.gm[g];
+      float* const out = gm.out;
       const Items r = items_of(gm.K, gm.n_tiles, G, c);
       const int KB = r.KB;
       for (int64_t it = r.lo; it < r.hi;) {
@@ -393,7 +379,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         }
         tc_fence_after();
         const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * C::kAccCols;
-        float* col = gm.out + tile * kTileM + t;        // output feature n = tile * 128 + t
+        float* col = out + tile * kTileM + t;           // output feature n = tile * 128 + t
 #pragma unroll
         for (int cc = 0; cc < BN; cc += 16) {
           float v[16];
@@ -411,6 +397,46 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       }
     };
 
+    // GEMM operand X = bf16(gain * h) over every row, each CTA a slice of the columns, and
+    // the CTA's partial sums of h^2 per row into ssp[c][j] (RMSNorm is a per-row scale: the
+    // GEMM sums are multiplied by 1/rms afterwards)
+    auto gain_operand = [&](const float* gain, __nv_bfloat16* X, float* ssp) {
+      const int n4 = p.d >> 2;
+      const int q0 = static_cast<int>(static_cast<int64_t>(n4) * c / G);
+      const int q1 = static_cast<int>(static_cast<int64_t>(n4) * (c + 1) / G);
+      const int w4 = q1 - q0;
+      if (t < 32) s_ss[t] = 0.f;
+      epi_bar();
+      for (int u = t; u < m_rows * w4; u += 128) {
+        const int jj = u / w4;
+        const int k = (q0 + u - jj * w4) * 4;
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.h + static_cast<int64_t>(s_rows[jj]) * p.d + k));
+        const float4 g4 = __ldg(reinterpret_cast<const float4*>(gain + k));
+        __nv_bfloat162 lo = __floats2bfloat162_rn(g4.x * v.x, g4.y * v.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(g4.z * v.z, g4.w * v.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(X + static_cast<int64_t>(jj) * p.d + k) = pk;
+        atomicAdd(&s_ss[jj], v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w);
+      }
+      epi_bar();
+      if (t < m_rows) ssp[c * kMaxRows + t] = s_ss[t];
+    };
+    // 1/rms of every row from the partials of all CTAs (after the phase that wrote them)
+    auto rinv_from = [&](const float* ssp, float* rinv) {
+      const int jj = t & 31;
+      float acc = 0.f;
+      if (jj < m_rows)
+        for (int cc = t >> 5; cc < G; cc += 4) acc += __ldcg(ssp + cc * kMaxRows + jj);
+      if (t < 32) s_ss[t] = 0.f;
+      epi_bar();
+      if (jj < m_rows) atomicAdd(&s_ss[jj], acc);
+      epi_bar();
+      if (t < m_rows) rinv[t] = rsqrtf(s_ss[t] / static_cast<float>(p.d) + p.eps);
+      epi_bar();
+    };
+
     for (int li = 0; li < p.n_layers; ++li) {
       const int l = p.l0 + li;
       const int target = (li + 1) * G;
@@ -418,22 +444,21 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       __nv_bfloat16* vc = p.vc + static_cast<int64_t>(l) * p.kv_layer;
       // the previous layer's down sums are complete in h (and its sums have been read)
       if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t)) s_flag[0] = 1;
-      // zero the fp32 sums of this layer's rows, RMSNorm before attention
       if (!s_flag[0]) {
+        // zero this layer's sums (every CTA passes this phase before any adds into them)
         const int64_t nq = static_cast<int64_t>(m_rows) * p.qkvd / 4;
         const int64_t ng = static_cast<int64_t>(m_rows) * 2 * p.F / 4;
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int64_t x = gt; x < nq; x += gstride) reinterpret_cast<float4*>(p.s_qkv)[x] = z;
         for (int64_t x = gt; x < ng; x += gstride) reinterpret_cast<float4*>(p.s_gu)[x] = z;
-        for (int r = c; r < m_rows; r += G)
-          norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_attn + static_cast<int64_t>(l) * p.d, p.eps, p.d,
-                   p.z1 + static_cast<int64_t>(r) * p.d, t, red);
+        gain_operand(p.g_attn + static_cast<int64_t>(l) * p.d, p.z1, p.ssp1);   // QKV operand
       }
-      signal_phase(p.sync + S_NORM1, t);
-      gemm_epilogues(0);                                           // QKV sums
+      signal_phase(p.sync + S_X1, t);
+      if (epi_wait_phase(p.sync + S_X1, target, s_flag, t)) rinv_from(p.ssp1, s_rinv1);   // while QKV streams
+      gemm_epilogues(0, li);                                       // QKV sums
       signal_phase(p.sync + S_QKV, t);
-      // RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention operand, k and v
-      // scattered into the cache rows of their positions
+      // RMSNorm scale and RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention
+      // operand, k and v scattered into the cache rows of their positions
       if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t)) {
         const int pairs = p.qkvd >> 1;
         const int64_t total = static_cast<int64_t>(m_rows) * pairs;
@@ -443,7 +468,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           const int pi = rr % half;
           const int n_lo = (rr / half) * p.hd + pi;
           const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
-          const float xl = __ldcg(srow + n_lo), xh = __ldcg(srow + n_lo + half);
+          const float ri = s_rinv1[jr];
+          const float xl = __ldcg(srow + n_lo) * ri, xh = __ldcg(srow + n_lo + half) * ri;
           const int flat = s_rows[jr];
           const int b = flat / p.N;
           const int pos = flat - b * p.N;
@@ -513,30 +539,41 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         }
       }
       signal_phase(p.sync + S_COMB, t);
-      gemm_epilogues(1);                                           // O, added into h
+      gemm_epilogues(1, li);                                       // O, added into h
       signal_phase(p.sync + S_O, t);
-      // RMSNorm before the FFN
-      if (epi_wait_phase(p.sync + S_O, target, s_flag, t)) {
-        for (int r = c; r < m_rows; r += G)
-          norm_row(p.h + static_cast<int64_t>(s_rows[r]) * p.d, p.g_ffn + static_cast<int64_t>(l) * p.d, p.eps, p.d,
-                   p.z2 + static_cast<int64_t>(r) * p.d, t, red);
-      }
-      signal_phase(p.sync + S_NORM2, t);
-      gemm_epilogues(2);                                           // gate/up sums
+      // gate/up operand g_ffn * h once every O sum is in h
+      if (epi_wait_phase(p.sync + S_O, target, s_flag, t))
+        gain_operand(p.g_ffn + static_cast<int64_t>(l) * p.d, p.z2, p.ssp2);
+      signal_phase(p.sync + S_X2, t);
+      if (epi_wait_phase(p.sync + S_X2, target, s_flag, t)) rinv_from(p.ssp2, s_rinv2);   // while gate/up streams
+      gemm_epilogues(2, li);                                       // gate/up sums
       signal_phase(p.sync + S_GU, t);
-      // SwiGLU: act = silu(gate) * up
+      // SwiGLU on the RMSNorm-scaled sums: act = silu(gate) * up
       if (epi_wait_phase(p.sync + S_GU, target, s_flag, t)) {
-        const int64_t total = static_cast<int64_t>(m_rows) * p.F;
+        const int f4 = p.F >> 2;
+        const int64_t total = static_cast<int64_t>(m_rows) * f4;
         for (int64_t uu = gt; uu < total; uu += gstride) {
-          const int jr = static_cast<int>(uu / p.F);
-          const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * p.F);
+          const int jr = static_cast<int>(uu / f4);
+          const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * f4) * 4;
           const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
-          const float g = __ldcg(srow + f), up = __ldcg(srow + p.F + f);
-          p.act[static_cast<int64_t>(jr) * p.F + f] = __float2bfloat16(g / (1.f + __expf(-g)) * up);
+          const float ri = s_rinv2[jr];
+          const float4 g4 = __ldcg(reinterpret_cast<const float4*>(srow + f));
+          const float4 u4 = __ldcg(reinterpret_cast<const float4*>(srow + p.F + f));
+          const float g[4] = {g4.x * ri, g4.y * ri, g4.z * ri, g4.w * ri};
+          const float u[4] = {u4.x * ri, u4.y * ri, u4.z * ri, u4.w * ri};
+          float a[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a[e] = g[e] / (1.f + __expf(-g[e])) * u[e];
+          __nv_bfloat162 lo = __floats2bfloat162_rn(a[0], a[1]);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(a[2], a[3]);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(p.act + static_cast<int64_t>(jr) * p.F + f) = pk;
         }
       }
       signal_phase(p.sync + S_SWIGLU, t);
-      gemm_epilogues(3);                                           // down, added into h
+      gemm_epilogues(3, li);                                       // down, added into h
       signal_phase(p.sync + S_DOWN, t);
     }
   }
@@ -586,8 +623,9 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const F
 
 }  // namespace
 
-size_t fused_scratch_floats(int rows_cap, int qkvd, int F) {
-  return static_cast<size_t>(rows_cap) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F));
+size_t fused_scratch_floats(int qkvd, int F) {
+  return static_cast<size_t>(kMaxRows) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F)) +
+         2 * static_cast<size_t>(kNumSMs) * kMaxRows;
 }
 
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
@@ -596,7 +634,7 @@ int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
 }
 
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
-  if (a.rows_cap <= 0 || a.rows_cap > 32) return DLLM_ERR_UNSUPPORTED;
+  if (a.rows_cap <= 0 || a.rows_cap > kMaxRows) return DLLM_ERR_UNSUPPORTED;
   if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   if (a.n_layers <= 0 || a.l0 < 0 || a.l0 + a.n_layers > a.L) return DLLM_ERR_INVALID_ARG;
   const int bn = a.rows_cap <= 16 ? 16 : 32;
@@ -617,8 +655,9 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.l0 = a.l0;
   p.n_layers = a.n_layers;
   float* s_qkv = a.scratch;
-  float* s_gu = a.scratch + static_cast<size_t>(a.rows_cap) * a.qkvd;
-  const int waits[4] = {S_NORM1, S_COMB, S_NORM2, S_SWIGLU};
+  float* s_gu = s_qkv + static_cast<size_t>(kMaxRows) * a.qkvd;
+  float* ssp = s_gu + static_cast<size_t>(kMaxRows) * 2 * a.F;
+  const int waits[4] = {S_X1, S_COMB, S_X2, S_SWIGLU};
   float* outs[4] = {s_qkv, a.h, s_gu, a.h};
   const int ldos[4] = {a.qkvd, a.d, 2 * a.F, a.d};
   for (int q = 0; q < 4; ++q) {
@@ -642,6 +681,8 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.z2 = a.z2;
   p.s_qkv = s_qkv;
   p.s_gu = s_gu;
+  p.ssp1 = ssp;
+  p.ssp2 = ssp + static_cast<size_t>(grid) * kMaxRows;
   p.qkvd = a.qkvd; p.qd = a.qd; p.kvd = a.kvd; p.hd = a.hd; p.Hkv = a.Hkv; p.N = a.N; p.F = a.F;
   p.rope_cos = a.rope_cos;
   p.rope_sin = a.rope_sin;

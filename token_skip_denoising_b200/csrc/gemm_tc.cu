@@ -369,6 +369,10 @@ __global__ void lmhead_combine_kernel(const float4* __restrict__ part, int n_vti
     }
     const int o = out_index ? out_index[j] : j;
     const float L = M + logf(S);
+    if (BI == 0x7fffffff) {   // no finite logit: report it, and never hand on an invalid token id
+      set_dev_status(DLLM_DEV_BAD_INDEX);
+      BI = 0;
+    }
     if (conf) conf[o] = expf(BV - L);
     if (amax) amax[o] = BI;
     if (lse) lse[o] = L;

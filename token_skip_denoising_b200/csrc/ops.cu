@@ -58,10 +58,11 @@ int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, 
   return rope_table_launch(cos_t, sin_t, N, head_dim, theta, static_cast<cudaStream_t>(stream));
 }
 
-int dllm_op_embed_rows(const void* embed, const int32_t* tokens, const int32_t* rows, const int32_t* count,
-                       int32_t rows_cap, int32_t d, float* h, void* stream) {
-  if (!embed || !tokens || !rows || !h || rows_cap < 0 || d <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad embed args");
-  return embed_rows_launch(static_cast<const __nv_bfloat16*>(embed), tokens, rows, count, rows_cap, d, h,
+int dllm_op_embed_rows(const void* embed, int32_t vocab, const int32_t* tokens, const int32_t* rows,
+                       const int32_t* count, int32_t rows_cap, int32_t d, float* h, void* stream) {
+  if (!embed || !tokens || !rows || !h || rows_cap < 0 || d <= 0 || vocab <= 0)
+    OP_FAIL(DLLM_ERR_INVALID_ARG, "bad embed args");
+  return embed_rows_launch(static_cast<const __nv_bfloat16*>(embed), vocab, tokens, rows, count, rows_cap, d, h,
                            static_cast<cudaStream_t>(stream));
 }
 

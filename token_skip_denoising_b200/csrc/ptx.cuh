@@ -8,6 +8,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/dllm.h"
+
 namespace dllm {
 
 // Device status word (one per device that loads the library).  Kernels
@@ -15,7 +17,6 @@ namespace dllm {
 // with dllm_device_status().
 extern __device__ int g_dev_status;
 
-enum : int { DLLM_DEV_OK = 0, DLLM_DEV_TIMEOUT = 1, DLLM_DEV_BAD_INDEX = 2 };
 
 __device__ __forceinline__ void set_dev_status(int code) { atomicCAS(&g_dev_status, 0, code); }
 

@@ -35,7 +35,7 @@ __global__ void rope_table_kernel(float* cos_t, float* sin_t, int N, int half, d
 // ------------------------------------------------------------------ embedding
 // h[row_map[j]] = E[tokens[row_map[j]]] (bf16 -> fp32), j < count
 __global__ void embed_rows_kernel(const __nv_bfloat16* __restrict__ E, const int* __restrict__ tokens,
-                                  const int* __restrict__ row_map, const int* count_dev, int rows_cap, int d,
+                                  const int* __restrict__ row_map, const int* count_dev, int rows_cap, int d, int V,
                                   float* __restrict__ h) {
   pdl_trigger();
   pdl_wait();
@@ -44,8 +44,13 @@ __global__ void embed_rows_kernel(const __nv_bfloat16* __restrict__ E, const int
   if (j >= m) return;
   const int flat = row_map[j];
   const int tok = tokens[flat];
-  const __nv_bfloat16* src = E + static_cast<int64_t>(tok) * d;
   float* dst = h + static_cast<int64_t>(flat) * d;
+  if (tok < 0 || tok >= V) {   // a token id outside the vocabulary is reported, never read
+    if (threadIdx.x == 0) set_dev_status(DLLM_DEV_BAD_INDEX);
+    for (int i = threadIdx.x; i < d; i += blockDim.x) dst[i] = 0.f;
+    return;
+  }
+  const __nv_bfloat16* src = E + static_cast<int64_t>(tok) * d;
   for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
     const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -564,6 +569,10 @@ __global__ void kl_step_kernel(KlStep k) {
     int I = 0x7fffffff;
     for (int i = 0; i < nw; ++i)
       if (sf[i] > B || (sf[i] == B && si[i] < I)) { B = sf[i]; I = si[i]; }
+    if (I == 0x7fffffff) {   // no finite logit: report it, and never hand on an invalid token id
+      set_dev_status(DLLM_DEV_BAD_INDEX);
+      I = 0;
+    }
     s_res[1] = B;
     si[31] = I;
   }
@@ -648,12 +657,12 @@ int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, c
   return DLLM_OK;
 }
 
-int embed_rows_launch(const __nv_bfloat16* E, const int* tokens, const int* row_map, const int* count_dev,
+int embed_rows_launch(const __nv_bfloat16* E, int V, const int* tokens, const int* row_map, const int* count_dev,
                       int rows_cap, int d, float* h, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
   if (d % 8) return DLLM_ERR_SHAPE;
 {
-    const int rc_ = launch_pdl(  embed_rows_kernel, dim3(rows_cap), dim3(128), 0, st, E, tokens, row_map, count_dev, rows_cap, d, h);
+    const int rc_ = launch_pdl(  embed_rows_kernel, dim3(rows_cap), dim3(128), 0, st, E, tokens, row_map, count_dev, rows_cap, d, V, h);
     if (rc_) return rc_;
   }
   return DLLM_OK;

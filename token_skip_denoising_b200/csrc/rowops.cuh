@@ -29,7 +29,7 @@ struct SelectParams {
 };
 
 int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st);
-int embed_rows_launch(const __nv_bfloat16* E, const int* tokens, const int* row_map, const int* count_dev,
+int embed_rows_launch(const __nv_bfloat16* E, int V, const int* tokens, const int* row_map, const int* count_dev,
                       int rows_cap, int d, float* h, cudaStream_t st);
 int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
                         float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st);
@@ -110,10 +110,11 @@ struct FusedLayerArgs {
   size_t attn_floats;
   int* attn_ctr;           // fused_attn_counters(...) ints, zero before the launch; left zero
   int n_attn_ctr;
-  float* scratch;          // fused_scratch_floats(rows_cap, qkvd, F): fp32 QKV and gate/up sums
+  float* scratch;          // fused_scratch_floats(qkvd, F): fp32 QKV (2 buffers) and gate/up sums;
+                           // zero before the first launch, the kernel leaves it zero
   int* sync;               // kFusedSyncInts counters, zero before the launch; the kernel leaves them zero
 };
-size_t fused_scratch_floats(int rows_cap, int qkvd, int F);
+size_t fused_scratch_floats(int qkvd, int F);
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap);
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st);
 

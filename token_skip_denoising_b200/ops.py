@@ -31,8 +31,8 @@ def rope_table(N: int, head_dim: int, theta: float):
 
 
 def embed_rows(embed, tokens, rows, count, rows_cap, h):
-    check(_L().dllm_op_embed_rows(ptr(embed), ptr(tokens), ptr(rows), ptr(count), rows_cap, embed.shape[1], ptr(h),
-                                  stream_ptr()), "embed_rows")
+    check(_L().dllm_op_embed_rows(ptr(embed), embed.shape[0], ptr(tokens), ptr(rows), ptr(count), rows_cap,
+                                  embed.shape[1], ptr(h), stream_ptr()), "embed_rows")
 
 
 def rmsnorm_rows(h, g, eps, rows=None, count=None, rows_cap=None, z=None):
