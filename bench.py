@@ -32,7 +32,6 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-PROF_EVERY = 7          # every 7th GEMM / attention launch is bracketed by CUDA events
 METRIC = "generated tokens/s, LLaDA-8B shape, 1×B200; step latency & roofline % vs active ratio"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -152,14 +151,12 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    # ---- device-timed region: K generations, profiling of the GEMMs / attention on
+    # ---- device-timed region: K generations, nothing else on the stream
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         uuid = None
-    eng.profile(PROF_EVERY, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"])
-    eng.profile_read()
     barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(uuid)
@@ -175,8 +172,6 @@ def run_ours(args, rank, world, local_rank):
     launches = kernel_launches() - launches0
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
-    prof = eng.profile_read()
-    eng.profile(0)
     ms_max = reduce_over_ranks([ms], world, dev)[0]
     value = whole_job_tokens_per_s(cfg.batch, cfg.gen_len, args.steps, world, ms_max / 1e3)
     assert not bool((tok == cfg.model.mask_id).any()), "generation left mask ids"
@@ -195,21 +190,38 @@ def run_ours(args, rank, world, local_rank):
     e2e_s = reduce_over_ranks([time.perf_counter() - w0], world, dev)[0]
     e2e_value = whole_job_tokens_per_s(cfg.batch, cfg.gen_len, args.steps, world, e2e_s)
 
-    # ---- roofline of the dominant kernel (the fused tcgen05 GEMM)
-    gemm_gbs = prof["gemm_bytes"] / (prof["gemm_ms"] / 1e3) / 1e9 if prof["gemm_ms"] > 0 else 0.0
-    roof = {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
-            "kernel": "gemm_tc_kernel (all QKV/O/gate-up/down/LM-head launches of the timed region)",
+    # ---- per-kernel figures: one more generation with every launch bracketed by CUDA events
+    # (on the engine's stream); the dominant kernel is the fused run of layers of the skip steps
+    eng.profile(1, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"])
+    eng.profile_read()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    one_generation()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prof = eng.profile_read()
+    eng.profile(0)
+    prof_ms = p0.elapsed_time(p1)
+    fused_gbs = prof["fused_bytes"] / (prof["fused_ms"] / 1e3) / 1e9 if prof["fused_ms"] > 0 else 0.0
+    roof = {"bound": "hbm", "achieved": round(fused_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(fused_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+            "kernel": "fused_layer_kernel (one persistent launch per run of layers with <= 32 rows)",
             "peak_source": peaks["source"],
-            "timed_launches": prof["gemm_launches"],
-            "sampling": f"every {PROF_EVERY}th launch of the timed region bracketed by CUDA events",
-            "avg_launch_us": round(1e3 * prof["gemm_ms"] / max(1, prof["gemm_launches"]), 3),
-            "time_share": round(PROF_EVERY * prof["gemm_ms"] / ms, 4),
-            "roofline_time_frac": round(prof["gemm_roofline_ms"] / prof["gemm_ms"], 4) if prof["gemm_ms"] else None,
-            "attention": {"timed_launches": prof["attn_launches"],
-                          "time_share": round(PROF_EVERY * prof["attn_ms"] / ms, 4),
-                          "achieved_gbs": round(prof["attn_bytes"] / (prof["attn_ms"] / 1e3) / 1e9, 1)
-                          if prof["attn_ms"] else None}}
+            "launches": prof["fused_launches"], "layers_per_launch": round(prof["fused_layers"] / max(1, prof[
+                "fused_launches"]), 2),
+            "avg_launch_us": round(1e3 * prof["fused_ms"] / max(1, prof["fused_launches"]), 2),
+            "bytes_per_launch": round(prof["fused_bytes"] / max(1, prof["fused_launches"])),
+            "time_share": round(prof["fused_ms"] / prof_ms, 4) if prof_ms else None,
+            "timing": "every launch of one extra generation bracketed by CUDA events on the engine stream",
+            "split_path": {"kernel": "gemm_tc_kernel + attn_kernel (rows > 32: refresh steps)",
+                           "gemm_launches": prof["gemm_launches"],
+                           "gemm_time_share": round(prof["gemm_ms"] / prof_ms, 4) if prof_ms else None,
+                           "gemm_achieved_tflops": round(prof["gemm_flops"] / (prof["gemm_ms"] / 1e3) / 1e12, 1)
+                           if prof["gemm_ms"] else None,
+                           "gemm_roofline_time_frac": round(prof["gemm_roofline_ms"] / prof["gemm_ms"], 4)
+                           if prof["gemm_ms"] else None,
+                           "attn_time_share": round(prof["attn_ms"] / prof_ms, 4) if prof_ms else None}}
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,

@@ -203,10 +203,13 @@ int dllm_reset(dllm_handle* h, void* stream);
  * dllm_profile_read synchronises, sums the records since the last read and
  * clears them. */
 typedef struct dllm_profile {
-  int64_t gemm_launches;
+  int64_t gemm_launches;   /* kernel-per-step path: each GEMM launch */
   double gemm_ms, gemm_bytes, gemm_flops, gemm_roofline_ms;
-  int64_t attn_launches;
+  int64_t attn_launches;   /* kernel-per-step path: each attention launch (with its merge) */
   double attn_ms, attn_bytes, attn_flops;
+  int64_t fused_launches;  /* fused runs of layers (one persistent kernel each) */
+  int64_t fused_layers;    /* layers those launches ran */
+  double fused_ms, fused_bytes, fused_flops;   /* bytes: weights + K/V read + row traffic */
 } dllm_profile;
 int dllm_profile_enable(dllm_handle* h, int32_t enable, double hbm_gbs, double tensor_tflops);
 int dllm_profile_read(dllm_handle* h, dllm_profile* out);

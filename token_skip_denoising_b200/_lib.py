@@ -60,7 +60,8 @@ class DllmStepInfo(ctypes.Structure):
 class DllmProfile(ctypes.Structure):
     _fields_ = [("gemm_launches", ctypes.c_int64), ("gemm_ms", c_f64), ("gemm_bytes", c_f64), ("gemm_flops", c_f64),
                 ("gemm_roofline_ms", c_f64), ("attn_launches", ctypes.c_int64), ("attn_ms", c_f64),
-                ("attn_bytes", c_f64), ("attn_flops", c_f64)]
+                ("attn_bytes", c_f64), ("attn_flops", c_f64), ("fused_launches", ctypes.c_int64),
+                ("fused_layers", ctypes.c_int64), ("fused_ms", c_f64), ("fused_bytes", c_f64), ("fused_flops", c_f64)]
 
 
 _SIGS = {

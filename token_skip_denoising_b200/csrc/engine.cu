@@ -135,12 +135,13 @@ std::atomic<int64_t> dllm::g_kernel_launches{0};
 struct Prof {
   struct Rec {
     cudaEvent_t a, b;
-    int cls;            // 0 GEMM, 1 attention
+    int cls;            // 0 GEMM, 1 attention, 2 fused run of layers
     double bytes, flops;
+    int layers;
   };
   bool on = false;
   int every = 1;                // bracket every n-th launch of each class
-  int64_t seen[2] = {0, 0};
+  int64_t seen[3] = {0, 0, 0};
   double hbm_gbs = 0, tflops = 0;
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -156,11 +157,11 @@ struct Prof {
     *a = get();
     cudaEventRecord(*a, st);
   }
-  void end(cudaStream_t st, cudaEvent_t a, int cls, double bytes, double flops) {
+  void end(cudaStream_t st, cudaEvent_t a, int cls, double bytes, double flops, int layers = 0) {
     if (!on || !a) return;
     cudaEvent_t b = get();
     cudaEventRecord(b, st);
-    recs.push_back({a, b, cls, bytes, flops});
+    recs.push_back({a, b, cls, bytes, flops, layers});
   }
   ~Prof() {
     for (auto& r : recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
@@ -402,9 +403,7 @@ int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_
 }
 
 // The fused persistent kernel serves row sets of at most 32 rows (not while GEMMs are timed).
-bool fused_applies(const LayerCtx& x, int rows_cap) {
-  return x.fused && x.fused_sync && rows_cap <= 32 && !(x.prof && x.prof->on);
-}
+bool fused_applies(const LayerCtx& x, int rows_cap) { return x.fused && x.fused_sync && rows_cap <= 32; }
 
 // Layers x.layer .. x.layer + n_layers - 1 as one fused persistent kernel (DLLM_ERR_UNSUPPORTED
 // when the shapes do not allow it).
@@ -422,7 +421,19 @@ int run_fused_layers(const LayerCtx& x, int n_layers, float* hbuf, const int* ro
   a.attn_ctr = x.fused_attn_ctr; a.n_attn_ctr = x.n_fused_attn_ctr;
   a.scratch = x.fused_scratch;
   a.sync = x.fused_sync;
-  return fused_layer_launch(a, st);
+  cudaEvent_t ev = nullptr;
+  if (x.prof) x.prof->begin(st, &ev, 2);
+  const int rc = fused_layer_launch(a, st);
+  if (x.prof && ev) {
+    // algorithmic traffic per layer: the four weight matrices, this layer's K and V cache (read by
+    // attention), and the rows' hidden state, operands and sums (bound: rows_cap rows)
+    const double P = static_cast<double>(x.qkvd) * x.d + static_cast<double>(x.d) * x.qd + 3.0 * x.d * x.F;
+    const double kv = 2.0 * x.B * x.Hkv * static_cast<double>(x.N) * x.hd * 2.0;
+    const double rowb = static_cast<double>(rows_cap) * (8.0 * x.d + 4.0 * (x.qkvd + 2.0 * x.F) + 2.0 * x.F);
+    const double fl = 2.0 * rows_cap * P + 4.0 * rows_cap * static_cast<double>(x.N) * x.Hq * x.hd;
+    x.prof->end(st, ev, 2, n_layers * (2.0 * P + kv + rowb), n_layers * fl, n_layers);
+  }
+  return rc;
 }
 
 // One transformer layer on rows[j] (j < *n) of the position-indexed hidden buffer hbuf:
@@ -883,11 +894,17 @@ int dllm_profile_read(dllm_handle* x, dllm_profile* out) {
       out->gemm_flops += r.flops;
       if (x->prof.hbm_gbs > 0 && x->prof.tflops > 0)
         out->gemm_roofline_ms += std::max(r.bytes / (x->prof.hbm_gbs * 1e6), r.flops / (x->prof.tflops * 1e9));
-    } else {
+    } else if (r.cls == 1) {
       out->attn_launches += 1;
       out->attn_ms += ms;
       out->attn_bytes += r.bytes;
       out->attn_flops += r.flops;
+    } else {
+      out->fused_launches += 1;
+      out->fused_layers += r.layers;
+      out->fused_ms += ms;
+      out->fused_bytes += r.bytes;
+      out->fused_flops += r.flops;
     }
     x->prof.pool.push_back(r.a);
     x->prof.pool.push_back(r.b);
