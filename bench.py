@@ -32,6 +32,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# DRAM bytes (read + write) per layer of fused_layer_kernel, from one ncu capture of the kernel on three
+# LLaDA-8B-shaped layers (kernel_bench case fused_m7_l3); roofline.traffic scales it by the layers a launch runs
+FUSED_DRAM_BYTES_PER_LAYER = 450.89e6
 METRIC = "generated tokens/s, LLaDA-8B shape, 1×B200; step latency & roofline % vs active ratio"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -204,12 +207,14 @@ def run_ours(args, rank, world, local_rank):
     eng.profile(0)
     prof_ms = p0.elapsed_time(p1)
     fused_gbs = prof["fused_bytes"] / (prof["fused_ms"] / 1e3) / 1e9 if prof["fused_ms"] > 0 else 0.0
+    layers_per_launch = prof["fused_layers"] / max(1, prof["fused_launches"])
     roof = {"bound": "hbm", "achieved": round(fused_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(fused_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+            "frac": round(fused_gbs / peaks["hbm_gbs"], 4),
+            "traffic": round(FUSED_DRAM_BYTES_PER_LAYER * layers_per_launch),
+            "traffic_source": "ncu dram read+write of one 3-layer launch (7 rows), per layer, x layers per launch",
             "kernel": "fused_layer_kernel (one persistent launch per run of layers with <= 32 rows)",
             "peak_source": peaks["source"],
-            "launches": prof["fused_launches"], "layers_per_launch": round(prof["fused_layers"] / max(1, prof[
-                "fused_launches"]), 2),
+            "launches": prof["fused_launches"], "layers_per_launch": round(layers_per_launch, 2),
             "avg_launch_us": round(1e3 * prof["fused_ms"] / max(1, prof["fused_launches"]), 2),
             "bytes_per_launch": round(prof["fused_bytes"] / max(1, prof["fused_launches"])),
             "time_share": round(prof["fused_ms"] / prof_ms, 4) if prof_ms else None,

@@ -4,8 +4,9 @@
 
 Cases time one kernel family at the LLaDA-8B shape on seeded inputs: the fused
 GEMM of each projection at the active-row counts of a skip step (7, 32) and of a
-refresh (768), the attention of the active rows over N = 768 cached keys, and
-the LM head.  Each weight matrix is replicated enough times that the working
+refresh (768), the attention of the active rows over N = 768 cached keys, the
+LM head, and the persistent run of layers of a skip step (7 or 32 rows over a
+few LLaDA-8B-shaped layers, through the engine).  Each weight matrix is replicated enough times that the working
 set exceeds L2 (126 MB) and the copies are used round-robin, so the timings
 are HBM timings.  Durations are CUDA-event medians; bytes and flops are the
 algorithmic ones (weights + activation rows + outputs).
@@ -102,6 +103,40 @@ def attn_case(rows, reps, N=768, H=32, hd=128, splits=0):
             "bytes": byts, "flops": flops}
 
 
+def fused_case(rows, reps, layers=3):
+    """A skip step's run of `layers` layers as one persistent kernel (7 kept or 32 candidate rows)."""
+    from synth import get_config, make_tokens, make_weights
+    from synth.configs import scaled
+    from .engine import Engine
+    base = scaled(get_config("llada_es"), n_layers=layers + 1, vocab=2048, mask_id=2047)
+    cfg = base.replace(skip_layer=1) if rows < base.block_len else base.replace(skip_layer=layers + 1)
+    m = cfg.model
+    w = make_weights(m, device="cuda")
+    eng = Engine(cfg, w, make_tokens(cfg).cuda(), layer_kernel="fused")
+    eng.step()                                   # refresh: fills every layer's K/V cache
+    eng.begin_step()
+    if rows < cfg.block_len:
+        eng.layers_forward(0, 1)
+        eng.select_active()
+        l0 = 1
+    else:
+        l0 = 0
+    n = int(eng.buffer("nrows")[0])
+    assert n == rows, (n, rows)
+
+    def fn(i):
+        eng.stream = torch.cuda.current_stream()
+        eng.layers_forward(l0, l0 + layers)
+
+    t = _time(fn, reps)
+    P = m.params_per_layer
+    kv = 2 * m.n_kv_heads * cfg.seq_len * m.head_dim * 2
+    byts = layers * (2 * P + kv)
+    flops = layers * (2.0 * rows * P + 4.0 * rows * cfg.seq_len * m.n_heads * m.head_dim)
+    return {"case": f"fused_m{rows}_l{layers}", "ms": t, "gbs": byts / t / 1e6, "tflops": flops / t / 1e9,
+            "bytes": byts, "flops": flops}
+
+
 CASES = {
     **{f"gemm_{k}_m{m}": (lambda k=k, m=m, **kw: gemm_case(k, m, **kw))
        for k in ("qkv", "o", "gu", "down") for m in (7, 32, 768)},
@@ -110,6 +145,8 @@ CASES = {
     "attn_m7": lambda **kw: attn_case(7, **kw),
     "attn_m32": lambda **kw: attn_case(32, **kw),
     "attn_m768": lambda **kw: attn_case(768, **kw),
+    "fused_m7_l3": lambda **kw: fused_case(7, **kw),
+    "fused_m32_l3": lambda **kw: fused_case(32, **kw),
 }
 
 
