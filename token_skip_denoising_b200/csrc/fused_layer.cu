@@ -514,8 +514,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           rem /= p.attn_qtiles;
           const int kvh = rem % ap.Hkv;
           const int b = rem / ap.Hkv;
-          if (p.hd == 128) attn::attn_item<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
-          else attn::attn_item<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          if (p.hd == 128) attn::attn_item_kp<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          else attn::attn_item_kp<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
           if (ap.splits > 1) {
             __threadfence();
             epi_bar();
