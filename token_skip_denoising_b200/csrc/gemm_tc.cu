@@ -172,8 +172,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
           for (int sub = 0; sub < KSUB; ++sub) {
             const int x = (kb * KSUB + sub) * kBK;
-            tma_load_2d(a + sub * kABytes, &tmW, &full_bar[s], x, row0, pol_w);
-            tma_load_2d(a + sub * kABytes + kABytes / 2, &tmW, &full_bar[s], x, row1, pol_w);
+            if (p.swiglu) {   // 64 gate rows and the matching 64 up rows: two boxes
+              tma_load_2d(a + sub * kABytes, &tmW, &full_bar[s], x, row0, pol_w);
+              tma_load_2d(a + sub * kABytes + kABytes / 2, &tmW, &full_bar[s], x, row1, pol_w);
+            } else {          // one 128-row box (fewer, larger TMA requests stream faster)
+              tma_load_2d(a + sub * kABytes, &tmW, &full_bar[s], x, row0, pol_w);
+            }
           }
           if (waited) {
 #pragma unroll
@@ -555,7 +559,7 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
     while (grid > 1 && tiles % grid != 0) --grid;
   }
   CUtensorMap tmW, tmX;
-  int rc = make_tmap(&tmW, a.W, a.w_rows_total, a.K, 64);
+  int rc = make_tmap(&tmW, a.W, a.w_rows_total, a.K, a.swiglu ? 64 : 128);
   if (rc) return rc;
   rc = make_tmap(&tmX, a.X, a.rows_cap, a.K, bn);
   if (rc) return rc;
