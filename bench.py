@@ -415,6 +415,30 @@ def variant_steps(peaks, steps=3, warm=2):
                      "tokens_per_s": round(B * cfg.gen_len / gen_s, 2)})
         del eng
         torch.cuda.empty_cache()
+    # ---- ES-dLLM with parallel decoding (several top-confidence tokens per step), same weights
+    es = get_config("llada_es")
+    rows = []
+    for n in (2, 4):
+        ecfg = es.replace(tokens_per_step=n)
+        etok = make_tokens(ecfg).cuda()
+        eng = Engine(ecfg, w, etok.clone(), stream=stream)
+        eng.generate()                                          # warm-up generation
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eng.reset(etok)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        eng.generate()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        gen_ms = e0.elapsed_time(e1)
+        steps = ecfg.n_blocks * math.ceil(ecfg.block_len / n)
+        rows.append({"tokens_per_step": n, "steps": steps, "generation_ms": round(gen_ms, 2),
+                     "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)})
+        del eng
+        torch.cuda.empty_cache()
+    res["es_parallel_decoding_llada8b"] = {
+        "workload": "llada_es with n top-confidence tokens committed per step (one generation, device-timed)",
+        "cases": rows}
     res["dllm_cache_dus_llada8b_b4"] = {
         "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "
                     f"{cfg.block_len}, DUS {R} rounds/block; prompt refresh every {cfg.prompt_interval} steps; "

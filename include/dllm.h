@@ -55,7 +55,13 @@ enum {
 };
 
 enum { DLLM_POLICY_VANILLA = 0, DLLM_POLICY_ES = 1, DLLM_POLICY_SURELOCK = 2, DLLM_POLICY_DLLM_CACHE = 3 };
-enum { DLLM_UNMASK_TOPCONF = 0, DLLM_UNMASK_DUS = 1 };
+/* TOPCONF: the tokens_per_step masked positions of the block with the highest confidence.
+   DUS: the dilated round of the step (Plan for Speed summary sec. 2).
+   CB_DUS: confidence-bounded with the dilation rule as a post-filter (the same summary, sec. 3):
+   positions with confidence >= cb_tau in confidence order (the first one always), none next to
+   another taken in the step, at most tokens_per_step; a block ends when nothing in it is masked
+   (the step count is data-dependent: the host reads B counts after each step). */
+enum { DLLM_UNMASK_TOPCONF = 0, DLLM_UNMASK_DUS = 1, DLLM_UNMASK_CB_DUS = 2 };
 enum { DLLM_SCOPE_BLOCK = 0, DLLM_SCOPE_ALL = 1 };
 /* How a layer over a small row set runs: AUTO lets the library choose, SPLIT launches one
    kernel per step of the layer, FUSED runs the whole layer as one persistent kernel whenever
@@ -88,6 +94,11 @@ typedef struct dllm_config {
   int32_t unmask;          /* DLLM_UNMASK_* */
   int32_t tokens_per_step; /* TOPCONF: n committed per step and sequence */
   int32_t layer_kernel;    /* DLLM_LAYER_* */
+  /* SureLock lock scope: 0 = unmasked positions only (prompt and decoded tokens); 1 = every
+     position, masked ones included (a locked masked position is still unmasked later from the
+     confidence and argmax stored when it locked) */
+  int32_t lock_masked;
+  float cb_tau;            /* CB_DUS confidence bound */
 } dllm_config;
 
 /* Device pointers to the weights (bf16 unless noted), all row-major [out, in]. */
@@ -344,12 +355,16 @@ int dllm_op_select(const float* scores, int32_t B, int32_t n, int32_t mode, int3
                    int32_t N, const uint8_t* lock, int32_t* act_pos, int32_t k_max, int32_t* count, int32_t* rows,
                    int32_t* seq_off, void* stream);
 
-/* Unmask within [blk_s, blk_s + blk_len) of each sequence: with round_mask (uint8 [blk_len])
- * null, the n_commit masked positions with the highest conf; else every masked position of
- * the round.  tokens[b, pos] = argmax[b*N + pos]. */
+/* Unmask within [blk_s, blk_s + blk_len) of each sequence.  mode DLLM_UNMASK_TOPCONF: the
+ * n_commit masked positions with the highest conf (round_mask null), or every masked position
+ * of the round (round_mask uint8 [blk_len], DUS); mode DLLM_UNMASK_CB_DUS: at most n_commit
+ * positions with conf >= cb_tau (the best one always), none adjacent to another taken, in
+ * confidence order (ties to the lower position).  tokens[b, pos] = argmax[b*N + pos].
+ * remain (nullable): masked positions left in the block of each sequence afterwards. */
 int dllm_op_unmask(int32_t* tokens, const float* conf, const int32_t* argmax, int32_t B, int32_t N, int32_t blk_s,
-                   int32_t blk_len, int32_t mask_id, int32_t n_commit, const uint8_t* round_mask, int32_t* pos_out,
-                   int32_t* tok_out, int32_t* n_out, int32_t max_out, void* stream);
+                   int32_t blk_len, int32_t mask_id, int32_t mode, int32_t n_commit, float cb_tau,
+                   const uint8_t* round_mask, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, int32_t max_out,
+                   int32_t* remain, void* stream);
 
 /* One transformer layer for the rows rows[j] (j < *count) of the hidden buffer h fp32 [B*N, d],
  * in place, with the layer's weights (pointers to layer l of w_qkv, w_o, w_gu, w_down, g_attn,

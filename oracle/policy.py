@@ -110,6 +110,30 @@ def unmask_topconf(conf: np.ndarray, masked: np.ndarray, n: int) -> np.ndarray:
     return np.array(sorted(cand[:n]), dtype=np.int64)
 
 
+def unmask_cb_dus(conf: np.ndarray, masked: np.ndarray, tau: float, cap: int) -> np.ndarray:
+    """Confidence-bounded unmasking with the dilation principle of DUS as a post-filter
+    (Plan for Speed summary, sec. 3 'complementary hybrid extension': spacing applied to an
+    adaptive, confidence-bounded sampler keeps it from picking densely clustered tokens).
+    Masked positions are taken in order of confidence (descending, ties to the lower
+    position) while their confidence is at least tau -- the first one always, so every step
+    unmasks something -- skipping any position next to one already taken in this step, at
+    most `cap` in all.  Confidences and tau compare as float32.  Ascending positions."""
+    tau32 = float(np.float32(tau))
+    order = sorted((i for i in range(len(conf)) if masked[i]), key=lambda i: _key_desc(conf[i], i))
+    taken, blocked = [], set()
+    for i in order:
+        if len(taken) >= cap:
+            break
+        v, nan = canonical_score(conf[i])
+        if taken and (nan or not v >= tau32):
+            break                      # confidences only fall from here on
+        if i in blocked:
+            continue
+        taken.append(i)
+        blocked.update((i - 1, i + 1))
+    return np.array(sorted(taken), dtype=np.int64)
+
+
 # ---------------------------------------------------------------- DUS
 
 def dus_rounds(length: int, n_rounds: int, base: int = 2):

@@ -19,8 +19,10 @@ denoising iteration of the configured policy:
   rows whose value vectors moved away from the cached ones (cosine < tau),
   at most ceil(rho * n_resp) of them.
 
-Unmasking is either top-n confidence within the current block or the DUS
-dilated rounds (Plan for Speed summary sec. 2).
+Unmasking is top-n confidence within the current block, the DUS dilated rounds
+(Plan for Speed summary sec. 2), or a confidence-bounded choice filtered by the
+dilation rule (the same summary, sec. 3); a block ends when it has no masked
+position left.
 """
 from __future__ import annotations
 
@@ -30,7 +32,7 @@ import numpy as np
 
 from .model import OracleModel, lm_confidence
 from .policy import (cosine_rows, dus_schedule, es_importance, kl_from_logits,
-                     threshold_cap_select, topk_select, unmask_topconf)
+                     threshold_cap_select, topk_select, unmask_cb_dus, unmask_topconf)
 
 
 class OracleRun:
@@ -105,6 +107,8 @@ class OracleRun:
                 r = self.step_in_block
                 local = [p for p in self.rounds[r] if masked[p]] if r < len(self.rounds) else \
                     [p for p in range(e - s) if masked[p]]
+            elif cfg.unmask == "cb_dus":
+                local = list(unmask_cb_dus(self.conf[b, s:e], masked, cfg.cb_tau, cfg.tokens_per_step))
             else:
                 local = list(unmask_topconf(self.conf[b, s:e], masked, cfg.tokens_per_step))
             for p in local:
@@ -225,7 +229,8 @@ class OracleRun:
         h = self.model.embed(self.tokens[b_idx, pos])
         h = self._layers(h, b_idx, pos, 0, m.n_layers)
         s, e = self.block_range()
-        eligible = ~masked0[b_idx, pos]
+        # lock-eligible rows: the unmasked ones, or every row in the all-positions mode
+        eligible = np.ones(len(pos), bool) if cfg.lock_masked else ~masked0[b_idx, pos]
         lm = eligible | (masked0[b_idx, pos] & (pos >= s) & (pos < e))
         r = np.nonzero(lm)[0]
         z = self.model.logits(h[r]) if len(r) else np.zeros((0, m.vocab))

@@ -18,6 +18,7 @@ POLICY_DLLM_CACHE = "dllm_cache"
 
 UNMASK_TOPCONF = "topconf"
 UNMASK_DUS = "dus"
+UNMASK_CB_DUS = "cb_dus"   # confidence-bounded, filtered by the dilation (non-adjacency) rule
 
 SCOPE_BLOCK = "block"   # candidates = rows of the current block
 SCOPE_ALL = "all"       # candidates = every row of the sequence
@@ -74,12 +75,16 @@ class RunConfig:
     # SureLock
     kl_eps: float = 1e-3
     conf_tau: float = 0.9
+    lock_masked: bool = False        # SureLock: masked positions may lock too
     # dLLM-Cache
     sim_tau: float = 0.95
     rho_cap: float = 0.25
     prompt_interval: int = 50
     # DUS
     dus_base: int = 2
+    # confidence-bounded unmasking (unmask = cb_dus): take tokens with confidence >= cb_tau,
+    # at most tokens_per_step, none next to another taken in the same step
+    cb_tau: float = 0.9
 
     @property
     def seq_len(self) -> int:

@@ -397,6 +397,37 @@ def test_unmask_topconf_bit_exact(n_commit):
         assert sorted(pos[b, :len(ref)].tolist()) == ref.tolist()
 
 
+@pytest.mark.parametrize("blk,tau,cap", [(32, 0.5, 4), (32, 2.0, 4), (200, 0.0, 64), (1000, 0.3, 7), (64, -1.0, 64)])
+def test_unmask_cb_dus_bit_exact(blk, tau, cap):
+    """Confidence-bounded, dilation-filtered unmasking against the oracle's rule, with ties
+    (confidences on a coarse grid), already-unmasked positions, ragged block lengths; and the
+    count of masked positions left in the block."""
+    B, P = 3, 8
+    N = P + blk + 5
+    rng = np.random.default_rng(blk + cap)
+    mask = 999
+    tok = np.full((B, N), mask, dtype=np.int32)
+    tok[:, :P] = rng.integers(0, 900, (B, P))
+    tok[:, P:P + blk][rng.random((B, blk)) < 0.3] = 7                  # some already unmasked
+    conf = (rng.integers(0, 16, (B, N)) / 16).astype(np.float32)
+    conf[0, P + 1] = np.nan                                             # NaN ranks last
+    amax = rng.integers(0, 900, (B, N)).astype(np.int32)
+    t = torch.tensor(tok, device=DEV)
+    remain = torch.full((B,), -1, dtype=torch.int32, device=DEV)
+    pos, tk, cnt = ops.unmask(t, torch.tensor(conf.reshape(-1), device=DEV), torch.tensor(amax.reshape(-1), device=DEV),
+                              P, blk, mask, cap, max_out=cap, mode=ops.UNMASK_CB_DUS, cb_tau=tau, remain=remain)
+    got = t.cpu().numpy()
+    for b in range(B):
+        masked = tok[b, P:P + blk] == mask
+        ref = op.unmask_cb_dus(conf[b, P:P + blk], masked, tau, cap) + P
+        exp = tok[b].copy()
+        exp[ref] = amax[b, ref]
+        np.testing.assert_array_equal(got[b], exp)
+        assert int(cnt[b]) == len(ref)
+        assert sorted(pos[b, :len(ref)].tolist()) == ref.tolist()
+        assert int(remain[b]) == int(masked.sum()) - len(ref)
+
+
 def test_unmask_dus_round():
     B, P, blk = 2, 8, 64
     N = P + blk

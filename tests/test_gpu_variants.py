@@ -49,8 +49,9 @@ def _force(eng, orc):
 
 # ------------------------------------------------------------------ SureLock
 
-def test_surelock_steps_match_oracle_with_lock_pattern(tiny_w):
-    cfg = TINY.replace(policy="surelock", tokens_per_step=2, batch=2)
+@pytest.mark.parametrize("lock_masked", [False, True])
+def test_surelock_steps_match_oracle_with_lock_pattern(tiny_w, lock_masked):
+    cfg = TINY.replace(policy="surelock", tokens_per_step=2, batch=2, lock_masked=lock_masked)
     N = cfg.seq_len
     tok0 = make_tokens(cfg)
     pattern = np.zeros((cfg.batch, N), bool)
@@ -168,3 +169,49 @@ def test_dllm_cache_forced_ratio_selects_exactly_the_cap(tiny_w):
         eng.layer_forward(l)
         assert int(eng.buffer("nsel")[0]) == math.ceil(0.25 * cfg.gen_len)
     eng.unmask()
+
+
+# ------------------------------------------------------------------ confidence-bounded DUS
+
+def test_cb_dus_generation(tiny_w):
+    """The engine with confidence-bounded, dilation-filtered unmasking: every masked position is
+    unmasked once, no two in one step are adjacent, at most tokens_per_step per step, and the
+    data-dependent block ends are followed (the run takes fewer steps than one token per step)."""
+    cfg = TINY.replace(policy="vanilla", unmask="cb_dus", cb_tau=0.0, tokens_per_step=4)
+    eng = Engine(cfg, _dev(tiny_w), make_tokens(cfg).to(DEV).contiguous())
+    pos = torch.full((1, 4), -1, dtype=torch.int32, device=DEV)
+    tk = torch.full_like(pos, -1)
+    cnt = torch.zeros(1, dtype=torch.int32, device=DEV)
+    seen = np.zeros(cfg.seq_len, int)
+    steps = 0
+    while not eng.done:
+        eng.begin_step()
+        for l in range(cfg.model.n_layers):
+            eng.layer_forward(l)
+        eng.unmask(pos, tk, cnt)
+        ps = sorted(pos[0, :int(cnt[0])].tolist())
+        assert 1 <= len(ps) <= 4 and all(q - p >= 2 for p, q in zip(ps, ps[1:]))
+        for p in ps:
+            seen[p] += 1
+        steps += 1
+    assert np.all(seen[cfg.prompt_len:] == 1) and np.all(seen[:cfg.prompt_len] == 0)
+    assert steps < cfg.gen_len
+    assert not bool((eng.tokens == cfg.model.mask_id).any())
+
+
+def test_cb_dus_unreachable_bound_is_top1(tiny_w):
+    """A bound no confidence reaches leaves the forced best token only: the same tokens as
+    top-1 decoding (vanilla steps: the kernel-per-step path, deterministic)."""
+    w = _dev(tiny_w)
+    tok0 = make_tokens(TINY).to(DEV).contiguous()
+    a = Engine(TINY.replace(policy="vanilla", unmask="cb_dus", cb_tau=2.0, tokens_per_step=4), w, tok0.clone())
+    b = Engine(TINY.replace(policy="vanilla", unmask="topconf", tokens_per_step=1), w, tok0.clone())
+    na = nb = 0
+    while not a.done:
+        a.step()
+        na += 1
+    while not b.done:
+        b.step()
+        nb += 1
+    assert na == nb == TINY.gen_len
+    assert torch.equal(a.tokens, b.tokens)

@@ -10,7 +10,7 @@ import scipy.stats
 
 from oracle.policy import (cosine_rows, dus_num_rounds, dus_rounds, dus_schedule,
                            es_importance, kl_from_logits, threshold_cap_select, topk_select,
-                           unmask_topconf)
+                           unmask_cb_dus, unmask_topconf)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 RNG = np.random.default_rng(99)
@@ -150,6 +150,47 @@ def test_unmask_topconf_properties():
     assert list(unmask_topconf(conf, masked, 2)) == [1, 2]     # 0.95 is not masked; tie -> lower pos
     assert list(unmask_topconf(conf, masked, 1)) == [1]
     assert list(unmask_topconf(conf, masked, 10)) == [0, 1, 2, 3, 5]
+
+
+def test_unmask_cb_dus_hand_example():
+    # confidences by position:       0     1     2     3     4     5
+    conf = np.array([0.90, 0.95, 0.20, 0.85, 0.99, 0.50])
+    masked = np.ones(6, bool)
+    # 4 (0.99) taken, 3 and 5 blocked; 1 (0.95) taken, 0 and 2 blocked; 0 and 3 skipped; 5 < tau: stop
+    assert list(unmask_cb_dus(conf, masked, 0.8, 4)) == [1, 4]
+    assert list(unmask_cb_dus(conf, masked, 0.8, 1)) == [4]                   # cap
+    assert list(unmask_cb_dus(conf, masked, 0.999, 4)) == [4]                 # the first is always taken
+    assert list(unmask_cb_dus(conf, masked, -1.0, 6)) == [1, 4]               # 0, 2, 3, 5 all blocked
+    m2 = masked.copy()
+    m2[4] = False                                                              # 4 already unmasked
+    assert list(unmask_cb_dus(conf, m2, 0.8, 4)) == [1, 3]                    # 1; 0 blocked; 3
+    assert list(unmask_cb_dus(np.array([0.5, 0.5, 0.5]), np.ones(3, bool), 0.0, 3)) == [0, 2]   # ties: lower first
+
+
+def test_unmask_cb_dus_properties():
+    rng = np.random.default_rng(7)
+    for trial in range(300):
+        n = int(rng.integers(1, 40))
+        conf = rng.random(n).astype(np.float32)
+        conf[rng.random(n) < 0.1] = rng.choice(conf)                           # ties
+        masked = rng.random(n) < 0.7
+        if not masked.any():
+            masked[int(rng.integers(n))] = True
+        tau = float(rng.choice([0.0, 0.3, 0.7, 0.95, 2.0]))
+        cap = int(rng.integers(1, 8))
+        got = list(unmask_cb_dus(conf, masked, tau, cap))
+        assert 1 <= len(got) <= cap and all(masked[i] for i in got)
+        assert all(b - a >= 2 for a, b in zip(got, got[1:]))                   # mutually non-adjacent
+        order = sorted(np.nonzero(masked)[0], key=lambda i: (-conf[i], i))
+        assert got[0] == order[0] or order[0] in got                           # the best is always taken
+        assert sum(conf[i] < np.float32(tau) for i in got) <= 1                # only the forced first may be below
+        if len(got) < cap:
+            # maximal: a qualifying position left out is next to a taken one of higher priority
+            rank = {i: r for r, i in enumerate(order)}
+            for i in order:
+                if i in got or conf[i] < np.float32(tau):
+                    continue
+                assert any(abs(i - j) == 1 and rank[j] < rank[i] for j in got), (conf, masked, tau, cap, got)
 
 
 # ---------------------------------------------------------------- DUS

@@ -111,6 +111,63 @@ def test_locked_rows_never_change(tiny_w, tiny_tok):
     assert len(run.last["rows"][1]) == cfg.seq_len - int(run.lock.sum()) or run.done
 
 
+def test_surelock_all_positions_lock_scope(tiny_w, tiny_tok):
+    """Lock scope 'all positions' (the SureLock summary's "each token position i", kept as a flag):
+    masked positions lock too.  A locked masked position is never recomputed, its K/V and stored
+    distribution never change, and it is still unmasked, exactly once, with the argmax stored when
+    it locked; with eps = 0 nothing locks (KL >= 0 and the rule is strict)."""
+    cfg = TINY.replace(policy="surelock", tokens_per_step=2, lock_masked=True)
+    pattern = np.zeros((1, cfg.seq_len), bool)
+    pattern[0, 1::3] = True
+    run = OracleRun(cfg, tiny_w, tiny_tok, lock_pattern=pattern)
+    snap, locked_masked = {}, {}
+    while not run.done:
+        masked_before = run.tokens == cfg.model.mask_id
+        run.step()
+        for b, p in zip(*np.nonzero(run.lock)):
+            key = (int(b), int(p))
+            if key not in snap:
+                snap[key] = (run.K[:, b, :, p].copy(), run.V[:, b, :, p].copy(), run.prev_logits[key][0].copy())
+                if masked_before[b, p]:
+                    locked_masked[key] = int(run.amax[b, p])
+            K, V, z = snap[key]
+            np.testing.assert_array_equal(run.K[:, b, :, p], K)
+            np.testing.assert_array_equal(run.V[:, b, :, p], V)
+            np.testing.assert_array_equal(run.prev_logits[key][0], z)
+    assert len(locked_masked) > 3
+    assert not (run.tokens == cfg.model.mask_id).any()
+    positions = [p for _, _, p, _ in run.unmask_events]
+    assert sorted(positions) == list(range(cfg.prompt_len, cfg.seq_len))     # each masked position once
+    for (b, p), tok in locked_masked.items():
+        assert run.tokens[b, p] == tok                                       # the argmax stored at lock time
+    none = generate(cfg.replace(kl_eps=0.0, conf_tau=-1.0), tiny_w, tiny_tok)
+    assert not none.lock.any()
+
+
+def test_cb_dus_with_unreachable_bound_is_top1_decoding(tiny_w, tiny_tok):
+    """A confidence bound no token reaches leaves only the forced best token per step: the
+    generation is exactly top-1-confidence decoding."""
+    a = generate(TINY.replace(unmask="cb_dus", cb_tau=2.0, tokens_per_step=4), tiny_w, tiny_tok)
+    b = generate(TINY.replace(unmask="topconf", tokens_per_step=1), tiny_w, tiny_tok)
+    np.testing.assert_array_equal(a.tokens, b.tokens)
+    assert a.n_steps == b.n_steps == TINY.gen_len
+
+
+def test_cb_dus_generation_unmasks_each_position_once(tiny_w, tiny_tok):
+    cfg = TINY.replace(unmask="cb_dus", cb_tau=0.0, tokens_per_step=4)
+    run = generate(cfg, tiny_w, tiny_tok)
+    assert not (run.tokens == cfg.model.mask_id).any()
+    positions = [p for _, _, p, _ in run.unmask_events]
+    assert sorted(positions) == list(range(cfg.prompt_len, cfg.seq_len))
+    by_step = {}
+    for step, b, p, _ in run.unmask_events:
+        by_step.setdefault(step, []).append(p)
+    for ps in by_step.values():                                 # each step: non-adjacent, at most 4
+        ps.sort()
+        assert len(ps) <= 4 and all(q - p >= 2 for p, q in zip(ps, ps[1:]))
+    assert run.n_steps < cfg.gen_len                            # several tokens per step on average
+
+
 def test_es_skip_step_rewrites_only_recomputed_rows(tiny_w, tiny_tok):
     cfg = TINY
     run = OracleRun(cfg, tiny_w, tiny_tok)

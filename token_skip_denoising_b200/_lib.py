@@ -25,7 +25,7 @@ DLLM_OK = 0
 STATUS_NAMES = {0: "DLLM_OK", 1: "DLLM_ERR_INVALID_ARG", 2: "DLLM_ERR_SHAPE", 3: "DLLM_ERR_UNSUPPORTED",
                 4: "DLLM_ERR_CUDA", 5: "DLLM_ERR_TIMEOUT", 6: "DLLM_ERR_DEVICE", 7: "DLLM_ERR_STATE"}
 POLICY = {"vanilla": 0, "es": 1, "surelock": 2, "dllm_cache": 3}
-UNMASK = {"topconf": 0, "dus": 1}
+UNMASK = {"topconf": 0, "dus": 1, "cb_dus": 2}
 SCOPE = {"block": 0, "all": 1}
 STEP_KIND = {0: "full", 1: "skip", 2: "locked", 3: "partial"}
 BUF = {"kcache": 0, "vcache": 1, "hidden": 2, "hprev": 3, "conf": 4, "argmax": 5, "rows": 6, "nrows": 7,
@@ -43,7 +43,8 @@ class DllmConfig(ctypes.Structure):
                 ("skip_layer", c_i32), ("keep_ratio", c_f32), ("alpha", c_f32), ("refresh_period", c_i32),
                 ("kl_eps", c_f32), ("conf_tau", c_f32),
                 ("sim_tau", c_f32), ("rho_cap", c_f32), ("prompt_interval", c_i32), ("forced_rho", c_i32),
-                ("unmask", c_i32), ("tokens_per_step", c_i32), ("layer_kernel", c_i32)]
+                ("unmask", c_i32), ("tokens_per_step", c_i32), ("layer_kernel", c_i32), ("lock_masked", c_i32),
+                ("cb_tau", c_f32)]
 
 
 class DllmWeights(ctypes.Structure):
@@ -104,8 +105,8 @@ _SIGS = {
                                        c_vp, c_vp, c_vp]),
     "dllm_op_select": (ctypes.c_int, [c_vp, c_i32, c_i32, c_i32, c_i32, c_f32, c_i32, c_i32, c_vp, c_vp, c_i32,
                                       c_vp, c_vp, c_vp, c_vp]),
-    "dllm_op_unmask": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp,
-                                      c_vp, c_vp, c_i32, c_vp]),
+    "dllm_op_unmask": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_f32,
+                                      c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp]),
     "dllm_op_layer": (ctypes.c_int, [P(DllmConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_sz, c_vp]),
     "dllm_op_layer_workspace": (ctypes.c_int, [P(DllmConfig), c_i32, c_i32, P(c_sz)]),
@@ -178,6 +179,8 @@ def make_config(run, **over) -> DllmConfig:
     c.unmask = UNMASK[run.unmask]
     c.tokens_per_step = run.tokens_per_step
     c.layer_kernel = 0
+    c.lock_masked = 1 if run.lock_masked else 0
+    c.cb_tau = run.cb_tau
     for k, v in over.items():
         if k == "layer_kernel" and isinstance(v, str):
             v = LAYER_KERNEL[v]

@@ -102,16 +102,18 @@ int validate(const dllm_config* c) {
   if (c->vocab % 128) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "vocab must be a multiple of 128");
   if (c->policy < DLLM_POLICY_VANILLA || c->policy > DLLM_POLICY_DLLM_CACHE)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown policy");
-  if (c->unmask != DLLM_UNMASK_TOPCONF && c->unmask != DLLM_UNMASK_DUS) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown unmask");
+  if (c->unmask != DLLM_UNMASK_TOPCONF && c->unmask != DLLM_UNMASK_DUS && c->unmask != DLLM_UNMASK_CB_DUS)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown unmask");
   if (c->cand_scope != DLLM_SCOPE_BLOCK && c->cand_scope != DLLM_SCOPE_ALL)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown candidate scope");
-  if (c->unmask == DLLM_UNMASK_TOPCONF && c->tokens_per_step <= 0)
+  if ((c->unmask == DLLM_UNMASK_TOPCONF || c->unmask == DLLM_UNMASK_CB_DUS) && c->tokens_per_step <= 0)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "tokens_per_step must be positive");
   if (c->unmask == DLLM_UNMASK_DUS && c->block_len == 2)
     DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "DUS: a block of 2 has no single-round non-adjacent schedule");
   if (c->block_len > 8192) DLLM_FAIL(DLLM_ERR_UNSUPPORTED, "block_len above 8192");
   if (c->layer_kernel < DLLM_LAYER_AUTO || c->layer_kernel > DLLM_LAYER_FUSED)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown layer_kernel");
+  if (c->lock_masked != 0 && c->lock_masked != 1) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "lock_masked must be 0 or 1");
   if (c->policy == DLLM_POLICY_ES && (c->skip_layer < 0 || c->skip_layer > c->n_layers))
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "skip_layer outside [0, n_layers]");
   if (c->policy == DLLM_POLICY_ES && !(c->keep_ratio > 0.f && c->keep_ratio <= 1.f))
@@ -217,6 +219,7 @@ struct dllm_handle {
   int* cur_seq_off = nullptr;
   int rows_first = 0;
   bool began = false;
+  int* blk_remain = nullptr;   // workspace: masked positions left in the block per sequence (CB_DUS)
   std::vector<uint8_t> round_host;
 };
 
@@ -274,6 +277,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->n_lm = w.take<int>(1);
   x->act_idx = w.take<int>(BN);
   x->act_count = w.take<int>(x->B);
+  x->blk_remain = w.take<int>(x->B);
   x->scores = w.take<float>(BN);
   x->kl = w.take<float>(BN);
   const int64_t R = BN;   // row bound of any step
@@ -343,7 +347,9 @@ void fill_dims(dllm_handle* x, const dllm_config* c) {
   x->n_cand = c->cand_scope == DLLM_SCOPE_ALL ? x->N : c->block_len;
   x->k_keep = c->policy == DLLM_POLICY_ES ? keep_count(c->keep_ratio, x->n_cand) : x->n_cand;
   x->n_rounds = dus_rounds_for(c->block_len);
-  x->steps_per_block = c->unmask == DLLM_UNMASK_DUS ? x->n_rounds : ceil_div(c->block_len, c->tokens_per_step);
+  x->steps_per_block = c->unmask == DLLM_UNMASK_DUS      ? x->n_rounds
+                       : c->unmask == DLLM_UNMASK_CB_DUS ? c->block_len   // an upper bound: the block ends when done
+                                                         : ceil_div(c->block_len, c->tokens_per_step);
   x->resp_start = c->cand_scope == DLLM_SCOPE_ALL ? 0 : c->prompt_len;
   x->n_resp = x->N - x->resp_start;
   x->resp_cap = rho_cap_count(c->rho_cap, x->n_resp);
@@ -742,8 +748,11 @@ int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_o
                                                           : x->h;
   const int lm_cap = std::min(lm_cap_of(x), x->cur_rows_cap);
   const bool surelock = c.policy == DLLM_POLICY_SURELOCK;
-  DLLM_TRY(lm_rows_launch(x->cur_rows, x->cur_n, x->cur_rows_cap, x->tokens, c.mask_id, x->N, bs, bs + c.block_len,
-                          rmask, surelock ? 1 : 0, x->lm_rows, x->n_lm, st));
+  // SureLock needs the distribution of every lock-eligible row (with lock_masked: every row)
+  const bool all_rows = surelock && c.lock_masked;
+  DLLM_TRY(lm_rows_launch(x->cur_rows, x->cur_n, x->cur_rows_cap, x->tokens, c.mask_id, x->N, all_rows ? 0 : bs,
+                          all_rows ? x->N : bs + c.block_len, all_rows ? nullptr : rmask, surelock ? 1 : 0,
+                          x->lm_rows, x->n_lm, st));
   DLLM_TRY(rmsnorm_rows_launch(hsrc, x->lm_rows, x->n_lm, lm_cap, x->d, x->w.g_final, c.rms_eps, x->z, x->d, st));
   GemmArgs g;
   g.W = x->w.lm_head; g.w_rows_total = x->V; g.X = x->z; g.rows_cap = lm_cap; g.rows_dev = x->n_lm; g.K = x->d;
@@ -762,6 +771,7 @@ int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_o
     k.z_cur = zcur; k.z_prev = zprev; k.lse_prev = lprev; k.lse_cur = lcur; k.stamp = x->has_prev;
     k.step = x->n_steps; k.rows = x->lm_rows; k.count = x->n_lm; k.rows_cap = lm_cap; k.V = x->V;
     k.mask_id = c.mask_id; k.tokens = x->tokens; k.lock = x->lock; k.pattern = x->lock_pattern;
+    k.lock_masked = c.lock_masked;
     k.kl_eps = c.kl_eps; k.conf_tau = c.conf_tau; k.conf = x->conf; k.amax = x->amax; k.kl_out = x->kl;
     DLLM_TRY(kl_step_launch(k, st));
   } else {
@@ -770,12 +780,22 @@ int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_o
     DLLM_TRY(lmhead_combine_launch(x->lm_part, x->V / 128, lm_cap, x->n_lm, x->lm_rows, x->conf, x->amax, x->lse, st));
   }
   const int max_out = c.unmask == DLLM_UNMASK_DUS ? c.block_len : c.tokens_per_step;
+  const bool cb = c.unmask == DLLM_UNMASK_CB_DUS;
   DLLM_TRY(unmask_launch(x->tokens, x->conf, x->amax, x->B, x->N, bs, c.block_len, c.mask_id, c.tokens_per_step, rmask,
-                         pos_out, tok_out, n_out, max_out, st));
-  // schedule
+                         cb ? 1 : 0, c.cb_tau, pos_out, tok_out, n_out, max_out, cb ? x->blk_remain : nullptr, st));
+  // schedule: a confidence-bounded step unmasks a data-dependent number of positions, so the host
+  // reads how many are left in the block (B ints, the one synchronisation of such a step)
+  bool block_done = false;
+  if (cb) {
+    std::vector<int> left(x->B);
+    DLLM_CUDA_TRY(cudaMemcpyAsync(left.data(), x->blk_remain, x->B * sizeof(int), cudaMemcpyDeviceToHost, st));
+    DLLM_CUDA_TRY(cudaStreamSynchronize(st));
+    block_done = true;
+    for (int v : left) block_done = block_done && v == 0;
+  }
   x->n_steps += 1;
   x->step_in_block += 1;
-  if (x->step_in_block >= x->steps_per_block) {
+  if (block_done || x->step_in_block >= x->steps_per_block) {
     x->block += 1;
     x->step_in_block = 0;
   }

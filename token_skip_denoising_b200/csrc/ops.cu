@@ -227,13 +227,18 @@ int dllm_op_select(const float* scores, int32_t B, int32_t n, int32_t mode, int3
 }
 
 int dllm_op_unmask(int32_t* tokens, const float* conf, const int32_t* argmax, int32_t B, int32_t N, int32_t blk_s,
-                   int32_t blk_len, int32_t mask_id, int32_t n_commit, const uint8_t* round_mask, int32_t* pos_out,
-                   int32_t* tok_out, int32_t* n_out, int32_t max_out, void* stream) {
+                   int32_t blk_len, int32_t mask_id, int32_t mode, int32_t n_commit, float cb_tau,
+                   const uint8_t* round_mask, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, int32_t max_out,
+                   int32_t* remain, void* stream) {
   if (!tokens || !conf || !argmax || B <= 0 || blk_s < 0 || blk_s + blk_len > N)
     OP_FAIL(DLLM_ERR_INVALID_ARG, "bad unmask args");
+  if (mode != DLLM_UNMASK_TOPCONF && mode != DLLM_UNMASK_CB_DUS) OP_FAIL(DLLM_ERR_INVALID_ARG, "unknown unmask mode");
+  if (mode == DLLM_UNMASK_CB_DUS && (round_mask || n_commit <= 0))
+    OP_FAIL(DLLM_ERR_INVALID_ARG, "the confidence-bounded mode takes no round mask and n_commit >= 1");
   if (pos_out && (!tok_out || max_out <= 0)) OP_FAIL(DLLM_ERR_INVALID_ARG, "pos_out needs tok_out and max_out");
-  return unmask_launch(tokens, conf, argmax, B, N, blk_s, blk_len, mask_id, n_commit, round_mask, pos_out, tok_out,
-                       n_out, max_out, static_cast<cudaStream_t>(stream));
+  return unmask_launch(tokens, conf, argmax, B, N, blk_s, blk_len, mask_id, n_commit, round_mask,
+                       mode == DLLM_UNMASK_CB_DUS ? 1 : 0, cb_tau, pos_out, tok_out, n_out, max_out, remain,
+                       static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -476,8 +476,9 @@ __global__ void snapshot_rows_kernel(const float* __restrict__ h, float* __restr
 // round_mask (DUS): commit every masked position of this round.
 __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict__ conf, const int* __restrict__ amax,
                               int N, int blk_s, int blk_len, int mask_id, int n_commit,
-                              const uint8_t* __restrict__ round_mask, int* __restrict__ pos_out,
-                              int* __restrict__ tok_out, int* __restrict__ n_out, int max_out) {
+                              const uint8_t* __restrict__ round_mask, int cb_mode, float cb_tau,
+                              int* __restrict__ pos_out, int* __restrict__ tok_out, int* __restrict__ n_out,
+                              int max_out, int* __restrict__ remain) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ float s_conf[];
@@ -493,9 +494,45 @@ __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict_
     s_conf[i] = c;
   }
   __syncthreads();
+  if (cb_mode) {
+    // confidence-bounded, dilation-filtered: take the best eligible position (confidence
+    // descending, ties to the lower position) while it reaches cb_tau (the first always),
+    // making its neighbours ineligible, at most n_commit times.  s_masked: 1 eligible,
+    // 2 taken, 3 masked but next to a taken position.
+    __shared__ float s_bv[32];
+    __shared__ int s_bi[32];
+    __shared__ int s_stop;
+    for (int k = 0; k < n_commit; ++k) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int i = threadIdx.x; i < blk_len; i += blockDim.x)
+        if (s_masked[i] == 1 && (s_conf[i] > bv || (s_conf[i] == bv && i < bi))) { bv = s_conf[i]; bi = i; }
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((threadIdx.x & 31) == 0) { s_bv[threadIdx.x >> 5] = bv; s_bi[threadIdx.x >> 5] = bi; }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w)
+          if (s_bv[w] > bv || (s_bv[w] == bv && s_bi[w] < bi)) { bv = s_bv[w]; bi = s_bi[w]; }
+        s_stop = (bi == 0x7fffffff || (k > 0 && !(bv >= cb_tau))) ? 1 : 0;
+        if (!s_stop) {
+          s_masked[bi] = 2;
+          if (bi > 0 && s_masked[bi - 1] == 1) s_masked[bi - 1] = 3;
+          if (bi + 1 < blk_len && s_masked[bi + 1] == 1) s_masked[bi + 1] = 3;
+        }
+      }
+      __syncthreads();
+      if (s_stop) break;
+    }
+  }
   for (int i = threadIdx.x; i < blk_len; i += blockDim.x) {
     bool commit = false;
-    if (s_masked[i]) {
+    if (cb_mode) {
+      commit = s_masked[i] == 2;
+    } else if (s_masked[i]) {
       if (round_mask) {
         commit = round_mask[i] != 0;
       } else {
@@ -520,6 +557,16 @@ __global__ void unmask_kernel(int* __restrict__ tokens, const float* __restrict_
   }
   __syncthreads();
   if (threadIdx.x == 0 && n_out) n_out[b] = min(s_cnt, max_out);
+  if (remain) {   // masked positions of the block left after this step
+    __shared__ int s_left;
+    if (threadIdx.x == 0) s_left = 0;
+    __syncthreads();
+    int left = 0;
+    for (int i = threadIdx.x; i < blk_len; i += blockDim.x) left += tokens[base + i] == mask_id;
+    atomicAdd(&s_left, left);
+    __syncthreads();
+    if (threadIdx.x == 0) remain[b] = s_left;
+  }
 }
 
 // SureLock per LM row (one CTA): lse, argmax (mask id excluded), conf = p(argmax) of this
@@ -622,7 +669,7 @@ __global__ void kl_step_kernel(KlStep k) {
     k.amax[flat] = BI;
     k.lse_cur[flat] = L;
     if (k.kl_out) k.kl_out[j] = kl;
-    const bool eligible = k.tokens[flat] != k.mask_id;
+    const bool eligible = k.lock_masked || k.tokens[flat] != k.mask_id;
     if (k.lock && eligible && has_prev) {
       const bool lock_now = k.pattern ? (k.pattern[flat] != 0) : (kl < k.kl_eps && conf > k.conf_tau);
       if (lock_now) k.lock[flat] = 1;
@@ -757,14 +804,14 @@ int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8
 }
 
 int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N, int blk_s, int blk_len, int mask_id,
-                  int n_commit, const uint8_t* round_mask, int* pos_out, int* tok_out, int* n_out, int max_out,
-                  cudaStream_t st) {
+                  int n_commit, const uint8_t* round_mask, int cb_mode, float cb_tau, int* pos_out, int* tok_out,
+                  int* n_out, int max_out, int* remain, cudaStream_t st) {
   if (blk_len <= 0 || blk_len > 8192) return DLLM_ERR_UNSUPPORTED;
   const int threads = std::min(1024, ((blk_len + 31) / 32) * 32);
   const size_t smem = blk_len * sizeof(float) + blk_len;
 {
-    const int rc_ = launch_pdl(  unmask_kernel, dim3(B), dim3(threads), smem, st, tokens, conf, amax, N, blk_s, blk_len, mask_id, n_commit, round_mask, pos_out,
-                                          tok_out, n_out, max_out);
+    const int rc_ = launch_pdl(  unmask_kernel, dim3(B), dim3(threads), smem, st, tokens, conf, amax, N, blk_s, blk_len, mask_id, n_commit, round_mask,
+                                          cb_mode, cb_tau, pos_out, tok_out, n_out, max_out, remain);
     if (rc_) return rc_;
   }
   return DLLM_OK;

@@ -54,6 +54,7 @@ struct KlStep {
   const int* tokens = nullptr;            // eligibility: token != mask at the start of the step
   uint8_t* lock = nullptr;
   const uint8_t* pattern = nullptr;       // forced locks (measurement mode) instead of the KL rule
+  int lock_masked = 0;                    // masked positions are lock-eligible too
   float kl_eps = 0.f, conf_tau = 0.f;
   float* conf = nullptr;
   int* amax = nullptr;
@@ -75,9 +76,11 @@ int lm_rows_launch(const int* rows, const int* count_dev, int rows_cap, const in
                    cudaStream_t st);
 int snapshot_rows_launch(const float* h, float* h_prev, const int* tokens, uint8_t* masked_prev, int mask_id,
                          const int* rows, int n_rows, int d, cudaStream_t st);
+// cb_mode: confidence-bounded, dilation-filtered choice (at most n_commit, conf >= cb_tau after the
+// first, none adjacent); remain (nullable): masked positions left in the block per sequence.
 int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N, int blk_s, int blk_len, int mask_id,
-                  int n_commit, const uint8_t* round_mask, int* pos_out, int* tok_out, int* n_out, int max_out,
-                  cudaStream_t st);
+                  int n_commit, const uint8_t* round_mask, int cb_mode, float cb_tau, int* pos_out, int* tok_out,
+                  int* n_out, int max_out, int* remain, cudaStream_t st);
 
 size_t attn_partial_floats(int rows_cap, int Hq, int hd, int splits);
 int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N);

@@ -10,6 +10,7 @@ from ._lib import check, ptr, stream_ptr
 
 EPI_STORE_F32, EPI_STORE_BF16, EPI_RESID_ADD = 0, 1, 3
 SEL_TOPK_DESC, SEL_BELOW_CAP_ASC, SEL_FORCED_ASC, SEL_ALL_ELIGIBLE = 0, 1, 2, 3
+UNMASK_TOPCONF, UNMASK_CB_DUS = 0, 2
 
 _DEFAULT_WS = 256 << 20
 
@@ -140,13 +141,15 @@ def select(scores, B, n, mode, k, tau=0.0, cand_start=0, N=None, lock=None, k_ma
     return act, cnt, rows, off
 
 
-def unmask(tokens, conf, amax, blk_s, blk_len, mask_id, n_commit, round_mask=None, max_out=64):
+def unmask(tokens, conf, amax, blk_s, blk_len, mask_id, n_commit, round_mask=None, max_out=64,
+           mode=UNMASK_TOPCONF, cb_tau=0.0, remain=None):
     B, N = tokens.shape
     pos = torch.full((B, max_out), -1, dtype=torch.int32, device="cuda")
     tok = torch.full((B, max_out), -1, dtype=torch.int32, device="cuda")
     cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
-    check(_L().dllm_op_unmask(ptr(tokens), ptr(conf), ptr(amax), B, N, blk_s, blk_len, mask_id, n_commit,
-                              ptr(round_mask), ptr(pos), ptr(tok), ptr(cnt), max_out, stream_ptr()), "unmask")
+    check(_L().dllm_op_unmask(ptr(tokens), ptr(conf), ptr(amax), B, N, blk_s, blk_len, mask_id, mode, n_commit,
+                              float(cb_tau), ptr(round_mask), ptr(pos), ptr(tok), ptr(cnt), max_out, ptr(remain),
+                              stream_ptr()), "unmask")
     return pos, tok, cnt
 
 
