@@ -334,7 +334,9 @@ def _step_roofline_ms(peaks, m, n_layers_rows, lm_rows, N, batch, extra_bytes=0.
 def variant_steps(peaks, steps=3, warm=2):
     """Per-step device latency of the SureLock (Dream-7B shape, batch 8) and dLLM-Cache + DUS
     (long-context LLaDA-8B shape, batch 4) generations, at the measured selection and at
-    forced lock fractions / a forced cap, with tokens/s extrapolated to a whole run."""
+    forced lock fractions / a forced cap, with tokens/s extrapolated to a whole run; and whole
+    LLaDA-8B ES-dLLM generations with several tokens per step (top-n confidence, and the
+    confidence-bounded sampler filtered by the DUS dilation rule)."""
     import numpy as np
     import torch
 
@@ -438,6 +440,34 @@ def variant_steps(peaks, steps=3, warm=2):
         torch.cuda.empty_cache()
     res["es_parallel_decoding_llada8b"] = {
         "workload": "llada_es with n top-confidence tokens committed per step (one generation, device-timed)",
+        "cases": rows}
+    # ---- ES-dLLM with confidence-bounded unmasking filtered by the DUS dilation rule; random
+    # weights give every token a confidence near 1/V, so the bound is set to 0 and the cap and the
+    # non-adjacency rule decide how many tokens a step takes
+    rows = []
+    for n in (2, 4, 8):
+        ecfg = es.replace(unmask="cb_dus", cb_tau=0.0, tokens_per_step=n)
+        etok = make_tokens(ecfg).cuda()
+        eng = Engine(ecfg, w, etok.clone(), stream=stream)
+        eng.generate()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eng.reset(etok)
+        torch.cuda.synchronize()
+        n_steps = 0
+        e0.record(stream)
+        while not eng.done:
+            eng.step()
+            n_steps += 1
+        e1.record(stream)
+        torch.cuda.synchronize()
+        gen_ms = e0.elapsed_time(e1)
+        rows.append({"cap": n, "steps": n_steps, "generation_ms": round(gen_ms, 2),
+                     "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)})
+        del eng
+        torch.cuda.empty_cache()
+    res["es_cb_dus_llada8b"] = {
+        "workload": "llada_es, unmask = confidence-bounded (tau 0) with the dilation post-filter, cap n per step; "
+                    "each step syncs the host once (data-dependent block ends)",
         "cases": rows}
     res["dllm_cache_dus_llada8b_b4"] = {
         "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "

@@ -254,228 +254,6 @@ __device__ __forceinline__ void attn_item(const AttnParams& p, int qt, int b, in
   }
 }
 
-// The same item with each key block also split across the four warps: when the item has
-// few query units (one or two 16-row MMA tiles, e.g. 7 rows of an MHA model), the warps
-// that would sit idle in attn_item take a slice of every key block instead.  The blocks are
-// loaded as in attn_item (all 128 threads, double-buffered 64-key blocks); warp w computes
-// query tile w / KP against keys [kp * 64 / KP, (kp + 1) * 64 / KP) of each block with its
-// own online softmax, and the KP states of a query tile are combined once at the end in
-// shared memory into the item's partial (or final) output.
-template <int HD, int KP, class Bar>
-__device__ __forceinline__ void attn_item_kp_impl(const AttnParams& p, int u0, int n_units, int off, int b, int kvh,
-                                                  int split, int blk0, int blk1, uint8_t* smem, int tid, Bar bar) {
-  constexpr int kChunks = HD / 8;                      // 16-byte chunks per key row
-  constexpr int kTileBytes = kKeysPerBlock * HD * 2;
-  constexpr int NT = 8 / KP;                           // 8-key n-tiles of a warp's slice
-  constexpr int kSlice = kKeysPerBlock / KP;
-  uint8_t* kbuf[2] = {smem, smem + 2 * kTileBytes};
-  uint8_t* vbuf[2] = {smem + kTileBytes, smem + 3 * kTileBytes};
-  const int G = p.Hq / p.Hkv;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int mt = warp / KP, kp = warp % KP;
-  const int mtiles = (min(kUnitsPerCta, n_units - u0) + 15) / 16;
-  const bool active = mt < mtiles;
-  const int wu0 = u0 + mt * 16;
-  const int ks0 = kp * kSlice;                         // first key of the slice inside a block
-  const __nv_bfloat16* kbase = p.kc + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N * HD;
-  const __nv_bfloat16* vbase = p.vc + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N * HD;
-
-  auto load_block = [&](int blk, int buf) {
-    const int key0 = blk * kKeysPerBlock;
-    for (int i = tid; i < kKeysPerBlock * kChunks; i += 128) {
-      const int r = i / kChunks, ch = i % kChunks;
-      const int key = key0 + r;
-      const bool ok = key < p.N;
-      const int64_t go = static_cast<int64_t>(ok ? key : 0) * HD + ch * 8;
-      const int so = r * (HD * 2) + ((ch ^ (r & 7)) * 16);
-      cp_async16(kbuf[buf] + so, kbase + go, ok);
-      cp_async16(vbuf[buf] + so, vbase + go, ok);
-    }
-    cp_async_commit();
-  };
-
-  uint32_t qa[HD / 16][4];
-  {
-    const int ua = wu0 + g, ub = wu0 + g + 8;
-    const bool va = active && ua < n_units, vb = active && ub < n_units;
-    const __nv_bfloat16* qa_row = p.q + (static_cast<int64_t>(off + (va ? ua / G : 0)) * p.Hq + kvh * G + (va ? ua % G : 0)) * HD;
-    const __nv_bfloat16* qb_row = p.q + (static_cast<int64_t>(off + (vb ? ub / G : 0)) * p.Hq + kvh * G + (vb ? ub % G : 0)) * HD;
-#pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-      const int d0 = kk * 16 + 2 * c;
-      qa[kk][0] = va ? __ldcg(reinterpret_cast<const unsigned int*>(qa_row + d0)) : 0u;
-      qa[kk][1] = vb ? __ldcg(reinterpret_cast<const unsigned int*>(qb_row + d0)) : 0u;
-      qa[kk][2] = va ? __ldcg(reinterpret_cast<const unsigned int*>(qa_row + d0 + 8)) : 0u;
-      qa[kk][3] = vb ? __ldcg(reinterpret_cast<const unsigned int*>(qb_row + d0 + 8)) : 0u;
-    }
-  }
-
-  float o[HD / 8][4];
-#pragma unroll
-  for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-
-  load_block(blk0, 0);
-  for (int blk = blk0, it = 0; blk < blk1; ++blk, ++it) {
-    const int buf = it & 1;
-    if (blk + 1 < blk1) {
-      load_block(blk + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    bar();
-    if (active) {
-      const uint32_t ks = smem_u32(kbuf[buf]);
-      const uint32_t vs = smem_u32(vbuf[buf]);
-      float s[NT][4];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-#pragma unroll
-        for (int nt = 0; nt < NT; nt += 2) {
-          const int mi = lane >> 3;
-          const int key = ks0 + (nt + (mi >> 1)) * 8 + (lane & 7);
-          const int ch = 2 * kk + (mi & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(ks + key * (HD * 2) + ((ch ^ (key & 7)) * 16), b0, b1, b2, b3);
-          mma_bf16(s[nt], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-          mma_bf16(s[nt + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
-        }
-      }
-      const int key0 = blk * kKeysPerBlock + ks0;
-      float mx_a = m_a, mx_b = m_b;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + nt * 8 + 2 * c + (e & 1);
-          s[nt][e] = key < p.N ? s[nt][e] * p.scale_log2 : -INFINITY;
-        }
-        mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
-        mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
-      }
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-      // a slice entirely past N leaves the running max at -inf: keep the state unchanged then
-      const float corr_a = mx_a == -INFINITY ? 1.f : exp2f(m_a - mx_a);
-      const float corr_b = mx_b == -INFINITY ? 1.f : exp2f(m_b - mx_b);
-      m_a = mx_a;
-      m_b = mx_b;
-      float rs_a = 0.f, rs_b = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        s[nt][0] = mx_a == -INFINITY ? 0.f : exp2f(s[nt][0] - m_a);
-        s[nt][1] = mx_a == -INFINITY ? 0.f : exp2f(s[nt][1] - m_a);
-        s[nt][2] = mx_b == -INFINITY ? 0.f : exp2f(s[nt][2] - m_b);
-        s[nt][3] = mx_b == -INFINITY ? 0.f : exp2f(s[nt][3] - m_b);
-        rs_a += s[nt][0] + s[nt][1];
-        rs_b += s[nt][2] + s[nt][3];
-      }
-      l_a = l_a * corr_a + rs_a;
-      l_b = l_b * corr_b + rs_b;
-#pragma unroll
-      for (int i = 0; i < HD / 8; ++i) {
-        o[i][0] *= corr_a;
-        o[i][1] *= corr_a;
-        o[i][2] *= corr_b;
-        o[i][3] *= corr_b;
-      }
-#pragma unroll
-      for (int t = 0; t < NT / 2; ++t) {
-        const uint32_t a0 = pack_bf16(s[2 * t][0], s[2 * t][1]);
-        const uint32_t a1 = pack_bf16(s[2 * t][2], s[2 * t][3]);
-        const uint32_t a2 = pack_bf16(s[2 * t + 1][0], s[2 * t + 1][1]);
-        const uint32_t a3 = pack_bf16(s[2 * t + 1][2], s[2 * t + 1][3]);
-#pragma unroll
-        for (int dn = 0; dn < HD / 8; dn += 2) {
-          const int mi = lane >> 3;
-          const int key = ks0 + 16 * t + (mi & 1) * 8 + (lane & 7);
-          const int ch = dn + (mi >> 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vs + key * (HD * 2) + ((ch ^ (key & 7)) * 16), b0, b1, b2, b3);
-          mma_bf16(o[dn], a0, a1, a2, a3, b0, b1);
-          mma_bf16(o[dn + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-    }
-    bar();
-  }
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-
-  // combine the KP slices of each query tile: per warp m[16], l[16], O[16][HD] in shared memory
-  float* st = reinterpret_cast<float*>(smem) + warp * (32 + 16 * HD);
-  if (active) {
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = g + half * 8;
-      if (c == 0) {
-        st[r] = half ? m_b : m_a;
-        st[16 + r] = half ? l_b : l_a;
-      }
-#pragma unroll
-      for (int dn = 0; dn < HD / 8; ++dn) {
-        const int d = dn * 8 + 2 * c;
-        *reinterpret_cast<float2*>(st + 32 + r * HD + d) = make_float2(o[dn][half * 2], o[dn][half * 2 + 1]);
-      }
-    }
-  }
-  bar();
-  for (int e = tid; e < mtiles * 16 * HD; e += 128) {
-    const int tmt = e / (16 * HD);
-    const int r = (e / HD) % 16;
-    const int d = e % HD;
-    const int u = u0 + tmt * 16 + r;
-    if (u >= n_units) continue;
-    const float* s0 = reinterpret_cast<float*>(smem) + tmt * KP * (32 + 16 * HD);
-    float M = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < KP; ++k) M = fmaxf(M, s0[k * (32 + 16 * HD) + r]);
-    float acc = 0.f, L = 0.f;
-#pragma unroll
-    for (int k = 0; k < KP; ++k) {
-      const float* sk = s0 + k * (32 + 16 * HD);
-      const float w = sk[r] == -INFINITY ? 0.f : exp2f(sk[r] - M);
-      acc += w * sk[32 + r * HD + d];
-      L += w * sk[16 + r];
-    }
-    const int row = off + u / G;
-    const int h = kvh * G + u % G;
-    if (p.splits == 1) {
-      p.out[(static_cast<int64_t>(row) * p.Hq + h) * HD + d] = __float2bfloat16(acc / L);
-    } else {
-      const int64_t base = (static_cast<int64_t>(split) * p.rows_cap + row) * p.Hq + h;
-      p.opart[base * HD + d] = acc;
-      if (d == 0) p.ml[base] = make_float2(M, L);
-    }
-  }
-}
-
-template <int HD, class Bar>
-__device__ __forceinline__ void attn_item_kp(const AttnParams& p, int qt, int b, int kvh, int split, uint8_t* smem,
-                                             int tid, Bar bar) {
-  const int G = p.Hq / p.Hkv;
-  const int off = p.seq_off[b];
-  const int n_units = (p.seq_off[b + 1] - off) * G;
-  const int u0 = qt * kUnitsPerCta;
-  if (u0 >= n_units) return;
-  const int n_blocks = (p.N + kKeysPerBlock - 1) / kKeysPerBlock;
-  const int blk0 = split * p.blocks_per_split;
-  const int blk1 = min(n_blocks, blk0 + p.blocks_per_split);
-  if (blk0 >= blk1) return;
-  const int mtiles = (min(kUnitsPerCta, n_units - u0) + 15) / 16;
-  if (mtiles == 1) attn_item_kp_impl<HD, 4>(p, u0, n_units, off, b, kvh, split, blk0, blk1, smem, tid, bar);
-  else if (mtiles == 2) attn_item_kp_impl<HD, 2>(p, u0, n_units, off, b, kvh, split, blk0, blk1, smem, tid, bar);
-  else attn_item<HD>(p, qt, b, kvh, split, smem, tid, bar);
-}
-
 // Merge of the split partials for one (row, head), one warp (lane 0..31).
 template <int HD>
 __device__ __forceinline__ void attn_merge(const AttnParams& p, int row, int h, int lane) {

@@ -286,6 +286,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
               for (int sub = 0; sub < kKsub; ++sub) {
                 const int x = (kb * kKsub + sub) * kBK;
                 tma_load_2d(a + sub * kABytes, tmW[g], &full_bar[s], x, wrow0 + tile * kTileM, pol_w);
+                tma_load_2d(a + sub * kABytes + kABytes / 2, tmW[g], &full_bar[s], x, wrow0 + tile * kTileM + 64,
+                            pol_w);
               }
               if (!ready && x_ready(g)) flush();
               if (ready) {
@@ -460,54 +462,39 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t)) {
         const int pairs = p.qkvd >> 1;
         const int64_t total = static_cast<int64_t>(m_rows) * pairs;
-        // four pairs per thread and round: every load of the round is issued before any use
-        constexpr int kB = 4;
-        for (int64_t base = gt; base < total; base += kB * gstride) {
-          float xl[kB], xh[kB], cs[kB], sn[kB];
-          int jr[kB], pi[kB], n_lo[kB];
-#pragma unroll
-          for (int e = 0; e < kB; ++e) {
-            const int64_t uu = base + e * gstride;
-            const bool ok = uu < total;
-            jr[e] = ok ? static_cast<int>(uu / pairs) : 0;
-            const int rr = ok ? static_cast<int>(uu - static_cast<int64_t>(jr[e]) * pairs) : 0;
-            pi[e] = rr % half;
-            n_lo[e] = ok ? (rr / half) * p.hd + pi[e] : -1;
-            const float* srow = p.s_qkv + static_cast<int64_t>(jr[e]) * p.qkvd;
-            const int pos = s_rows[jr[e]] % p.N;
-            const int nl = ok ? n_lo[e] : 0;
-            xl[e] = __ldcg(srow + nl);
-            xh[e] = __ldcg(srow + nl + half);
-            cs[e] = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi[e]);
-            sn[e] = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi[e]);
+        for (int64_t uu = gt; uu < total; uu += gstride) {
+          const int jr = static_cast<int>(uu / pairs);
+          const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
+          const int pi = rr % half;
+          const int n_lo = (rr / half) * p.hd + pi;
+          const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
+          const float ri = s_rinv1[jr];
+          const float xl = __ldcg(srow + n_lo) * ri, xh = __ldcg(srow + n_lo + half) * ri;
+          const int flat = s_rows[jr];
+          const int b = flat / p.N;
+          const int pos = flat - b * p.N;
+          float yl = xl, yh = xh;
+          if (n_lo < p.qd + p.kvd) {
+            const float cs = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi);
+            const float sn = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi);
+            yl = xl * cs - xh * sn;
+            yh = xh * cs + xl * sn;
           }
-#pragma unroll
-          for (int e = 0; e < kB; ++e) {
-            if (n_lo[e] < 0) continue;
-            const float ri = s_rinv1[jr[e]];
-            const float x0 = xl[e] * ri, x1 = xh[e] * ri;
-            const bool rot = n_lo[e] < p.qd + p.kvd;
-            const float yl = rot ? x0 * cs[e] - x1 * sn[e] : x0;
-            const float yh = rot ? x1 * cs[e] + x0 * sn[e] : x1;
-            const int flat = s_rows[jr[e]];
-            const int b = flat / p.N;
-            const int pos = flat - b * p.N;
-            if (n_lo[e] < p.qd) {
-              __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr[e]) * p.qd + n_lo[e];
-              dst[0] = __float2bfloat16(yl);
-              dst[half] = __float2bfloat16(yh);
-            } else {
-              int nn = n_lo[e] - p.qd;
-              __nv_bfloat16* cache = kc;
-              if (nn >= p.kvd) {
-                nn -= p.kvd;
-                cache = vc;
-              }
-              const int kvh = nn / p.hd;
-              __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi[e];
-              dst[0] = __float2bfloat16(yl);
-              dst[half] = __float2bfloat16(yh);
+          if (n_lo < p.qd) {
+            __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
+            dst[0] = __float2bfloat16(yl);
+            dst[half] = __float2bfloat16(yh);
+          } else {
+            int nn = n_lo - p.qd;
+            __nv_bfloat16* cache = kc;
+            if (nn >= p.kvd) {
+              nn -= p.kvd;
+              cache = vc;
             }
+            const int kvh = nn / p.hd;
+            __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
+            dst[0] = __float2bfloat16(yl);
+            dst[half] = __float2bfloat16(yh);
           }
         }
       }
@@ -527,8 +514,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           rem /= p.attn_qtiles;
           const int kvh = rem % ap.Hkv;
           const int b = rem / ap.Hkv;
-          if (p.hd == 128) attn::attn_item_kp<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
-          else attn::attn_item_kp<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          if (p.hd == 128) attn::attn_item<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
+          else attn::attn_item<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
           if (ap.splits > 1) {
             __threadfence();
             epi_bar();
@@ -565,36 +552,24 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       if (epi_wait_phase(p.sync + S_GU, target, s_flag, t)) {
         const int f4 = p.F >> 2;
         const int64_t total = static_cast<int64_t>(m_rows) * f4;
-        constexpr int kB = 4;   // four float4 units per thread and round, loads first
-        for (int64_t base = gt; base < total; base += kB * gstride) {
-          float4 g4[kB], u4[kB];
-          int jr[kB], f[kB];
+        for (int64_t uu = gt; uu < total; uu += gstride) {
+          const int jr = static_cast<int>(uu / f4);
+          const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * f4) * 4;
+          const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
+          const float ri = s_rinv2[jr];
+          const float4 g4 = __ldcg(reinterpret_cast<const float4*>(srow + f));
+          const float4 u4 = __ldcg(reinterpret_cast<const float4*>(srow + p.F + f));
+          const float g[4] = {g4.x * ri, g4.y * ri, g4.z * ri, g4.w * ri};
+          const float u[4] = {u4.x * ri, u4.y * ri, u4.z * ri, u4.w * ri};
+          float a[4];
 #pragma unroll
-          for (int e = 0; e < kB; ++e) {
-            const int64_t uu = base + e * gstride;
-            const bool ok = uu < total;
-            jr[e] = ok ? static_cast<int>(uu / f4) : -1;
-            f[e] = ok ? static_cast<int>(uu - static_cast<int64_t>(jr[e]) * f4) * 4 : 0;
-            const float* srow = p.s_gu + static_cast<int64_t>(ok ? jr[e] : 0) * 2 * p.F;
-            g4[e] = __ldcg(reinterpret_cast<const float4*>(srow + f[e]));
-            u4[e] = __ldcg(reinterpret_cast<const float4*>(srow + p.F + f[e]));
-          }
-#pragma unroll
-          for (int e = 0; e < kB; ++e) {
-            if (jr[e] < 0) continue;
-            const float ri = s_rinv2[jr[e]];
-            const float g[4] = {g4[e].x * ri, g4[e].y * ri, g4[e].z * ri, g4[e].w * ri};
-            const float u[4] = {u4[e].x * ri, u4[e].y * ri, u4[e].z * ri, u4[e].w * ri};
-            float a4[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) a4[q] = g[q] / (1.f + __expf(-g[q])) * u[q];
-            __nv_bfloat162 lo = __floats2bfloat162_rn(a4[0], a4[1]);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(a4[2], a4[3]);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(p.act + static_cast<int64_t>(jr[e]) * p.F + f[e]) = pk;
-          }
+          for (int e = 0; e < 4; ++e) a[e] = g[e] / (1.f + __expf(-g[e])) * u[e];
+          __nv_bfloat162 lo = __floats2bfloat162_rn(a[0], a[1]);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(a[2], a[3]);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(p.act + static_cast<int64_t>(jr) * p.F + f) = pk;
         }
       }
       signal_phase(p.sync + S_SWIGLU, t);
@@ -671,7 +646,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   const int K[4] = {a.d, a.qd, a.d, a.F};
   const void* X[4] = {a.z1, a.attn, a.z2, a.act};
   for (int q = 0; q < 4; ++q) {
-    int rc = make_tmap(&tw[q], W[q], wrows[q] * a.L, K[q], kTileM);   // one 128-row box per k-block
+    int rc = make_tmap(&tw[q], W[q], wrows[q] * a.L, K[q], 64);
     if (rc) return rc;
     rc = make_tmap(&tx[q], X[q], a.rows_cap, K[q], bn);
     if (rc) return rc;
