@@ -65,7 +65,7 @@ enum { DLLM_UNMASK_TOPCONF = 0, DLLM_UNMASK_DUS = 1, DLLM_UNMASK_CB_DUS = 2 };
 enum { DLLM_SCOPE_BLOCK = 0, DLLM_SCOPE_ALL = 1 };
 /* How a layer over a small row set runs: AUTO lets the library choose, SPLIT launches one
    kernel per step of the layer, FUSED runs the whole layer as one persistent kernel whenever
-   at most 32 rows are recomputed (larger row sets always take SPLIT). */
+   at most 64 rows are recomputed (larger row sets always take SPLIT). */
 enum { DLLM_LAYER_AUTO = 0, DLLM_LAYER_SPLIT = 1, DLLM_LAYER_FUSED = 2 };
 enum { DLLM_STEP_FULL = 0, DLLM_STEP_SKIP = 1, DLLM_STEP_LOCKED = 2, DLLM_STEP_PARTIAL = 3 };
 
@@ -165,7 +165,7 @@ int dllm_begin_step(dllm_handle* h, int32_t* kind_out, void* stream);
 int dllm_layer_forward(dllm_handle* h, int32_t layer, void* stream);
 
 /* Runs layers l0 .. l1-1 for the current row set, with the same result as
- * dllm_layer_forward on each in turn.  When at most 32 rows are recomputed (and
+ * dllm_layer_forward on each in turn.  When at most 64 rows are recomputed (and
  * layer_kernel allows it) the whole run is one persistent kernel whose weight
  * stream continues across the layer boundaries.  Same algorithm and page
  * passages as dllm_layer_forward; l0 == l1 is a no-op; DLLM_ERR_INVALID_ARG when

@@ -34,6 +34,9 @@ CASES = {
                   ffn_dim=2816, vocab=2048, mask_id=2047).replace(skip_layer=1, prompt_len=96, gen_len=64),
     # LLaDA-8B layer shape, 3 layers: every GEMM has more items than SMs
     "llada": scaled(get_config("llada_es"), n_layers=3, vocab=2048, mask_id=2047).replace(skip_layer=1),
+    # the widest row sets the fused kernel takes: 64 candidates, 48 kept (64-wide MMA tiles)
+    "rows64": scaled(get_config("llada_es"), n_layers=2, vocab=2048, mask_id=2047).replace(
+        skip_layer=1, prompt_len=64, gen_len=64, block_len=64, keep_ratio=0.75),
 }
 
 
@@ -104,7 +107,7 @@ def test_fused_layer_repeats_without_reset():
             B.buffer(buf).copy_(A.buffer(buf))
 
 
-@pytest.mark.parametrize("name", ["tiny", "gqa", "llada"])
+@pytest.mark.parametrize("name", ["tiny", "gqa", "llada", "rows64"])
 def test_layer_runs_match_single_layers(name):
     """dllm_layers_forward (one persistent kernel per run of layers) against the split path
     layer by layer: hidden rows, every layer's K/V cache and the unmasked tokens."""

@@ -23,11 +23,11 @@ def _rowrel(a, b):
     return float((np.abs(a - b).max(1) / np.maximum(np.abs(b).max(1), 1e-30)).max())
 
 
-def _run_layer_case(dims, B, N, rows_per_seq, seed, h_scale=1.0, gain_jitter=0.1):
+def _run_layer_case(dims, B, N, rows_per_seq, seed, h_scale=1.0, gain_jitter=0.1, layer_kernel="auto"):
     w = make_weights(dims, seed=seed, device=DEV, gain_jitter=gain_jitter, layers=[0])
     run = RunConfig(name="t", model=dims, batch=B, prompt_len=N - 64 if N > 64 else 0,
                     gen_len=64 if N > 64 else N, block_len=64 if N > 64 else N)
-    cfg = _lib.make_config(run)
+    cfg = _lib.make_config(run, layer_kernel=layer_kernel)
     g = torch.Generator(device=DEV).manual_seed(seed + 1)
     h0 = torch.randn((B * N, dims.d_model), generator=g, device=DEV) * h_scale
     kc0 = torch.randn((B, dims.n_kv_heads, N, dims.head_dim), generator=g, device=DEV).to(torch.bfloat16)
@@ -55,14 +55,17 @@ def _run_layer_case(dims, B, N, rows_per_seq, seed, h_scale=1.0, gain_jitter=0.1
     return h, h0, kc, vc, kc0, vc0, flat, ref, K, V
 
 
+@pytest.mark.parametrize("layer_kernel", ["auto", "split"])   # auto: the fused kernel up to 64 rows
 @pytest.mark.parametrize("dims,B,N,rows", [
     (TINY, 1, 64, [8]),
     (TINY, 2, 96, [5, 33]),
     (ModelDims(n_layers=1, d_model=512, n_heads=4, n_kv_heads=2, head_dim=128, ffn_dim=1408, vocab=1024,
+               mask_id=1023), 2, 130, [27, 37]),
+    (ModelDims(n_layers=1, d_model=512, n_heads=4, n_kv_heads=2, head_dim=128, ffn_dim=1408, vocab=1024,
                mask_id=1023), 3, 130, [1, 70, 130]),
 ])
-def test_layer_matches_oracle(dims, B, N, rows):
-    h, h0, kc, vc, kc0, vc0, flat, ref, K, V = _run_layer_case(dims, B, N, rows, seed=3)
+def test_layer_matches_oracle(dims, B, N, rows, layer_kernel):
+    h, h0, kc, vc, kc0, vc0, flat, ref, K, V = _run_layer_case(dims, B, N, rows, seed=3, layer_kernel=layer_kernel)
     got = h.cpu().double().numpy()
     assert _rowrel(got[flat], ref) < TOL_HIDDEN
     others = np.setdiff1d(np.arange(B * N), flat)

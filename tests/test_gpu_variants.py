@@ -201,11 +201,14 @@ def test_cb_dus_generation(tiny_w):
 
 def test_cb_dus_unreachable_bound_is_top1(tiny_w):
     """A bound no confidence reaches leaves the forced best token only: the same tokens as
-    top-1 decoding (vanilla steps: the kernel-per-step path, deterministic)."""
+    top-1 decoding (both on the kernel-per-step layer, whose sums are bit-reproducible; the
+    fused layer adds fp32 pieces in arbitrary order)."""
     w = _dev(tiny_w)
     tok0 = make_tokens(TINY).to(DEV).contiguous()
-    a = Engine(TINY.replace(policy="vanilla", unmask="cb_dus", cb_tau=2.0, tokens_per_step=4), w, tok0.clone())
-    b = Engine(TINY.replace(policy="vanilla", unmask="topconf", tokens_per_step=1), w, tok0.clone())
+    a = Engine(TINY.replace(policy="vanilla", unmask="cb_dus", cb_tau=2.0, tokens_per_step=4), w, tok0.clone(),
+               layer_kernel="split")
+    b = Engine(TINY.replace(policy="vanilla", unmask="topconf", tokens_per_step=1), w, tok0.clone(),
+               layer_kernel="split")
     na = nb = 0
     while not a.done:
         a.step()

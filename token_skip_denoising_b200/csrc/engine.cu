@@ -253,7 +253,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->lock = s.take<uint8_t>(BN);
   x->has_prev = s.take<int>(BN);
   x->fused_sync = s.take<int>(kFusedSyncInts);
-  x->n_fused_attn_ctr = fused_attn_counters(x->B, c.n_heads, c.n_kv_heads, 32);
+  x->n_fused_attn_ctr = fused_attn_counters(x->B, c.n_heads, c.n_kv_heads, kFusedMaxRows);
   x->fused_attn_ctr = s.take<int>(x->n_fused_attn_ctr);
   if (c.policy == DLLM_POLICY_SURELOCK) {
     x->zstore = s.take<__nv_bfloat16>(2 * BN * x->V);
@@ -318,9 +318,9 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   size_t ml = af / std::max(1, x->hd);
   x->attn_ml = w.take<float2>(ml);
   // fused small-row layer scratch
-  x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(32) * x->d);
+  x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(kFusedMaxRows) * x->d);
   x->fused_scratch = w.take<float>(fused_scratch_floats(x->qkvd, x->F));
-  x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * 32 * c.n_heads * x->hd;
+  x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * kFusedMaxRows * c.n_heads * x->hd;
   x->fused_opart = w.take<float>(x->fused_attn_floats);
   x->fused_ml = w.take<float2>(x->fused_attn_floats / x->hd);
   int actr = 0;
@@ -408,8 +408,8 @@ int timed_gemm(Prof* prof, const GemmArgs& g, const GemmScratch& gs, cudaStream_
   return rc;
 }
 
-// The fused persistent kernel serves row sets of at most 32 rows (not while GEMMs are timed).
-bool fused_applies(const LayerCtx& x, int rows_cap) { return x.fused && x.fused_sync && rows_cap <= 32; }
+// The fused persistent kernel serves row sets of at most kFusedMaxRows rows.
+bool fused_applies(const LayerCtx& x, int rows_cap) { return x.fused && x.fused_sync && rows_cap <= kFusedMaxRows; }
 
 // Layers x.layer .. x.layer + n_layers - 1 as one fused persistent kernel (DLLM_ERR_UNSUPPORTED
 // when the shapes do not allow it).
@@ -523,6 +523,38 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
+}
+
+// The single-layer op's share of the fused kernel's buffers (row sets of at most
+// kFusedMaxRows rows, unless the configuration asks for the kernel-per-step layer); with a
+// null context only sizes are taken.  Its counters rely on the op workspace being zeroed once.
+void carve_fused_op(Carver& w, const dllm_config* cfg, int rows_cap, LayerCtx* L) {
+  if (rows_cap > kFusedMaxRows || cfg->layer_kernel == DLLM_LAYER_SPLIT) return;
+  const int d = cfg->d_model, qd = cfg->n_heads * cfg->head_dim, kvd = cfg->n_kv_heads * cfg->head_dim;
+  const int N = cfg->prompt_len + cfg->gen_len;
+  int* sync = w.take<int>(kFusedSyncInts);
+  const int n_ctr = fused_attn_counters(cfg->batch, cfg->n_heads, cfg->n_kv_heads, kFusedMaxRows);
+  int* ctr = w.take<int>(n_ctr);
+  __nv_bfloat16* z2 = w.take<__nv_bfloat16>(static_cast<size_t>(kFusedMaxRows) * d);
+  float* scratch = w.take<float>(fused_scratch_floats(qd + 2 * kvd, cfg->ffn_dim));
+  const size_t af = static_cast<size_t>((N + 63) / 64) * kFusedMaxRows * cfg->n_heads * cfg->head_dim;
+  float* opart = w.take<float>(af);
+  float2* ml = w.take<float2>(af / cfg->head_dim);
+  if (!L) return;
+  L->fused = true;
+  L->layer = 0;
+  L->n_layers_total = 1;
+  L->Wqkv0 = L->Wqkv; L->Wo0 = L->Wo; L->Wgu0 = L->Wgu; L->Wdn0 = L->Wdn;
+  L->g_attn0 = L->g_attn; L->g_ffn0 = L->g_ffn;
+  L->kc0 = L->kc; L->vc0 = L->vc;
+  L->z2 = z2;
+  L->fused_scratch = scratch;
+  L->fused_sync = sync;
+  L->fused_attn_ctr = ctr;
+  L->n_fused_attn_ctr = n_ctr;
+  L->fused_opart = opart;
+  L->fused_ml = ml;
+  L->fused_attn_floats = af;
 }
 
 }  // namespace
@@ -936,6 +968,7 @@ int dllm_profile_read(dllm_handle* x, dllm_profile* out) {
 int64_t dllm_kernel_launches(void) { return dllm::g_kernel_launches.load(); }
 
 int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t rows_per_seq_cap, size_t* bytes) {
+  DLLM_TRY(validate(cfg));
   if (!cfg || !bytes || rows_cap <= 0) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "bad layer workspace args");
   const int d = cfg->d_model, qd = cfg->n_heads * cfg->head_dim, kvd = cfg->n_kv_heads * cfg->head_dim;
   const int qkvd = qd + 2 * kvd, F = cfg->ffn_dim;
@@ -958,6 +991,7 @@ int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t ro
   const size_t af = sp > 1 ? attn_partial_floats(rows_cap, cfg->n_heads, cfg->head_dim, sp) : 0;
   w.take<float>(af);
   w.take<float2>(af / cfg->head_dim);
+  carve_fused_op(w, cfg, rows_cap, nullptr);
   *bytes = (w.off + 255) & ~size_t(255);
   return DLLM_OK;
 }
@@ -1002,6 +1036,7 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
   L.attn_floats = sp > 1 ? attn_partial_floats(rows_cap, L.Hq, L.hd, sp) : 0;
   L.attn_opart = w.take<float>(L.attn_floats);
   L.attn_ml = w.take<float2>(L.attn_floats / L.hd);
+  carve_fused_op(w, cfg, rows_cap, &L);
   return run_layer(L, h, rows, count, seq_off, rows_cap, rows_per_seq_cap, st);
 }
 

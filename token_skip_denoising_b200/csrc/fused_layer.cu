@@ -1,6 +1,6 @@
 // A run of transformer layers for a few recomputed rows as a single persistent kernel.
 //
-// With at most 32 active rows (the ES-dLLM skip step: the block's rows below the
+// With at most 64 active rows (the ES-dLLM skip step: the block's rows below the
 // skip layer, the kept rows above it) a layer is four weight streams (QKV, O,
 // gate/up, down: 436 MB for the LLaDA-8B shape) separated by small dependent
 // steps (RMSNorm, RoPE, attention over the cached K/V, the split merge, SwiGLU).
@@ -43,12 +43,13 @@ using namespace gemm;
 
 constexpr int kThreads = 192;
 constexpr int kKsub = 2;                          // 64-column k-blocks per ring stage
-constexpr int kMaxRows = 32;                      // rows of the fp32 sum buffers (any launch's row count)
+constexpr int kMaxRows = kFusedMaxRows;           // rows of the fp32 sum buffers (any launch's row count)
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
 enum Phase : int { S_X1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_X2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
 static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
+static_assert(kMaxRows <= 128 && 128 % kMaxRows == 0, "rows are handled by the 128 step threads");
 
 template <int BN>
 struct FCfg {
@@ -59,7 +60,7 @@ struct FCfg {
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr size_t kAttnBytes = 4 * 64 * 128 * 2;   // K/V double buffer for hd <= 128
-  static constexpr size_t kMiscBytes = 512;                 // row map, 1/rms of the rows, operand flag
+  static constexpr size_t kMiscBytes = 4 * kMaxRows * 4;    // row map, 1/rms before attention and FFN, partial sums
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + kMiscBytes + (2 * kStages + 4) * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "fused layer does not fit shared memory");
 };
@@ -184,9 +185,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   uint8_t* stage_base = smem;
   uint8_t* attn_smem = smem + C::kStages * C::kStageBytes;
   int* s_rows = reinterpret_cast<int*>(attn_smem + C::kAttnBytes);   // [32]
-  float* s_rinv1 = reinterpret_cast<float*>(s_rows + 32);             // [32] 1/rms before attention
-  float* s_rinv2 = s_rinv1 + 32;                                      // [32] 1/rms before the FFN
-  float* s_ss = s_rinv2 + 32;                                         // [32] partial sums of squares
+  float* s_rinv1 = reinterpret_cast<float*>(s_rows + kMaxRows);       // 1/rms before attention
+  float* s_rinv2 = s_rinv1 + kMaxRows;                                // 1/rms before the FFN
+  float* s_ss = s_rinv2 + kMaxRows;                                   // partial sums of squares
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(attn_smem + C::kAttnBytes + C::kMiscBytes);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* acc_full = empty_bar + C::kStages;
@@ -353,7 +354,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     // ---------------- warps 0-3: reductions of the GEMM pieces and the steps between GEMMs
     const int t = threadIdx.x;
     const int m_rows = min(*p.n_rows, p.rows_cap);
-    if (t < 32) s_rows[t] = t < m_rows ? p.rows[t] : 0;
+    if (t < kMaxRows) s_rows[t] = t < m_rows ? p.rows[t] : 0;
     epi_bar();
     const int64_t gt = static_cast<int64_t>(c) * 128 + t;   // grid-wide epilogue thread index
     const int64_t gstride = static_cast<int64_t>(G) * 128;
@@ -405,7 +406,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       const int q0 = static_cast<int>(static_cast<int64_t>(n4) * c / G);
       const int q1 = static_cast<int>(static_cast<int64_t>(n4) * (c + 1) / G);
       const int w4 = q1 - q0;
-      if (t < 32) s_ss[t] = 0.f;
+      if (t < kMaxRows) s_ss[t] = 0.f;
       epi_bar();
       for (int u = t; u < m_rows * w4; u += 128) {
         const int jj = u / w4;
@@ -425,11 +426,11 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     };
     // 1/rms of every row from the partials of all CTAs (after the phase that wrote them)
     auto rinv_from = [&](const float* ssp, float* rinv) {
-      const int jj = t & 31;
+      const int jj = t % kMaxRows;
       float acc = 0.f;
       if (jj < m_rows)
-        for (int cc = t >> 5; cc < G; cc += 4) acc += __ldcg(ssp + cc * kMaxRows + jj);
-      if (t < 32) s_ss[t] = 0.f;
+        for (int cc = t / kMaxRows; cc < G; cc += 128 / kMaxRows) acc += __ldcg(ssp + cc * kMaxRows + jj);
+      if (t < kMaxRows) s_ss[t] = 0.f;
       epi_bar();
       if (jj < m_rows) atomicAdd(&s_ss[jj], acc);
       epi_bar();
@@ -637,7 +638,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.rows_cap <= 0 || a.rows_cap > kMaxRows) return DLLM_ERR_UNSUPPORTED;
   if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   if (a.n_layers <= 0 || a.l0 < 0 || a.l0 + a.n_layers > a.L) return DLLM_ERR_INVALID_ARG;
-  const int bn = a.rows_cap <= 16 ? 16 : 32;
+  const int bn = a.rows_cap <= 16 ? 16 : (a.rows_cap <= 32 ? 32 : 64);
   const int grid = kNumSMs;
   CUtensorMap tw[4], tx[4];
   // every layer of a weight stack in one map: layer l's tile rows start at l * rows per layer
@@ -721,7 +722,8 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.attn_ctr = a.attn_ctr;
   p.sync = a.sync;
   if (bn == 16) return launch_fused<16>(tw, tx, p, grid, st);
-  return launch_fused<32>(tw, tx, p, grid, st);
+  if (bn == 32) return launch_fused<32>(tw, tx, p, grid, st);
+  return launch_fused<64>(tw, tx, p, grid, st);
 }
 
 }  // namespace dllm

@@ -91,9 +91,9 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
                 int splits, float* opart, float2* ml, size_t partial_floats, int* counters, int n_counters,
                 cudaStream_t st);
 
-// One transformer layer for at most 32 rows as a single persistent kernel (fused_layer.cu).
-// A run of layers over at most 32 rows as one persistent kernel (fused_layer.cu).
+// A run of layers over at most kFusedMaxRows rows as one persistent kernel (fused_layer.cu).
 constexpr int kFusedSyncInts = 16;
+constexpr int kFusedMaxRows = 64;   // row sets the fused kernel serves (its sum buffers' rows)
 struct FusedLayerArgs {
   int B, N, d, qd, kvd, qkvd, F, hd, Hq, Hkv;
   int L, l0, n_layers;              // layers l0 .. l0 + n_layers - 1 of L
