@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 # DRAM bytes (read + write) per layer of fused_layer_kernel, from one ncu capture of the kernel on three
 # LLaDA-8B-shaped layers (kernel_bench case fused_m7_l3); roofline.traffic scales it by the layers a launch runs
-FUSED_DRAM_BYTES_PER_LAYER = 450.89e6
+FUSED_DRAM_BYTES_PER_LAYER = 451.75e6
 METRIC = "generated tokens/s, LLaDA-8B shape, 1×B200; step latency & roofline % vs active ratio"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -212,14 +212,14 @@ def run_ours(args, rank, world, local_rank):
             "frac": round(fused_gbs / peaks["hbm_gbs"], 4),
             "traffic": round(FUSED_DRAM_BYTES_PER_LAYER * layers_per_launch),
             "traffic_source": "ncu dram read+write of one 3-layer launch (7 rows), per layer, x layers per launch",
-            "kernel": "fused_layer_kernel (one persistent launch per run of layers with <= 32 rows)",
+            "kernel": "fused_layer_kernel (one persistent launch per run of layers with <= 64 rows)",
             "peak_source": peaks["source"],
             "launches": prof["fused_launches"], "layers_per_launch": round(layers_per_launch, 2),
             "avg_launch_us": round(1e3 * prof["fused_ms"] / max(1, prof["fused_launches"]), 2),
             "bytes_per_launch": round(prof["fused_bytes"] / max(1, prof["fused_launches"])),
             "time_share": round(prof["fused_ms"] / prof_ms, 4) if prof_ms else None,
             "timing": "every launch of one extra generation bracketed by CUDA events on the engine stream",
-            "split_path": {"kernel": "gemm_tc_kernel + attn_kernel (rows > 32: refresh steps)",
+            "split_path": {"kernel": "gemm_tc_kernel + attn_kernel (rows > 64: refresh steps)",
                            "gemm_launches": prof["gemm_launches"],
                            "gemm_time_share": round(prof["gemm_ms"] / prof_ms, 4) if prof_ms else None,
                            "gemm_achieved_tflops": round(prof["gemm_flops"] / (prof["gemm_ms"] / 1e3) / 1e12, 1)
@@ -419,7 +419,7 @@ def variant_steps(peaks, steps=3, warm=2):
         torch.cuda.empty_cache()
     # ---- ES-dLLM with parallel decoding (several top-confidence tokens per step), same weights
     es = get_config("llada_es")
-    rows = []
+    es_rows = []
     for n in (2, 4):
         ecfg = es.replace(tokens_per_step=n)
         etok = make_tokens(ecfg).cuda()
@@ -434,17 +434,17 @@ def variant_steps(peaks, steps=3, warm=2):
         torch.cuda.synchronize()
         gen_ms = e0.elapsed_time(e1)
         steps = ecfg.n_blocks * math.ceil(ecfg.block_len / n)
-        rows.append({"tokens_per_step": n, "steps": steps, "generation_ms": round(gen_ms, 2),
+        es_rows.append({"tokens_per_step": n, "steps": steps, "generation_ms": round(gen_ms, 2),
                      "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)})
         del eng
         torch.cuda.empty_cache()
     res["es_parallel_decoding_llada8b"] = {
         "workload": "llada_es with n top-confidence tokens committed per step (one generation, device-timed)",
-        "cases": rows}
+        "cases": es_rows}
     # ---- ES-dLLM with confidence-bounded unmasking filtered by the DUS dilation rule; random
     # weights give every token a confidence near 1/V, so the bound is set to 0 and the cap and the
     # non-adjacency rule decide how many tokens a step takes
-    rows = []
+    es_rows = []
     for n in (2, 4, 8):
         ecfg = es.replace(unmask="cb_dus", cb_tau=0.0, tokens_per_step=n)
         etok = make_tokens(ecfg).cuda()
@@ -453,22 +453,22 @@ def variant_steps(peaks, steps=3, warm=2):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         eng.reset(etok)
         torch.cuda.synchronize()
-        n_steps = 0
+        gen_steps = 0
         e0.record(stream)
         while not eng.done:
             eng.step()
-            n_steps += 1
+            gen_steps += 1
         e1.record(stream)
         torch.cuda.synchronize()
         gen_ms = e0.elapsed_time(e1)
-        rows.append({"cap": n, "steps": n_steps, "generation_ms": round(gen_ms, 2),
+        es_rows.append({"cap": n, "steps": gen_steps, "generation_ms": round(gen_ms, 2),
                      "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)})
         del eng
         torch.cuda.empty_cache()
     res["es_cb_dus_llada8b"] = {
         "workload": "llada_es, unmask = confidence-bounded (tau 0) with the dilation post-filter, cap n per step; "
                     "each step syncs the host once (data-dependent block ends)",
-        "cases": rows}
+        "cases": es_rows}
     res["dllm_cache_dus_llada8b_b4"] = {
         "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "
                     f"{cfg.block_len}, DUS {R} rounds/block; prompt refresh every {cfg.prompt_interval} steps; "

@@ -42,8 +42,8 @@ def _flat(b_idx, pos, N):
     return np.asarray(b_idx) * N + np.asarray(pos)
 
 
-def _engine(cfg, w, tokens):
-    return Engine(cfg, _to_dev(w), tokens.to(DEV).contiguous())
+def _engine(cfg, w, tokens, **over):
+    return Engine(cfg, _to_dev(w), tokens.to(DEV).contiguous(), **over)
 
 
 @pytest.mark.parametrize("cfg", [TINY, TINY.replace(batch=2), TINY.replace(policy="vanilla"),
@@ -129,9 +129,12 @@ def test_es_steps_match_oracle_teacher_forced(tiny_w_cpu):
 
 
 def test_keep_all_equals_vanilla_on_gpu(tiny_w_cpu):
+    """keep ratio 1 over all rows is the full recompute, bit for bit, on the kernel-per-step
+    layer (the fused layer's fp32 reductions are order-dependent, so it is held to the
+    tolerances of the oracle comparisons instead)."""
     tok0 = make_tokens(TINY)
-    a = _engine(TINY.replace(keep_ratio=1.0, cand_scope="all"), tiny_w_cpu, tok0)
-    b = _engine(TINY.replace(policy="vanilla"), tiny_w_cpu, tok0)
+    a = _engine(TINY.replace(keep_ratio=1.0, cand_scope="all"), tiny_w_cpu, tok0, layer_kernel="split")
+    b = _engine(TINY.replace(policy="vanilla"), tiny_w_cpu, tok0, layer_kernel="split")
     a.generate()
     b.generate()
     torch.cuda.synchronize()
