@@ -47,7 +47,7 @@ enum {
   DLLM_OK = 0,
   DLLM_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum value */
   DLLM_ERR_SHAPE = 2,       /* sizes that do not fit the layout */
-  DLLM_ERR_UNSUPPORTED = 3, /* a valid request this build does not implement */
+  DLLM_ERR_UNSUPPORTED = 3, /* a valid request the library does not implement */
   DLLM_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
   DLLM_ERR_TIMEOUT = 5,     /* a bounded device wait ran out */
   DLLM_ERR_DEVICE = 6,      /* the device status word was set */
