@@ -11,6 +11,11 @@ denoising iteration of the configured policy:
   `refresh_period` steps) recomputes all rows; other steps recompute the
   current block's rows up to the skip layer, score them by Eq. 1, keep the
   top k = ceil(keep * n) and run only those through the remaining layers.
+  With `es_per_layer` the choice is made again at the start of every layer
+  from the skip layer on (ES-dLLM summary sec. 2.1, item 2): Eq. 1 compares
+  each candidate's input of that layer with the one of the previous
+  iteration, and a row skipped at a layer carries its cached output of that
+  layer (from the last iteration that computed it) into the next one.
 * surelock: SureLock summary sec. 2.1.  Unlocked rows run every layer; locked
   rows are never recomputed and keep the K/V written when they locked; a row
   locks when KL(p_t || p_t-1) < eps and its confidence > tau.
@@ -56,6 +61,8 @@ class OracleRun:
         self.prev_logits = {}          # (b, pos) -> (z, lse) of the last computed distribution
         self.forced_rho = forced_rho
         self.h_cache = None            # dLLM-Cache per-layer outputs [L, B, N, d]
+        self.es_in = None              # ES per-layer: input of layer l last iteration [L, B, N, d]
+        self.es_out = None             # ES per-layer: last computed output of layer l [L, B, N, d]
         self.block = 0
         self.step_in_block = 0
         self.n_steps = 0
@@ -150,7 +157,15 @@ class OracleRun:
         if store_hprev_rows is not None:
             sel = store_hprev_rows[b_idx, pos]
             self.h_prev[b_idx[sel], pos[sel]] = h[sel]
-        h = self._layers(h, b_idx, pos, ls, m.n_layers, keep_outputs)
+        if store_hprev_rows is not None and cfg.es_per_layer:
+            self._es_layer_state()
+            sb, sp = b_idx[sel], pos[sel]
+            for l in range(ls, m.n_layers):
+                self.es_in[l][sb, sp] = h[sel]
+                h = self._layers(h, b_idx, pos, l, l + 1)
+                self.es_out[l][sb, sp] = h[sel]
+        else:
+            h = self._layers(h, b_idx, pos, ls, m.n_layers, keep_outputs)
         r = self._lm_rows_for(b_idx, pos, masked0)
         z, lse = self._lm(h[r], b_idx[r], pos[r])
         return b_idx, pos, h, r, z, lse
@@ -189,6 +204,12 @@ class OracleRun:
         rp = self.cfg.refresh_period
         return self.step_in_block == 0 or (rp > 0 and self.step_in_block % rp == 0)
 
+    def _es_layer_state(self):
+        if self.es_in is None:
+            shape = (self.dims.n_layers, self.B, self.N, self.dims.d_model)
+            self.es_in = np.zeros(shape)
+            self.es_out = np.zeros(shape)
+
     def _es_step(self, forced_scores):
         cfg, m = self.cfg, self.dims
         masked0 = self.tokens == m.mask_id
@@ -204,6 +225,8 @@ class OracleRun:
         h = self.model.embed(self.tokens[b_idx, pos])
         h = self._layers(h, b_idx, pos, 0, ls)
         c = np.where(self.masked_prev[b_idx, pos], self.conf[b_idx, pos], 0.0)
+        if cfg.es_per_layer:
+            return self._es_per_layer_skip(h, b_idx, pos, c, masked0, forced_scores)
         scores = es_importance(cfg.alpha, c, h, self.h_prev[b_idx, pos])
         self.h_prev[b_idx, pos] = h
         h_skip = h.copy()
@@ -219,6 +242,43 @@ class OracleRun:
         r = self._lm_rows_for(ab, ap, masked0)
         z, lse = self._lm(ha[r], ab[r], ap[r])
         return {"kind": "skip", "rows": (ab, ap), "cand": (b_idx, pos), "scores": scores,
+                "h_skip": h_skip, "active": act, "h_out": ha, "lm_rows": r, "k": k}
+
+    def _es_per_layer_skip(self, x, b_idx, pos, c, masked0, forced_scores):
+        """Layers skip_layer .. L-1 of a skip step, choosing the top k at each layer.
+
+        x holds every candidate's input of the current layer.  forced_scores, when
+        given, is one score vector per layer from the skip layer on (teacher forcing).
+        """
+        cfg, m = self.cfg, self.dims
+        ls = cfg.skip_layer
+        n = len(pos) // self.B
+        k = cfg.keep_count(n)
+        h_skip = x.copy()
+        layer_scores, layer_active, layer_in = [], [], []
+        for l in range(ls, m.n_layers):
+            # Eq. 1 on this layer's input: H^(t)_l against H^(t-1)_l
+            scores = es_importance(cfg.alpha, c, x, self.es_in[l][b_idx, pos])
+            self.es_in[l][b_idx, pos] = x
+            if forced_scores is not None:
+                scores = np.asarray(forced_scores[l - ls], dtype=np.float64).reshape(-1)
+            act = np.concatenate([b * n + topk_select(scores[b * n:(b + 1) * n], k)
+                                  for b in range(self.B)])
+            out = self.model.layer(l, x[act], b_idx[act], pos[act], self.K[l], self.V[l])
+            self.es_out[l][b_idx[act], pos[act]] = out
+            layer_scores.append(scores)
+            layer_active.append(act)
+            layer_in.append(x)
+            # every candidate enters the next layer with its latest output of this one:
+            # just computed for the chosen rows, cached for the skipped ones
+            x = self.es_out[l][b_idx, pos].copy()
+        self.masked_prev = masked0
+        ab, ap = b_idx[act], pos[act]
+        ha = x[act]
+        r = self._lm_rows_for(ab, ap, masked0)
+        self._lm(ha[r], ab[r], ap[r])
+        return {"kind": "skip", "rows": (ab, ap), "cand": (b_idx, pos), "scores": layer_scores[0],
+                "layer_scores": layer_scores, "layer_active": layer_active, "layer_in": layer_in,
                 "h_skip": h_skip, "active": act, "h_out": ha, "lm_rows": r, "k": k}
 
     def _surelock_step(self):

@@ -72,6 +72,7 @@ class RunConfig:
     alpha: float = 0.5
     cand_scope: str = SCOPE_BLOCK
     refresh_period: int = 0          # 0: refresh only at the first step of a block
+    es_per_layer: bool = False       # re-select the top k at every layer from skip_layer on
     # SureLock
     kl_eps: float = 1e-3
     conf_tau: float = 0.9
