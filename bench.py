@@ -441,6 +441,26 @@ def variant_steps(peaks, steps=3, warm=2):
     res["es_parallel_decoding_llada8b"] = {
         "workload": "llada_es with n top-confidence tokens committed per step (one generation, device-timed)",
         "cases": es_rows}
+    # ---- ES-dLLM with the top k chosen again at every layer from the skip layer on
+    ecfg = es.replace(es_per_layer=True)
+    etok = make_tokens(ecfg).cuda()
+    eng = Engine(ecfg, w, etok.clone(), stream=stream)
+    eng.generate()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    eng.reset(etok)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    eng.generate()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    gen_ms = e0.elapsed_time(e1)
+    res["es_per_layer_llada8b"] = {
+        "workload": "llada_es with the top k re-chosen by Eq. 1 at every layer from the skip layer on "
+                    "(one score, selection and layer launch per layer; one generation, device-timed)",
+        "generation_ms": round(gen_ms, 2), "steps": ecfg.n_blocks * ecfg.block_len,
+        "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)}
+    del eng
+    torch.cuda.empty_cache()
     # ---- ES-dLLM with confidence-bounded unmasking filtered by the DUS dilation rule; random
     # weights give every token a confidence near 1/V, so the bound is set to 0 and the cap and the
     # non-adjacency rule decide how many tokens a step takes

@@ -99,6 +99,10 @@ typedef struct dllm_config {
      confidence and argmax stored when it locked) */
   int32_t lock_masked;
   float cb_tau;            /* CB_DUS confidence bound */
+  /* ES-dLLM: 0 = one top-k choice at skip_layer for the rest of the step; 1 = the choice is
+     made again at the start of every layer from skip_layer on (ES-dLLM sec. 2.1, item 2),
+     Eq. 1 on that layer's input; needs skip_layer < n_layers */
+  int32_t es_per_layer;
 } dllm_config;
 
 /* Device pointers to the weights (bf16 unless noted), all row-major [out, in]. */
@@ -177,7 +181,17 @@ int dllm_layers_forward(dllm_handle* h, int32_t l0, int32_t l1, void* stream);
  * the top k per sequence (ties to the lower position) and makes them the row
  * set of the remaining layers.  active_idx (device int32 [B, k], ascending
  * positions) and active_count (device int32 [B]) are optional outputs.
- * On a refresh step it only snapshots the candidates' hidden states. */
+ * On a refresh step it only snapshots the candidates' hidden states.
+ *
+ * With es_per_layer the call is made before every layer from skip_layer on
+ * (the first call applies to skip_layer, each next one to the following
+ * layer) and the layer then runs alone (dllm_layer_forward, or
+ * dllm_layers_forward over that one layer).  Eq. 1 compares each candidate's
+ * input of that layer with its input of the previous iteration; a row the
+ * previous layer skipped enters with its cached output of that layer and a
+ * zero variation term, and the chosen rows become the layer's row set.
+ * Calls out of this order return DLLM_ERR_STATE, as does dllm_unmask before
+ * the last layer's call. */
 int dllm_select_active(dllm_handle* h, const float* scores_or_null, int32_t* active_idx, int32_t* active_count,
                        void* stream);
 

@@ -44,7 +44,7 @@ class DllmConfig(ctypes.Structure):
                 ("kl_eps", c_f32), ("conf_tau", c_f32),
                 ("sim_tau", c_f32), ("rho_cap", c_f32), ("prompt_interval", c_i32), ("forced_rho", c_i32),
                 ("unmask", c_i32), ("tokens_per_step", c_i32), ("layer_kernel", c_i32), ("lock_masked", c_i32),
-                ("cb_tau", c_f32)]
+                ("cb_tau", c_f32), ("es_per_layer", c_i32)]
 
 
 class DllmWeights(ctypes.Structure):
@@ -181,6 +181,7 @@ def make_config(run, **over) -> DllmConfig:
     c.layer_kernel = 0
     c.lock_masked = 1 if run.lock_masked else 0
     c.cb_tau = run.cb_tau
+    c.es_per_layer = 1 if run.es_per_layer else 0
     for k, v in over.items():
         if k == "layer_kernel" and isinstance(v, str):
             v = LAYER_KERNEL[v]

@@ -114,6 +114,9 @@ int validate(const dllm_config* c) {
   if (c->layer_kernel < DLLM_LAYER_AUTO || c->layer_kernel > DLLM_LAYER_FUSED)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown layer_kernel");
   if (c->lock_masked != 0 && c->lock_masked != 1) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "lock_masked must be 0 or 1");
+  if (c->es_per_layer != 0 && c->es_per_layer != 1) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "es_per_layer must be 0 or 1");
+  if (c->policy == DLLM_POLICY_ES && c->es_per_layer && c->skip_layer >= c->n_layers)
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "per-layer selection needs skip_layer < n_layers");
   if (c->policy == DLLM_POLICY_ES && (c->skip_layer < 0 || c->skip_layer > c->n_layers))
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "skip_layer outside [0, n_layers]");
   if (c->policy == DLLM_POLICY_ES && !(c->keep_ratio > 0.f && c->keep_ratio <= 1.f))
@@ -220,10 +223,18 @@ struct dllm_handle {
   int rows_first = 0;
   bool began = false;
   int* blk_remain = nullptr;   // workspace: masked positions left in the block per sequence (CB_DUS)
+  // ES per-layer re-selection: the input of layer l seen last iteration for l > skip_layer
+  // (layer skip_layer uses h_prev), the rows chosen at the previous layer, the next layer
+  // select_active applies to
+  float* es_in = nullptr;
+  uint8_t* act_flag = nullptr;
+  int es_layer = 0;
   std::vector<uint8_t> round_host;
 };
 
 namespace {
+
+bool es_per_layer(const dllm_handle* x) { return x->c.policy == DLLM_POLICY_ES && x->c.es_per_layer; }
 
 int lm_cap_of(const dllm_handle* hd) {
   const auto& c = hd->c;
@@ -263,6 +274,8 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
     x->lse_store = nullptr;
   }
   x->hcache = c.policy == DLLM_POLICY_DLLM_CACHE ? s.take<float>(static_cast<size_t>(x->L) * BN * x->d) : nullptr;
+  const int n_es_in = es_per_layer(x) ? x->L - c.skip_layer - 1 : 0;
+  x->es_in = n_es_in > 0 ? s.take<float>(static_cast<size_t>(n_es_in) * BN * x->d) : nullptr;
   x->state_total = (s.off + 255) & ~size_t(255);
   if (state_bytes) *state_bytes = x->state_total;
 
@@ -278,6 +291,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->act_idx = w.take<int>(BN);
   x->act_count = w.take<int>(x->B);
   x->blk_remain = w.take<int>(x->B);
+  x->act_flag = es_per_layer(x) ? w.take<uint8_t>(BN) : nullptr;
   x->scores = w.take<float>(BN);
   x->kl = w.take<float>(BN);
   const int64_t R = BN;   // row bound of any step
@@ -557,6 +571,55 @@ void carve_fused_op(Carver& w, const dllm_config* cfg, int rows_cap, LayerCtx* L
   L->fused_attn_floats = af;
 }
 
+// Per-layer ES selection: from the skip layer on, each layer runs alone and right after
+// its select_active call.
+int per_layer_order(const dllm_handle* x, int l0, int l1) {
+  if (!es_per_layer(x) || l1 <= x->c.skip_layer) return DLLM_OK;
+  if (l1 - l0 == 1 && l0 >= x->c.skip_layer && x->es_layer == l0 + 1) return DLLM_OK;
+  DLLM_FAIL(DLLM_ERR_STATE, "per-layer selection: each layer from skip_layer on runs alone, after select_active");
+}
+
+// ES-dLLM sec. 2.1 item 2, per layer: the top k chosen at the start of layer es_layer.
+// Refresh steps snapshot each candidate's input of the layer instead.
+int select_layer(dllm_handle* x, const float* forced, int32_t* active_idx, int32_t* active_count, cudaStream_t st) {
+  const auto& c = x->c;
+  const int l = x->es_layer, ls = c.skip_layer;
+  if (l >= x->L) DLLM_FAIL(DLLM_ERR_STATE, "select_active after the last layer");
+  const int64_t BNd = static_cast<int64_t>(x->B) * x->N * x->d;
+  float* prev = l == ls ? x->h_prev : x->es_in + (l - ls - 1) * BNd;
+  const int ncand = x->B * x->n_cand;
+  if (x->kind == DLLM_STEP_FULL) {
+    if (l == ls) {
+      DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->n_cand, x->rows2, x->seq_off2, x->nrows2, st));
+      DLLM_TRY(snapshot_rows_launch(x->h, x->h_prev, x->tokens, x->masked_prev, c.mask_id, x->rows2, ncand, x->d, st));
+    } else {
+      DLLM_TRY(copy_rows_launch(x->h, prev, x->rows2, x->nrows2, ncand, x->d, st));
+    }
+    x->es_layer += 1;
+    return DLLM_OK;
+  }
+  if (x->kind != DLLM_STEP_SKIP) DLLM_FAIL(DLLM_ERR_STATE, "select_active outside an ES step");
+  // Eq. 1 on this layer's input; rows the previous layer skipped take their cached output
+  // (their input last iteration) and score the confidence term alone.  masked_prev rolls
+  // forward at the last layer, after every layer has read it.
+  DLLM_TRY(score_es_launch(x->h, prev, x->conf, x->masked_prev, l == x->L - 1 ? x->tokens : nullptr, c.mask_id,
+                           x->rows, ncand, x->d, c.alpha, 1, l > ls ? x->act_flag : nullptr, x->scores, st));
+  SelectParams sp;
+  sp.scores = forced ? forced : x->scores;
+  sp.B = x->B; sp.n = x->n_cand; sp.mode = SEL_TOPK_DESC; sp.k = x->k_keep; sp.cand_start = cand_first(x);
+  sp.seq_n = x->N; sp.act_pos = active_idx ? active_idx : x->act_idx; sp.k_max = x->k_keep;
+  sp.count = active_count ? active_count : x->act_count; sp.row_map = x->rows2; sp.seq_off = x->seq_off2;
+  sp.total = x->nrows2; sp.flag = x->act_flag;
+  DLLM_TRY(select_launch(sp, st));
+  x->cur_rows = x->rows2;
+  x->cur_n = x->nrows2;
+  x->cur_seq_off = x->seq_off2;
+  x->cur_rows_cap = x->B * x->k_keep;
+  x->cur_rows_per_seq = x->k_keep;
+  x->es_layer += 1;
+  return DLLM_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -671,6 +734,7 @@ int dllm_begin_step(dllm_handle* x, int32_t* kind_out, void* stream) {
   DLLM_TRY(embed_rows_launch(static_cast<const __nv_bfloat16*>(x->w.embed), x->V, x->tokens, x->rows, x->nrows,
                              x->cur_rows_cap, x->d, x->h, st));
   x->began = true;
+  x->es_layer = c.skip_layer;
   if (kind_out) *kind_out = kind;
   return DLLM_OK;
 }
@@ -679,6 +743,7 @@ int dllm_layer_forward(dllm_handle* x, int32_t layer, void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
   if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "layer_forward before begin_step");
   if (layer < 0 || layer >= x->L) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "layer out of range");
+  DLLM_TRY(per_layer_order(x, layer, layer + 1));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto& c = x->c;
   const int64_t BNd = static_cast<int64_t>(x->B) * x->N * x->d;
@@ -721,6 +786,7 @@ int dllm_layers_forward(dllm_handle* x, int32_t l0, int32_t l1, void* stream) {
   if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "layers_forward before begin_step");
   if (l0 < 0 || l1 > x->L || l0 > l1) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "layer range out of bounds");
   if (l0 == l1) return DLLM_OK;
+  DLLM_TRY(per_layer_order(x, l0, l1));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (x->c.policy != DLLM_POLICY_DLLM_CACHE) {   // dLLM-Cache picks its rows per layer
     const LayerCtx L0 = layer_ctx(x, l0);
@@ -741,6 +807,7 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto& c = x->c;
   if (c.policy != DLLM_POLICY_ES) return DLLM_OK;
+  if (c.es_per_layer) return select_layer(x, scores_or_null, active_idx, active_count, st);
   const int mask = c.mask_id;
   if (x->kind == DLLM_STEP_FULL) {
     // refresh: snapshot the candidates' hidden state at the skip layer
@@ -751,7 +818,7 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
   if (x->kind != DLLM_STEP_SKIP) DLLM_FAIL(DLLM_ERR_STATE, "select_active outside an ES step");
   // Eq. 1 (always evaluated: it also rolls h_prev and masked_prev forward)
   DLLM_TRY(score_es_launch(x->h, x->h_prev, x->conf, x->masked_prev, x->tokens, mask, x->rows, x->B * x->n_cand, x->d,
-                           c.alpha, 1, x->scores, st));
+                           c.alpha, 1, nullptr, x->scores, st));
   SelectParams sp;
   sp.scores = scores_or_null ? scores_or_null : x->scores;
   sp.B = x->B; sp.n = x->n_cand; sp.mode = SEL_TOPK_DESC; sp.k = x->k_keep; sp.cand_start = cand_first(x);
@@ -770,6 +837,8 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
 int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
   if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "unmask before begin_step");
+  if (es_per_layer(x) && x->es_layer != x->L)
+    DLLM_FAIL(DLLM_ERR_STATE, "per-layer selection: select_active before every layer from skip_layer on");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto& c = x->c;
   const int bs = blk_start(x);
@@ -843,8 +912,15 @@ int dllm_step(dllm_handle* x, dllm_step_info* info, void* stream) {
   const auto& c = x->c;
   const int ls = c.policy == DLLM_POLICY_ES ? c.skip_layer : x->L;
   DLLM_TRY(dllm_layers_forward(x, 0, ls, stream));
-  if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
-  DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));
+  if (es_per_layer(x)) {
+    for (int l = ls; l < x->L; ++l) {
+      DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+      DLLM_TRY(dllm_layers_forward(x, l, l + 1, stream));
+    }
+  } else {
+    if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
+    DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));
+  }
   DLLM_TRY(dllm_unmask(x, nullptr, nullptr, nullptr, stream));
   if (info) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);

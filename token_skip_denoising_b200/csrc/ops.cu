@@ -192,8 +192,9 @@ int dllm_op_score_es(const float* h, float* h_prev, const float* conf, uint8_t* 
                      float* score, void* stream) {
   if (!h || !h_prev || !conf || !score || n_rows < 0 || d <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad score_es args");
   if (update && (!masked_prev || !tokens)) OP_FAIL(DLLM_ERR_INVALID_ARG, "update needs masked_prev and tokens");
-  return score_es_launch(h, h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha, update, score,
-                         static_cast<cudaStream_t>(stream));
+  // without a previous-layer choice (act_prev null) the kernel only reads h
+  return score_es_launch(const_cast<float*>(h), h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
+                         update, nullptr, score, static_cast<cudaStream_t>(stream));
 }
 
 int dllm_op_score_cos(const float* vnew, const void* vcache, const int32_t* rows, const int32_t* count,

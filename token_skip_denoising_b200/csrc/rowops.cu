@@ -112,25 +112,36 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int* __re
 //   var = ||h - h_prev||_1 / (sqrt(d) ||h_prev||_2)   (0 when ||h_prev|| = 0)
 //   score[j] = alpha c + (1 - alpha) var
 // then h_prev[flat] := h[flat] and masked_prev[flat] := (tokens[flat] == mask_id)
+// (tokens null: masked_prev is read but not rolled).
+// Per-layer re-selection: with act_prev non-null, a row whose act_prev[flat] is 0 was
+// skipped by the previous layer, so its input here is its cached output of that layer,
+// h_prev[flat] itself: var = 0 and the row of h is overwritten with h_prev (the carry of
+// the cached state into this layer), h_prev unchanged.
 // One warp per row.
-__global__ void score_es_kernel(const float* __restrict__ h, float* __restrict__ h_prev,
+__global__ void score_es_kernel(float* __restrict__ h, float* __restrict__ h_prev,
                                 const float* __restrict__ conf, uint8_t* __restrict__ masked_prev,
                                 const int* __restrict__ tokens, int mask_id, const int* __restrict__ rows,
-                                int n_rows, int d, float alpha, int update, float* __restrict__ score) {
+                                int n_rows, int d, float alpha, int update, const uint8_t* __restrict__ act_prev,
+                                float* __restrict__ score) {
   pdl_trigger();
   pdl_wait();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= n_rows) return;
   const int flat = rows ? rows[wid] : wid;
-  const float* x = h + static_cast<int64_t>(flat) * d;
+  float* x = h + static_cast<int64_t>(flat) * d;
   float* xp = h_prev + static_cast<int64_t>(flat) * d;
+  const bool carried = act_prev && !act_prev[flat];
   float l1 = 0.f, l2 = 0.f;
   for (int i = lane * 4; i < d; i += 128) {
-    const float4 a = *reinterpret_cast<const float4*>(x + i);
     const float4 b = *reinterpret_cast<const float4*>(xp + i);
-    l1 += fabsf(a.x - b.x) + fabsf(a.y - b.y) + fabsf(a.z - b.z) + fabsf(a.w - b.w);
     l2 += b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+    if (carried) {
+      *reinterpret_cast<float4*>(x + i) = b;
+      continue;
+    }
+    const float4 a = *reinterpret_cast<const float4*>(x + i);
+    l1 += fabsf(a.x - b.x) + fabsf(a.y - b.y) + fabsf(a.z - b.z) + fabsf(a.w - b.w);
     if (update) *reinterpret_cast<float4*>(xp + i) = a;
   }
   l1 = warp_sum_f(l1);
@@ -390,6 +401,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
       const bool sel = e && (take_all || keys[i] > T || (eq && eqr < need_eq));
       int tot_sel;
       const int o = block_scan_excl(sel ? 1 : 0, s_warp, tot_sel) + carry_sel;
+      if (p.flag && in) p.flag[static_cast<int64_t>(b) * p.seq_n + p.cand_start + i] = (sel && kk > 0) ? 1 : 0;
       if (sel && kk > 0) {
         const int pos = p.cand_start + i;
         if (p.act_pos) p.act_pos[static_cast<int64_t>(b) * p.k_max + o] = pos;
@@ -726,15 +738,15 @@ int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev
   return DLLM_OK;
 }
 
-int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
-                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update, float* score,
-                    cudaStream_t st) {
+int score_es_launch(float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
+                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update,
+                    const uint8_t* act_prev, float* score, cudaStream_t st) {
   if (n_rows <= 0) return DLLM_OK;
   if (d % 4) return DLLM_ERR_SHAPE;
   const int blocks = (n_rows * 32 + 255) / 256;
 {
     const int rc_ = launch_pdl(  score_es_kernel, dim3(blocks), dim3(256), 0, st, h, h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
-                                          update, score);
+                                          update, act_prev, score);
     if (rc_) return rc_;
   }
   return DLLM_OK;

@@ -26,6 +26,7 @@ struct SelectParams {
   int* row_map = nullptr;          // flat rows, b-major
   int* seq_off = nullptr;          // [B + 1]
   int* total = nullptr;
+  uint8_t* flag = nullptr;         // [B, seq_n]: 1 where a candidate is chosen, 0 where not
 };
 
 int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st);
@@ -33,9 +34,9 @@ int embed_rows_launch(const __nv_bfloat16* E, int V, const int* tokens, const in
                       int rows_cap, int d, float* h, cudaStream_t st);
 int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
                         float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st);
-int score_es_launch(const float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
-                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update, float* score,
-                    cudaStream_t st);
+int score_es_launch(float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
+                    int mask_id, const int* rows, int n_rows, int d, float alpha, int update,
+                    const uint8_t* act_prev, float* score, cudaStream_t st);
 int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, const int* rows, const int* count_dev,
                      int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st);
 // SureLock: statistics of the stored logits of each LM row, its divergence from the
