@@ -456,7 +456,8 @@ def variant_steps(peaks, steps=3, warm=2):
     gen_ms = e0.elapsed_time(e1)
     res["es_per_layer_llada8b"] = {
         "workload": "llada_es with the top k re-chosen by Eq. 1 at every layer from the skip layer on "
-                    "(one score, selection and layer launch per layer; one generation, device-timed)",
+                    "(skip steps: layers 4-31 in one persistent launch that scores and chooses the rows at the "
+                    "start of each layer; one generation, device-timed)",
         "generation_ms": round(gen_ms, 2), "steps": ecfg.n_blocks * ecfg.block_len,
         "tokens_per_s": round(ecfg.batch * ecfg.gen_len / (gen_ms / 1e3), 2)}
     del eng

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     from token_skip_denoising_b200._lib import DllmError
-    from token_skip_denoising_b200.engine import Engine
+    from token_skip_denoising_b200.engine import Engine, kernel_launches
 
 DEV = "cuda"
 BASE = scaled(get_config("tiny"), n_layers=4)
@@ -147,6 +147,94 @@ def test_forced_layer_choices_that_differ(w4):
                        orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_fused_per_layer_run_matches_oracle_teacher_forced(w4, batch):
+    """dllm_select_layers_forward: on skip steps one persistent launch scores and chooses the
+    rows at the start of every layer itself.  With the oracle's per-layer scores forced, the
+    chosen rows are exact and outputs, confidences and caches agree within tolerance; the
+    scores it computes (the last layer's are kept) agree with Eq. 1 on the score scale."""
+    cfg = PL.replace(batch=batch)
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, w4, tok0.numpy())
+    eng = Engine(cfg, _dev(w4), tok0.to(DEV).contiguous())
+    N, L, ls = cfg.seq_len, cfg.model.n_layers, cfg.skip_layer
+    kc, vc = eng.buffer("kcache"), eng.buffer("vcache")
+    hid, conf, amax = eng.buffer("hidden"), eng.buffer("conf"), eng.buffer("argmax")
+    n_skip = 0
+    while not orc.done:
+        rec = orc.step()
+        kind = eng.begin_step()
+        eng.layers_forward(0, ls)
+        forced = None
+        if kind == "skip":
+            forced = torch.tensor(np.stack(rec["layer_scores"]), dtype=torch.float32, device=DEV).contiguous()
+        torch.cuda.synchronize()
+        n0 = kernel_launches()
+        eng.select_layers_forward(forced)
+        torch.cuda.synchronize()
+        if kind == "skip":
+            assert kernel_launches() - n0 == 2            # the row counts, then one fused launch
+            gs = eng.buffer("scores")[:len(rec["cand"][0])].cpu().numpy().astype(np.float64)
+            ref = rec["layer_scores"][-1]
+            assert np.abs(gs - ref).max() <= 0.1 * np.abs(ref).max()
+            n_skip += 1
+        rows = eng.buffer("rows")
+        nrows = int(eng.buffer("nrows")[0])
+        flat = _flat(*rec["rows"], N)
+        np.testing.assert_array_equal(rows[:nrows].cpu().numpy(), flat)
+        assert _rowrel(hid[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
+        eng.unmask()
+        torch.cuda.synchronize()
+        lm = flat[rec["lm_rows"]]
+        np.testing.assert_allclose(conf[torch.tensor(lm, device=DEV)].cpu().numpy(), orc.conf.reshape(-1)[lm],
+                                   rtol=5e-2, atol=1e-5)
+        for l in range(L):
+            assert _rowrel(kc[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
+                           orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
+            assert _rowrel(vc[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
+                           orc.V[l].reshape(-1, cfg.model.head_dim)) < 2e-2
+        eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
+        conf.copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
+        amax.copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
+    assert n_skip == 7
+    assert eng.done
+
+
+def test_fused_per_layer_run_with_differing_forced_choices(w4):
+    """Forced choices that move from layer to layer (rows 4j .. 4j+7 at the j-th scored layer)
+    through the in-kernel choice: the same rows, inputs carried the same way as the oracle."""
+    cfg = PL
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, w4, tok0.numpy())
+    eng = Engine(cfg, _dev(w4), tok0.to(DEV).contiguous())
+    orc.step()
+    eng.step()
+    eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
+    eng.buffer("conf").copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
+    eng.buffer("argmax").copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
+    L, ls, n, N = cfg.model.n_layers, cfg.skip_layer, cfg.block_len, cfg.seq_len
+    forced = np.zeros((L - ls, n))
+    for j in range(L - ls):
+        forced[j, 4 * j + np.arange(8)] = 1.0
+    rec = orc.step(forced_scores=list(forced))
+    k0 = eng.buffer("kcache").clone()
+    assert eng.begin_step() == "skip"
+    eng.layers_forward(0, ls)
+    eng.select_layers_forward(torch.tensor(forced, dtype=torch.float32, device=DEV).contiguous())
+    flat = _flat(*rec["rows"], N)
+    np.testing.assert_array_equal(eng.buffer("rows")[:8].cpu().numpy(), flat)
+    assert _rowrel(eng.buffer("hidden")[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
+    eng.unmask()
+    torch.cuda.synchronize()
+    k1 = eng.buffer("kcache")
+    for j, l in enumerate(range(ls, L)):
+        chosen = cfg.prompt_len + 4 * j + np.arange(8)
+        changed = (k1[l] != k0[l]).any(dim=-1).any(dim=1)[0].cpu().numpy()
+        assert set(np.nonzero(changed)[0].tolist()) <= set(chosen.tolist())
+        assert _rowrel(k1[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
+                       orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
+
+
 def test_keep_all_per_layer_equals_vanilla(w4):
     tok0 = make_tokens(BASE)
     a = Engine(PL.replace(keep_ratio=1.0, cand_scope="all"), _dev(w4), tok0.to(DEV).contiguous(),
@@ -189,3 +277,5 @@ def test_out_of_order_calls_are_refused(w4):
         eng.layers_forward(cfg.skip_layer, cfg.model.n_layers)   # more than one layer at once
     with pytest.raises(DllmError):
         eng.unmask()                                 # layers left
+    with pytest.raises(DllmError):
+        eng.select_layers_forward()                  # a per-layer call was made in this step

@@ -75,6 +75,7 @@ _SIGS = {
     "dllm_layer_forward": (ctypes.c_int, [c_vp, c_i32, c_vp]),
     "dllm_layers_forward": (ctypes.c_int, [c_vp, c_i32, c_i32, c_vp]),
     "dllm_select_active": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "dllm_select_layers_forward": (ctypes.c_int, [c_vp, c_vp, c_vp]),
     "dllm_unmask": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     "dllm_step": (ctypes.c_int, [c_vp, P(DllmStepInfo), c_vp]),
     "dllm_done": (ctypes.c_int, [c_vp]),

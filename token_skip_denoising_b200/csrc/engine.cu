@@ -428,8 +428,9 @@ bool fused_applies(const LayerCtx& x, int rows_cap) { return x.fused && x.fused_
 // Layers x.layer .. x.layer + n_layers - 1 as one fused persistent kernel (DLLM_ERR_UNSUPPORTED
 // when the shapes do not allow it).
 int run_fused_layers(const LayerCtx& x, int n_layers, float* hbuf, const int* rows, const int* n, const int* seq_off,
-                     int rows_cap, int rows_per_seq, cudaStream_t st) {
+                     int rows_cap, int rows_per_seq, cudaStream_t st, const FusedEs* es = nullptr) {
   FusedLayerArgs a;
+  if (es) a.es = *es;
   a.B = x.B; a.N = x.N; a.d = x.d; a.qd = x.qd; a.kvd = x.kvd; a.qkvd = x.qkvd; a.F = x.F; a.hd = x.hd;
   a.Hq = x.Hq; a.Hkv = x.Hkv; a.eps = x.eps;
   a.L = x.n_layers_total; a.l0 = x.layer; a.n_layers = n_layers;
@@ -617,6 +618,35 @@ int select_layer(dllm_handle* x, const float* forced, int32_t* active_idx, int32
   x->cur_rows_cap = x->B * x->k_keep;
   x->cur_rows_per_seq = x->k_keep;
   x->es_layer += 1;
+  return DLLM_OK;
+}
+
+// Layers skip_layer .. L-1 of a per-layer ES skip step as one fused launch that scores and
+// chooses the rows at the start of each layer itself (DLLM_ERR_UNSUPPORTED when it does not apply).
+int fused_per_layer_run(dllm_handle* x, const float* forced, cudaStream_t st) {
+  const auto& c = x->c;
+  const int ls = c.skip_layer;
+  const LayerCtx L0 = layer_ctx(x, ls);
+  const int cap = x->B * x->k_keep;
+  if (!fused_applies(L0, cap) || x->n_cand > kFusedEsMaxCand) return DLLM_ERR_UNSUPPORTED;
+  // the row counts and sequence offsets of k rows per sequence (the kernel fills the rows)
+  DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->k_keep, x->rows2, x->seq_off2, x->nrows2, st));
+  FusedEs e;
+  e.on = 1;
+  e.ls = ls; e.L = x->L;
+  e.B = x->B; e.n_cand = x->n_cand; e.cand_start = cand_first(x); e.k = x->k_keep;
+  e.alpha = c.alpha; e.mask_id = c.mask_id;
+  e.h_prev = x->h_prev; e.es_in = x->es_in;
+  e.conf = x->conf; e.masked_prev = x->masked_prev; e.tokens = x->tokens;
+  e.flag = x->act_flag; e.rows = x->rows2; e.scores = x->scores; e.forced = forced;
+  const int rc = run_fused_layers(L0, x->L - ls, x->h, x->rows2, x->nrows2, x->seq_off2, cap, x->k_keep, st, &e);
+  if (rc) return rc;
+  x->cur_rows = x->rows2;
+  x->cur_n = x->nrows2;
+  x->cur_seq_off = x->seq_off2;
+  x->cur_rows_cap = cap;
+  x->cur_rows_per_seq = x->k_keep;
+  x->es_layer = x->L;
   return DLLM_OK;
 }
 
@@ -834,6 +864,25 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
   return DLLM_OK;
 }
 
+int dllm_select_layers_forward(dllm_handle* x, const float* scores_or_null, void* stream) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward before begin_step");
+  if (!es_per_layer(x)) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward needs ES with es_per_layer");
+  if (x->es_layer != x->c.skip_layer) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward starts at skip_layer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int ls = x->c.skip_layer;
+  if (x->kind == DLLM_STEP_SKIP) {
+    const int rc = fused_per_layer_run(x, scores_or_null, st);
+    if (rc != DLLM_ERR_UNSUPPORTED) return rc;
+  }
+  const int64_t per = static_cast<int64_t>(x->B) * x->n_cand;
+  for (int l = ls; l < x->L; ++l) {
+    DLLM_TRY(select_layer(x, scores_or_null ? scores_or_null + (l - ls) * per : nullptr, nullptr, nullptr, st));
+    DLLM_TRY(dllm_layers_forward(x, l, l + 1, stream));
+  }
+  return DLLM_OK;
+}
+
 int dllm_unmask(dllm_handle* x, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
   if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "unmask before begin_step");
@@ -913,10 +962,7 @@ int dllm_step(dllm_handle* x, dllm_step_info* info, void* stream) {
   const int ls = c.policy == DLLM_POLICY_ES ? c.skip_layer : x->L;
   DLLM_TRY(dllm_layers_forward(x, 0, ls, stream));
   if (es_per_layer(x)) {
-    for (int l = ls; l < x->L; ++l) {
-      DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
-      DLLM_TRY(dllm_layers_forward(x, l, l + 1, stream));
-    }
+    DLLM_TRY(dllm_select_layers_forward(x, nullptr, stream));
   } else {
     if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
     DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));

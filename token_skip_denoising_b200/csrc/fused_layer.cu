@@ -22,6 +22,10 @@
 //     QKV sums -> RoPE and K/V scatter -> attention (the last split of a query tile
 //     merges the partials) -> O in h -> operand g * h -> gate/up sums -> SwiGLU ->
 //     down in h.
+//   With per-layer re-selection (ES-dLLM, the top k chosen at the start of every layer)
+//   two phases open each layer: Eq. 1 for every candidate (one warp per row; a row the
+//   previous layer skipped first takes its cached output) and the top k of each sequence
+//   (one CTA per sequence, rank counting), which rewrites the row map the layer then uses.
 // Every cross-CTA wait is bounded; on expiry the kernel records a timeout in the
 // device status word and every role stops.
 #include <algorithm>
@@ -29,6 +33,7 @@
 
 #include "attn_dev.cuh"
 #include "common.cuh"
+#include "es_dev.cuh"
 #include "gemm_dev.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
@@ -47,7 +52,7 @@ constexpr int kMaxRows = kFusedMaxRows;           // rows of the fp32 sum buffer
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
-enum Phase : int { S_X1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_X2, S_GU, S_SWIGLU, S_DOWN, S_COUNT };
+enum Phase : int { S_X1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_X2, S_GU, S_SWIGLU, S_DOWN, S_SCORE, S_PICK, S_COUNT };
 static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
 static_assert(kMaxRows <= 128 && 128 % kMaxRows == 0, "rows are handled by the 128 step threads");
 
@@ -105,6 +110,8 @@ struct FParams {
   int attn_items;
   int* attn_ctr;          // [B * Hkv * attn_qtiles] split arrivals, zero between uses
   int* sync;              // [S_COUNT] phase counters + exit counter, zero at launch
+  FusedEs es;             // per-layer re-selection at the start of every layer (es.on)
+  float* es_acc;          // [2 * B * n_cand] Eq. 1 sums of the candidates, zero between layers
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -445,6 +452,80 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       __nv_bfloat16* vc = p.vc + static_cast<int64_t>(l) * p.kv_layer;
       // the previous layer's down sums are complete in h (and its sums have been read)
       if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t)) s_flag[0] = 1;
+      if (p.es.on) {
+        // ES-dLLM Eq. 1 on every candidate's input of this layer: each row split into column
+        // slices over the grid's warps, whose partial sums meet in es_acc[2 u .. 2 u + 1]
+        const FusedEs& es = p.es;
+        const int n = es.n_cand;
+        const int nrow = es.B * n;
+        if (!s_flag[0]) {
+          const int64_t BNd = static_cast<int64_t>(es.B) * p.N * p.d;
+          float* prev = l == es.ls ? es.h_prev : es.es_in + static_cast<int64_t>(l - es.ls - 1) * BNd;
+          const int nch = p.d >> 7;                                  // 128-column chunks of a row
+          const int S = max(1, min(nch, (G * 4) / nrow));            // slices per row
+          for (int w = c * 4 + warp; w < nrow * S; w += G * 4) {
+            const int u = w / S, sl = w - (w / S) * S;
+            const int b = u / n;
+            const int flat = b * p.N + es.cand_start + (u - b * n);
+            const bool carried = l > es.ls && __ldcg(es.flag + flat) == 0;
+            float l1 = 0.f, l2 = 0.f;
+            es_eq1_part(p.h + static_cast<int64_t>(flat) * p.d, prev + static_cast<int64_t>(flat) * p.d,
+                        (nch * sl / S) << 7, min(p.d, (nch * (sl + 1) / S) << 7), 1, carried, lane, l1, l2);
+            l1 = es_warp_sum(l1);
+            l2 = es_warp_sum(l2);
+            if (lane == 0) {
+              atomicAdd(p.es_acc + 2 * u, l1);
+              atomicAdd(p.es_acc + 2 * u + 1, l2);
+            }
+          }
+        }
+        signal_phase(p.sync + S_SCORE, t);
+        // the top k of sequence b by CTA b: a candidate is chosen when fewer than k others
+        // rank above it (higher key, or an equal key at a lower position)
+        if (epi_wait_phase(p.sync + S_SCORE, target, s_flag, t) && c < es.B) {
+          const int b = c;
+          const bool last = l == es.L - 1;
+          uint8_t* s_pick = attn_smem;                                         // idle outside attention
+          uint32_t* s_key = reinterpret_cast<uint32_t*>(attn_smem + kFusedEsMaxCand);
+          const float* fv = es.forced ? es.forced + (static_cast<int64_t>(li) * es.B + b) * n : nullptr;
+          for (int i = t; i < n; i += 128) {
+            const int u = b * n + i;
+            const int flat = b * p.N + es.cand_start + i;
+            const float l1 = __ldcg(p.es_acc + 2 * u), l2 = __ldcg(p.es_acc + 2 * u + 1);
+            p.es_acc[2 * u] = 0.f;                                           // zero for the next layer
+            p.es_acc[2 * u + 1] = 0.f;
+            const float cf = __ldcg(es.masked_prev + flat) ? __ldcg(es.conf + flat) : 0.f;
+            const float sc = es_eq1_score(l1, l2, p.d, cf, es.alpha);
+            es.scores[u] = sc;
+            // masked_prev rolls forward once every layer has read it
+            if (last) es.masked_prev[flat] = __ldcg(es.tokens + flat) == es.mask_id ? 1 : 0;
+            s_key[i] = order_key(fv ? __ldcg(fv + i) : sc);
+          }
+          epi_bar();
+          for (int i = t; i < n; i += 128) {
+            const uint32_t ki = s_key[i];
+            int rank = 0;
+            for (int jn = 0; jn < n; ++jn) {
+              const uint32_t kj = s_key[jn];
+              rank += (kj > ki || (kj == ki && jn < i)) ? 1 : 0;
+            }
+            const uint8_t ch = rank < es.k ? 1 : 0;
+            s_pick[i] = ch;
+            es.flag[b * p.N + es.cand_start + i] = ch;
+          }
+          epi_bar();
+          for (int i = t; i < n; i += 128) {
+            if (!s_pick[i]) continue;
+            int o = 0;
+            for (int jn = 0; jn < i; ++jn) o += s_pick[jn];
+            es.rows[b * es.k + o] = b * p.N + es.cand_start + i;
+          }
+        }
+        signal_phase(p.sync + S_PICK, t);
+        if (epi_wait_phase(p.sync + S_PICK, target, s_flag, t) && t < kMaxRows)
+          s_rows[t] = t < m_rows ? __ldcg(es.rows + t) : 0;
+        epi_bar();
+      }
       if (!s_flag[0]) {
         // zero this layer's sums (every CTA passes this phase before any adds into them)
         const int64_t nq = static_cast<int64_t>(m_rows) * p.qkvd / 4;
@@ -626,7 +707,7 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const F
 
 size_t fused_scratch_floats(int qkvd, int F) {
   return static_cast<size_t>(kMaxRows) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F)) +
-         2 * static_cast<size_t>(kNumSMs) * kMaxRows;
+         2 * static_cast<size_t>(kNumSMs) * kMaxRows + 2 * static_cast<size_t>(kMaxRows) * kFusedEsMaxCand;
 }
 
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
@@ -684,6 +765,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.s_gu = s_gu;
   p.ssp1 = ssp;
   p.ssp2 = ssp + static_cast<size_t>(grid) * kMaxRows;
+  p.es_acc = ssp + 2 * static_cast<size_t>(kNumSMs) * kMaxRows;
   p.qkvd = a.qkvd; p.qd = a.qd; p.kvd = a.kvd; p.hd = a.hd; p.Hkv = a.Hkv; p.N = a.N; p.F = a.F;
   p.rope_cos = a.rope_cos;
   p.rope_sin = a.rope_sin;
@@ -721,6 +803,16 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.attn_items = a.B * a.Hkv * qtiles * splits;
   p.attn_ctr = a.attn_ctr;
   p.sync = a.sync;
+  p.es = a.es;
+  if (a.es.on) {
+    const FusedEs& e = a.es;
+    if (e.n_cand <= 0 || e.n_cand > kFusedEsMaxCand || e.k <= 0 || e.k > e.n_cand || e.B != a.B || e.B > grid ||
+        e.B * e.k > a.rows_cap || e.ls < 0 || a.l0 < e.ls || a.l0 + a.n_layers > e.L || e.L != a.L)
+      return DLLM_ERR_UNSUPPORTED;
+    if (!e.h_prev || (a.l0 + a.n_layers - 1 > e.ls && !e.es_in) || !e.conf || !e.masked_prev || !e.tokens ||
+        !e.flag || !e.rows || !e.scores || e.rows != a.rows)
+      return DLLM_ERR_INVALID_ARG;
+  }
   if (bn == 16) return launch_fused<16>(tw, tx, p, grid, st);
   if (bn == 32) return launch_fused<32>(tw, tx, p, grid, st);
   return launch_fused<64>(tw, tx, p, grid, st);

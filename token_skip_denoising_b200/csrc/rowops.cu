@@ -5,6 +5,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "es_dev.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
 
@@ -129,28 +130,12 @@ __global__ void score_es_kernel(float* __restrict__ h, float* __restrict__ h_pre
   const int lane = threadIdx.x & 31;
   if (wid >= n_rows) return;
   const int flat = rows ? rows[wid] : wid;
-  float* x = h + static_cast<int64_t>(flat) * d;
-  float* xp = h_prev + static_cast<int64_t>(flat) * d;
   const bool carried = act_prev && !act_prev[flat];
-  float l1 = 0.f, l2 = 0.f;
-  for (int i = lane * 4; i < d; i += 128) {
-    const float4 b = *reinterpret_cast<const float4*>(xp + i);
-    l2 += b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
-    if (carried) {
-      *reinterpret_cast<float4*>(x + i) = b;
-      continue;
-    }
-    const float4 a = *reinterpret_cast<const float4*>(x + i);
-    l1 += fabsf(a.x - b.x) + fabsf(a.y - b.y) + fabsf(a.z - b.z) + fabsf(a.w - b.w);
-    if (update) *reinterpret_cast<float4*>(xp + i) = a;
-  }
-  l1 = warp_sum_f(l1);
-  l2 = warp_sum_f(l2);
+  const float c = (masked_prev && masked_prev[flat]) ? conf[flat] : 0.f;
+  const float s = es_eq1_row(h + static_cast<int64_t>(flat) * d, h_prev + static_cast<int64_t>(flat) * d, d, c,
+                             alpha, update, carried, lane);
   if (lane == 0) {
-    const float c = (masked_prev && masked_prev[flat]) ? conf[flat] : 0.f;
-    const float nrm = sqrtf(l2);
-    const float var = nrm > 0.f ? l1 / (sqrtf(static_cast<float>(d)) * nrm) : 0.f;
-    score[wid] = alpha * c + (1.f - alpha) * var;
+    score[wid] = s;
     if (update && masked_prev && tokens) masked_prev[flat] = tokens[flat] == mask_id ? 1 : 0;
   }
 }
@@ -293,13 +278,6 @@ __global__ void kl_conf_kernel(const __nv_bfloat16* __restrict__ z, int64_t ldz,
 // ------------------------------------------------------------------ selection
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxN = 8192;
-
-__device__ __forceinline__ uint32_t order_key(float x) {
-  if (x != x) return 0u;               // NaN: lowest
-  x = x + 0.0f;                        // -0 -> +0
-  uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // exclusive block scan for 1024 threads; returns the exclusive prefix, total via ref
 __device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int& total) {

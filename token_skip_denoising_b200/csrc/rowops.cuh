@@ -95,6 +95,28 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
 // A run of layers over at most kFusedMaxRows rows as one persistent kernel (fused_layer.cu).
 constexpr int kFusedSyncInts = 16;
 constexpr int kFusedMaxRows = 64;   // row sets the fused kernel serves (its sum buffers' rows)
+// ES-dLLM per-layer re-selection inside the fused layer run (every layer of the run is
+// scored and re-chosen at its start).  Same definition as the score and select kernels:
+// Eq. 1 on each candidate's layer input with the carry of skipped rows, the top k of each
+// sequence (ties to the lower position) in ascending position order.
+struct FusedEs {
+  int on = 0;
+  int ls = 0, L = 0;                 // skip layer, layers of the model
+  int B = 0, n_cand = 0, cand_start = 0, k = 0;
+  float alpha = 0.f;
+  int mask_id = 0;
+  float* h_prev = nullptr;           // inputs of layer ls last iteration, position-indexed [B*N, d]
+  float* es_in = nullptr;            // the same for layers ls+1 .. L-1: [L - ls - 1, B*N, d]
+  const float* conf = nullptr;       // [B*N]
+  uint8_t* masked_prev = nullptr;    // [B*N], rolled forward at the last layer
+  const int* tokens = nullptr;       // [B*N]
+  uint8_t* flag = nullptr;           // [B*N] chosen at the previous layer
+  int* rows = nullptr;               // [B*k] the chosen rows (the run's row map)
+  float* scores = nullptr;           // [B*n_cand] the latest layer's Eq. 1 scores
+  const float* forced = nullptr;     // [n_layers, B, n_cand] scores used for the choice, or null
+};
+constexpr int kFusedEsMaxCand = 512;  // candidates per sequence the in-kernel choice ranks
+
 struct FusedLayerArgs {
   int B, N, d, qd, kvd, qkvd, F, hd, Hq, Hkv;
   int L, l0, n_layers;              // layers l0 .. l0 + n_layers - 1 of L
@@ -117,6 +139,7 @@ struct FusedLayerArgs {
   float* scratch;          // fused_scratch_floats(qkvd, F): fp32 QKV (2 buffers) and gate/up sums;
                            // zero before the first launch, the kernel leaves it zero
   int* sync;               // kFusedSyncInts counters, zero before the launch; the kernel leaves them zero
+  FusedEs es;              // per-layer re-selection (es.on = 0: the row map is fixed)
 };
 size_t fused_scratch_floats(int qkvd, int F);
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap);

@@ -90,6 +90,12 @@ class Engine:
         check(self.lib.dllm_select_active(self.handle, ptr(scores), ptr(active_idx), ptr(active_count),
                                           stream_ptr(self.stream)), "dllm_select_active")
 
+    def select_layers_forward(self, scores: torch.Tensor | None = None):
+        """Per-layer ES: every layer from the skip layer on, each after its own choice
+        (scores: optional fp32 [L - skip_layer, B, n_cand] used for the choices)."""
+        check(self.lib.dllm_select_layers_forward(self.handle, ptr(scores), stream_ptr(self.stream)),
+              "dllm_select_layers_forward")
+
     def unmask(self, pos_out=None, tok_out=None, n_out=None):
         check(self.lib.dllm_unmask(self.handle, ptr(pos_out), ptr(tok_out), ptr(n_out), stream_ptr(self.stream)),
               "dllm_unmask")
