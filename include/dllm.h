@@ -195,16 +195,17 @@ int dllm_layers_forward(dllm_handle* h, int32_t l0, int32_t l1, void* stream);
 int dllm_select_active(dllm_handle* h, const float* scores_or_null, int32_t* active_idx, int32_t* active_count,
                        void* stream);
 
-/* ES-dLLM with es_per_layer: layers skip_layer .. n_layers-1 of the step with the
- * choice made again before each of them, the same result as dllm_select_active ->
- * dllm_layer_forward for each layer in turn.  On a skip step whose kept rows fit the
- * fused layer kernel (B * k <= 64, n_cand <= 512, layer_kernel not SPLIT) the whole
- * run is one persistent launch that scores (Eq. 1, with the carry of skipped rows)
- * and chooses the rows at the start of every layer itself.  `scores_or_null`: fp32
- * device [n_layers - skip_layer, B, n_cand], the scores each layer's choice uses
- * (teacher forcing), or NULL for Eq. 1.  Call after dllm_layers_forward(0,
- * skip_layer) and before dllm_unmask; DLLM_ERR_STATE when es_per_layer is off or a
- * per-layer call has already been made in this step. */
+/* ES-dLLM: the choice and layers skip_layer .. n_layers-1 of the step, with the same
+ * result as dllm_select_active -> dllm_layers_forward(skip_layer, n_layers), or with
+ * es_per_layer as dllm_select_active -> dllm_layer_forward for each layer in turn.
+ * On a skip step whose kept rows fit the fused layer kernel (B * k <= 64,
+ * n_cand <= 512, layer_kernel not SPLIT) the whole run is one persistent launch
+ * that scores (Eq. 1; per layer with the carry of skipped rows) and chooses the
+ * rows itself, at the skip layer or at the start of every layer.
+ * `scores_or_null`: fp32 device [S, B, n_cand], S = 1 (or n_layers - skip_layer
+ * with es_per_layer), the scores each choice uses (teacher forcing), or NULL for
+ * Eq. 1.  Call after dllm_layers_forward(0, skip_layer) and before dllm_unmask;
+ * DLLM_ERR_STATE outside the ES policy or when the step's choice was already made. */
 int dllm_select_layers_forward(dllm_handle* h, const float* scores_or_null, void* stream);
 
 /* Ends the step: final RMSNorm and vocabulary projection of the recomputed

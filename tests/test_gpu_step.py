@@ -16,7 +16,7 @@ from synth import get_config, make_tokens, make_weights
 pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
-    from token_skip_denoising_b200.engine import Engine
+    from token_skip_denoising_b200.engine import Engine, kernel_launches
 
 DEV = "cuda"
 TINY = get_config("tiny")
@@ -121,6 +121,55 @@ def test_es_steps_match_oracle_teacher_forced(tiny_w_cpu):
             assert _rowrel(kc[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
                            orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
         # teacher forcing of the decisions
+        eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
+        conf.copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
+        amax.copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
+    assert n_skip == 7
+    assert eng.done
+
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_es_choice_inside_the_fused_run_teacher_forced(tiny_w_cpu, batch):
+    """dllm_select_layers_forward on a skip step: one persistent launch scores the candidates
+    by Eq. 1, keeps the top k of each sequence and runs the remaining layers on them.  With the
+    oracle's scores forced the kept rows are exact; its own Eq. 1 scores, the outputs, the
+    confidences and the caches agree with the oracle within tolerance."""
+    cfg = TINY.replace(batch=batch)
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, tiny_w_cpu, tok0.numpy())
+    eng = _engine(cfg, tiny_w_cpu, tok0)
+    N, L, ls = cfg.seq_len, cfg.model.n_layers, cfg.skip_layer
+    kc = eng.buffer("kcache")
+    hid, conf, amax = eng.buffer("hidden"), eng.buffer("conf"), eng.buffer("argmax")
+    n_skip = 0
+    while not orc.done:
+        rec = orc.step()
+        kind = eng.begin_step()
+        eng.layers_forward(0, ls)
+        forced = None
+        if kind == "skip":
+            forced = torch.tensor(rec["scores"][None], dtype=torch.float32, device=DEV).contiguous()
+        torch.cuda.synchronize()
+        n0 = kernel_launches()
+        eng.select_layers_forward(forced)
+        torch.cuda.synchronize()
+        if kind == "skip":
+            assert kernel_launches() - n0 == 2            # the row counts, then one fused launch
+            gs = eng.buffer("scores")[:len(rec["scores"])].cpu().numpy().astype(np.float64)
+            assert np.abs(gs - rec["scores"]).max() <= 0.1 * np.abs(rec["scores"]).max()
+            n_skip += 1
+        nrows = int(eng.buffer("nrows")[0])
+        flat = _flat(*rec["rows"], N)
+        np.testing.assert_array_equal(eng.buffer("rows")[:nrows].cpu().numpy(), flat)
+        assert _rowrel(hid[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
+        eng.unmask()
+        torch.cuda.synchronize()
+        lm = flat[rec["lm_rows"]]
+        np.testing.assert_allclose(conf[torch.tensor(lm, device=DEV)].cpu().numpy(), orc.conf.reshape(-1)[lm],
+                                   rtol=5e-2, atol=1e-5)
+        for l in range(L):
+            assert _rowrel(kc[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
+                           orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
         eng.tokens.copy_(torch.tensor(orc.tokens, dtype=torch.int32))
         conf.copy_(torch.tensor(orc.conf.reshape(-1), dtype=torch.float32))
         amax.copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))

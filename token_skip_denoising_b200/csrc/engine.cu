@@ -291,7 +291,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->act_idx = w.take<int>(BN);
   x->act_count = w.take<int>(x->B);
   x->blk_remain = w.take<int>(x->B);
-  x->act_flag = es_per_layer(x) ? w.take<uint8_t>(BN) : nullptr;
+  x->act_flag = c.policy == DLLM_POLICY_ES ? w.take<uint8_t>(BN) : nullptr;
   x->scores = w.take<float>(BN);
   x->kl = w.take<float>(BN);
   const int64_t R = BN;   // row bound of any step
@@ -621,9 +621,10 @@ int select_layer(dllm_handle* x, const float* forced, int32_t* active_idx, int32
   return DLLM_OK;
 }
 
-// Layers skip_layer .. L-1 of a per-layer ES skip step as one fused launch that scores and
-// chooses the rows at the start of each layer itself (DLLM_ERR_UNSUPPORTED when it does not apply).
-int fused_per_layer_run(dllm_handle* x, const float* forced, cudaStream_t st) {
+// Layers skip_layer .. L-1 of an ES skip step as one fused launch that scores and chooses the
+// rows itself: at the skip layer, or at the start of every layer with es_per_layer
+// (DLLM_ERR_UNSUPPORTED when it does not apply).
+int fused_es_run(dllm_handle* x, const float* forced, cudaStream_t st) {
   const auto& c = x->c;
   const int ls = c.skip_layer;
   const LayerCtx L0 = layer_ctx(x, ls);
@@ -633,6 +634,7 @@ int fused_per_layer_run(dllm_handle* x, const float* forced, cudaStream_t st) {
   DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->k_keep, x->rows2, x->seq_off2, x->nrows2, st));
   FusedEs e;
   e.on = 1;
+  e.n_scored = c.es_per_layer ? x->L - ls : 1;
   e.ls = ls; e.L = x->L;
   e.B = x->B; e.n_cand = x->n_cand; e.cand_start = cand_first(x); e.k = x->k_keep;
   e.alpha = c.alpha; e.mask_id = c.mask_id;
@@ -843,6 +845,7 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
     // refresh: snapshot the candidates' hidden state at the skip layer
     DLLM_TRY(range_rows_launch(x->B, x->N, cand_first(x), x->n_cand, x->rows2, x->seq_off2, x->nrows2, st));
     DLLM_TRY(snapshot_rows_launch(x->h, x->h_prev, x->tokens, x->masked_prev, mask, x->rows2, x->B * x->n_cand, x->d, st));
+    x->es_layer = x->L;
     return DLLM_OK;
   }
   if (x->kind != DLLM_STEP_SKIP) DLLM_FAIL(DLLM_ERR_STATE, "select_active outside an ES step");
@@ -861,19 +864,24 @@ int dllm_select_active(dllm_handle* x, const float* scores_or_null, int32_t* act
   x->cur_seq_off = x->seq_off2;
   x->cur_rows_cap = x->B * x->k_keep;
   x->cur_rows_per_seq = x->k_keep;
+  x->es_layer = x->L;
   return DLLM_OK;
 }
 
 int dllm_select_layers_forward(dllm_handle* x, const float* scores_or_null, void* stream) {
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
   if (!x->began) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward before begin_step");
-  if (!es_per_layer(x)) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward needs ES with es_per_layer");
+  if (x->c.policy != DLLM_POLICY_ES) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward needs the ES policy");
   if (x->es_layer != x->c.skip_layer) DLLM_FAIL(DLLM_ERR_STATE, "select_layers_forward starts at skip_layer");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int ls = x->c.skip_layer;
-  if (x->kind == DLLM_STEP_SKIP) {
-    const int rc = fused_per_layer_run(x, scores_or_null, st);
+  if (x->kind == DLLM_STEP_SKIP && ls < x->L) {
+    const int rc = fused_es_run(x, scores_or_null, st);
     if (rc != DLLM_ERR_UNSUPPORTED) return rc;
+  }
+  if (!x->c.es_per_layer) {
+    DLLM_TRY(dllm_select_active(x, scores_or_null, nullptr, nullptr, stream));
+    return dllm_layers_forward(x, ls, x->L, stream);
   }
   const int64_t per = static_cast<int64_t>(x->B) * x->n_cand;
   for (int l = ls; l < x->L; ++l) {
@@ -961,12 +969,8 @@ int dllm_step(dllm_handle* x, dllm_step_info* info, void* stream) {
   const auto& c = x->c;
   const int ls = c.policy == DLLM_POLICY_ES ? c.skip_layer : x->L;
   DLLM_TRY(dllm_layers_forward(x, 0, ls, stream));
-  if (es_per_layer(x)) {
-    DLLM_TRY(dllm_select_layers_forward(x, nullptr, stream));
-  } else {
-    if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_active(x, nullptr, nullptr, nullptr, stream));
-    DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));
-  }
+  if (c.policy == DLLM_POLICY_ES) DLLM_TRY(dllm_select_layers_forward(x, nullptr, stream));
+  else DLLM_TRY(dllm_layers_forward(x, ls, x->L, stream));
   DLLM_TRY(dllm_unmask(x, nullptr, nullptr, nullptr, stream));
   if (info) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);

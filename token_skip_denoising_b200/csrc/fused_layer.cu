@@ -22,8 +22,8 @@
 //     QKV sums -> RoPE and K/V scatter -> attention (the last split of a query tile
 //     merges the partials) -> O in h -> operand g * h -> gate/up sums -> SwiGLU ->
 //     down in h.
-//   With per-layer re-selection (ES-dLLM, the top k chosen at the start of every layer)
-//   two phases open each layer: Eq. 1 for every candidate (one warp per row; a row the
+//   With the ES-dLLM choice in the run (the top k at the skip layer, or again at the start
+//   of every layer) two phases open each choosing layer: Eq. 1 for every candidate (one warp per row; a row the
 //   previous layer skipped first takes its cached output) and the top k of each sequence
 //   (one CTA per sequence, rank counting), which rewrites the row map the layer then uses.
 // Every cross-CTA wait is bounded; on expiry the kernel records a timeout in the
@@ -452,7 +452,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       __nv_bfloat16* vc = p.vc + static_cast<int64_t>(l) * p.kv_layer;
       // the previous layer's down sums are complete in h (and its sums have been read)
       if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t)) s_flag[0] = 1;
-      if (p.es.on) {
+      if (p.es.on && li < p.es.n_scored) {
         // ES-dLLM Eq. 1 on every candidate's input of this layer: each row split into column
         // slices over the grid's warps, whose partial sums meet in es_acc[2 u .. 2 u + 1]
         const FusedEs& es = p.es;
@@ -484,7 +484,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         // rank above it (higher key, or an equal key at a lower position)
         if (epi_wait_phase(p.sync + S_SCORE, target, s_flag, t) && c < es.B) {
           const int b = c;
-          const bool last = l == es.L - 1;
+          const bool last = li == es.n_scored - 1;
           uint8_t* s_pick = attn_smem;                                         // idle outside attention
           uint32_t* s_key = reinterpret_cast<uint32_t*>(attn_smem + kFusedEsMaxCand);
           const float* fv = es.forced ? es.forced + (static_cast<int64_t>(li) * es.B + b) * n : nullptr;
@@ -807,9 +807,10 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.es.on) {
     const FusedEs& e = a.es;
     if (e.n_cand <= 0 || e.n_cand > kFusedEsMaxCand || e.k <= 0 || e.k > e.n_cand || e.B != a.B || e.B > grid ||
-        e.B * e.k > a.rows_cap || e.ls < 0 || a.l0 < e.ls || a.l0 + a.n_layers > e.L || e.L != a.L)
+        e.B * e.k > a.rows_cap || e.ls < 0 || a.l0 < e.ls || a.l0 + a.n_layers > e.L || e.L != a.L ||
+        e.n_scored < 1 || e.n_scored > a.n_layers)
       return DLLM_ERR_UNSUPPORTED;
-    if (!e.h_prev || (a.l0 + a.n_layers - 1 > e.ls && !e.es_in) || !e.conf || !e.masked_prev || !e.tokens ||
+    if (!e.h_prev || (a.l0 + e.n_scored - 1 > e.ls && !e.es_in) || !e.conf || !e.masked_prev || !e.tokens ||
         !e.flag || !e.rows || !e.scores || e.rows != a.rows)
       return DLLM_ERR_INVALID_ARG;
   }

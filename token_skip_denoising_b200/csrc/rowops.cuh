@@ -95,12 +95,14 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
 // A run of layers over at most kFusedMaxRows rows as one persistent kernel (fused_layer.cu).
 constexpr int kFusedSyncInts = 16;
 constexpr int kFusedMaxRows = 64;   // row sets the fused kernel serves (its sum buffers' rows)
-// ES-dLLM per-layer re-selection inside the fused layer run (every layer of the run is
-// scored and re-chosen at its start).  Same definition as the score and select kernels:
+// ES-dLLM choice inside the fused layer run: the first n_scored layers of the run are scored
+// and the rows re-chosen at their start (1: the per-step choice at the skip layer; all: the
+// per-layer re-selection).  Same definition as the score and select kernels:
 // Eq. 1 on each candidate's layer input with the carry of skipped rows, the top k of each
 // sequence (ties to the lower position) in ascending position order.
 struct FusedEs {
   int on = 0;
+  int n_scored = 0;                  // layers of the run, from its first, that choose (1: per step)
   int ls = 0, L = 0;                 // skip layer, layers of the model
   int B = 0, n_cand = 0, cand_start = 0, k = 0;
   float alpha = 0.f;
