@@ -60,7 +60,7 @@ template <int BN>
 struct FCfg {
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr uint32_t kStageBytes = kKsub * (kABytes + kBBytes);
-  static constexpr int kFit = static_cast<int>((144u * 1024u) / kStageBytes);
+  static constexpr int kFit = static_cast<int>((160u * 1024u) / kStageBytes);
   static constexpr int kStages = kFit > 8 ? 8 : (kFit < 2 ? 2 : kFit);
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
