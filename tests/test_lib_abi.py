@@ -51,6 +51,7 @@ def test_state_bytes_covers_kv_cache(lib):
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 96, 3), ("gen_len", 33, 2), ("n_kv_heads", 3, 2), ("mask_id", 5000, 1),
     ("policy", 9, 1), ("keep_ratio", 0.0, 1), ("skip_layer", 99, 1), ("vocab", 1000, 3),
+    ("es_per_layer", 2, 1), ("lock_masked", 2, 1), ("layer_kernel", 7, 1), ("unmask", 9, 1),
 ])
 def test_invalid_configs_are_rejected(lib, field, value, status):
     cfg = _lib.make_config(get_config("tiny"))
@@ -76,3 +77,37 @@ def test_null_arguments_are_rejected_without_a_gpu(lib):
     cfg = _lib.make_config(get_config("tiny"))
     assert lib.dllm_step_init(ctypes.byref(h), ctypes.byref(cfg), None, None, None, None, None) == 1
     assert lib.dllm_op_select(None, 1, 4, 0, 2, 0.0, 0, 4, None, None, 0, None, None, None, None) == 1
+
+
+def test_per_layer_selection_needs_a_layer_after_the_skip_layer(lib):
+    run = get_config("tiny").replace(es_per_layer=True)
+    sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+    cfg = _lib.make_config(run.replace(skip_layer=run.model.n_layers))
+    assert lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb)) == 1
+    cfg = _lib.make_config(run.replace(skip_layer=run.model.n_layers - 1))
+    assert lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb)) == 0
+
+
+def test_per_layer_state_holds_one_input_snapshot_per_layer_above_the_skip_layer(lib):
+    # the per-layer choice keeps, for every layer above the skip layer, each row's input of
+    # that layer last iteration: (L - L_s - 1) fp32 [B*N, d] slabs more than the per-step choice
+    run = get_config("llada_es")
+    m = run.model
+    sizes = []
+    for per_layer in (False, True):
+        cfg = _lib.make_config(run.replace(es_per_layer=per_layer))
+        sb, wb = ctypes.c_size_t(), ctypes.c_size_t()
+        assert lib.dllm_state_bytes(ctypes.byref(cfg), ctypes.byref(sb), ctypes.byref(wb)) == 0
+        sizes.append((sb.value, wb.value))
+    slab = run.batch * run.seq_len * m.d_model * 4
+    extra = (m.n_layers - run.skip_layer - 1) * slab
+    assert extra <= sizes[1][0] - sizes[0][0] <= extra + 4096
+    assert sizes[1][1] == sizes[0][1]
+
+
+def test_step_calls_reject_a_null_handle_without_a_gpu(lib):
+    assert lib.dllm_begin_step(None, None, None) == 1
+    assert lib.dllm_select_active(None, None, None, None, None) == 1
+    assert lib.dllm_select_layers_forward(None, None, None) == 1
+    assert lib.dllm_layers_forward(None, 0, 1, None) == 1
+    assert lib.dllm_unmask(None, None, None, None, None) == 1
