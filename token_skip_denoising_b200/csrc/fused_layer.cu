@@ -191,7 +191,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* attn_smem = smem + C::kStages * C::kStageBytes;
-  int* s_rows = reinterpret_cast<int*>(attn_smem + C::kAttnBytes);   // [32]
+  int* s_rows = reinterpret_cast<int*>(attn_smem + C::kAttnBytes);   // [kMaxRows]
   float* s_rinv1 = reinterpret_cast<float*>(s_rows + kMaxRows);       // 1/rms before attention
   float* s_rinv2 = s_rinv1 + kMaxRows;                                // 1/rms before the FFN
   float* s_ss = s_rinv2 + kMaxRows;                                   // partial sums of squares

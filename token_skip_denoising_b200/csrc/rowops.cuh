@@ -138,8 +138,9 @@ struct FusedLayerArgs {
   size_t attn_floats;
   int* attn_ctr;           // fused_attn_counters(...) ints, zero before the launch; left zero
   int n_attn_ctr;
-  float* scratch;          // fused_scratch_floats(qkvd, F): fp32 QKV (2 buffers) and gate/up sums;
-                           // zero before the first launch, the kernel leaves it zero
+  float* scratch;          // fused_scratch_floats(qkvd, F): fp32 QKV and gate/up sums, per-CTA partial
+                           // sums of squares, the ES choice's row sums; zero before the first launch,
+                           // the kernel leaves it zero
   int* sync;               // kFusedSyncInts counters, zero before the launch; the kernel leaves them zero
   FusedEs es;              // per-layer re-selection (es.on = 0: the row map is fixed)
 };
