@@ -147,25 +147,47 @@ int dllm_device_status(int32_t* status, int32_t reset);
 /* Bytes of caller-allocated device memory a configuration needs: `state`
  * persists across steps (K/V cache, hidden snapshots, confidences, locks,
  * stored distributions, per-layer output cache), `workspace` is scratch for
- * one step.  Both must be 256-byte aligned.  Validates the configuration. */
+ * one step.  Both must be 256-byte aligned.  Validates the configuration.
+ * What persists follows what each policy keeps between iterations: ES-dLLM
+ * sec. 2.1 (the skip layer's hidden state and confidence of the previous
+ * iteration, the partially updated K/V cache), SureLock sec. 2.1 (the lock
+ * flags and the previous step's distribution of every lock-eligible row, the
+ * frozen K/V), the dLLM-Cache explainer sec. 3 (per-layer cached outputs).
+ * state_bytes / workspace_bytes must be non-null; returns
+ * DLLM_ERR_INVALID_ARG / _SHAPE / _UNSUPPORTED for a configuration the
+ * library cannot serve.  Host only: launches nothing. */
 int dllm_state_bytes(const dllm_config* cfg, size_t* state_bytes, size_t* workspace_bytes);
 
 /* Creates a handle over caller memory and zero-initialises the caches.
  * tokens: device int32 [B, N], the prompt followed by mask ids; updated in
- * place by every step.  Enqueued on `stream`. */
+ * place by every step.  Enqueued on `stream`.
+ * The start of a generation as the pages describe it: the prompt is followed
+ * by masked positions that the iterations unmask (ES-dLLM sec. 1; Plan for
+ * Speed sec. 2, blocks generated in order).  state / workspace must hold the
+ * sizes dllm_state_bytes gives, 256-byte aligned, else DLLM_ERR_INVALID_ARG;
+ * every pointer must stay valid until dllm_destroy.  Synchronises `stream`
+ * once (the host copy of the DUS round masks must outlive its upload). */
 int dllm_step_init(dllm_handle** out, const dllm_config* cfg, const dllm_weights* w, void* state, void* workspace,
                    int32_t* tokens, void* stream);
 
 /* Starts one denoising step: decides from the schedule whether it is a full
  * refresh (ES-dLLM sec. 2.2; dLLM-Cache prompt interval), chooses the rows
  * that enter layer 0 (all rows; the current block; SureLock's unlocked rows)
- * and gathers their embeddings.  *kind_out (nullable) gets DLLM_STEP_*. */
+ * and gathers their embeddings.  *kind_out (nullable) gets DLLM_STEP_*.
+ * DLLM_ERR_STATE once every block is finished.  Asynchronous on `stream`. */
 int dllm_begin_step(dllm_handle* h, int32_t* kind_out, void* stream);
 
 /* Runs one transformer layer for the current row set, in place: new K/V rows
  * are written into the cache before attention, attention reads all N cached
  * rows of the sequence.  Under dLLM-Cache the layer first scores the response
- * rows by value-vector cosine and recomputes only the selected ones. */
+ * rows by value-vector cosine and recomputes only the selected ones.
+ * Follows ES-dLLM sec. 2.1 item 3 (the computed rows' K/V are updated in
+ * place in the cache, the skipped rows' entries are kept), SureLock sec. 2.1
+ * item 3 (active queries attend over all positions, locked ones through their
+ * frozen K/V) and the dLLM-Cache explainer sec. 3 (per-layer partial update of
+ * the response rows).  layer in [0, n_layers) else DLLM_ERR_INVALID_ARG;
+ * DLLM_ERR_STATE before dllm_begin_step or out of the per-layer selection
+ * order.  Asynchronous on `stream`; reads and writes only caller memory. */
 int dllm_layer_forward(dllm_handle* h, int32_t layer, void* stream);
 
 /* Runs layers l0 .. l1-1 for the current row set, with the same result as
@@ -213,11 +235,25 @@ int dllm_select_layers_forward(dllm_handle* h, const float* scores_or_null, void
  * argmax (mask id excluded), SureLock's KL and locking, and unmasking
  * (top-n confidence, or the DUS round).  pos_out / tok_out (device int32
  * [B, max(n, round size)]) and n_out (device int32 [B]) are optional.
- * Advances the schedule. */
+ * Advances the schedule.
+ * Follows ES-dLLM sec. 1 (a few tokens of highest confidence are unmasked per
+ * iteration; the confidences are stored for the next iteration's Eq. 1),
+ * SureLock sec. 2.1 items 1-2 (KL(p_t || p_t-1) per position from the step's
+ * logits and the stored ones; lock when KL < eps and the confidence > tau) and
+ * Plan for Speed sec. 2 (the round's dilated group is unmasked together).
+ * DLLM_ERR_STATE before dllm_begin_step or with per-layer choices left; with
+ * the CB_DUS unmasking the call reads B ints back and synchronises `stream`,
+ * otherwise it is asynchronous. */
 int dllm_unmask(dllm_handle* h, int32_t* pos_out, int32_t* tok_out, int32_t* n_out, void* stream);
 
 /* One whole denoising step (begin, layers, selection, unmask).  With `info`
- * non-null the call synchronises the stream and fills it. */
+ * non-null the call synchronises the stream and fills it.
+ * The iteration of the pages: choose the rows to compute (ES-dLLM sec. 2.1
+ * Eq. 1 and early skip; SureLock sec. 2.1 locks; dLLM-Cache sec. 3 similarity
+ * gate), compute them over the cached K/V, unmask; refresh steps per ES-dLLM
+ * sec. 2.2 and the dLLM-Cache prompt interval.  DLLM_ERR_STATE once
+ * dllm_done() is 1; a failing call leaves the step unfinished (the handle
+ * stays valid; dllm_reset starts over). */
 int dllm_step(dllm_handle* h, dllm_step_info* info_or_null, void* stream);
 
 /* Host-side schedule: 1 when every block is finished. */
@@ -231,7 +267,11 @@ int dllm_done(const dllm_handle* h);
 int dllm_set_lock_pattern(dllm_handle* h, const uint8_t* pattern);
 
 /* Starts a new generation on the same handle: zeroes the caches and rewinds
- * the schedule, asynchronously on `stream` (the caller rewrites `tokens`). */
+ * the schedule, asynchronously on `stream` (the caller rewrites `tokens`).
+ * It also clears the GEMM tile and attention split counters of the workspace:
+ * every launch leaves them at zero except one that gave up a wait, so after
+ * dllm_device_status reports DLLM_DEV_TIMEOUT call dllm_reset (or destroy the
+ * handle) before further steps. */
 int dllm_reset(dllm_handle* h, void* stream);
 
 /* Per-kernel timing of the fused GEMMs and the attention, for roofline
@@ -251,6 +291,38 @@ typedef struct dllm_profile {
 } dllm_profile;
 int dllm_profile_enable(dllm_handle* h, int32_t enable, double hbm_gbs, double tensor_tflops);
 int dllm_profile_read(dllm_handle* h, dllm_profile* out);
+
+/* Position of the generation schedule (host state of a handle).  Together with the
+ * caller-owned `state` buffer and the token buffer it is the whole generation state:
+ * copying state and tokens to a fresh handle of the same configuration and setting
+ * its progress resumes the generation exactly (checkpoint / resume).  The pages have
+ * no counterpart; this is a facility of this library. */
+typedef struct dllm_progress {
+  int32_t step;           /* steps run so far */
+  int32_t block;          /* current block */
+  int32_t step_in_block;  /* steps run in it */
+} dllm_progress;
+/* Reads the schedule position; valid between steps. */
+int dllm_get_progress(const dllm_handle* h, dllm_progress* out);
+/* Sets it (between steps): DLLM_ERR_INVALID_ARG for a position outside the schedule of
+ * the configuration, DLLM_ERR_STATE in the middle of a step. */
+int dllm_set_progress(dllm_handle* h, const dllm_progress* p);
+
+/* dLLM-Cache teacher forcing: with a device fp32 [L, B, n_resp] array the partial
+ * steps choose each layer's rows from these similarities instead of the cosine of
+ * the value vectors (n_resp = gen_len, or prompt_len + gen_len over all rows); the
+ * cosine is still computed and left in DLLM_BUF_SCORES.  The threshold, the cap and
+ * the tie rule are those of the dLLM-Cache explainer sec. 3 as configured.  NULL
+ * restores the cosine; the array must outlive the handle's steps.
+ * DLLM_ERR_STATE outside the dLLM-Cache policy. */
+int dllm_set_forced_similarities(dllm_handle* h, const float* sims);
+
+/* Poll limit of the grid-wide waits of the fused layer kernel (0: the default, about
+ * 0.4 s).  Failure-detection tests lower it so that a wait they make unsatisfiable
+ * (DLLM_BUF_FUSED_SYNC) runs out quickly: the kernel then records DLLM_DEV_TIMEOUT,
+ * stops its work, waits for its own copies in flight, frees its tensor memory and
+ * returns, and the next launch starts clean.  The pages have no counterpart. */
+int dllm_set_wait_limit(dllm_handle* h, uint32_t polls);
 
 /* Number of CUDA kernels this library has launched in the process so far. */
 int64_t dllm_kernel_launches(void);
@@ -281,10 +353,24 @@ enum {
                                layer keeps g * h there and scales the sums by 1/rms instead) */
   DLLM_BUF_LAYER_Q = 19,    /* bf16 [rows, Hq*hd] rotated queries */
   DLLM_BUF_LAYER_ATTN = 20, /* bf16 [rows, Hq*hd] attention output */
-  DLLM_BUF_LAYER_ACT = 21   /* bf16 [rows, F] SwiGLU activation */
+  DLLM_BUF_LAYER_ACT = 21,  /* bf16 [rows, F] SwiGLU activation */
+  DLLM_BUF_ES_IN = 22,      /* fp32 [L - skip_layer - 1, B*N, d] per-layer ES: each candidate's input
+                               of layer skip_layer + 1 + i in the last iteration that scored it */
+  DLLM_BUF_ZSTORE = 23,     /* bf16 [2, B*N, V] SureLock: stored logits, buffer (step & 1) written
+                               by step `step` */
+  DLLM_BUF_LSE_STORE = 24,  /* fp32 [2, B*N] their log-sum-exp */
+  DLLM_BUF_STAMP = 25,      /* int32 [B*N] step + 1 of the last stored distribution per position */
+  DLLM_BUF_VNEW = 26,       /* fp32 [B*n_resp, Hkv*hd] dLLM-Cache: value vectors of the last layer's probe */
+  DLLM_BUF_FUSED_SYNC = 27  /* int32 [16] phase counters of the fused layer kernel, zero between launches;
+                               element 0 gates every CTA's first QKV step of a launch */
 };
 int dllm_get_buffer(dllm_handle* h, int32_t which, void** ptr, size_t* bytes);
 
+/* Frees the handle's host metadata (the pages have no counterpart: ownership
+ * rule of this library).  Caller memory (weights, tokens, state, workspace)
+ * is not touched and stays owned by the caller; NULL is a no-op.  Kernels
+ * already enqueued keep running: synchronise the stream first if the caller
+ * frees its buffers next. */
 void dllm_destroy(dllm_handle* h);
 
 /* ------------------------------------------------------------------ ops
@@ -292,7 +378,8 @@ void dllm_destroy(dllm_handle* h);
  * single-layer microbenchmark).  Device pointers, stream as above.
  * `workspace` (where taken) is caller scratch: zero it before its first use;
  * its first 256 KB hold GEMM tile counters that every call leaves at zero, so
- * calls on one stream may share it; calls that overlap on the GPU may not.  */
+ * calls on one stream may share it; calls that overlap on the GPU may not.
+ * After dllm_device_status reports DLLM_DEV_TIMEOUT, zero it again.  */
 
 /* RoPE tables cos/sin fp32 [N, hd/2] with angle pos * theta^(-2i/hd). */
 int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, double theta, void* stream);

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle.policy import es_importance, topk_select
 from oracle.steps import OracleRun
 from synth import get_config, make_tokens, make_weights
 from synth.configs import scaled
@@ -26,6 +27,23 @@ DEV = "cuda"
 BASE = scaled(get_config("tiny"), n_layers=4)
 PL = BASE.replace(es_per_layer=True, skip_layer=1)
 TOL_HIDDEN = 2e-2
+
+
+TOL_SCORE = 1e-4     # Eq. 1 in fp32 on the GPU's own inputs
+
+
+def _c_term(eng, flat):
+    idx = torch.tensor(flat, device=DEV)
+    return np.where(eng.buffer("masked_prev")[idx].cpu().numpy() != 0,
+                    eng.buffer("conf")[idx].double().cpu().numpy(), 0.0)
+
+
+def _prev_input(eng, l, ls, flat):
+    """The GPU's record of each candidate's input of layer l in the last iteration."""
+    idx = torch.tensor(flat, device=DEV)
+    if l == ls:
+        return eng.buffer("hprev")[idx].double().cpu().numpy()
+    return eng.buffer("es_in")[l - ls - 1][idx].double().cpu().numpy()
 
 
 def _rowrel(a, b):
@@ -62,18 +80,24 @@ def test_per_layer_steps_match_oracle_teacher_forced(w4, layer_kernel, batch):
         rec = orc.step()
         kind = eng.begin_step()
         assert kind == ("full" if rec["kind"] == "refresh" else "skip")
+        if kind == "skip":
+            c_g = _c_term(eng, _flat(*rec["cand"], N))     # masked_prev rolls forward at the last layer
         for l in range(L):
             if l >= ls:
                 if kind == "skip":
                     j = l - ls
                     flat = _flat(*rec["cand"], N)
+                    prev = _prev_input(eng, l, ls, flat)
                     eng.select_active(torch.tensor(rec["layer_scores"][j], dtype=torch.float32, device=DEV))
                     # every candidate's input of this layer, skipped rows carrying their cached output
                     hx = hid[torch.tensor(flat, device=DEV)].cpu().numpy()
                     assert _rowrel(hx, rec["layer_in"][j]) < TOL_HIDDEN
                     gs = eng.buffer("scores")[:len(flat)].cpu().numpy().astype(np.float64)
                     ref = rec["layer_scores"][j]
-                    assert np.abs(gs - ref).max() <= 0.1 * np.abs(ref).max()
+                    # Eq. 1 element by element on the GPU's own input of this layer and its record of
+                    # the previous iteration's
+                    np.testing.assert_allclose(gs, es_importance(cfg.alpha, c_g, hx.astype(np.float64), prev),
+                                               rtol=TOL_SCORE, atol=1e-7)
                     if j:
                         # rows the previous layer skipped: variation exactly zero, confidence term only
                         skipped = np.setdiff1d(np.arange(len(flat)), rec["layer_active"][j - 1])
@@ -168,6 +192,9 @@ def test_fused_per_layer_run_matches_oracle_teacher_forced(w4, batch):
         forced = None
         if kind == "skip":
             forced = torch.tensor(np.stack(rec["layer_scores"]), dtype=torch.float32, device=DEV).contiguous()
+            cflat = _flat(*rec["cand"], N)
+            c_g = _c_term(eng, cflat)
+            prev_last = _prev_input(eng, L - 1, ls, cflat)
         torch.cuda.synchronize()
         n0 = kernel_launches()
         eng.select_layers_forward(forced)
@@ -175,8 +202,12 @@ def test_fused_per_layer_run_matches_oracle_teacher_forced(w4, batch):
         if kind == "skip":
             assert kernel_launches() - n0 == 2            # the row counts, then one fused launch
             gs = eng.buffer("scores")[:len(rec["cand"][0])].cpu().numpy().astype(np.float64)
-            ref = rec["layer_scores"][-1]
-            assert np.abs(gs - ref).max() <= 0.1 * np.abs(ref).max()
+            # the last layer's in-kernel Eq. 1, element by element: its input is what the run left in
+            # the per-layer record, the previous iteration's what the record held before the run
+            cur_last = _prev_input(eng, L - 1, ls, cflat)
+            np.testing.assert_allclose(gs, es_importance(cfg.alpha, c_g, cur_last, prev_last),
+                                       rtol=TOL_SCORE, atol=1e-7)
+            assert _rowrel(cur_last, rec["layer_in"][-1]) < TOL_HIDDEN
             n_skip += 1
         rows = eng.buffer("rows")
         nrows = int(eng.buffer("nrows")[0])
@@ -233,6 +264,38 @@ def test_fused_per_layer_run_with_differing_forced_choices(w4):
         assert set(np.nonzero(changed)[0].tolist()) <= set(chosen.tolist())
         assert _rowrel(k1[l].float().cpu().numpy().reshape(-1, cfg.model.head_dim),
                        orc.K[l].reshape(-1, cfg.model.head_dim)) < 2e-2
+
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_fused_per_layer_choice_on_its_own_scores_is_the_top_k(w4, batch):
+    """No teacher forcing: after each fused per-layer run, the last layer's scores match Eq. 1
+    on the GPU's own inputs of that layer and the rows it kept are the top k of those scores,
+    bit for bit."""
+    cfg = PL.replace(batch=batch)
+    eng = Engine(cfg, _dev(w4), make_tokens(cfg).to(DEV).contiguous())
+    N, L, ls, n = cfg.seq_len, cfg.model.n_layers, cfg.skip_layer, cfg.block_len
+    k = cfg.keep_count(n)
+    n_skip = 0
+    while not eng.done:
+        kind = eng.begin_step()
+        eng.layers_forward(0, ls)
+        if kind == "skip":
+            s0 = cfg.prompt_len + eng.progress()["block"] * cfg.block_len
+            cflat = np.concatenate([b * N + s0 + np.arange(n) for b in range(cfg.batch)])
+            c_g = _c_term(eng, cflat)
+            prev_last = _prev_input(eng, L - 1, ls, cflat)
+        eng.select_layers_forward()
+        torch.cuda.synchronize()
+        if kind == "skip":
+            gs = eng.buffer("scores")[:cfg.batch * n].cpu().numpy().astype(np.float64)
+            cur_last = _prev_input(eng, L - 1, ls, cflat)
+            np.testing.assert_allclose(gs, es_importance(cfg.alpha, c_g, cur_last, prev_last),
+                                       rtol=TOL_SCORE, atol=1e-7)
+            want = np.concatenate([b * N + s0 + topk_select(gs[b * n:(b + 1) * n], k) for b in range(cfg.batch)])
+            np.testing.assert_array_equal(eng.buffer("rows")[:cfg.batch * k].cpu().numpy(), want)
+            n_skip += 1
+        eng.unmask()
+    assert n_skip == 7
 
 
 def test_keep_all_per_layer_equals_vanilla(w4):

@@ -19,6 +19,7 @@ if torch.cuda.is_available():
     from token_skip_denoising_b200.engine import Engine, device_status
 
 TOL = 2e-2
+TOL_CONF = 5e-2
 
 
 def _rel(a, b):
@@ -80,7 +81,12 @@ def test_fused_layer_matches_split_layer(name):
     for e in (A, B):
         e.unmask()
     torch.cuda.synchronize()
-    assert torch.equal(A.tokens, B.tokens) or _rel(B.buffer("conf"), A.buffer("conf")) < TOL
+    # the fused sums land in a different order, so a near-tie between two confidences may
+    # resolve differently: the confidences themselves are compared.  conf = exp(z_max - lse):
+    # a relative error e of the hidden rows moves the logits by about e * |z| (|z| up to ~2 std
+    # here), so conf carries about twice the hidden-state tolerance -- the 5e-2 that every
+    # confidence comparison with the oracle uses
+    assert _rel(B.buffer("conf"), A.buffer("conf")) < TOL_CONF
     assert device_status() == 0
 
 

@@ -81,9 +81,12 @@ def test_layer_matches_oracle(dims, B, N, rows, layer_kernel):
         assert _rowrel(vg[b, :, p].reshape(1, -1), V[b, :, p].reshape(1, -1)) < 1e-2
 
 
-@pytest.mark.parametrize("dims,N,rows", [(LLADA8B, 768, [7]), (LLADA8B, 768, [32]), (DREAM7B, 1536, [9])])
+@pytest.mark.parametrize("dims,N,rows", [(LLADA8B, 768, [7]), (LLADA8B, 768, [32]), (DREAM7B, 1536, [9]),
+                                         (LLADA8B, 768, [768]), (DREAM7B, 1536, [1536]), (LLADA8B, 2048, [205])])
 def test_layer_full_width(dims, N, rows):
-    """LLaDA-8B / Dream-7B layer width with the row counts of the ES skip step."""
+    """LLaDA-8B / Dream-7B layer width with the row counts of the ES skip step, of a refresh
+    (every row: 128-wide GEMM tiles and 768 x 768 attention for LLaDA, 256-wide tiles and GQA
+    28/4 over 1536 x 1536 for Dream) and of the single-layer microbenchmark at active ratio 0.1."""
     d1 = ModelDims(n_layers=1, d_model=dims.d_model, n_heads=dims.n_heads, n_kv_heads=dims.n_kv_heads,
                    head_dim=dims.head_dim, ffn_dim=dims.ffn_dim, vocab=1024, mask_id=1023,
                    rope_theta=dims.rope_theta)

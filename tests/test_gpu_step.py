@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle.policy import es_importance, topk_select
 from oracle.steps import OracleRun
 from synth import get_config, make_tokens, make_weights
 
@@ -21,6 +22,25 @@ if torch.cuda.is_available():
 DEV = "cuda"
 TINY = get_config("tiny")
 TOL_HIDDEN = 2e-2
+
+
+TOL_SCORE = 1e-4     # Eq. 1 in fp32 on the GPU's own inputs: relative to each score
+
+
+def _eq1_inputs(eng, flat):
+    """The GPU's own Eq. 1 inputs for the candidate rows `flat`: current hidden state at the
+    skip layer, the snapshot of the previous iteration, and c = conf if the row was masked at
+    the start of the previous step, else 0."""
+    idx = torch.tensor(flat, device=DEV)
+    h = eng.buffer("hidden")[idx].double().cpu().numpy()
+    hp = eng.buffer("hprev")[idx].double().cpu().numpy()
+    c = np.where(eng.buffer("masked_prev")[idx].cpu().numpy() != 0, eng.buffer("conf")[idx].double().cpu().numpy(),
+                 0.0)
+    return h, hp, c
+
+
+def _assert_scores(gs, want):
+    np.testing.assert_allclose(gs, want, rtol=TOL_SCORE, atol=1e-7)
 
 
 def _rowrel(a, b):
@@ -96,12 +116,12 @@ def test_es_steps_match_oracle_teacher_forced(tiny_w_cpu):
                     # hidden state of the candidates at the skip layer (Eq. 1 input)
                     hc = hid[torch.tensor(_flat(b_idx, pos, N), device=DEV)].cpu().numpy()
                     assert _rowrel(hc, rec["h_skip"]) < TOL_HIDDEN
+                    h_g, hp_g, c_g = _eq1_inputs(eng, _flat(b_idx, pos, N))
                     forced = torch.tensor(rec["scores"], dtype=torch.float32, device=DEV)
                     eng.select_active(forced)
-                    gpu_scores = eng.buffer("scores")[:len(rec["scores"])].cpu().numpy()
-                    # Eq. 1 on the bf16 path: the variation term differences two nearby states,
-                    # so compare against the score scale rather than element-wise
-                    assert np.abs(gpu_scores - rec["scores"]).max() <= 0.1 * np.abs(rec["scores"]).max()
+                    gpu_scores = eng.buffer("scores")[:len(rec["scores"])].double().cpu().numpy()
+                    # Eq. 1 element by element on the GPU's own inputs
+                    _assert_scores(gpu_scores, es_importance(cfg.alpha, c_g, h_g, hp_g))
                     n_skip += 1
                 else:
                     eng.select_active()
@@ -149,6 +169,7 @@ def test_es_choice_inside_the_fused_run_teacher_forced(tiny_w_cpu, batch):
         forced = None
         if kind == "skip":
             forced = torch.tensor(rec["scores"][None], dtype=torch.float32, device=DEV).contiguous()
+            h_g, hp_g, c_g = _eq1_inputs(eng, _flat(*rec["cand"], N))
         torch.cuda.synchronize()
         n0 = kernel_launches()
         eng.select_layers_forward(forced)
@@ -156,7 +177,8 @@ def test_es_choice_inside_the_fused_run_teacher_forced(tiny_w_cpu, batch):
         if kind == "skip":
             assert kernel_launches() - n0 == 2            # the row counts, then one fused launch
             gs = eng.buffer("scores")[:len(rec["scores"])].cpu().numpy().astype(np.float64)
-            assert np.abs(gs - rec["scores"]).max() <= 0.1 * np.abs(rec["scores"]).max()
+            # the in-kernel Eq. 1, element by element on the GPU's own inputs
+            _assert_scores(gs, es_importance(cfg.alpha, c_g, h_g, hp_g))
             n_skip += 1
         nrows = int(eng.buffer("nrows")[0])
         flat = _flat(*rec["rows"], N)
@@ -175,6 +197,43 @@ def test_es_choice_inside_the_fused_run_teacher_forced(tiny_w_cpu, batch):
         amax.copy_(torch.tensor(orc.amax.reshape(-1), dtype=torch.int32))
     assert n_skip == 7
     assert eng.done
+
+
+@pytest.mark.parametrize("path", ["fused", "split"])
+@pytest.mark.parametrize("batch", [1, 2])
+def test_es_choice_on_its_own_scores_is_the_top_k(tiny_w_cpu, path, batch):
+    """No teacher forcing: on every skip step the GPU's Eq. 1 scores match Eq. 1 evaluated on
+    the GPU's own inputs, and the kept rows are exactly the top k of those scores (ties to the
+    lower position), bit for bit: the in-kernel rank count of the fused run, and the radix
+    select of the split path."""
+    cfg = TINY.replace(batch=batch)
+    eng = _engine(cfg, tiny_w_cpu, make_tokens(cfg), layer_kernel=path)
+    N, ls, n = cfg.seq_len, cfg.skip_layer, cfg.block_len
+    k = cfg.keep_count(n)
+    n_skip = 0
+    while not eng.done:
+        kind = eng.begin_step()
+        eng.layers_forward(0, ls)
+        if kind == "skip":
+            s0 = cfg.prompt_len + eng.progress()["block"] * cfg.block_len
+            flat = np.concatenate([b * N + s0 + np.arange(n) for b in range(cfg.batch)])
+            h_g, hp_g, c_g = _eq1_inputs(eng, flat)
+        if path == "fused":
+            eng.select_layers_forward()
+        else:
+            eng.select_active()
+            eng.layers_forward(ls, cfg.model.n_layers)
+        torch.cuda.synchronize()
+        if kind == "skip":
+            gs = eng.buffer("scores")[:cfg.batch * n].cpu().numpy().astype(np.float64)
+            _assert_scores(gs, es_importance(cfg.alpha, c_g, h_g, hp_g))
+            want = np.concatenate([b * N + s0 + topk_select(gs[b * n:(b + 1) * n], k)
+                                   for b in range(cfg.batch)])
+            nrows = int(eng.buffer("nrows")[0])
+            np.testing.assert_array_equal(eng.buffer("rows")[:nrows].cpu().numpy(), want)
+            n_skip += 1
+        eng.unmask()
+    assert n_skip == 7
 
 
 def test_keep_all_equals_vanilla_on_gpu(tiny_w_cpu):

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle.policy import dus_schedule
+from oracle.policy import cosine_rows, dus_schedule, kl_from_logits, threshold_cap_select
 from oracle.steps import OracleRun
 from synth import get_config, make_tokens, make_weights
 
@@ -73,19 +73,79 @@ def test_surelock_steps_match_oracle_with_lock_pattern(tiny_w, lock_masked):
         assert _rowrel(hid[torch.tensor(flat, device=DEV)].cpu().numpy(), rec["h_out"]) < TOL_HIDDEN
         np.testing.assert_array_equal(eng.buffer("lock").cpu().numpy().reshape(cfg.batch, N),
                                       orc.lock.astype(np.uint8))
-        # KL of the eligible rows that had a previous distribution
+        # KL of the eligible rows that had a previous distribution: present exactly where the
+        # oracle has one, and equal to KL(p_t || p_t-1) of the GPU's own two stored bf16 logit rows
         n_lm = int(eng.buffer("nlmrows")[0])
         assert n_lm == len(rec["lm_rows"])
-        kl_g = eng.buffer("kl")[:n_lm].cpu().numpy()
-        ok = ~np.isnan(rec["kl"])
-        if ok.any():
-            np.testing.assert_allclose(kl_g[ok], rec["kl"][ok], rtol=0.1, atol=2e-3)
+        kl_g = eng.buffer("kl")[:n_lm].cpu().numpy().astype(np.float64)
+        ok = ~np.isnan(rec["kl"])            # the oracle's: eligible rows with a previous distribution
+        assert not np.isnan(kl_g[ok]).any()  # (the GPU also reports it for masked rows that have one)
+        has = ~np.isnan(kl_g)
+        if has.any():
+            _check_kl_on_own_logits(eng, info["step"], eng.buffer("lmrows")[:n_lm].cpu().numpy()[has], kl_g[has])
         lm = flat[rec["lm_rows"]]
         np.testing.assert_allclose(eng.buffer("conf")[torch.tensor(lm, device=DEV)].cpu().numpy(),
                                    orc.conf.reshape(-1)[lm], rtol=5e-2, atol=1e-5)
         locked_max = max(locked_max, int(orc.lock.sum()))
         _force(eng, orc)
     assert locked_max > 10 and eng.done
+
+
+TOL_KL_REL, TOL_KL_ABS = 1e-3, 1e-5     # well below the lock threshold eps = 1e-3
+
+
+def _check_kl_on_own_logits(eng, step, flat, kl_gpu):
+    """KL(p_t || p_t-1) in fp64 from the bf16 logits the GPU stored at steps t and t-1."""
+    z = eng.buffer("zstore")
+    cur = z[step & 1][torch.tensor(flat, device=DEV)].double().cpu().numpy()
+    prv = z[(step + 1) & 1][torch.tensor(flat, device=DEV)].double().cpu().numpy()
+
+    def lse(a):
+        mx = a.max(1, keepdims=True)
+        return (mx + np.log(np.exp(a - mx).sum(1, keepdims=True)))[:, 0]
+    want = kl_from_logits(cur, lse(cur), prv, lse(prv))
+    np.testing.assert_allclose(kl_gpu, want, rtol=TOL_KL_REL, atol=TOL_KL_ABS)
+
+
+@pytest.mark.parametrize("lock_masked", [False, True])
+def test_surelock_kl_rule_decisions(tiny_w, lock_masked):
+    """The lock rule itself (no pattern), teacher-forced on the oracle's tokens:
+    * kl_eps = 1e30, conf_tau = -1 makes the rule true wherever a KL exists, so the locks do not
+      depend on floating point: the GPU's lock flags equal the oracle's at every step;
+    * kl_eps = 1e-3: every LM row's decision equals "KL < eps and conf > tau" on the GPU's own
+      KL and confidence (the decision is taken in the kernel's fp32 on both sides), and the KL
+      equals fp64 KL of the GPU's stored logits to 1e-3 relative / 1e-5 absolute."""
+    for eps, tau in ((1e30, -1.0), (1e-3, -1.0)):
+        cfg = TINY.replace(policy="surelock", tokens_per_step=2, kl_eps=eps, conf_tau=tau, lock_masked=lock_masked)
+        N = cfg.seq_len
+        tok0 = make_tokens(cfg)
+        orc = OracleRun(cfg, tiny_w, tok0.numpy())
+        eng = Engine(cfg, _dev(tiny_w), tok0.to(DEV).contiguous())
+        n_new = 0
+        while not orc.done:
+            lock0 = eng.buffer("lock").cpu().numpy().copy()
+            tok_before = eng.tokens.cpu().numpy().reshape(-1).copy()
+            orc.step()
+            info = eng.step(info=True)
+            lock1 = eng.buffer("lock").cpu().numpy()
+            n_lm = int(eng.buffer("nlmrows")[0])
+            flat = eng.buffer("lmrows")[:n_lm].cpu().numpy()
+            kl_g = eng.buffer("kl")[:n_lm].cpu().numpy()
+            conf_g = eng.buffer("conf")[torch.tensor(flat, device=DEV)].cpu().numpy()
+            has = ~np.isnan(kl_g)
+            if has.any():
+                _check_kl_on_own_logits(eng, info["step"], flat[has], kl_g[has].astype(np.float64))
+            if eps > 1e29:
+                np.testing.assert_array_equal(lock1.reshape(cfg.batch, N), orc.lock.astype(np.uint8))
+            else:
+                eligible = np.ones(n_lm, bool) if lock_masked else tok_before[flat] != cfg.model.mask_id
+                rule = eligible & has & (kl_g < np.float32(eps)) & (conf_g > np.float32(tau))
+                np.testing.assert_array_equal(lock1[flat] != 0, (lock0[flat] != 0) | rule)
+            n_new += int((lock1 != lock0).sum())
+            _force(eng, orc)
+            eng.buffer("lock").copy_(torch.tensor(orc.lock.reshape(-1).astype(np.uint8)))
+        if eps > 1e29:
+            assert n_new > 10
 
 
 def test_surelock_eps_zero_never_locks(tiny_w):
@@ -128,6 +188,79 @@ def test_dllm_cache_full_selection_matches_oracle(tiny_w):
         n_partial += kind == "partial"
         _force(eng, orc)
     assert n_partial > 0 and eng.done
+
+
+def _check_cos_on_own_values(eng, cfg, vcache_before):
+    """The GPU's cosine scores of a layer against fp64 cosine of its own value vectors and the
+    cached V rows the layer read."""
+    n = cfg.gen_len
+    N = cfg.seq_len
+    sims = eng.buffer("scores")[:cfg.batch * n].double().cpu().numpy()
+    vnew = eng.buffer("vnew")[:cfg.batch * n].double().cpu().numpy()
+    flat = np.concatenate([b * N + cfg.prompt_len + np.arange(n) for b in range(cfg.batch)])
+    vc = vcache_before.double().cpu().numpy()             # [B, Hkv, N, hd]
+    vrows = vc[flat // N, :, flat % N, :].reshape(len(flat), -1)
+    np.testing.assert_allclose(sims, cosine_rows(vnew, vrows), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("forced", [False, True])
+def test_dllm_cache_capped_selection_teacher_forced(tiny_w, forced):
+    """dLLM-Cache with tau = 0.95 and rho = 0.25: the oracle's per-layer similarities are fed to
+    the GPU's selection (dllm_set_forced_similarities), and the rows chosen at every layer equal
+    the oracle's, bit for bit; outputs agree within tolerance and the GPU's own cosine equals
+    fp64 cosine of its own value vectors.  forced=True uses similarities where both the
+    threshold and the cap bind (12 of 32 rows below 0.5, cap 8)."""
+    cfg = TINY.replace(policy="dllm_cache", sim_tau=0.5 if forced else 0.95, rho_cap=0.25,
+                       prompt_interval=5, tokens_per_step=2, batch=2)
+    N, L, n = cfg.seq_len, cfg.model.n_layers, cfg.gen_len
+    tok0 = make_tokens(cfg)
+    orc = OracleRun(cfg, tiny_w, tok0.numpy())
+    eng = Engine(cfg, _dev(tiny_w), tok0.to(DEV).contiguous())
+    fsims = torch.zeros((L, cfg.batch, n), dtype=torch.float32, device=DEV)
+    eng.set_forced_similarities(fsims)
+    cap = math.ceil(cfg.rho_cap * n - 1e-9)
+    rng = np.random.default_rng(5)
+    n_partial = n_capped = 0
+    while not orc.done:
+        fs = None
+        if forced and orc.n_steps % cfg.prompt_interval:
+            fs = []
+            for l in range(L):
+                sims = np.full(cfg.batch * n, 0.9)
+                for b in range(cfg.batch):
+                    low = rng.choice(n, 12, replace=False)
+                    sims[b * n + low] = rng.permutation(np.linspace(0.05, 0.45, 12))
+                fs.append(sims)
+        rec = orc.step(forced_scores=fs)
+        kind = eng.begin_step()
+        assert kind == ("full" if rec["kind"] == "refresh" else "partial")
+        if kind == "partial":
+            fsims.copy_(torch.tensor(np.stack([lay["sims"] for lay in rec["layers"]]).reshape(L, cfg.batch, n)))
+        for l in range(L):
+            vc0 = eng.buffer("vcache")[l].clone()
+            eng.layer_forward(l)
+            if kind == "partial":
+                want = rec["layers"][l]["sel"]
+                nsel = int(eng.buffer("nsel")[0])
+                got = eng.buffer("selrows")[:nsel].cpu().numpy()
+                np.testing.assert_array_equal(got, (want // n) * N + cfg.prompt_len + want % n)
+                for b in range(cfg.batch):
+                    sims_b = rec["layers"][l]["sims"][b * n:(b + 1) * n]
+                    np.testing.assert_array_equal(
+                        np.sort(want[(want >= b * n) & (want < (b + 1) * n)] - b * n),
+                        threshold_cap_select(sims_b, cfg.sim_tau, cap))
+                    n_capped += int((np.asarray(sims_b) < cfg.sim_tau).sum() > cap)
+                _check_cos_on_own_values(eng, cfg, vc0)
+        eng.unmask()
+        torch.cuda.synchronize()
+        b_idx, pos = rec["rows"]
+        got = eng.buffer("hcache")[L - 1][torch.tensor(b_idx * N + pos, device=DEV)].cpu().numpy()
+        assert _rowrel(got, rec["h_out"]) < TOL_HIDDEN
+        n_partial += kind == "partial"
+        _force(eng, orc)
+    assert n_partial > 0 and eng.done
+    if forced:
+        assert n_capped > 0
 
 
 def test_dllm_cache_dus_generation(tiny_w):

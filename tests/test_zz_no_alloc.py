@@ -47,6 +47,25 @@ def test_noalloc_matches_workspace_gemm_on_two_calls(lib, rows, n_out, K):
         _noalloc(lib, 0, W, X, got)
         torch.cuda.synchronize()
         assert _rowrel(got.cpu().numpy(), ref.cpu().numpy()) < 1e-4, f"call {call}"
+        # and the definition itself, X W^T in fp64 on the same bf16 operands
+        exact = X.cpu().double().numpy() @ W.cpu().double().numpy().T
+        assert _rowrel(got.cpu().numpy(), exact) < 1e-4, f"call {call}"
+
+
+def test_noalloc_bf16_output_on_split_tiles(lib):
+    """kind 1 (bf16 store) at the shape whose tiles are split across CTAs (12288 x 4096)."""
+    from token_skip_denoising_b200 import ops
+    g = torch.Generator(device=DEV).manual_seed(11)
+    for call in range(2):
+        W = (torch.randn((12288, 4096), generator=g, device=DEV) * 0.05).to(torch.bfloat16)
+        X = torch.randn((32, 4096), generator=g, device=DEV).to(torch.bfloat16)
+        ref = ops.gemm(W, X, kind=1)
+        got = torch.zeros((32, 12288), dtype=torch.bfloat16, device=DEV)
+        _noalloc(lib, 1, W, X, got)
+        torch.cuda.synchronize()
+        exact = X.cpu().double().numpy() @ W.cpu().double().numpy().T
+        assert _rowrel(got.float().cpu().numpy(), ref.float().cpu().numpy()) < 2 ** -8, f"call {call}"
+        assert _rowrel(got.float().cpu().numpy(), exact) < 2 ** -8, f"call {call}"
 
 
 def test_noalloc_residual_with_device_count(lib):

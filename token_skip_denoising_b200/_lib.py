@@ -30,7 +30,8 @@ SCOPE = {"block": 0, "all": 1}
 STEP_KIND = {0: "full", 1: "skip", 2: "locked", 3: "partial"}
 BUF = {"kcache": 0, "vcache": 1, "hidden": 2, "hprev": 3, "conf": 4, "argmax": 5, "rows": 6, "nrows": 7,
        "scores": 8, "lock": 9, "masked_prev": 10, "lmrows": 11, "nlmrows": 12, "kl": 13, "hcache": 14, "lse": 15,
-       "selrows": 16, "nsel": 17, "layer_z": 18, "layer_q": 19, "layer_attn": 20, "layer_act": 21}
+       "selrows": 16, "nsel": 17, "layer_z": 18, "layer_q": 19, "layer_attn": 20, "layer_act": 21,
+       "es_in": 22, "zstore": 23, "lse_store": 24, "stamp": 25, "vnew": 26, "fused_sync": 27}
 LAYER_KERNEL = {"auto": 0, "split": 1, "fused": 2}
 
 
@@ -58,6 +59,10 @@ class DllmStepInfo(ctypes.Structure):
                 ("done", c_i32)]
 
 
+class DllmProgress(ctypes.Structure):
+    _fields_ = [("step", c_i32), ("block", c_i32), ("step_in_block", c_i32)]
+
+
 class DllmProfile(ctypes.Structure):
     _fields_ = [("gemm_launches", ctypes.c_int64), ("gemm_ms", c_f64), ("gemm_bytes", c_f64), ("gemm_flops", c_f64),
                 ("gemm_roofline_ms", c_f64), ("attn_launches", ctypes.c_int64), ("attn_ms", c_f64),
@@ -83,6 +88,10 @@ _SIGS = {
     "dllm_set_lock_pattern": (ctypes.c_int, [c_vp, c_vp]),
     "dllm_profile_enable": (ctypes.c_int, [c_vp, c_i32, c_f64, c_f64]),
     "dllm_profile_read": (ctypes.c_int, [c_vp, P(DllmProfile)]),
+    "dllm_get_progress": (ctypes.c_int, [c_vp, P(DllmProgress)]),
+    "dllm_set_progress": (ctypes.c_int, [c_vp, P(DllmProgress)]),
+    "dllm_set_forced_similarities": (ctypes.c_int, [c_vp, c_vp]),
+    "dllm_set_wait_limit": (ctypes.c_int, [c_vp, ctypes.c_uint32]),
     "dllm_kernel_launches": (ctypes.c_int64, []),
     "dllm_get_buffer": (ctypes.c_int, [c_vp, c_i32, P(c_vp), P(c_sz)]),
     "dllm_destroy": (None, [c_vp]),

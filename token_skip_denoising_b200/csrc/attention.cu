@@ -61,8 +61,9 @@ int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N) {
   const int qtiles = (rows_per_seq * G + kUnitsPerCta - 1) / kUnitsPerCta;
   const int ctas = qtiles * B * Hkv;
   const int n_blocks = (N + kKeysPerBlock - 1) / kKeysPerBlock;
-  if (ctas >= kNumSMs) return 1;
-  int s = (2 * kNumSMs + ctas - 1) / ctas;
+  const int sms = num_sms();
+  if (ctas >= sms) return 1;
+  int s = (2 * sms + ctas - 1) / ctas;
   s = std::min(s, n_blocks);
   return std::max(1, s);
 }
@@ -97,13 +98,12 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
   const int qtiles = (rows_per_seq_cap * G + kUnitsPerCta - 1) / kUnitsPerCta;
   dim3 grid(qtiles, B * Hkv, splits);
   const size_t smem = 4 * kKeysPerBlock * hd * 2;
-  static bool attr_done = false;
-  if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(4 * kKeysPerBlock * 128 * 2)));
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(4 * kKeysPerBlock * 64 * 2)));
-    attr_done = true;
+  {
+    const int rc = hd == 128 ? ensure_smem_attr(reinterpret_cast<const void*>(attn_kernel<128>),
+                                                static_cast<int>(4 * kKeysPerBlock * 128 * 2))
+                             : ensure_smem_attr(reinterpret_cast<const void*>(attn_kernel<64>),
+                                                static_cast<int>(4 * kKeysPerBlock * 64 * 2));
+    if (rc) return rc;
   }
   if (hd == 128) {
     const int rc = launch_pdl(attn_kernel<128>, grid, dim3(128), smem, st, p);

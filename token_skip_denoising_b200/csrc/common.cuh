@@ -15,7 +15,14 @@
 
 namespace dllm {
 
-constexpr int kNumSMs = 148;
+// SMs of the current device, queried once per device (148 on a B200).  Grids and the
+// scratch sized from them follow the device; with no device at all (a sizing call on a
+// host without a GPU) it returns kDefaultSMs.
+constexpr int kDefaultSMs = 148;
+int num_sms();
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) for `fn`, once per device and function
+// (thread-safe): a launch on a second device sets it there too.
+int ensure_smem_attr(const void* fn, int bytes);
 
 #define DLLM_CUDA_TRY(expr)                                                   \
   do {                                                                        \

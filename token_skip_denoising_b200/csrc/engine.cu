@@ -18,8 +18,11 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <set>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -34,6 +37,44 @@ void set_last_error(const char* msg, const char* file, int line) {
   char buf[512];
   snprintf(buf, sizeof buf, "%s (%s:%d)", msg, file, line);
   g_last_error = buf;
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_sms[kMaxDevices] = {};
+std::set<std::pair<const void*, int>> g_attr_done;
+}  // namespace
+
+int num_sms() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return kDefaultSMs;
+  }
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (g_sms[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return kDefaultSMs;
+    }
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+int ensure_smem_attr(const void* fn, int bytes) {
+  int dev = -1;
+  DLLM_CUDA_TRY(cudaGetDevice(&dev));
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_attr_done.count({fn, dev})) return DLLM_OK;
+  }
+  DLLM_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  g_attr_done.insert({fn, dev});
+  return DLLM_OK;
 }
 
 #define DLLM_FAIL(code, msg)                              \
@@ -209,6 +250,9 @@ struct dllm_handle {
   int* fused_sync;         // state: phase counters of the fused layer kernel (zero between launches)
   int* fused_attn_ctr;     // state: split arrival counters of its attention step (zero between uses)
   int n_fused_attn_ctr;
+  int n_sms = kDefaultSMs;          // SMs the fused kernel's per-CTA scratch was sized for
+  uint32_t spin_limit = 0;          // fused kernel grid-phase wait limit (0: default)
+  const float* forced_sims = nullptr;   // dLLM-Cache teacher forcing: [L, B, n_resp] (caller-owned)
   float* fused_opart;
   float2* fused_ml;
   size_t fused_attn_floats;
@@ -333,7 +377,8 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->attn_ml = w.take<float2>(ml);
   // fused small-row layer scratch
   x->z2 = w.take<__nv_bfloat16>(static_cast<size_t>(kFusedMaxRows) * x->d);
-  x->fused_scratch = w.take<float>(fused_scratch_floats(x->qkvd, x->F));
+  x->n_sms = num_sms();
+  x->fused_scratch = w.take<float>(fused_scratch_floats(x->qkvd, x->F, x->n_sms));
   x->fused_attn_floats = static_cast<size_t>((x->N + 63) / 64) * kFusedMaxRows * c.n_heads * x->hd;
   x->fused_opart = w.take<float>(x->fused_attn_floats);
   x->fused_ml = w.take<float2>(x->fused_attn_floats / x->hd);
@@ -406,6 +451,8 @@ struct LayerCtx {
   float* fused_opart = nullptr;
   float2* fused_ml = nullptr;
   size_t fused_attn_floats = 0;
+  int max_ctas = kDefaultSMs;       // grid bound its per-CTA scratch was sized for
+  uint32_t spin_limit = 0;
 };
 
 // GEMM launch with optional event bracketing; bytes / flops are the algorithmic figures
@@ -442,6 +489,8 @@ int run_fused_layers(const LayerCtx& x, int n_layers, float* hbuf, const int* ro
   a.attn_ctr = x.fused_attn_ctr; a.n_attn_ctr = x.n_fused_attn_ctr;
   a.scratch = x.fused_scratch;
   a.sync = x.fused_sync;
+  a.max_ctas = x.max_ctas;
+  a.spin_limit = x.spin_limit;
   cudaEvent_t ev = nullptr;
   if (x.prof) x.prof->begin(st, &ev, 2);
   const int rc = fused_layer_launch(a, st);
@@ -536,6 +585,8 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.z2 = x->z2; L.fused_scratch = x->fused_scratch; L.fused_sync = x->fused_sync;
   L.fused_attn_ctr = x->fused_attn_ctr; L.n_fused_attn_ctr = x->n_fused_attn_ctr;
   L.fused_opart = x->fused_opart; L.fused_ml = x->fused_ml; L.fused_attn_floats = x->fused_attn_floats;
+  L.max_ctas = x->n_sms;
+  L.spin_limit = x->spin_limit;
   L.prof = const_cast<Prof*>(&x->prof);
   return L;
 }
@@ -551,7 +602,8 @@ void carve_fused_op(Carver& w, const dllm_config* cfg, int rows_cap, LayerCtx* L
   const int n_ctr = fused_attn_counters(cfg->batch, cfg->n_heads, cfg->n_kv_heads, kFusedMaxRows);
   int* ctr = w.take<int>(n_ctr);
   __nv_bfloat16* z2 = w.take<__nv_bfloat16>(static_cast<size_t>(kFusedMaxRows) * d);
-  float* scratch = w.take<float>(fused_scratch_floats(qd + 2 * kvd, cfg->ffn_dim));
+  const int sms = num_sms();
+  float* scratch = w.take<float>(fused_scratch_floats(qd + 2 * kvd, cfg->ffn_dim, sms));
   const size_t af = static_cast<size_t>((N + 63) / 64) * kFusedMaxRows * cfg->n_heads * cfg->head_dim;
   float* opart = w.take<float>(af);
   float2* ml = w.take<float2>(af / cfg->head_dim);
@@ -570,6 +622,7 @@ void carve_fused_op(Carver& w, const dllm_config* cfg, int rows_cap, LayerCtx* L
   L->fused_opart = opart;
   L->fused_ml = ml;
   L->fused_attn_floats = af;
+  L->max_ctas = sms;
 }
 
 // Per-layer ES selection: from the skip layer on, each layer runs alone and right after
@@ -800,7 +853,8 @@ int dllm_layer_forward(dllm_handle* x, int32_t layer, void* stream) {
     DLLM_TRY(timed_gemm(&x->prof, v, x->gs, st, 4.0 * x->kvd));
     DLLM_TRY(score_cos_launch(x->vnew, x->kvd, L.vc, x->rows, x->nrows, cap, x->N, c.n_kv_heads, x->hd, x->scores, st));
     SelectParams sp;
-    sp.scores = x->scores; sp.B = x->B; sp.n = x->n_resp; sp.mode = c.forced_rho ? SEL_FORCED_ASC : SEL_BELOW_CAP_ASC;
+    sp.scores = x->forced_sims ? x->forced_sims + static_cast<int64_t>(layer) * x->B * x->n_resp : x->scores;
+    sp.B = x->B; sp.n = x->n_resp; sp.mode = c.forced_rho ? SEL_FORCED_ASC : SEL_BELOW_CAP_ASC;
     sp.k = x->resp_cap; sp.tau = c.sim_tau; sp.cand_start = x->resp_start; sp.seq_n = x->N;
     sp.act_pos = x->act_idx; sp.k_max = std::max(1, x->resp_cap); sp.count = x->act_count;
     sp.row_map = x->rows2; sp.seq_off = x->seq_off2; sp.total = x->nrows2;
@@ -1020,6 +1074,15 @@ int dllm_get_buffer(dllm_handle* x, int32_t which, void** ptr, size_t* bytes) {
     case DLLM_BUF_LAYER_Q: p = x->q; b = BN * x->qd * 2; break;
     case DLLM_BUF_LAYER_ATTN: p = x->attn; b = BN * x->qd * 2; break;
     case DLLM_BUF_LAYER_ACT: p = x->act; b = BN * x->F * 2; break;
+    case DLLM_BUF_ES_IN:
+      p = x->es_in;
+      b = x->es_in ? static_cast<size_t>(x->L - x->c.skip_layer - 1) * BN * x->d * 4 : 0;
+      break;
+    case DLLM_BUF_ZSTORE: p = x->zstore; b = x->zstore ? 2 * BN * static_cast<size_t>(x->V) * 2 : 0; break;
+    case DLLM_BUF_LSE_STORE: p = x->lse_store; b = x->lse_store ? 2 * BN * 4 : 0; break;
+    case DLLM_BUF_STAMP: p = x->has_prev; b = BN * 4; break;
+    case DLLM_BUF_VNEW: p = x->vnew; b = x->vnew ? static_cast<size_t>(x->B) * x->n_resp * x->kvd * 4 : 0; break;
+    case DLLM_BUF_FUSED_SYNC: p = x->fused_sync; b = kFusedSyncInts * 4; break;
     default: DLLM_FAIL(DLLM_ERR_INVALID_ARG, "unknown buffer");
   }
   *ptr = p;
@@ -1041,10 +1104,48 @@ int dllm_reset(dllm_handle* x, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = reinterpret_cast<uint8_t*>(x->rope_cos);
   DLLM_CUDA_TRY(cudaMemsetAsync(base + x->const_bytes, 0, x->state_total - x->const_bytes, st));
+  // GEMM tile and attention split counters of the workspace: every launch leaves them at
+  // zero, except one that gave up a wait (DLLM_DEV_TIMEOUT)
+  if (x->gs.n_counters) DLLM_CUDA_TRY(cudaMemsetAsync(x->gs.counters, 0, x->gs.n_counters * sizeof(int), st));
+  if (x->n_attn_ctr) DLLM_CUDA_TRY(cudaMemsetAsync(x->attn_ctr, 0, x->n_attn_ctr * sizeof(int), st));
   x->block = 0;
   x->step_in_block = 0;
   x->n_steps = 0;
   x->began = false;
+  return DLLM_OK;
+}
+
+int dllm_get_progress(const dllm_handle* x, dllm_progress* out) {
+  if (!x || !out) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  out->step = x->n_steps;
+  out->block = x->block;
+  out->step_in_block = x->step_in_block;
+  return DLLM_OK;
+}
+
+int dllm_set_progress(dllm_handle* x, const dllm_progress* p) {
+  if (!x || !p) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  if (x->began) DLLM_FAIL(DLLM_ERR_STATE, "set_progress in the middle of a step");
+  const int n_blocks = x->c.gen_len / x->c.block_len;
+  if (p->step < 0 || p->block < 0 || p->block > n_blocks || p->step_in_block < 0 ||
+      p->step_in_block >= x->steps_per_block || (p->block == n_blocks && p->step_in_block != 0))
+    DLLM_FAIL(DLLM_ERR_INVALID_ARG, "progress outside the schedule");
+  x->n_steps = p->step;
+  x->block = p->block;
+  x->step_in_block = p->step_in_block;
+  return DLLM_OK;
+}
+
+int dllm_set_forced_similarities(dllm_handle* x, const float* sims) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  if (x->c.policy != DLLM_POLICY_DLLM_CACHE) DLLM_FAIL(DLLM_ERR_STATE, "forced similarities apply to dLLM-Cache");
+  x->forced_sims = sims;
+  return DLLM_OK;
+}
+
+int dllm_set_wait_limit(dllm_handle* x, uint32_t polls) {
+  if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null handle");
+  x->spin_limit = polls;
   return DLLM_OK;
 }
 

@@ -49,11 +49,12 @@ using namespace gemm;
 constexpr int kThreads = 192;
 constexpr int kKsub = 2;                          // 64-column k-blocks per ring stage
 constexpr int kMaxRows = kFusedMaxRows;           // rows of the fp32 sum buffers (any launch's row count)
-constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kSpinLimit = 1u << 22;          // default polls of a grid-phase wait (~0.4 s)
 constexpr size_t kMaxKvPrefetch = 64ull << 20;    // larger caches are not prefetched
 
 enum Phase : int { S_X1 = 0, S_QKV, S_ROPE, S_COMB, S_O, S_X2, S_GU, S_SWIGLU, S_DOWN, S_SCORE, S_PICK, S_COUNT };
-static_assert(S_COUNT + 1 <= kFusedSyncInts, "phase counters + exit counter");
+constexpr int S_ABORT = S_COUNT + 1;              // set by a CTA that gave up a wait
+static_assert(S_ABORT + 1 <= kFusedSyncInts, "phase counters + exit counter + abort word");
 static_assert(kMaxRows <= 128 && 128 % kMaxRows == 0, "rows are handled by the 128 step threads");
 
 template <int BN>
@@ -66,7 +67,7 @@ struct FCfg {
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr size_t kAttnBytes = 4 * 64 * 128 * 2;   // K/V double buffer for hd <= 128
   static constexpr size_t kMiscBytes = 4 * kMaxRows * 4;    // row map, 1/rms before attention and FFN, partial sums
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + kMiscBytes + (2 * kStages + 4) * 8 + 64;
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kAttnBytes + kMiscBytes + (2 * kStages + 5) * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "fused layer does not fit shared memory");
 };
 
@@ -109,9 +110,11 @@ struct FParams {
   int attn_qtiles;
   int attn_items;
   int* attn_ctr;          // [B * Hkv * attn_qtiles] split arrivals, zero between uses
-  int* sync;              // [S_COUNT] phase counters + exit counter, zero at launch
+  int* sync;              // [S_COUNT] phase counters + exit counter + abort word, zero at launch
   FusedEs es;             // per-layer re-selection at the start of every layer (es.on)
   float* es_acc;          // [2 * B * n_cand] Eq. 1 sums of the candidates, zero between layers
+  int n_attn_ctr;         // attention split counters (cleared after an aborted launch)
+  uint32_t spin_limit;    // polls of a grid-phase wait before it gives up
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -141,24 +144,39 @@ __device__ __forceinline__ Items items_of(int K, int n_tiles, int G, int c) {
   return r;
 }
 
-// Bounded wait until counter >= target.
-__device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile int* abort) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+// Bounded wait until counter >= target.  On expiry the CTA records the timeout, raises its
+// abort flag and marks the launch aborted (the last CTA out then clears what an unfinished
+// layer leaves behind).
+__device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile int* abort, uint32_t limit,
+                                           int* abort_word) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (ld_acquire(ctr) >= target) return true;
     if (*abort) return false;
     __nanosleep(64);
   }
   set_dev_status(DLLM_DEV_TIMEOUT);
   *abort = 1;
+  atomicExch(abort_word, 1);
+  return false;
+}
+
+// Bounded wait on an mbarrier phase that also gives up as soon as the CTA's abort flag is up.
+__device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31) == 31 && *abort) return false;
+  }
+  set_dev_status(DLLM_DEV_TIMEOUT);
   return false;
 }
 
 // The 128 epilogue threads wait for a phase of every CTA: thread 0 polls, the barrier
 // vote hands the outcome to all of them (true: go on).
-__device__ __forceinline__ bool epi_wait_phase(const int* ctr, int target, volatile int* abort, int tid) {
+__device__ __forceinline__ bool epi_wait_phase(const int* ctr, int target, volatile int* abort, int tid,
+                                               uint32_t limit, int* abort_word) {
   bool ok = true;
   if (tid == 0) {
-    ok = wait_count(ctr, target, abort);
+    ok = wait_count(ctr, target, abort, limit, abort_word);
     __threadfence();
   }
   return !epi_any(!ok || *abort);   // the barrier orders the other threads' reads after the acquire
@@ -199,7 +217,8 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* acc_full = empty_bar + C::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* mma_done = acc_empty + 2;                                 // every MMA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last split
 
   const CUtensorMap* tmW[4] = {&tmW0, &tmW1, &tmW2, &tmW3};
@@ -222,6 +241,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    mbar_init(mma_done, 1);
     s_flag[0] = 0;
     s_flag[1] = 0;
     fence_barrier_init();
@@ -256,7 +276,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         }
         // bounded wait for the activation operand of GEMM g of this layer (a grid phase)
         auto x_ready = [&](int g) -> bool { return ld_acquire(p.sync + p.gm[g].wait_slot) >= target; };
-        auto wait_x = [&](int g) -> bool { return wait_count(p.sync + p.gm[g].wait_slot, target, s_flag); };
+        auto wait_x = [&](int g) -> bool {
+          return wait_count(p.sync + p.gm[g].wait_slot, target, s_flag, p.spin_limit, p.sync + S_ABORT);
+        };
         for (int g = 0; g < 4 && !s_flag[0]; ++g) {
           const FGemm& gm = p.gm[g];
           const int KB = R[g].KB;
@@ -287,7 +309,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
                 if (!wait_x(g)) break;
                 flush();
               }
-              if (!mbar_wait(&empty_bar[s], ph ^ 1)) { s_flag[0] = 1; break; }
+              if (!mbar_wait_ab(&empty_bar[s], ph ^ 1, s_flag)) { s_flag[0] = 1; break; }
               uint8_t* a = stage_base + s * C::kStageBytes;
               mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
 #pragma unroll
@@ -314,7 +336,13 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           if (!ready && n_pend > 0 && !s_flag[0]) {
             if (wait_x(g)) flush();
           }
+          if (s_flag[0] && n_pend > 0) flush();   // aborting: complete the stages already requested
         }
+      }
+      if (s_flag[0]) {
+        // aborting: wait (bounded) until the copies of the last stages requested have landed
+        for (int q = i > C::kStages ? i - C::kStages : 0; q < i; ++q)
+          mbar_wait(&full_bar[q % C::kStages], (q / C::kStages) & 1);
       }
     }
   } else if (warp == 5) {
@@ -333,13 +361,13 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
             const int b = j & 1;
             const uint32_t u = static_cast<uint32_t>(j >> 1);
             ++j;
-            if (!mbar_wait(&acc_empty[b], (u & 1) ^ 1)) { s_flag[0] = 1; break; }
+            if (!mbar_wait_ab(&acc_empty[b], (u & 1) ^ 1, s_flag)) { s_flag[0] = 1; break; }
             tc_fence_after();
             const uint32_t d = tmem + b * C::kAccCols;
             for (int kb = kb0; kb < kb1; ++kb, ++i) {
               const int s = i % C::kStages;
               const uint32_t ph = (i / C::kStages) & 1;
-              if (!mbar_wait(&full_bar[s], ph)) { s_flag[0] = 1; break; }
+              if (!mbar_wait_ab(&full_bar[s], ph, s_flag)) { s_flag[0] = 1; break; }
               tc_fence_after();
               const uint32_t a = smem_u32(stage_base + s * C::kStageBytes);
               const uint32_t bb = a + kKsub * kABytes;
@@ -356,6 +384,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           }
         }
       }
+      // every MMA issued has completed before the tensor memory is freed
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0);
     }
   } else {
     // ---------------- warps 0-3: reductions of the GEMM pieces and the steps between GEMMs
@@ -380,7 +411,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         const int b = j & 1;
         const uint32_t u = static_cast<uint32_t>(j >> 1);
         ++j;
-        const bool late = !mbar_wait(&acc_full[b], u & 1);
+        const bool late = !mbar_wait_ab(&acc_full[b], u & 1, s_flag);
         if (epi_any(late || s_flag[0])) {              // one decision for all epilogue threads
           s_flag[0] = 1;
           return;
@@ -451,7 +482,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       __nv_bfloat16* kc = p.kc + static_cast<int64_t>(l) * p.kv_layer;
       __nv_bfloat16* vc = p.vc + static_cast<int64_t>(l) * p.kv_layer;
       // the previous layer's down sums are complete in h (and its sums have been read)
-      if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t)) s_flag[0] = 1;
+      if (li > 0 && !epi_wait_phase(p.sync + S_DOWN, li * G, s_flag, t, p.spin_limit, p.sync + S_ABORT)) s_flag[0] = 1;
       if (p.es.on && li < p.es.n_scored) {
         // ES-dLLM Eq. 1 on every candidate's input of this layer: each row split into column
         // slices over the grid's warps, whose partial sums meet in es_acc[2 u .. 2 u + 1]
@@ -482,7 +513,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         signal_phase(p.sync + S_SCORE, t);
         // the top k of sequence b by CTA b: a candidate is chosen when fewer than k others
         // rank above it (higher key, or an equal key at a lower position)
-        if (epi_wait_phase(p.sync + S_SCORE, target, s_flag, t) && c < es.B) {
+        if (epi_wait_phase(p.sync + S_SCORE, target, s_flag, t, p.spin_limit, p.sync + S_ABORT) && c < es.B) {
           const int b = c;
           const bool last = li == es.n_scored - 1;
           uint8_t* s_pick = attn_smem;                                         // idle outside attention
@@ -522,7 +553,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           }
         }
         signal_phase(p.sync + S_PICK, t);
-        if (epi_wait_phase(p.sync + S_PICK, target, s_flag, t) && t < kMaxRows)
+        if (epi_wait_phase(p.sync + S_PICK, target, s_flag, t, p.spin_limit, p.sync + S_ABORT) && t < kMaxRows)
           s_rows[t] = t < m_rows ? __ldcg(es.rows + t) : 0;
         epi_bar();
       }
@@ -536,12 +567,12 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         gain_operand(p.g_attn + static_cast<int64_t>(l) * p.d, p.z1, p.ssp1);   // QKV operand
       }
       signal_phase(p.sync + S_X1, t);
-      if (epi_wait_phase(p.sync + S_X1, target, s_flag, t)) rinv_from(p.ssp1, s_rinv1);   // while QKV streams
+      if (epi_wait_phase(p.sync + S_X1, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ssp1, s_rinv1);   // while QKV streams
       gemm_epilogues(0, li);                                       // QKV sums
       signal_phase(p.sync + S_QKV, t);
       // RMSNorm scale and RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention
       // operand, k and v scattered into the cache rows of their positions
-      if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t)) {
+      if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         const int pairs = p.qkvd >> 1;
         const int64_t total = static_cast<int64_t>(m_rows) * pairs;
         for (int64_t uu = gt; uu < total; uu += gstride) {
@@ -583,7 +614,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       signal_phase(p.sync + S_ROPE, t);
       // attention items over the cached K/V (the new rows are in the cache now); the last
       // split of a (sequence, KV head, query tile) to finish merges the partials
-      if (epi_wait_phase(p.sync + S_ROPE, target, s_flag, t)) {
+      if (epi_wait_phase(p.sync + S_ROPE, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         attn::AttnParams ap = p.ap;
         ap.kc = kc;
         ap.vc = vc;
@@ -624,14 +655,14 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       gemm_epilogues(1, li);                                       // O, added into h
       signal_phase(p.sync + S_O, t);
       // gate/up operand g_ffn * h once every O sum is in h
-      if (epi_wait_phase(p.sync + S_O, target, s_flag, t))
+      if (epi_wait_phase(p.sync + S_O, target, s_flag, t, p.spin_limit, p.sync + S_ABORT))
         gain_operand(p.g_ffn + static_cast<int64_t>(l) * p.d, p.z2, p.ssp2);
       signal_phase(p.sync + S_X2, t);
-      if (epi_wait_phase(p.sync + S_X2, target, s_flag, t)) rinv_from(p.ssp2, s_rinv2);   // while gate/up streams
+      if (epi_wait_phase(p.sync + S_X2, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ssp2, s_rinv2);   // while gate/up streams
       gemm_epilogues(2, li);                                       // gate/up sums
       signal_phase(p.sync + S_GU, t);
       // SwiGLU on the RMSNorm-scaled sums: act = silu(gate) * up
-      if (epi_wait_phase(p.sync + S_GU, target, s_flag, t)) {
+      if (epi_wait_phase(p.sync + S_GU, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         const int f4 = p.F >> 2;
         const int64_t total = static_cast<int64_t>(m_rows) * f4;
         for (int64_t uu = gt; uu < total; uu += gstride) {
@@ -663,11 +694,19 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 5) tmem_dealloc(tmem, C::kTmemCols);
-  // the last CTA out clears the counters, so every launch (a graph replay too) starts from zero
+  // the last CTA out clears the counters, so every launch (a graph replay too) starts from zero;
+  // after an aborted launch it also clears what an unfinished layer can leave behind (attention
+  // split arrivals, the ES choice's row sums)
   if (threadIdx.x == 0) {
+    if (s_flag[0]) atomicExch(p.sync + S_ABORT, 1);
     __threadfence();
     if (atomicAdd(p.sync + S_COUNT, 1) == G - 1) {
-      for (int q = 0; q <= S_COUNT; ++q) atomicExch(p.sync + q, 0);
+      if (atomicAdd(p.sync + S_ABORT, 0) != 0) {
+        for (int q = 0; q < p.n_attn_ctr; ++q) p.attn_ctr[q] = 0;
+        if (p.es.on)
+          for (int q = 0; q < 2 * p.es.B * p.es.n_cand; ++q) p.es_acc[q] = 0.f;
+      }
+      for (int q = 0; q <= S_ABORT; ++q) atomicExch(p.sync + q, 0);
       __threadfence();
     }
   }
@@ -677,12 +716,8 @@ template <int BN>
 int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const FParams& p, int grid,
                  cudaStream_t st) {
   using C = FCfg<BN>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(fused_layer_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::kSmem)));
-    attr_done = true;
-  }
+  const int rc = ensure_smem_attr(reinterpret_cast<const void*>(fused_layer_kernel<BN>), static_cast<int>(C::kSmem));
+  if (rc) return rc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -705,9 +740,9 @@ int launch_fused(const CUtensorMap (&tw)[4], const CUtensorMap (&tx)[4], const F
 
 }  // namespace
 
-size_t fused_scratch_floats(int qkvd, int F) {
+size_t fused_scratch_floats(int qkvd, int F, int max_ctas) {
   return static_cast<size_t>(kMaxRows) * (static_cast<size_t>(qkvd) + 2 * static_cast<size_t>(F)) +
-         2 * static_cast<size_t>(kNumSMs) * kMaxRows + 2 * static_cast<size_t>(kMaxRows) * kFusedEsMaxCand;
+         2 * static_cast<size_t>(max_ctas) * kMaxRows + 2 * static_cast<size_t>(kMaxRows) * kFusedEsMaxCand;
 }
 
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
@@ -720,7 +755,8 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
   if (a.n_layers <= 0 || a.l0 < 0 || a.l0 + a.n_layers > a.L) return DLLM_ERR_INVALID_ARG;
   const int bn = a.rows_cap <= 16 ? 16 : (a.rows_cap <= 32 ? 32 : 64);
-  const int grid = kNumSMs;
+  if (a.max_ctas <= 0) return DLLM_ERR_INVALID_ARG;
+  const int grid = std::min(num_sms(), a.max_ctas);   // one CTA per SM, all resident (cooperative)
   CUtensorMap tw[4], tx[4];
   // every layer of a weight stack in one map: layer l's tile rows start at l * rows per layer
   const void* W[4] = {a.Wqkv, a.Wo, a.Wgu, a.Wdn};
@@ -765,7 +801,9 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.s_gu = s_gu;
   p.ssp1 = ssp;
   p.ssp2 = ssp + static_cast<size_t>(grid) * kMaxRows;
-  p.es_acc = ssp + 2 * static_cast<size_t>(kNumSMs) * kMaxRows;
+  p.es_acc = ssp + 2 * static_cast<size_t>(a.max_ctas) * kMaxRows;
+  p.n_attn_ctr = a.n_attn_ctr;
+  p.spin_limit = a.spin_limit ? a.spin_limit : kSpinLimit;
   p.qkvd = a.qkvd; p.qd = a.qd; p.kvd = a.kvd; p.hd = a.hd; p.Hkv = a.Hkv; p.N = a.N; p.F = a.F;
   p.rope_cos = a.rope_cos;
   p.rope_sin = a.rope_sin;
@@ -787,7 +825,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
     return e ? std::max(0, atoi(e)) : 0;
   }();
   const int groups = a.B * a.Hkv * qtiles;
-  int splits = splits_env > 0 ? splits_env : std::max(1, kNumSMs / groups);
+  int splits = splits_env > 0 ? splits_env : std::max(1, grid / groups);
   splits = std::max(1, std::min(n_blocks, splits));
   const int bps = (n_blocks + splits - 1) / splits;
   splits = (n_blocks + bps - 1) / bps;

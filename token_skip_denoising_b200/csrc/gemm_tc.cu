@@ -478,23 +478,16 @@ int pick_bn(int rows) {
 // Grid of the persistent kernel: one CTA per SM, never more CTAs than k-block iterations.
 int pick_grid(int tiles, int KB) {
   const int64_t T = static_cast<int64_t>(tiles) * KB;
-  return static_cast<int>(std::min<int64_t>(kNumSMs, T));
+  return static_cast<int>(std::min<int64_t>(num_sms(), T));
 }
 
 template <int BN, int KSUB, bool BIG>
 int launch_cfg2(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int grid, cudaStream_t st) {
   using C = Cfg<BN, KSUB, BIG>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    DLLM_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, KSUB, BIG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::kSmem)));
-    attr_done = true;
-  }
-{
-    const int rc_ = launch_pdl(gemm_tc_kernel<BN, KSUB, BIG>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
-    if (rc_) return rc_;
-  }
-  return DLLM_OK;
+  const int rc = ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, KSUB, BIG>),
+                                  static_cast<int>(C::kSmem));
+  if (rc) return rc;
+  return launch_pdl(gemm_tc_kernel<BN, KSUB, BIG>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
 }
 
 template <int BN, int KSUB>
@@ -537,7 +530,7 @@ size_t gemm_partial_floats(int rows_cap, int n_tiles_w, int K) {
   (void)n_tiles_w;
   (void)K;
   const int bn = pick_bn(rows_cap);
-  return static_cast<size_t>(kNumSMs) * 2 * bn * 128;
+  return static_cast<size_t>(num_sms()) * 2 * bn * 128;
 }
 
 int gemm_counters_needed(int rows_cap, int n_tiles_w) {

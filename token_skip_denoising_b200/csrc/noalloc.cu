@@ -7,6 +7,7 @@
 // because it synchronises the device and can fail under memory pressure.  For
 // them dllm_op_gemm_noalloc keeps that scratch in a fixed array in this
 // library's device image, so the call itself allocates nothing.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -15,11 +16,14 @@ namespace dllm {
 namespace {
 
 // Largest problem the fixed scratch serves: up to 32 activation rows (one tile
-// of the 32-wide MMA) and up to 4096 output tiles of 128 rows.
+// of the 32-wide MMA) and up to 4096 output tiles of 128 rows, with one partial
+// tile pair per CTA of a grid of at most 148 CTAs (a device with more SMs runs
+// this call on 148 of them).
 constexpr int kNoAllocMaxRows = 32;
 constexpr int kNoAllocMaxTiles = 4096;
+constexpr int kNoAllocMaxGrid = 148;
 constexpr size_t kNoAllocCounterBytes = kNoAllocMaxTiles * sizeof(int);
-constexpr size_t kNoAllocPartialFloats = static_cast<size_t>(kNumSMs) * 2 * kNoAllocMaxRows * 128;
+constexpr size_t kNoAllocPartialFloats = static_cast<size_t>(kNoAllocMaxGrid) * 2 * kNoAllocMaxRows * 128;
 constexpr size_t kNoAllocBytes = kNoAllocCounterBytes + kNoAllocPartialFloats * sizeof(float);   // ~4.9 MB
 
 // The scratch: one copy per device that loads the library, held until the process exits.
@@ -101,5 +105,5 @@ extern "C" int dllm_op_gemm_noalloc(int32_t kind, const void* W, int32_t n_out, 
   } else {
     a.epi.out = out; a.epi.ldo = n_out;
   }
-  return gemm_launch(a, gs, st, 0, 0);
+  return gemm_launch(a, gs, st, std::min(num_sms(), kNoAllocMaxGrid), 0);
 }

@@ -143,8 +143,10 @@ struct FusedLayerArgs {
                            // the kernel leaves it zero
   int* sync;               // kFusedSyncInts counters, zero before the launch; the kernel leaves them zero
   FusedEs es;              // per-layer re-selection (es.on = 0: the row map is fixed)
+  int max_ctas = 0;        // grid bound the scratch was sized for (fused_scratch_floats)
+  uint32_t spin_limit = 0; // polls of a grid-phase wait (0: the default)
 };
-size_t fused_scratch_floats(int qkvd, int F);
+size_t fused_scratch_floats(int qkvd, int F, int max_ctas);
 int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap);
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st);
 

@@ -111,6 +111,25 @@ class Engine:
         self._lock_pattern = pattern
         check(self.lib.dllm_set_lock_pattern(self.handle, ptr(pattern)), "dllm_set_lock_pattern")
 
+    def set_forced_similarities(self, sims: torch.Tensor | None):
+        """dLLM-Cache teacher forcing: per-layer similarities fp32 [L, B, n_resp] on the device."""
+        self._forced_sims = sims
+        check(self.lib.dllm_set_forced_similarities(self.handle, ptr(sims)), "dllm_set_forced_similarities")
+
+    def set_wait_limit(self, polls: int):
+        """Poll limit of the fused layer kernel's grid-phase waits (0: the default)."""
+        check(self.lib.dllm_set_wait_limit(self.handle, int(polls)), "dllm_set_wait_limit")
+
+    def progress(self) -> dict:
+        """Schedule position (with the state buffer and the tokens: the whole generation state)."""
+        p = _lib.DllmProgress()
+        check(self.lib.dllm_get_progress(self.handle, ctypes.byref(p)), "dllm_get_progress")
+        return {f: getattr(p, f) for f, _ in p._fields_}
+
+    def set_progress(self, prog: dict):
+        p = _lib.DllmProgress(**prog)
+        check(self.lib.dllm_set_progress(self.handle, ctypes.byref(p)), "dllm_set_progress")
+
     def profile(self, every: int, hbm_gbs: float = 0.0, tensor_tflops: float = 0.0):
         """Bracket every `every`-th GEMM / attention launch with CUDA events (0: off)."""
         check(self.lib.dllm_profile_enable(self.handle, int(every), hbm_gbs, tensor_tflops),
@@ -148,10 +167,18 @@ class Engine:
             "layer_z": (torch.bfloat16, (-1, c.d_model)), "layer_q": (torch.bfloat16, (-1, c.n_heads * c.head_dim)),
             "layer_attn": (torch.bfloat16, (-1, c.n_heads * c.head_dim)),
             "layer_act": (torch.bfloat16, (-1, c.ffn_dim)),
+            "es_in": (torch.float32, (-1, B * N, c.d_model)),
+            "zstore": (torch.bfloat16, (2, B * N, c.vocab)), "lse_store": (torch.float32, (2, B * N)),
+            "stamp": (torch.int32, (B * N,)),
+            "vnew": (torch.float32, (-1, c.n_kv_heads * c.head_dim)),
+            "fused_sync": (torch.int32, (16,)),
         }
         dt, shp = defaults[name]
         if shape is None and shp[0] == -1:
-            shp = (nb.value // (shp[1] * torch.empty(0, dtype=dt).element_size()), shp[1])
+            inner = 1
+            for v in shp[1:]:
+                inner *= v
+            shp = (nb.value // (inner * torch.empty(0, dtype=dt).element_size()),) + tuple(shp[1:])
         return _lib.view(p.value, shape or shp, dtype or dt)
 
 
