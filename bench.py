@@ -29,6 +29,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -120,6 +122,45 @@ def reduce_over_ranks(values, world: int, device="cpu"):
 
 def whole_job_tokens_per_s(batch: int, gen_len: int, steps: int, world: int, seconds: float) -> float:
     return batch * gen_len * steps * world / seconds
+
+
+def step_work(m, rows_per_layer, lm_rows, N, batch):
+    """Algorithmic bytes and FLOPs of one denoising step: every layer streams its weights
+    (2 P bytes) and reads its K/V cache, the recomputed rows of each layer do 2 P FLOPs of
+    GEMM and 4 N Hq hd of attention, the vocabulary projection streams V d weights."""
+    P = m.params_per_layer
+    byts = sum(2.0 * P + 2.0 * batch * N * m.kv_dim * 2 + r * (2 * m.kv_dim + 2 * m.d_model) * 2
+               for r in rows_per_layer) + 2.0 * m.vocab * m.d_model
+    flops = sum(2.0 * r * P + 4.0 * r * N * m.n_heads * m.head_dim for r in rows_per_layer)
+    flops += 2.0 * lm_rows * m.vocab * m.d_model
+    return byts, flops
+
+
+def generation_roofline(cfg, peaks, measured_ms):
+    """Roofline of one whole ES-dLLM generation: each step is bound by its bytes at the measured
+    HBM bandwidth or its FLOPs at the sustained bf16 peak (the generation is a long loop),
+    whichever is slower; refresh steps recompute every row, skip steps the block's rows below
+    the skip layer and the kept rows above it."""
+    m, N, B = cfg.model, cfg.seq_len, cfg.batch
+    L, ls, n_c = m.n_layers, cfg.skip_layer, cfg.block_len
+    k = cfg.keep_count(n_c)
+    steps_per_block = math.ceil(cfg.block_len / cfg.tokens_per_step)
+    n_ref = cfg.n_blocks
+    n_skip = cfg.n_blocks * (steps_per_block - 1)
+    hbm, tc = peaks["hbm_gbs"] * 1e6, peaks["bf16_tflops_sustained"] * 1e9        # bytes / ms, flops / ms
+    b_s, f_s = step_work(m, [B * n_c] * ls + [B * k] * (L - ls), B * k, N, B)
+    b_r, f_r = step_work(m, [B * N] * L, B * n_c, N, B)
+    t_s, t_r = max(b_s / hbm, f_s / tc), max(b_r / hbm, f_r / tc)
+    roof_ms = n_ref * t_r + n_skip * t_s
+    return {"roofline_ms": round(roof_ms, 2), "measured_ms": round(measured_ms, 2),
+            "frac": round(roof_ms / measured_ms, 4),
+            "tokens_per_s_at_roofline": round(B * cfg.gen_len / (roof_ms / 1e3), 2),
+            "skip_step": {"count": n_skip, "roofline_ms": round(t_s, 4), "bound": "hbm" if b_s / hbm >= f_s / tc else "tensor",
+                          "bytes": round(b_s), "flops": round(f_s)},
+            "refresh_step": {"count": n_ref, "roofline_ms": round(t_r, 4),
+                             "bound": "hbm" if b_r / hbm >= f_r / tc else "tensor", "bytes": round(b_r), "flops": round(f_r)},
+            "peaks": f"HBM {peaks['hbm_gbs']} GB/s, bf16 {peaks['bf16_tflops_sustained']} TFLOP/s sustained "
+                     f"({peaks['source']})"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -237,6 +278,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: every denoising step streams all 16 GB of weights",
                    "parallelism": f"replicas x{world} (no collective)"},
         "roofline": roof,
+        "generation_roofline": generation_roofline(cfg, peaks, ms_max / args.steps),
         "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(tok0_host.numel() * 4), "d2h_bytes_per_step": int(out_host.numel() * 4)},
         "gpu_launches": int(launches),
@@ -268,8 +310,22 @@ def micro_sweep(peaks, reps=20):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     out = []
     P = m.params_per_layer
+    # the oracle's single-layer step on the host: Eq. 1 over the N rows, the top k, the layer on
+    # the k rows (measured up to 512 rows, scaled by rows beyond: labelled extrapolated)
+    from oracle.policy import es_importance, topk_select
+    lw_host = layer_weights_cpu(w, 0)
+    h_host, hp_host = hin["h_cur"].double().cpu().numpy(), hin["h_prev"].double().cpu().numpy()
+    c_host = hin["conf"].double().cpu().numpy() * hin["masked_prev"].cpu().numpy()
+    rng = np.random.default_rng(0)
+    cores = host_cores()
     for rho in (0.03, 0.1, 0.25, 0.5, 1.0):
         k = max(1, math.ceil(rho * N - 1e-9))
+        t = time.perf_counter()
+        topk_select(es_importance(0.5, c_host, h_host, hp_host), k)
+        o_ms = 1e3 * (time.perf_counter() - t + oracle_layer_s(m, lw_host, k, N, rng, cap=512))
+        oracle = {"ms": round(o_ms, 1), "cores": cores, "kind": "oracle",
+                  "sample": "fp64 oracle: Eq. 1, top k, one layer" + (f" (layer measured at 512 rows, scaled x{k / 512:.2f}:"
+                                                                     " extrapolated)" if k > 512 else "")}
         ws = torch.zeros(ops.layer_workspace_bytes(ccfg, k, k), dtype=torch.uint8, device="cuda")
         for pattern in ("random", "contiguous"):
             h = hin["h_cur"].clone()
@@ -297,6 +353,7 @@ def micro_sweep(peaks, reps=20):
             roof_ms = max(byts / (peaks["hbm_gbs"] * 1e6), flops / (peaks["bf16_tflops"] * 1e9))
             out.append({"rho": rho, "k": k, "pattern": pattern, "ms": round(t, 4),
                         "roofline_ms": round(roof_ms, 4), "roofline_frac": round(roof_ms / t, 4),
+                        "cpu_baseline": oracle,
                         "bound": "hbm" if byts / (peaks["hbm_gbs"] * 1e6) >= flops / (peaks["bf16_tflops"] * 1e9)
                         else "tensor"})
     del w
@@ -352,6 +409,14 @@ def variant_steps(peaks, steps=3, warm=2):
     tok0 = make_tokens(cfg).cuda()
     eng = Engine(cfg, w, tok0.clone(), stream=stream)
     rows = []
+    rng = np.random.default_rng(0)
+    lw_host = layer_weights_cpu(w, 0)
+    lm_host, gf_host = w["lm_head"].cpu(), w["g_final"].cpu()
+    cores = host_cores()
+    # oracle seconds per layer (weight conversion) and per active row of a layer (a 256-row sample),
+    # per vocabulary-projection row (a 64-row sample)
+    o_conv, o_row = oracle_layer_cost(m, lw_host, 256, N, rng)
+    o_lm_row = oracle_lm_s(m, lm_host, gf_host, 64, rng) / 64
     for frac in (None, 0.25, 0.5, 0.75):
         eng.reset(tok0)
         pat = lock_pattern(B, N, frac).cuda() if frac is not None else None
@@ -364,10 +429,14 @@ def variant_steps(peaks, steps=3, warm=2):
         # logits of the recomputed rows: one store, three reads of this step's, one of the previous
         logit_bytes = 5.0 * n_lm * m.vocab * 2
         roof, bound = _step_roofline_ms(peaks, m, [active] * m.n_layers, n_lm, N, B, logit_bytes)
+        o_ms = 1e3 * (m.n_layers * (o_conv + active * o_row) + n_lm * o_lm_row)
         rows.append({"lock": "rule (KL < eps and conf > tau)" if frac is None else f"forced {frac:.2f} of positions",
                      "locked_frac": round(locked / (B * N), 4), "active_rows": active, "lm_rows": n_lm,
                      "ms_per_step": round(t, 3), "tokens_per_s": round(B * cfg.tokens_per_step / (t / 1e3), 2),
-                     "roofline_ms": round(roof, 3), "roofline_frac": round(roof / t, 4), "bound": bound})
+                     "roofline_ms": round(roof, 3), "roofline_frac": round(roof / t, 4), "bound": bound,
+                     "cpu_baseline": {"ms_per_step": round(o_ms, 1), "cores": cores, "kind": "oracle",
+                                      "sample": "fp64 oracle, one layer at 256 rows and the vocabulary projection "
+                                                "of 64 rows, scaled to the step's rows and layers: extrapolated"}})
     eng.set_lock_pattern(None)
     res["surelock_dream7b_b8"] = {
         "workload": f"{cfg.name}: batch {B}, prompt {cfg.prompt_len}, gen {cfg.gen_len} in blocks of "
@@ -384,6 +453,17 @@ def variant_steps(peaks, steps=3, warm=2):
     w = make_weights(m, device="cuda")
     tok0 = make_tokens(cfg).cuda()
     n_resp = B * cfg.gen_len
+    rng = np.random.default_rng(0)
+    lw_host = layer_weights_cpu(w, 0)
+    o_conv, o_row = oracle_layer_cost(m, lw_host, 256, N, rng)
+    o_lm_row = oracle_lm_s(m, w["lm_head"].cpu(), w["g_final"].cpu(), 64, rng) / 64
+    from oracle.model import OracleModel
+    hv = rng.standard_normal((256, m.d_model))
+    om_v = OracleModel(m, lw_host)
+    t = time.perf_counter()
+    om_v.value_only(0, hv)
+    o_probe_row = (time.perf_counter() - t) / 256          # the value-vector probe of one response row
+    cores = host_cores()
     R = max(1, math.ceil(math.log2(cfg.block_len)))
     n_steps = cfg.n_blocks * R
     n_ref = math.ceil(n_steps / cfg.prompt_interval)
@@ -408,7 +488,14 @@ def variant_steps(peaks, steps=3, warm=2):
         roof_p = max(roof_p, vproj)
         roof_f, _ = _step_roofline_ms(peaks, m, [B * N] * m.n_layers, lm_rows, N, B)
         gen_s = (n_ref * t_full + (n_steps - n_ref) * t_part) / 1e3
-        rows.append({"selection": "forced: exactly the cap" if forced else f"cos < {cfg.sim_tau}, capped",
+        o_part = 1e3 * (m.n_layers * o_conv + sum(sel) * o_row + m.n_layers * n_resp * o_probe_row + lm_rows * o_lm_row)
+        o_full = 1e3 * (m.n_layers * (o_conv + B * N * o_row) + lm_rows * o_lm_row)
+        rows.append({"cpu_baseline": {"partial_ms": round(o_part, 1), "refresh_ms": round(o_full, 1), "cores": cores,
+                                      "kind": "oracle",
+                                      "sample": "fp64 oracle, one layer at 256 rows, the value probe of 256 rows and "
+                                                "the vocabulary projection of 64 rows, scaled to the step's rows and "
+                                                "layers: extrapolated"},
+                     "selection": "forced: exactly the cap" if forced else f"cos < {cfg.sim_tau}, capped",
                      "rho_mean": round(float(np.mean(sel)) / n_resp, 4), "sel_rows_per_layer_max": max(sel),
                      "refresh_ms": round(t_full, 3), "partial_ms": round(t_part, 3),
                      "partial_roofline_ms": round(roof_p, 3), "partial_roofline_frac": round(roof_p / t_part, 4),
@@ -502,118 +589,131 @@ def variant_steps(peaks, steps=3, warm=2):
 
 
 # ---------------------------------------------------------------- oracle timing (CPU)
-def oracle_sample_timing(cfg, w_dev, seconds_cap=40.0):
-    """Time the oracle on a bounded sample of the workload on the host cores and
-    extrapolate to one whole generation: one layer at the three row counts a
-    generation uses (all rows at a refresh, the block below the skip layer, the
-    kept rows above it) and the vocabulary projection of the kept rows."""
-    import numpy as np
-    import torch
-
-    from oracle.model import OracleModel
-
+def host_cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] + [1]))
     except Exception:
-        cores = os.cpu_count()
+        return int(os.cpu_count() or 1)
+
+
+def layer_weights_cpu(w, layer):
+    """One layer of a weight dict (device or host tensors) as the oracle's host weights."""
+    lw = {key: w[key][layer:layer + 1].cpu() for key in ("w_qkv", "w_o", "w_gu", "w_down", "g_attn", "g_ffn")}
+    lw["layers"] = [0]
+    return lw
+
+
+def oracle_layer_cost(m, lw, r, N, rng):
+    """(seconds of the fp64 oracle's weight conversion for one layer, seconds per row of the layer
+    itself) from one layer on r rows of one sequence of N positions: every layer of an oracle step
+    converts its weights once, and the rest of its work is linear in its rows."""
+    from oracle.model import OracleModel
+    om = OracleModel(m, lw)
+    K = np.zeros((1, m.n_kv_heads, N, m.head_dim))
+    V = np.zeros_like(K)
+    h = rng.standard_normal((r, m.d_model))
+    pos = np.sort(rng.choice(N, r, replace=False))
+    t = time.perf_counter()
+    om.layer_weights(0)
+    t_conv = time.perf_counter() - t
+    t = time.perf_counter()
+    om.layer(0, h, np.zeros(r, dtype=np.int64), pos, K, V)
+    return t_conv, (time.perf_counter() - t) / r
+
+
+def oracle_layer_s(m, lw, rows, N, rng, cap=None):
+    """Host seconds of one fp64 oracle layer on `rows` rows, its weight conversion included; with a
+    cap, the rows' part is measured at `cap` rows and scaled by rows / cap."""
+    r = rows if cap is None else min(rows, cap)
+    t_conv, t_row = oracle_layer_cost(m, lw, r, N, rng)
+    return t_conv + t_row * rows
+
+
+def oracle_lm_s(m, lm_head, g_final, rows, rng, cap=None):
+    """Host seconds of the oracle's final RMSNorm + vocabulary projection + confidence of `rows`
+    rows (scaled from `cap` rows when capped)."""
+    from oracle.model import OracleModel, lm_confidence
+    r = rows if cap is None else min(rows, cap)
+    om = OracleModel(m, {"lm_head": lm_head, "g_final": g_final, "layers": []})
+    h = rng.standard_normal((r, m.d_model))
+    t = time.perf_counter()
+    lm_confidence(om.logits(h), m.mask_id)
+    return (time.perf_counter() - t) * rows / r
+
+
+def oracle_generation_sample(cfg, layers_w, lm_head, g_final, rng):
+    """One bounded sample of an ES-dLLM generation on the oracle: one layer at each row count a
+    generation uses (every row at a refresh, the block below the skip layer, the kept rows above
+    it) and the vocabulary projection of the block's rows at a refresh and of the kept rows at a
+    skip step.  Returns (generation seconds extrapolated to every step and layer, sample seconds)."""
     m = cfg.model
-    N = cfg.seq_len
-    n_c = cfg.block_len
+    N, n_c = cfg.seq_len, cfg.block_len
     k = cfg.keep_count(n_c)
-    rng = np.random.default_rng(0)
-
-    def layer_time(rows, layer):
-        lw = {key: w_dev[key][layer:layer + 1].cpu() for key in ("w_qkv", "w_o", "w_gu", "w_down", "g_attn",
-                                                                 "g_ffn")}
-        lw.update({"embed": w_dev["embed"], "lm_head": w_dev["lm_head"], "g_final": w_dev["g_final"].cpu(),
-                   "layers": [layer]})
-        om = OracleModel(m, lw)
-        K = np.zeros((1, m.n_kv_heads, N, m.head_dim))
-        V = np.zeros_like(K)
-        h = rng.standard_normal((rows, m.d_model))
-        pos = np.sort(rng.choice(N, rows, replace=False))
-        t = time.perf_counter()
-        om.layer(layer, h, np.zeros(rows, dtype=np.int64), pos, K, V)   # includes its lazy weight conversion
-        return time.perf_counter() - t
-
-    def lm_time(rows):
-        om = OracleModel(m, {"lm_head": w_dev["lm_head"], "g_final": w_dev["g_final"].cpu(), "layers": []})
-        h = rng.standard_normal((rows, m.d_model))
-        t = time.perf_counter()
-        om.logits(h)
-        return time.perf_counter() - t
-
-    t_start = time.perf_counter()
-    t_full = layer_time(N, 0)
-    t_pre = layer_time(n_c, 1)
-    t_post = layer_time(k, 2)
-    t_lm = lm_time(k)
-    spent = time.perf_counter() - t_start
+    B = cfg.batch
+    t0 = time.perf_counter()
+    t_full = oracle_layer_s(m, layers_w[0], N, N, rng)
+    t_pre = oracle_layer_s(m, layers_w[1], n_c, N, rng)
+    t_post = oracle_layer_s(m, layers_w[2], k, N, rng)
+    t_lm_ref = oracle_lm_s(m, lm_head, g_final, n_c, rng)
+    t_lm = oracle_lm_s(m, lm_head, g_final, k, rng)
+    spent = time.perf_counter() - t0
     steps_per_block = math.ceil(cfg.block_len / cfg.tokens_per_step)
-    n_ref = cfg.n_blocks
-    n_skip = cfg.n_blocks * (steps_per_block - 1)
+    n_ref, n_skip = cfg.n_blocks, cfg.n_blocks * (steps_per_block - 1)
     L, ls = m.n_layers, cfg.skip_layer
-    gen_s = n_ref * (L * t_full + t_lm) + n_skip * (ls * t_pre + (L - ls) * t_post + t_lm)
-    return {"value": round(cfg.batch * cfg.gen_len / gen_s, 6), "unit": "tokens/s", "cores": int(cores),
-            "kind": "oracle",
-            "sample": (f"fp64 oracle on one layer at {N}, {n_c} and {k} rows and the vocabulary projection of "
-                       f"{k} rows ({spent:.1f} s of host time, weight conversion included), extrapolated to "
-                       f"{n_ref} refresh + {n_skip} skip steps of {L} layers")}
+    gen_s = B * (n_ref * (L * t_full + t_lm_ref) + n_skip * (ls * t_pre + (L - ls) * t_post + t_lm))
+    return gen_s, spent
+
+
+def generation_sample_desc(cfg):
+    m = cfg.model
+    k = cfg.keep_count(cfg.block_len)
+    steps_per_block = math.ceil(cfg.block_len / cfg.tokens_per_step)
+    return (f"fp64 oracle, per sample: one layer at {cfg.seq_len}, {cfg.block_len} and {k} rows and the "
+            f"vocabulary projection of {cfg.block_len} and {k} rows (weight conversion included), extrapolated "
+            f"to {cfg.n_blocks} refresh + {cfg.n_blocks * (steps_per_block - 1)} skip steps of {m.n_layers} layers")
+
+
+def oracle_sample_timing(cfg, w_dev):
+    """cpu_baseline of our arm: the oracle on one sample of the generation (host cores)."""
+    rng = np.random.default_rng(0)
+    layers_w = [layer_weights_cpu(w_dev, l) for l in range(3)]
+    gen_s, spent = oracle_generation_sample(cfg, layers_w, w_dev["lm_head"].cpu(), w_dev["g_final"].cpu(), rng)
+    return {"value": round(cfg.batch * cfg.gen_len / gen_s, 6), "unit": "tokens/s", "cores": host_cores(),
+            "kind": "oracle", "sample": generation_sample_desc(cfg) + f" ({spent:.1f} s of host time)"}
 
 
 # ---------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args):
-    import numpy as np
-
-    from oracle.model import OracleModel
     from synth import get_config
+    from synth.gen import make_weights
 
     cfg = get_config(args.workload)
     m = cfg.model
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
-    # weights of the sampled layers only (host, bf16 values), seeded like the GPU arm's draw
-    import torch
-    from synth.gen import make_weights
-    w = make_weights(m, device="cpu", layers=[0], with_vocab=False)
-    N, n_c, k = cfg.seq_len, cfg.block_len, cfg.keep_count(cfg.block_len)
+    # host weights of the three sampled layers and the vocabulary, seeded like the GPU arm's draw
+    w = make_weights(m, device="cpu", layers=[0, 1, 2])
+    layers_w = [layer_weights_cpu(w, i) for i in range(3)]
     rng = np.random.default_rng(0)
-
-    def one_sample():
-        """One skip step's worth of the layer stack, scaled to a whole generation.  Each
-        layer call converts its weights, as the oracle does for every layer of a run."""
-        K = np.zeros((1, m.n_kv_heads, N, m.head_dim))
-        V = np.zeros_like(K)
-        t = time.perf_counter()
-        OracleModel(m, w).layer(0, rng.standard_normal((n_c, m.d_model)), np.zeros(n_c, np.int64),
-                                np.arange(n_c), K, V)
-        t_pre = time.perf_counter() - t
-        t = time.perf_counter()
-        OracleModel(m, w).layer(0, rng.standard_normal((k, m.d_model)), np.zeros(k, np.int64), np.arange(k), K, V)
-        t_post = time.perf_counter() - t
-        steps = cfg.n_blocks * math.ceil(cfg.block_len / cfg.tokens_per_step)
-        return steps * (cfg.skip_layer * t_pre + (m.n_layers - cfg.skip_layer) * t_post)
-
     for _ in range(args.warmup):
-        one_sample()
-    times = [one_sample() for _ in range(args.steps)]
-    gen_s = sum(times)
-    value = cfg.batch * cfg.gen_len * args.steps / gen_s
+        oracle_generation_sample(cfg, layers_w, w["lm_head"], w["g_final"], rng)
+    gens, samples = [], []
+    for _ in range(args.steps):
+        g, sp = oracle_generation_sample(cfg, layers_w, w["lm_head"], w["g_final"], rng)
+        gens.append(g)
+        samples.append(sp)
+    value = cfg.batch * cfg.gen_len * args.steps / sum(gens)
+    desc = generation_sample_desc(cfg)
     line = {"metric": METRIC, "value": round(value, 6), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(1e3 * gen_s / args.steps, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+            "warmup": args.warmup, "ms_per_step": round(1e3 * sum(samples) / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
             "data": "synthetic: seeded random-init N(0,0.02) bf16 weights, uniform-random prompt ids",
             "config": {"workload": workload_desc(cfg), "batch": cfg.batch, "seq_len": cfg.seq_len,
-                       "gen_len": cfg.gen_len, "step": "one whole generation, extrapolated from a sample",
+                       "gen_len": cfg.gen_len,
+                       "step": "one bounded sample of the generation (ms_per_step is its host time); value is the "
+                               "generation's tokens/s extrapolated from the samples",
                        "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
-                             "sample": ("per step: one layer of the fp64 oracle at the block's rows and at the "
-                                        "kept rows (weight conversion included), scaled to every skip step "
-                                        "and layer of the generation")},
+            "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                             "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

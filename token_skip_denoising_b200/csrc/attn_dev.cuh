@@ -257,12 +257,43 @@ __device__ __forceinline__ void attn_item(const AttnParams& p, int qt, int b, in
 // Merge of the split partials for one (row, head), one warp (lane 0..31).
 template <int HD>
 __device__ __forceinline__ void attn_merge(const AttnParams& p, int row, int h, int lane) {
+  constexpr int PER = HD / 32;
+  constexpr int kMaxUnrolled = 8;
+  if (p.splits <= kMaxUnrolled) {
+    // every split's (m, l) and partial row requested at once: two round trips in all
+    float2 v[kMaxUnrolled];
+#pragma unroll
+    for (int s = 0; s < kMaxUnrolled; ++s)
+      v[s] = s < p.splits ? __ldcg(&p.ml[(static_cast<int64_t>(s) * p.rows_cap + row) * p.Hq + h])
+                          : make_float2(-INFINITY, 0.f);
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxUnrolled; ++s) M = fmaxf(M, v[s].x);
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    float L = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxUnrolled; ++s) {
+      if (s < p.splits) {
+        const int64_t base = (static_cast<int64_t>(s) * p.rows_cap + row) * p.Hq + h;
+        const float w = (v[s].x == -INFINITY) ? 0.f : exp2f(v[s].x - M);
+        L += w * v[s].y;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] += w * __ldcg(p.opart + base * HD + lane + 32 * i);
+      }
+    }
+    const float inv = 1.f / L;
+    __nv_bfloat16* dst = p.out + (static_cast<int64_t>(row) * p.Hq + h) * HD;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) dst[lane + 32 * i] = __float2bfloat16(acc[i] * inv);
+    return;
+  }
   float M = -INFINITY;
   for (int s = 0; s < p.splits; ++s) {
     const float2 v = __ldcg(&p.ml[(static_cast<int64_t>(s) * p.rows_cap + row) * p.Hq + h]);
     M = fmaxf(M, v.x);
   }
-  constexpr int PER = HD / 32;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;

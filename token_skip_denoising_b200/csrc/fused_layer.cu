@@ -109,6 +109,7 @@ struct FParams {
   attn::AttnParams ap;    // q, out (O operand), seq_off, split partials (caches set per layer)
   int attn_qtiles;
   int attn_items;
+  int attn_group_merge;   // every item in one round: the splits of a group merge together
   int* attn_ctr;          // [B * Hkv * attn_qtiles] split arrivals, zero between uses
   int* sync;              // [S_COUNT] phase counters + exit counter + abort word, zero at launch
   FusedEs es;             // per-layer re-selection at the start of every layer (es.on)
@@ -575,23 +576,39 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         const int pairs = p.qkvd >> 1;
         const int64_t total = static_cast<int64_t>(m_rows) * pairs;
-        for (int64_t uu = gt; uu < total; uu += gstride) {
-          const int jr = static_cast<int>(uu / pairs);
-          const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
-          const int pi = rr % half;
-          const int n_lo = (rr / half) * p.hd + pi;
-          const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
+        constexpr int U = 4;                    // pairs per thread in flight: their loads go out together
+        for (int64_t u0 = gt; u0 < total; u0 += U * gstride) {
+          float xl[U], xh[U], cs[U], sn[U];
+          int jrs[U], nlo[U], pis[U];
+#pragma unroll
+          for (int e = 0; e < U; ++e) {
+            const int64_t uu = u0 + e * gstride < total ? u0 + e * gstride : 0;   // in bounds either way
+            const int jr = static_cast<int>(uu / pairs);
+            const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
+            pis[e] = rr % half;
+            nlo[e] = (rr / half) * p.hd + pis[e];
+            jrs[e] = jr;
+            const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
+            xl[e] = __ldcg(srow + nlo[e]);
+            xh[e] = __ldcg(srow + nlo[e] + half);
+            const int flat = s_rows[jr];
+            const int pos = flat - (flat / p.N) * p.N;
+            cs[e] = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pis[e]);
+            sn[e] = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pis[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < U; ++e) {
+          if (u0 + e * gstride >= total) break;
+          const int jr = jrs[e], n_lo = nlo[e], pi = pis[e];
           const float ri = s_rinv1[jr];
-          const float xl = __ldcg(srow + n_lo) * ri, xh = __ldcg(srow + n_lo + half) * ri;
+          const float x_l = xl[e] * ri, x_h = xh[e] * ri;
           const int flat = s_rows[jr];
           const int b = flat / p.N;
           const int pos = flat - b * p.N;
-          float yl = xl, yh = xh;
+          float yl = x_l, yh = x_h;
           if (n_lo < p.qd + p.kvd) {
-            const float cs = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pi);
-            const float sn = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pi);
-            yl = xl * cs - xh * sn;
-            yh = xh * cs + xl * sn;
+            yl = x_l * cs[e] - x_h * sn[e];
+            yh = x_h * cs[e] + x_l * sn[e];
           }
           if (n_lo < p.qd) {
             __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
@@ -608,6 +625,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
             __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
             dst[0] = __float2bfloat16(yl);
             dst[half] = __float2bfloat16(yh);
+          }
           }
         }
       }
@@ -629,7 +647,27 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           const int b = rem / ap.Hkv;
           if (p.hd == 128) attn::attn_item<128>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
           else attn::attn_item<64>(ap, qt, b, kvh, split, attn_smem, t, NamedBar{});
-          if (ap.splits > 1) {
+          if (ap.splits > 1 && p.attn_group_merge) {
+            // every split of the group is another CTA's item of this same round, all resident:
+            // each waits for all of them, then merges its share of the query tile's units
+            __threadfence();
+            epi_bar();
+            const int grp = (b * ap.Hkv + kvh) * p.attn_qtiles + qt;
+            if (t == 0) atomicAdd(p.attn_ctr + grp, 1);
+            if (epi_wait_phase(p.attn_ctr + grp, ap.splits, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
+              const int off = ap.seq_off[b];
+              const int n_units = (ap.seq_off[b + 1] - off) * Gq;
+              const int u1 = min(n_units, (qt + 1) * 64);
+              for (int uu = qt * 64 + split + ap.splits * warp; uu < u1; uu += 4 * ap.splits) {
+                const int row = off + uu / Gq, hh = kvh * Gq + uu % Gq;
+                if (p.hd == 128) attn::attn_merge<128>(ap, row, hh, lane);
+                else attn::attn_merge<64>(ap, row, hh, lane);
+              }
+            }
+            // a second arrival once the partials are read: the last one re-arms the counter
+            epi_bar();
+            if (t == 0 && atomicAdd(p.attn_ctr + grp, 1) == 2 * ap.splits - 1) p.attn_ctr[grp] = 0;
+          } else if (ap.splits > 1) {
             __threadfence();
             epi_bar();
             const int grp = (b * ap.Hkv + kvh) * p.attn_qtiles + qt;
@@ -665,13 +703,26 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       if (epi_wait_phase(p.sync + S_GU, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         const int f4 = p.F >> 2;
         const int64_t total = static_cast<int64_t>(m_rows) * f4;
-        for (int64_t uu = gt; uu < total; uu += gstride) {
+        constexpr int U = 4;                    // groups per thread in flight: their loads go out together
+        for (int64_t u0 = gt; u0 < total; u0 += U * gstride) {
+          float4 g4s[U], u4s[U];
+#pragma unroll
+          for (int e = 0; e < U; ++e) {
+            const int64_t uu = u0 + e * gstride < total ? u0 + e * gstride : 0;   // in bounds either way
+            const int jr = static_cast<int>(uu / f4);
+            const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * f4) * 4;
+            const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
+            g4s[e] = __ldcg(reinterpret_cast<const float4*>(srow + f));
+            u4s[e] = __ldcg(reinterpret_cast<const float4*>(srow + p.F + f));
+          }
+#pragma unroll
+          for (int e = 0; e < U; ++e) {
+          const int64_t uu = u0 + e * gstride;
+          if (uu >= total) break;
           const int jr = static_cast<int>(uu / f4);
           const int f = static_cast<int>(uu - static_cast<int64_t>(jr) * f4) * 4;
-          const float* srow = p.s_gu + static_cast<int64_t>(jr) * 2 * p.F;
           const float ri = s_rinv2[jr];
-          const float4 g4 = __ldcg(reinterpret_cast<const float4*>(srow + f));
-          const float4 u4 = __ldcg(reinterpret_cast<const float4*>(srow + p.F + f));
+          const float4 g4 = g4s[e], u4 = u4s[e];
           const float g[4] = {g4.x * ri, g4.y * ri, g4.z * ri, g4.w * ri};
           const float u[4] = {u4.x * ri, u4.y * ri, u4.z * ri, u4.w * ri};
           float a[4];
@@ -683,6 +734,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
           pk.x = *reinterpret_cast<uint32_t*>(&lo);
           pk.y = *reinterpret_cast<uint32_t*>(&hi);
           *reinterpret_cast<uint2*>(p.act + static_cast<int64_t>(jr) * p.F + f) = pk;
+          }
         }
       }
       signal_phase(p.sync + S_SWIGLU, t);
@@ -839,6 +891,7 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   ap.opart = a.attn_opart; ap.ml = a.attn_ml;
   p.attn_qtiles = qtiles;
   p.attn_items = a.B * a.Hkv * qtiles * splits;
+  p.attn_group_merge = p.attn_items <= grid ? 1 : 0;
   p.attn_ctr = a.attn_ctr;
   p.sync = a.sync;
   p.es = a.es;

@@ -137,6 +137,126 @@ def fused_case(rows, reps, layers=3):
             "bytes": byts, "flops": flops}
 
 
+def _copies_of(make, nbytes):
+    """Enough copies of an input set that their total exceeds L2 (used round-robin)."""
+    return [make(i) for i in range(_copies(nbytes))]
+
+
+def score_es_case(rows, reps, d=4096):
+    """ES-dLLM Eq. 1 over `rows` candidates (two fp32 hidden states per row)."""
+    g = torch.Generator(device="cuda").manual_seed(3)
+    nbytes = 2 * rows * d * 4
+    sets = _copies_of(lambda i: (torch.randn((rows, d), generator=g, device="cuda"),
+                                 torch.randn((rows, d), generator=g, device="cuda")), nbytes)
+    conf = torch.rand((rows,), generator=g, device="cuda")
+    mp = (torch.rand((rows,), generator=g, device="cuda") < 0.5).to(torch.uint8)
+    fn = lambda i: ops.score_es(sets[i % len(sets)][0], sets[i % len(sets)][1], conf, 0.5, masked_prev=mp)
+    t = _time(fn, reps)
+    byts = nbytes + rows * 9
+    return {"case": f"score_es_n{rows}", "ms": t, "gbs": byts / t / 1e6, "tflops": 0.0, "bytes": byts, "flops": 0}
+
+
+def score_cos_case(reps, B=4, N=5120, n_resp=1024, Hkv=32, hd=128):
+    """dLLM-Cache value cosine of the response rows (long-context LLaDA-8B shape, batch 4)."""
+    g = torch.Generator(device="cuda").manual_seed(4)
+    rows = B * n_resp
+    kvd = Hkv * hd
+    nbytes = rows * kvd * 4 + rows * kvd * 2
+    sets = _copies_of(lambda i: (torch.randn((rows, kvd), generator=g, device="cuda"),
+                                 torch.randn((B, Hkv, N, hd), generator=g, device="cuda").to(torch.bfloat16)), nbytes)
+    rmap = torch.tensor([b * N + (N - n_resp) + p for b in range(B) for p in range(n_resp)], dtype=torch.int32,
+                        device="cuda")
+    fn = lambda i: ops.score_cos(sets[i % len(sets)][0], sets[i % len(sets)][1], rmap, N, Hkv, hd)
+    t = _time(fn, reps)
+    return {"case": f"score_cos_n{rows}", "ms": t, "gbs": nbytes / t / 1e6, "tflops": 0.0, "bytes": nbytes,
+            "flops": 0}
+
+
+def rmsnorm_case(rows, reps, d=4096):
+    """Gathered RMSNorm of `rows` rows of the fp32 hidden state into the bf16 GEMM operand."""
+    g = torch.Generator(device="cuda").manual_seed(5)
+    nbytes = rows * d * 6
+    sets = _copies_of(lambda i: torch.randn((rows, d), generator=g, device="cuda"), nbytes)
+    gain = torch.ones(d, device="cuda")
+    z = torch.empty((rows, d), dtype=torch.bfloat16, device="cuda")
+    fn = lambda i: ops.rmsnorm_rows(sets[i % len(sets)], gain, 1e-5, z=z)
+    t = _time(fn, reps)
+    return {"case": f"rmsnorm_m{rows}", "ms": t, "gbs": nbytes / t / 1e6, "tflops": 0.0, "bytes": nbytes,
+            "flops": 0}
+
+
+def select_case(n, k, reps, B=1):
+    """Top-k of n scores per sequence (the ES-dLLM choice at the single-layer benchmark's size)."""
+    g = torch.Generator(device="cuda").manual_seed(6)
+    s = torch.rand((B * n,), generator=g, device="cuda")
+    fn = lambda i: ops.select(s, B, n, ops.SEL_TOPK_DESC, k)
+    t = _time(fn, reps)
+    return {"case": f"select_n{n}_k{k}", "ms": t, "gbs": B * n * 4 / t / 1e6, "tflops": 0.0, "bytes": B * n * 4,
+            "flops": 0}
+
+
+def unmask_case(reps, B=4, N=5120, blk=64):
+    """Top-1 confidence unmasking of the current block of B sequences."""
+    g = torch.Generator(device="cuda").manual_seed(7)
+    tokens = torch.full((B, N), 999, dtype=torch.int32, device="cuda")
+    conf = torch.rand((B * N,), generator=g, device="cuda")
+    amax = torch.randint(0, 998, (B * N,), generator=g, device="cuda", dtype=torch.int32)
+
+    def fn(i):
+        tokens[:, N - blk:] = 999                            # the block is masked again every call
+        ops.unmask(tokens, conf, amax, N - blk, blk, 999, 1, max_out=1)
+    t = _time(fn, reps)
+    return {"case": f"unmask_b{B}_blk{blk}", "ms": t, "gbs": 0.0, "tflops": 0.0, "bytes": 0, "flops": 0}
+
+
+def attn_gqa_case(rows, reps, N=1536, Hq=28, Hkv=4, hd=128):
+    """Attention of `rows` queries over N keys, GQA 28/4 (Dream-7B shape)."""
+    from synth.configs import DREAM7B
+    g = torch.Generator(device="cuda").manual_seed(8)
+    kvb = 2 * Hkv * N * hd * 2
+    ncop = _copies(kvb)
+    caches = [(torch.randn((1, Hkv, N, hd), generator=g, device="cuda").to(torch.bfloat16),
+               torch.randn((1, Hkv, N, hd), generator=g, device="cuda").to(torch.bfloat16)) for _ in range(ncop)]
+    q = torch.randn((rows, Hq * hd), generator=g, device="cuda").to(torch.bfloat16)
+    off = torch.tensor([0, rows], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256 << 20, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    fn = lambda i: ops.attention(q, caches[i % ncop][0], caches[i % ncop][1], off, DREAM7B, rows, out=out, ws=ws)
+    t = _time(fn, reps)
+    byts = kvb + 2 * rows * Hq * hd * 2
+    flops = 4.0 * rows * N * Hq * hd
+    return {"case": f"attn_gqa_m{rows}_n{N}", "ms": t, "gbs": byts / t / 1e6, "tflops": flops / t / 1e9,
+            "bytes": byts, "flops": flops}
+
+
+def surelock_step_case(reps, layers=2):
+    """One SureLock step of a Dream-7B-shaped model cut to `layers` layers (batch 1, prompt 256, gen
+    64): the vocabulary projection of every recomputed row into stored bf16 logits, then the KL step
+    (KL against the previous step's logits, confidence, locks).  Times whole steps."""
+    from synth import get_config, make_tokens, make_weights
+    from synth.configs import scaled
+    from .engine import Engine
+    cfg = scaled(get_config("dream_surelock"), n_layers=layers).replace(batch=1, prompt_len=256, gen_len=64)
+    w = make_weights(cfg.model, device="cuda")
+    eng = Engine(cfg, w, make_tokens(cfg).cuda())
+    for _ in range(2):
+        eng.step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(max(3, reps // 4)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        eng.step()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    t = statistics.median(ts)
+    n_lm = int(eng.buffer("nlmrows")[0])
+    kl_bytes = 3 * n_lm * cfg.model.vocab * 2       # this step's logits twice, the previous step's once
+    return {"case": f"surelock_step_l{layers}", "ms": t, "gbs": 0.0, "tflops": 0.0, "bytes": kl_bytes, "flops": 0,
+            "lm_rows": n_lm}
+
+
 CASES = {
     **{f"gemm_{k}_m{m}": (lambda k=k, m=m, **kw: gemm_case(k, m, **kw))
        for k in ("qkv", "o", "gu", "down") for m in (7, 32, 768)},
@@ -147,6 +267,14 @@ CASES = {
     "attn_m768": lambda **kw: attn_case(768, **kw),
     "fused_m7_l3": lambda **kw: fused_case(7, **kw),
     "fused_m32_l3": lambda **kw: fused_case(32, **kw),
+    "score_es_n8192": lambda **kw: score_es_case(8192, **kw),
+    "score_cos_n4096": lambda **kw: score_cos_case(**kw),
+    "rmsnorm_m8192": lambda **kw: rmsnorm_case(8192, **kw),
+    "select_n2048_k205": lambda **kw: select_case(2048, 205, **kw),
+    "unmask_b4": lambda **kw: unmask_case(**kw),
+    "attn_gqa_m1536": lambda **kw: attn_gqa_case(1536, **kw),
+    "attn_gqa_m7": lambda **kw: attn_gqa_case(7, **kw),
+    "surelock_step_l2": lambda **kw: surelock_step_case(**kw),
 }
 
 
@@ -165,7 +293,7 @@ def main():
             kw.update(splits=a.splits)
             if "gu" not in n:
                 kw.update(bn=a.bn)
-        elif n.startswith("attn"):
+        elif n.startswith("attn") and "gqa" not in n:
             kw.update(splits=a.splits)
         r = CASES[n](**kw)
         if a.json:
