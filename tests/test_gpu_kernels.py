@@ -306,6 +306,28 @@ def test_kl_conf_matches_oracle():
     assert abs(g[1]) < 2e-5 and np.all(g[ok] >= 0)
 
 
+def test_kl_conf_large_vocab_and_shape_guard():
+    """The one-pass statistics at the Dream-7B vocabulary (152064 = 8 x 19008, several thousand
+    16-byte loads per thread) against fp64, and a vocabulary that is not a multiple of 8 refused
+    (the kernel reads rows in 16-byte vectors)."""
+    rows, V = 3, 152064
+    z = _bf16((rows, V), 41, 3.0)
+    zp = _bf16((rows, V), 42, 3.0)
+    zf, zpf = _f64(z), _f64(zp)
+    lse_p = torch.tensor([float(np.log(np.exp(r - r.max()).sum()) + r.max()) for r in zpf], dtype=torch.float32)
+    has = torch.ones(rows, dtype=torch.int32)
+    conf, amax, lse, kl = ops.kl_conf(z.to(DEV), V - 1, rows=torch.arange(rows, dtype=torch.int32).to(DEV),
+                                      zp_store=zp.to(DEV), lse_prev=lse_p.to(DEV), has_prev=has.to(DEV))
+    rc, rt, rl = om.lm_confidence(zf, V - 1)
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=1e-6, atol=1e-5)
+    np.testing.assert_array_equal(amax.cpu().numpy(), rt)
+    np.testing.assert_allclose(conf.cpu().numpy(), rc, rtol=1e-4)
+    np.testing.assert_allclose(kl.cpu().numpy(), op.kl_from_logits(zf, rl, zpf, _f64(lse_p)), rtol=1e-3, atol=2e-5)
+    from token_skip_denoising_b200._lib import DllmError
+    with pytest.raises(DllmError):
+        ops.kl_conf(_bf16((2, 1001), 43).to(DEV), 1000)
+
+
 # ------------------------------------------------------------------ selection (bit-exact)
 
 def _scores_with_ties(B, n, seed):

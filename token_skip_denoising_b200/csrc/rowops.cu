@@ -154,15 +154,25 @@ __global__ void score_cos_kernel(const float* __restrict__ vnew, int64_t ldv, co
   if (wid >= m) return;
   const int flat = rows[wid];
   const int b = flat / N, pos = flat % N;
+  // one warp per row, 8 elements per lane and step: 16 bytes of the cached V row, 32 of v_new
+  const int chunks = Hkv * hd / 8;
+  const int per_head = hd / 8;
+  const float* nv = vnew + static_cast<int64_t>(wid) * ldv;
   float dot = 0.f, na = 0.f, nb = 0.f;
-  for (int kvh = 0; kvh < Hkv; ++kvh) {
-    const __nv_bfloat16* cv = vc + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd;
-    const float* nv = vnew + static_cast<int64_t>(wid) * ldv + kvh * hd;
-    for (int i = lane; i < hd; i += 32) {
-      const float a = nv[i], c = __bfloat162float(cv[i]);
-      dot += a * c;
-      na += a * a;
-      nb += c * c;
+#pragma unroll 4
+  for (int c = lane; c < chunks; c += 32) {
+    const int kvh = c / per_head, off = (c - kvh * per_head) * 8;
+    const uint4 cv = __ldg(reinterpret_cast<const uint4*>(vc + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd + off));
+    const float4 a0 = __ldg(reinterpret_cast<const float4*>(nv + c * 8));
+    const float4 a1 = __ldg(reinterpret_cast<const float4*>(nv + c * 8 + 4));
+    const __nv_bfloat162* cp = reinterpret_cast<const __nv_bfloat162*>(&cv);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 cf = __bfloat1622float2(cp[e]);
+      dot += av[2 * e] * cf.x + av[2 * e + 1] * cf.y;
+      na += av[2 * e] * av[2 * e] + av[2 * e + 1] * av[2 * e + 1];
+      nb += cf.x * cf.x + cf.y * cf.y;
     }
   }
   dot = warp_sum_f(dot);
@@ -177,6 +187,88 @@ __global__ void score_cos_kernel(const float* __restrict__ vnew, int64_t ldv, co
 }
 
 // ------------------------------------------------------------------ SureLock KL + confidence
+// Statistics of one logit row z [V] (bf16), by the whole CTA in one pass of 16-byte loads:
+// M = max z, S = sum exp(z - M), the argmax over v != mask_id (ties to the lower id), and with
+// a previous row zp: T = sum exp(z - M) (z - zp).  The running (M, S, T) of a thread is
+// rescaled by exp(M_old - M_new) whenever its maximum grows (online softmax).  Then
+// lse = M + log S, p(v) = exp(z - lse), and KL(p || p_prev) = sum p (z - lse - zp + lse_p)
+// = T / S - (lse - lse_p).  V % 8 == 0 and 16-byte aligned rows.
+struct RowStats {
+  float M, S, T, BV;
+  int BI;
+};
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+__device__ __forceinline__ RowStats row_stats(const __nv_bfloat16* __restrict__ z, const __nv_bfloat16* __restrict__ zp,
+                                              int V, int mask_id, float* s_f, int* s_i) {
+  float m = -INFINITY, sum = 0.f, tt = 0.f, bv = -INFINITY;
+  int bi = 0x7fffffff;
+  const uint4* z4 = reinterpret_cast<const uint4*>(z);
+  const uint4* p4 = reinterpret_cast<const uint4*>(zp);
+  const int n8 = V >> 3;
+#pragma unroll 2
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    float x[8];
+    unpack8(__ldg(z4 + i), x);
+    float y[8];
+    if (zp) unpack8(__ldg(p4 + i), y);
+    float lm = x[0];
+#pragma unroll
+    for (int e = 1; e < 8; ++e) lm = fmaxf(lm, x[e]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int v = i * 8 + e;
+      if (v != mask_id && (x[e] > bv || (x[e] == bv && v < bi))) { bv = x[e]; bi = v; }
+    }
+    if (lm > m) {
+      const float r = __expf(m - lm);
+      sum *= r;
+      tt *= r;
+      m = lm;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float ex = __expf(x[e] - m);
+      sum += ex;
+      if (zp) tt += ex * (x[e] - y[e]);
+    }
+  }
+  // combine the threads: warps by shuffles, then the warps through shared memory
+  auto combine = [](float& m1, float& s1, float& t1, float& b1, int& i1, float m2, float s2, float t2, float b2, int i2) {
+    const float mn = fmaxf(m1, m2);
+    const float r1 = m1 == -INFINITY ? 0.f : __expf(m1 - mn), r2 = m2 == -INFINITY ? 0.f : __expf(m2 - mn);
+    s1 = s1 * r1 + s2 * r2;
+    t1 = t1 * r1 + t2 * r2;
+    m1 = mn;
+    if (b2 > b1 || (b2 == b1 && i2 < i1)) { b1 = b2; i1 = i2; }
+  };
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    const float t2 = __shfl_xor_sync(0xffffffffu, tt, o), b2 = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+    combine(m, sum, tt, bv, bi, m2, s2, t2, b2, i2);
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (l == 0) {
+    s_f[4 * w] = m; s_f[4 * w + 1] = sum; s_f[4 * w + 2] = tt; s_f[4 * w + 3] = bv;
+    s_i[w] = bi;
+  }
+  __syncthreads();
+  RowStats r;
+  r.M = s_f[0]; r.S = s_f[1]; r.T = s_f[2]; r.BV = s_f[3]; r.BI = s_i[0];
+  for (int q = 1; q < nw; ++q)
+    combine(r.M, r.S, r.T, r.BV, r.BI, s_f[4 * q], s_f[4 * q + 1], s_f[4 * q + 2], s_f[4 * q + 3], s_i[q]);
+  __syncthreads();
+  return r;
+}
 // For LM row j with logits z[j, :] (bf16): lse, conf = p(argmax over v != mask), argmax,
 // and when has_prev: D = sum_v p_t (z_t - lse_t - z_p + lse_p), clamped at 0.
 // One CTA (256 threads) per row.
@@ -191,87 +283,22 @@ __global__ void kl_conf_kernel(const __nv_bfloat16* __restrict__ z, int64_t ldz,
   const int j = blockIdx.x;
   if (j >= m) return;
   const int flat = rows ? rows[j] : j;
-  const __nv_bfloat16* zr = z + static_cast<int64_t>(j) * ldz;
-  __shared__ float sf[32];
-  __shared__ int si[32];
-  // pass 1: max and argmax (mask id excluded from the argmax)
-  float mx = -INFINITY, bv = -INFINITY;
-  int bi = 0x7fffffff;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) {
-    const float x = __bfloat162float(zr[v]);
-    mx = fmaxf(mx, x);
-    if (v != mask_id && (x > bv || (x == bv && v < bi))) { bv = x; bi = v; }
-  }
-  for (int o = 16; o; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-  }
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
-  if (l == 0) { sf[w] = mx; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int i = 0; i < nw; ++i) M = fmaxf(M, sf[i]);
-    sf[31] = M;
-  }
-  __syncthreads();
-  const float M = sf[31];
-  __syncthreads();
-  if (l == 0) { sf[w] = bv; si[w] = bi; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float B = -INFINITY;
-    int I = 0x7fffffff;
-    for (int i = 0; i < nw; ++i)
-      if (sf[i] > B || (sf[i] == B && si[i] < I)) { B = sf[i]; I = si[i]; }
-    sf[30] = B;
-    si[30] = I;
-  }
-  __syncthreads();
-  const float BV = sf[30];
-  const int BI = si[30];
-  __syncthreads();
-  // pass 2: sum exp
-  float se = 0.f;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) se += __expf(__bfloat162float(zr[v]) - M);
-  se = warp_sum_f(se);
-  if (l == 0) sf[w] = se;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float S = 0.f;
-    for (int i = 0; i < nw; ++i) S += sf[i];
-    sf[29] = S;
-  }
-  __syncthreads();
-  const float L = M + logf(sf[29]);
+  __shared__ float s_f[4 * 32];
+  __shared__ int s_i[32];
   const bool hp = has_prev && has_prev[flat];
-  float kl = 0.f;
-  if (hp) {
-    const __nv_bfloat16* pr = zp_store + static_cast<int64_t>(flat) * ldp;
-    const float Lp = lse_prev[flat];
-    for (int v = threadIdx.x; v < V; v += blockDim.x) {
-      const float zt = __bfloat162float(zr[v]) - L;
-      const float zq = __bfloat162float(pr[v]) - Lp;
-      kl += __expf(zt) * (zt - zq);
-    }
-    kl = warp_sum_f(kl);
-    __syncthreads();
-    if (l == 0) sf[w] = kl;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float K = 0.f;
-      for (int i = 0; i < nw; ++i) K += sf[i];
-      sf[28] = fmaxf(K, 0.f);
-    }
-    __syncthreads();
-  }
+  const RowStats r = row_stats(z + static_cast<int64_t>(j) * ldz, hp ? zp_store + static_cast<int64_t>(flat) * ldp : nullptr,
+                               V, mask_id, s_f, s_i);
   if (threadIdx.x == 0) {
-    conf[flat] = __expf(BV - L);
+    const float L = r.M + logf(r.S);
+    int BI = r.BI;
+    if (BI == 0x7fffffff) {   // no finite logit: report it, and never hand on an invalid token id
+      set_dev_status(DLLM_DEV_BAD_INDEX);
+      BI = 0;
+    }
+    conf[flat] = __expf(r.BV - L);
     amax[flat] = BI;
     if (lse_out) lse_out[flat] = L;
-    if (kl_out) kl_out[j] = hp ? sf[28] : NAN;
+    if (kl_out) kl_out[j] = hp ? fmaxf(r.T / r.S - (L - lse_prev[flat]), 0.f) : NAN;
   }
 }
 
@@ -571,90 +598,21 @@ __global__ void kl_step_kernel(KlStep k) {
   if (j >= m) return;
   const int flat = k.rows[j];
   const int V = k.V;
-  const __nv_bfloat16* zr = k.z_cur + static_cast<int64_t>(flat) * V;
-  __shared__ float sf[32];
-  __shared__ int si[32];
-  __shared__ float s_res[4];
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
-  float mx = -INFINITY, bv = -INFINITY;
-  int bi = 0x7fffffff;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) {
-    const float x = __bfloat162float(zr[v]);
-    mx = fmaxf(mx, x);
-    if (v != k.mask_id && (x > bv || (x == bv && v < bi))) { bv = x; bi = v; }
-  }
-  for (int o = 16; o; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-  }
-  if (l == 0) { sf[w] = mx; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int i = 0; i < nw; ++i) M = fmaxf(M, sf[i]);
-    s_res[0] = M;
-  }
-  __syncthreads();
-  const float M = s_res[0];
-  __syncthreads();
-  if (l == 0) { sf[w] = bv; si[w] = bi; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float B = -INFINITY;
-    int I = 0x7fffffff;
-    for (int i = 0; i < nw; ++i)
-      if (sf[i] > B || (sf[i] == B && si[i] < I)) { B = sf[i]; I = si[i]; }
-    if (I == 0x7fffffff) {   // no finite logit: report it, and never hand on an invalid token id
-      set_dev_status(DLLM_DEV_BAD_INDEX);
-      I = 0;
-    }
-    s_res[1] = B;
-    si[31] = I;
-  }
-  __syncthreads();
-  const float BV = s_res[1];
-  const int BI = si[31];
-  __syncthreads();
-  float se = 0.f;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) se += __expf(__bfloat162float(zr[v]) - M);
-  se = warp_sum_f(se);
-  if (l == 0) sf[w] = se;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float S = 0.f;
-    for (int i = 0; i < nw; ++i) S += sf[i];
-    s_res[2] = M + logf(S);
-  }
-  __syncthreads();
-  const float L = s_res[2];
+  __shared__ float s_f[4 * 32];
+  __shared__ int s_i[32];
   // stamps hold step + 1 of the last store, so a store at the previous step reads k.step
   const bool has_prev = k.stamp && k.z_prev && k.step > 0 && k.stamp[flat] == k.step;
-  float kl = NAN;
-  if (has_prev) {
-    const __nv_bfloat16* pr = k.z_prev + static_cast<int64_t>(flat) * V;
-    const float Lp = k.lse_prev[flat];
-    float acc = 0.f;
-    for (int v = threadIdx.x; v < V; v += blockDim.x) {
-      const float zt = __bfloat162float(zr[v]) - L;
-      const float zq = __bfloat162float(pr[v]) - Lp;
-      acc += __expf(zt) * (zt - zq);
-    }
-    acc = warp_sum_f(acc);
-    __syncthreads();
-    if (l == 0) sf[w] = acc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float K = 0.f;
-      for (int i = 0; i < nw; ++i) K += sf[i];
-      s_res[3] = fmaxf(K, 0.f);
-    }
-    __syncthreads();
-    kl = s_res[3];
-  }
+  const RowStats r = row_stats(k.z_cur + static_cast<int64_t>(flat) * V,
+                               has_prev ? k.z_prev + static_cast<int64_t>(flat) * V : nullptr, V, k.mask_id, s_f, s_i);
   if (threadIdx.x == 0) {
-    const float conf = __expf(BV - L);
+    const float L = r.M + logf(r.S);
+    int BI = r.BI;
+    if (BI == 0x7fffffff) {   // no finite logit: report it, and never hand on an invalid token id
+      set_dev_status(DLLM_DEV_BAD_INDEX);
+      BI = 0;
+    }
+    const float kl = has_prev ? fmaxf(r.T / r.S - (L - k.lse_prev[flat]), 0.f) : NAN;
+    const float conf = __expf(r.BV - L);
     k.conf[flat] = conf;
     k.amax[flat] = BI;
     k.lse_cur[flat] = L;
@@ -733,6 +691,11 @@ int score_es_launch(float* h, float* h_prev, const float* conf, uint8_t* masked_
 int score_cos_launch(const float* vnew, int64_t ldv, const __nv_bfloat16* vc, const int* rows, const int* count_dev,
                      int rows_cap, int N, int Hkv, int hd, float* sim, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
+  // 16-byte vector loads: rows of 8-element multiples on 16-byte boundaries
+  if (hd % 8 || ldv % 4 || (reinterpret_cast<uintptr_t>(vnew) | reinterpret_cast<uintptr_t>(vc)) % 16) {
+    set_last_error("score_cos: head_dim a multiple of 8, 16-byte aligned rows", __FILE__, __LINE__);
+    return DLLM_ERR_SHAPE;
+  }
   const int blocks = (rows_cap * 32 + 255) / 256;
 {
     const int rc_ = launch_pdl(  score_cos_kernel, dim3(blocks), dim3(256), 0, st, vnew, ldv, vc, rows, count_dev, rows_cap, N, Hkv, hd, sim);
@@ -745,6 +708,12 @@ int kl_conf_launch(const __nv_bfloat16* z, int64_t ldz, const __nv_bfloat16* zp_
                    const float* lse_prev, const int* has_prev, const int* rows, const int* count_dev, int rows_cap,
                    int V, int mask_id, float* conf, int* amax, float* lse_out, float* kl_out, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
+  // 16-byte vector loads: rows of 8-element multiples on 16-byte boundaries
+  if (V % 8 || ldz % 8 || ldp % 8 ||
+      (reinterpret_cast<uintptr_t>(z) | reinterpret_cast<uintptr_t>(zp_store)) % 16) {
+    set_last_error("kl_conf: vocabulary and row strides multiples of 8, 16-byte aligned rows", __FILE__, __LINE__);
+    return DLLM_ERR_SHAPE;
+  }
 {
     const int rc_ = launch_pdl(  kl_conf_kernel, dim3(rows_cap), dim3(256), 0, st, z, ldz, zp_store, ldp, lse_prev, has_prev, rows, count_dev, rows_cap, V,
                                            mask_id, conf, amax, lse_out, kl_out);
@@ -813,6 +782,7 @@ namespace dllm {
 
 int kl_step_launch(const KlStep& k, cudaStream_t st) {
   if (k.rows_cap <= 0) return DLLM_OK;
+  if (k.V % 8 || (reinterpret_cast<uintptr_t>(k.z_cur) | reinterpret_cast<uintptr_t>(k.z_prev)) % 16) return DLLM_ERR_SHAPE;
   return launch_pdl(kl_step_kernel, dim3(k.rows_cap), dim3(256), 0, st, k);
 }
 
