@@ -71,7 +71,12 @@ struct KParams {
 
 // Persistent stream-K GEMM: grid = one CTA per SM (or fewer), each CTA walks its
 // contiguous share of the (tile, k-block) iterations; a tile split across CTAs is
-// summed by the last CTA to finish its piece, in k order.
+// summed by the last CTA to finish its piece, in k order.  Tiles are numbered weight
+// tile fastest (tile = ta * n_tiles_w + tw): with several activation tiles, the CTAs
+// whose ranges start n_tiles_w tiles apart stream the same weight tile at the same time,
+// so each weight k-block comes from DRAM once and from L2 for the other activation
+// tiles (numbered the other way, one CTA would reread a whole weight tile per activation
+// tile, a reuse distance of K x 256 B per CTA, beyond L2 across the grid).
 template <int BN, int KSUB, bool BIG>
 __global__ void __launch_bounds__(kThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams p) {
@@ -145,7 +150,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const int kb0 = static_cast<int>(it % KB);
         const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
         it += kb1 - kb0;
-        const int tw = tile / p.tiles_act, ta = tile % p.tiles_act;
+        const int tw = tile % p.n_tiles_w, ta = tile / p.n_tiles_w;
         const int act0 = ta * BN;
         if (!single && act0 >= m_rows) continue;     // tile without valid rows: skipped by every role
         const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
@@ -215,7 +220,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const int kb0 = static_cast<int>(it % KB);
         const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
         it += kb1 - kb0;
-        if (!single && (tile % p.tiles_act) * BN >= m_rows) continue;
+        if (!single && (tile / p.n_tiles_w) * BN >= m_rows) continue;
         const int b = j & 1;
         const uint32_t u = static_cast<uint32_t>(j >> 1);
         ++j;
@@ -253,7 +258,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       const int kb0 = static_cast<int>(it % KB);
       const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
       it += kb1 - kb0;
-      const int tw = tile / p.tiles_act, ta = tile % p.tiles_act;
+      const int tw = tile % p.n_tiles_w, ta = tile / p.n_tiles_w;
       const int act0 = ta * BN;
       if (!single && act0 >= m_rows) continue;
       const int b = j & 1;
@@ -463,15 +468,16 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 
 namespace {
 
-// Activation-tile width.  Up to 768 rows 128-wide tiles with two k-blocks per stage measure
-// faster than 256-wide ones with one (768 rows: QKV 755 vs 685, O 578 vs 367 TFLOP/s): more
-// tiles to balance over the SMs and more stages in flight.  From 1024 rows on the 256-wide
-// tile's higher reuse of each weight tile wins.
+// Activation-tile width: the narrowest tile that holds the rows up to 128, 256 above.  With
+// the weight-tile-fastest numbering every weight k-block is read from DRAM once whatever
+// the width, and the 256-wide tile halves the L2 rereads of the weights and the number of
+// tiles the epilogue drains (768 rows, TFLOP/s, 128 vs 256 wide: QKV 930 vs 1066, O 608 vs
+// 680, down 790 vs 951).
 int pick_bn(int rows) {
   if (rows <= 16) return 16;
   if (rows <= 32) return 32;
   if (rows <= 64) return 64;
-  if (rows <= 768) return 128;
+  if (rows <= 128) return 128;
   return 256;
 }
 
