@@ -12,6 +12,21 @@ constexpr int kTileM = 128;                  // weight rows per tile
 constexpr uint32_t kABytes = kTileM * kBK * 2;
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier `id` of 128 threads (one epilogue group of four warps).
+__device__ __forceinline__ void grp_bar(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+// Barrier `id` of `n` threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool bar_any(bool v, int id, int n) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 // Barrier of the 128 epilogue threads that also returns whether any of them passed true,
 // so that every branch taken after it is the same for all of them.
@@ -56,10 +71,11 @@ __device__ __forceinline__ int sk_first_cta(int64_t x, int64_t T, int G) {
 }
 
 // Epilogue of one 16-column chunk (columns = activation rows jbase..jbase+15) for the
-// weight row n held by TMEM lane t.  Exchange kinds synchronise the 128 epilogue threads.
+// weight row n held by TMEM lane t (warp = t / 32).  Exchange kinds synchronise the 128
+// threads of the epilogue group through named barrier `bar` and its buffer xb.
 template <int XP>
 __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[16], int t, int lane, int warp, int n,
-                                          int jbase, int m_rows, int tw, float* xb) {
+                                          int jbase, int m_rows, int tw, float* xb, int bar = 1) {
   switch (e.kind) {
     case EPI_STORE_F32: {
       float* o = static_cast<float*>(e.out);
@@ -81,17 +97,15 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
       break;
     }
     case EPI_RESID_ADD: {
-      // all loads of the chunk are issued before any store (no serialised round trips)
+      // one writer per element (the tile's owner), so a reduction adds exactly once and the
+      // result is the same as a load and a store, without waiting for the load
       int rr[16];
-      float old[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         rr[i] = (jbase + i < m_rows) ? (e.row_map ? __ldg(e.row_map + jbase + i) : jbase + i) : -1;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) old[i] = rr[i] >= 0 ? __ldcg(e.h + static_cast<int64_t>(rr[i]) * e.ldh + n) : 0.f;
-#pragma unroll
       for (int i = 0; i < 16; ++i)
-        if (rr[i] >= 0) e.h[static_cast<int64_t>(rr[i]) * e.ldh + n] = old[i] + v[i];
+        if (rr[i] >= 0) atomicAdd(e.h + static_cast<int64_t>(rr[i]) * e.ldh + n, v[i]);
       break;
     }
     case EPI_QKV_ROPE: {
@@ -121,7 +135,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
           sn[i] = __ldg(e.rope_sin + static_cast<int64_t>(pos[i]) * half + fi);
         }
       }
-      epi_bar();
+      grp_bar(bar);
       const int partner = t ^ half;
       float out[16];
 #pragma unroll
@@ -147,14 +161,14 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
             dst[((static_cast<int64_t>(bb[i]) * e.n_kv + kvh) * e.seq_n + pos[i]) * hd + (nn % hd)] =
                 __float2bfloat16(out[i]);
       }
-      epi_bar();
+      grp_bar(bar);
       break;
     }
     case EPI_SWIGLU: {
       // lanes 0-63 hold gate rows, lanes 64-127 the matching up rows
 #pragma unroll
       for (int i = 0; i < 16; ++i) xb[t * XP + i] = v[i];
-      epi_bar();
+      grp_bar(bar);
       if (t < 64) {
         const int f = tw * 64 + t;
 #pragma unroll
@@ -167,7 +181,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
           }
         }
       }
-      epi_bar();
+      grp_bar(bar);
       break;
     }
     case EPI_LMHEAD: {
@@ -183,7 +197,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
         warp_argmax(bv, bi);
         if (lane == 0) red[warp * 16 + i] = make_float4(mx, se, bv, __int_as_float(bi));
       }
-      epi_bar();
+      grp_bar(bar);
       if (t < 16 && jbase + t < m_rows) {
         float M = -INFINITY, S = 0.f, BV = -INFINITY;
         int BI = 0x7fffffff;
@@ -197,7 +211,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
         }
         e.lm_part[static_cast<int64_t>(jbase + t) * e.n_vtiles + tw] = make_float4(M, S, BV, __int_as_float(BI));
       }
-      epi_bar();
+      grp_bar(bar);
       break;
     }
     default:

@@ -48,13 +48,19 @@ struct Cfg {
   static constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // TMEM columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr int kXPitch = 17;                                 // epilogue exchange pitch (floats)
-  static constexpr size_t kSmem = 1024 /*align slack*/ + kStages * kStageBytes + 128 * kXPitch * 4 +
+  // Epilogue warps: one group of four (one thread per TMEM lane) drains a tile, or, from
+  // 128-wide tiles on, two groups that split its columns (a wide tile's epilogue would
+  // otherwise take longer than the next tile's MMAs); then the TMA producer warp and the
+  // MMA issuer warp (TMEM owner).
+  static constexpr int kGroups = BN >= 128 ? 2 : 1;
+  static constexpr int kEpiThreads = 128 * kGroups;
+  static constexpr int kThreads = kEpiThreads + 64;
+  static constexpr int kProducerWarp = kEpiThreads / 32, kMmaWarp = kProducerWarp + 1;
+  static constexpr size_t kSmem = 1024 /*align slack*/ + kStages * kStageBytes + kGroups * 128 * kXPitch * 4 +
                                   (2 * kStages + 4) * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "GEMM stage ring does not fit shared memory");
 };
-
-constexpr int kEpiThreads = 128;     // warps 0-3: epilogue, one thread per TMEM lane
-constexpr int kThreads = 192;        // + warp 4: TMA producer, warp 5: MMA issuer / TMEM owner
+constexpr int kEpiAllBar = 3;        // named barrier of every epilogue thread (groups use 1 and 2)
 
 struct KParams {
   int K;
@@ -62,6 +68,7 @@ struct KParams {
   const int* rows_dev;
   int n_tiles_w;
   int tiles_act;
+  int wt_fastest;      // tile numbering: 1 weight tile fastest, 0 activation tile fastest
   int swiglu;
   int ffn;
   float* partial;      // [gridDim.x][2][BN * 128]
@@ -71,21 +78,27 @@ struct KParams {
 
 // Persistent stream-K GEMM: grid = one CTA per SM (or fewer), each CTA walks its
 // contiguous share of the (tile, k-block) iterations; a tile split across CTAs is
-// summed by the last CTA to finish its piece, in k order.  Tiles are numbered weight
-// tile fastest (tile = ta * n_tiles_w + tw): with several activation tiles, the CTAs
-// whose ranges start n_tiles_w tiles apart stream the same weight tile at the same time,
-// so each weight k-block comes from DRAM once and from L2 for the other activation
-// tiles (numbered the other way, one CTA would reread a whole weight tile per activation
-// tile, a reuse distance of K x 256 B per CTA, beyond L2 across the grid).
+// summed by the last CTA to finish its piece, in k order.  The tile numbering decides
+// which operand the concurrently running CTAs share, since CTA c works on tiles near
+// c * tiles / grid:
+//   weight tile fastest (tile = ta * n_tiles_w + tw), for a few activation tiles (a
+//     refresh): the CTAs of the ~grid / tiles_act groups, one per activation tile, stream
+//     the same weight tile at about the same time, so each weight k-block comes from DRAM
+//     once (numbered the other way, a CTA would reread its whole weight tile once per
+//     activation tile, a reuse distance of K x 256 B per CTA, beyond L2 across the grid);
+//   activation tile fastest (tile = tw * tiles_act + ta), for many activation tiles (a
+//     batch of long sequences): each CTA keeps one weight tile and passes every
+//     activation tile under it, so a weight matrix larger than L2 (the vocabulary) is
+//     read once; the activations are shared by all CTAs.
 template <int BN, int KSUB, bool BIG>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(Cfg<BN, KSUB, BIG>::kThreads, BN >= 128 ? 1 : 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams p) {
   using C = Cfg<BN, KSUB, BIG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* xbuf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(xbuf + 128 * C::kXPitch);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(xbuf + C::kGroups * 128 * C::kXPitch);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* acc_full = empty_bar + C::kStages;     // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
@@ -116,19 +129,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiThreads);
+      mbar_init(&acc_empty[b], C::kEpiThreads);
     }
     s_flag[0] = 0;
     s_flag[1] = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (warp == C::kMmaWarp) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == C::kProducerWarp) {
     if (lane == 0) {
       // ---------------- TMA producer: one continuous ring over every segment
       // one activation tile: every weight tile is read once (evict first); several: each weight
@@ -150,7 +163,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const int kb0 = static_cast<int>(it % KB);
         const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
         it += kb1 - kb0;
-        const int tw = tile % p.n_tiles_w, ta = tile / p.n_tiles_w;
+        const int tw = p.wt_fastest ? tile % p.n_tiles_w : tile / p.tiles_act;
+        const int ta = p.wt_fastest ? tile / p.n_tiles_w : tile % p.tiles_act;
         const int act0 = ta * BN;
         if (!single && act0 >= m_rows) continue;     // tile without valid rows: skipped by every role
         const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
@@ -205,7 +219,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == C::kMmaWarp) {
     if (lane == 0) {
       // ---------------- MMA issuer: alternates between the two TMEM accumulators
       constexpr uint32_t idesc = make_idesc_bf16(kTileM, BN);
@@ -220,7 +234,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const int kb0 = static_cast<int>(it % KB);
         const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
         it += kb1 - kb0;
-        if (!single && (tile / p.n_tiles_w) * BN >= m_rows) continue;
+        if (!single && (p.wt_fastest ? tile / p.n_tiles_w : tile % p.tiles_act) * BN >= m_rows) continue;
         const int b = j & 1;
         const uint32_t u = static_cast<uint32_t>(j >> 1);
         ++j;
@@ -247,49 +261,56 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       }
     }
   } else {
-    // ---------------- epilogue warps 0-3
-    const int t = threadIdx.x;
+    // ---------------- epilogue warps (one or two groups of four)
     const EpiParams& e = p.epi;
     pdl_wait();
     const int m_rows = p.rows_dev ? min(*p.rows_dev, p.rows_cap) : p.rows_cap;
+    // group grp drains columns [c0, c1) of every tile; thread t holds TMEM lane t (weight row)
+    const int grp = warp >> 2, wq = warp & 3;
+    const int t = threadIdx.x & 127;
+    const int gbar = 1 + grp;
+    constexpr int kCols = BN / C::kGroups;
+    const int c0 = grp * kCols, c1 = c0 + kCols;
+    float* const xg = xbuf + grp * 128 * C::kXPitch;
     int j = 0;
     for (int64_t it = lo; it < hi;) {
       const int tile = static_cast<int>(it / KB);
       const int kb0 = static_cast<int>(it % KB);
       const int kb1 = (hi - it < KB - kb0) ? kb0 + static_cast<int>(hi - it) : KB;
       it += kb1 - kb0;
-      const int tw = tile % p.n_tiles_w, ta = tile / p.n_tiles_w;
+      const int tw = p.wt_fastest ? tile % p.n_tiles_w : tile / p.tiles_act;
+      const int ta = p.wt_fastest ? tile / p.n_tiles_w : tile % p.tiles_act;
       const int act0 = ta * BN;
       if (!single && act0 >= m_rows) continue;
       const int b = j & 1;
       const uint32_t u = static_cast<uint32_t>(j >> 1);
       ++j;
       const bool late = !mbar_wait(&acc_full[b], u & 1);
-      if (epi_any(late || s_flag[0])) {                // one decision for all epilogue threads
+      if (bar_any(late || s_flag[0], kEpiAllBar, C::kEpiThreads)) {   // one decision for all epilogue threads
         s_flag[0] = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * C::kAccCols;
+      const uint32_t tb = tmem + (static_cast<uint32_t>(wq * 32) << 16) + b * C::kAccCols;
       const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
       const int row1 = p.swiglu ? p.ffn + tw * 64 : tw * kTileM + 64;
       const int n = t < 64 ? row0 + t : row1 + (t - 64);
       const bool whole = (kb0 == 0 && kb1 == KB);
       if (whole) {
-        for (int cc = 0; cc < BN; cc += 16) {
+        for (int cc = c0; cc < c1; cc += 16) {
           float v[16];
           tmem_ld16(tb + cc, v);
-          if (cc + 16 >= BN) {                         // accumulator drained: hand it back
+          if (cc + 16 >= c1) {                         // this group's columns drained: hand them back
             tc_fence_before();
             mbar_arrive(&acc_empty[b]);
           }
-          epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, act0 + cc, m_rows, tw, xbuf);
+          epi_chunk<C::kXPitch>(e, v, t, lane, wq, n, act0 + cc, m_rows, tw, xg, gbar);
         }
       } else {
         // a piece of a split tile: store it, then the last piece to arrive sums all of them
         const int which = (tile == first_tile) ? 0 : 1;
         float* mine = p.partial + (static_cast<size_t>(c) * 2 + which) * (BN * 128);
-        for (int cc = 0; cc < BN; cc += 16) {
+        for (int cc = c0; cc < c1; cc += 16) {
           float v[16];
           tmem_ld16(tb + cc, v);
 #pragma unroll
@@ -298,18 +319,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
         __threadfence();
-        epi_bar();
+        bar_any(false, kEpiAllBar, C::kEpiThreads);
         const int64_t x0 = static_cast<int64_t>(tile) * KB;
         const int c_first = sk_first_cta(x0, T, G);
         const int c_last = sk_first_cta(x0 + KB - 1, T, G);
-        if (t == 0) {
+        if (threadIdx.x == 0) {
           const int old = atomicAdd(&p.counters[tile], 1);
           s_flag[1] = (old == c_last - c_first) ? 1 : 0;
         }
-        epi_bar();
+        bar_any(false, kEpiAllBar, C::kEpiThreads);
         if (s_flag[1]) {
           __threadfence();
-          for (int cc = 0; cc < BN; cc += 16) {
+          for (int cc = c0; cc < c1; cc += 16) {
             float v[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[q] = 0.f;
@@ -319,18 +340,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
               for (int q = 0; q < 16; ++q) v[q] += __ldcg(src + (cc + q) * 128 + t);
             }
-            epi_chunk<C::kXPitch>(e, v, t, lane, warp, n, act0 + cc, m_rows, tw, xbuf);
+            epi_chunk<C::kXPitch>(e, v, t, lane, wq, n, act0 + cc, m_rows, tw, xg, gbar);
           }
-          if (t == 0) p.counters[tile] = 0;
+          if (threadIdx.x == 0) p.counters[tile] = 0;
         }
-        epi_bar();
+        bar_any(false, kEpiAllBar, C::kEpiThreads);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == C::kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 __global__ void lmhead_combine_kernel(const float4* __restrict__ part, int n_vtiles, int rows_cap,
@@ -468,18 +489,27 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 
 namespace {
 
-// Activation-tile width: the narrowest tile that holds the rows up to 128, 256 above.  With
-// the weight-tile-fastest numbering every weight k-block is read from DRAM once whatever
-// the width, and the 256-wide tile halves the L2 rereads of the weights and the number of
-// tiles the epilogue drains (768 rows, TFLOP/s, 128 vs 256 wide: QKV 930 vs 1066, O 608 vs
-// 680, down 790 vs 951).
+// Activation-tile width.  Up to 768 rows the 128-wide tile: it keeps twice the weight bytes
+// in flight per stage (two 64-column k-blocks: 96 KB of weights in the ring against 64 KB at
+// 256 wide), and a 256-wide tile's epilogue (RoPE and K/V scatter, SwiGLU, the residual add)
+// outlasts its MMAs.  Whole 768-row layers, weight tile fastest, eight epilogue warps:
+// 583 us at 128 wide, 594 us at 256 wide; QKV with its RoPE epilogue 120 vs 162 us.
 int pick_bn(int rows) {
+  static const int wide = [] {
+    const char* e = getenv("DLLM_GEMM_WIDE_BN");   // A/B switch for measurements: width above 64 rows
+    return e ? atoi(e) : 0;
+  }();
   if (rows <= 16) return 16;
   if (rows <= 32) return 32;
   if (rows <= 64) return 64;
-  if (rows <= 128) return 128;
+  if (wide == 128 || wide == 256) return wide;
+  if (rows <= 768) return 128;
   return 256;
 }
+// Weight tile fastest up to 8 activation tiles (whole 768-row layers: 583 us against 638 us
+// activation tile fastest; 2048 rows: 1.68 -> 1.57 ms), activation tile fastest above
+// (batch-8 SureLock steps, 12288 rows: the vocabulary projection reads its 1.09 GB once).
+constexpr int kMaxActTilesWtFastest = 8;
 
 // Grid of the persistent kernel: one CTA per SM, never more CTAs than k-block iterations.
 int pick_grid(int tiles, int KB) {
@@ -493,7 +523,7 @@ int launch_cfg2(const CUtensorMap& tmW, const CUtensorMap& tmX, KParams& kp, int
   const int rc = ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, KSUB, BIG>),
                                   static_cast<int>(C::kSmem));
   if (rc) return rc;
-  return launch_pdl(gemm_tc_kernel<BN, KSUB, BIG>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, kp);
+  return launch_pdl(gemm_tc_kernel<BN, KSUB, BIG>, dim3(grid), dim3(C::kThreads), C::kSmem, st, tmW, tmX, kp);
 }
 
 template <int BN, int KSUB>
@@ -572,6 +602,11 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   kp.rows_dev = a.rows_dev;
   kp.n_tiles_w = a.n_tiles_w;
   kp.tiles_act = tiles_act;
+  static const int order_env = [] {
+    const char* e = getenv("DLLM_GEMM_ORDER");   // A/B switch for measurements: 0 activation, 1 weight tile fastest
+    return e ? atoi(e) : -1;
+  }();
+  kp.wt_fastest = order_env >= 0 ? order_env : (tiles_act <= kMaxActTilesWtFastest ? 1 : 0);
   kp.swiglu = a.swiglu ? 1 : 0;
   kp.ffn = a.epi.ffn;
   kp.partial = s.partial;

@@ -257,6 +257,70 @@ def surelock_step_case(reps, layers=2):
             "lm_rows": n_lm}
 
 
+def layer_case(rows, reps, N=768, dims=None):
+    """One whole layer on the kernel-per-step path (the refresh path: RMSNorm, QKV + RoPE + K/V
+    scatter, attention, O + residual, RMSNorm, gate/up + SwiGLU, down + residual) over `rows`
+    rows of one N-position sequence, LLaDA-8B layer shape."""
+    from synth import make_weights
+    from synth.configs import LLADA8B, RunConfig
+    from . import _lib
+    m = dims or LLADA8B
+    import dataclasses
+    m1 = dataclasses.replace(m, n_layers=1, vocab=1024, mask_id=1023)
+    run = RunConfig(name="layer", model=m1, batch=1, prompt_len=N - 64, gen_len=64, block_len=64, policy="vanilla")
+    cfg = _lib.make_config(run, layer_kernel="split")
+    nbytes = m1.params_per_layer * 2
+    ncop = _copies(nbytes)
+    ws_w = [make_weights(m1, seed=i, device="cuda", layers=[0], with_vocab=False) for i in range(ncop)]
+    lws = [{k: w[k][0] for k in ("w_qkv", "w_o", "w_gu", "w_down", "g_attn", "g_ffn")} for w in ws_w]
+    g = torch.Generator(device="cuda").manual_seed(9)
+    h = torch.randn((N, m1.d_model), generator=g, device="cuda")
+    kc = torch.randn((1, m1.n_kv_heads, N, m1.head_dim), generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn_like(kc, dtype=torch.float32).to(torch.bfloat16)
+    cos, sin = ops.rope_table(N, m1.head_dim, m1.rope_theta)
+    rows_t = torch.arange(rows, dtype=torch.int32, device="cuda") * (N // rows)
+    cnt = torch.tensor([rows], dtype=torch.int32, device="cuda")
+    off = torch.tensor([0, rows], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(ops.layer_workspace_bytes(cfg, rows, rows), dtype=torch.uint8, device="cuda")
+    fn = lambda i: ops.layer(cfg, lws[i % ncop], kc, vc, cos, sin, h, rows_t, cnt, off, rows, rows, ws=ws)
+    t = _time(fn, reps)
+    P = m1.params_per_layer
+    flops = 2.0 * rows * P + 4.0 * rows * N * m1.n_heads * m1.head_dim
+    byts = 2 * P + 2 * N * m1.kv_dim * 2
+    return {"case": f"layer_m{rows}_n{N}", "ms": t, "gbs": byts / t / 1e6, "tflops": flops / t / 1e9,
+            "bytes": byts, "flops": flops}
+
+
+def gemm_epi_case(kind, rows, reps, d=4096, F=12288, splits=0, bn=0):
+    """The refresh GEMMs with the epilogues the layer uses: QKV + RoPE + K/V scatter, and the
+    residual add into the hidden state of O and down."""
+    from synth.configs import LLADA8B
+    g = torch.Generator(device="cuda").manual_seed(10)
+    n_out, K = {"qkvrope": (3 * d, d), "oresid": (d, d), "downresid": (d, F)}[kind]
+    nbytes = n_out * K * 2
+    ncop = _copies(nbytes)
+    Ws = [(torch.randn((n_out, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16) for _ in range(ncop)]
+    X = torch.randn((rows, K), generator=g, device="cuda").to(torch.bfloat16)
+    ws = torch.zeros(256 << 20, dtype=torch.uint8, device="cuda")
+    N = rows
+    rmap = torch.arange(rows, dtype=torch.int32, device="cuda")
+    if kind == "qkvrope":
+        cos, sin = ops.rope_table(N, 128, LLADA8B.rope_theta)
+        kc = torch.zeros((1, 32, N, 128), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        fn = lambda i: ops.qkv_rope(Ws[i % ncop], X, LLADA8B, N, rmap, cos, sin, kc, vc, splits=splits, ws=ws)
+        out_bytes = rows * n_out * 2
+    else:
+        h = torch.zeros((rows, n_out), device="cuda")
+        fn = lambda i: ops.gemm(Ws[i % ncop], X, kind=3, out=h, rows_map=rmap, splits=splits, bn=bn, ws=ws)
+        out_bytes = rows * n_out * 8
+    t = _time(fn, reps)
+    byts = nbytes + rows * K * 2 + out_bytes
+    flops = 2.0 * rows * n_out * K
+    return {"case": f"gemm_{kind}_m{rows}", "ms": t, "gbs": byts / t / 1e6, "tflops": flops / t / 1e9,
+            "bytes": byts, "flops": flops}
+
+
 CASES = {
     **{f"gemm_{k}_m{m}": (lambda k=k, m=m, **kw: gemm_case(k, m, **kw))
        for k in ("qkv", "o", "gu", "down") for m in (7, 32, 768)},
@@ -275,6 +339,11 @@ CASES = {
     "attn_gqa_m1536": lambda **kw: attn_gqa_case(1536, **kw),
     "attn_gqa_m7": lambda **kw: attn_gqa_case(7, **kw),
     "surelock_step_l2": lambda **kw: surelock_step_case(**kw),
+    "layer_m768": lambda **kw: layer_case(768, **kw),
+    "layer_m205_n2048": lambda **kw: layer_case(205, N=2048, **kw),
+    "gemm_qkvrope_m768": lambda **kw: gemm_epi_case("qkvrope", 768, **kw),
+    "gemm_oresid_m768": lambda **kw: gemm_epi_case("oresid", 768, **kw),
+    "gemm_downresid_m768": lambda **kw: gemm_epi_case("downresid", 768, **kw),
 }
 
 
