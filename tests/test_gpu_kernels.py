@@ -202,6 +202,38 @@ def test_attention_vs_oracle(B, counts, N, hq, hkv, hd, splits):
         assert _rowrel(got[s:e], ref) < 2e-2
 
 
+# Tensor-core path (head dim 128, >= 64 query units per sequence and KV head): the refresh
+# shape (every row of the sequence), a Dream-7B GQA group (7 query heads per KV head), a
+# ragged last key tile, forced key splits and sequences of unequal length.  The operands are
+# bf16 on both sides, so what remains is the bf16 rounding of P (2^-9 of the largest weight)
+# and of the output: 8e-3 of each row's largest entry.
+TOL_ATTN_TC = 8e-3
+
+
+@pytest.mark.parametrize("B,counts,N,hq,hkv,splits", [
+    (1, [768], 768, 4, 4, 0), (1, [300], 1536, 28, 4, 0), (1, [200], 1000, 2, 2, 3),
+    (2, [129, 64], 300, 4, 4, 0), (2, [70, 5], 2048, 2, 2, 0), (1, [64], 128, 1, 1, 1),
+])
+def test_attention_tensor_core_vs_oracle(B, counts, N, hq, hkv, splits):
+    hd = 128
+    dims = ModelDims(n_layers=1, d_model=hq * hd, n_heads=hq, n_kv_heads=hkv, head_dim=hd, ffn_dim=64, vocab=128,
+                     mask_id=127)
+    rows = sum(counts)
+    q = _bf16((rows, hq * hd), 30)
+    K = _bf16((B, hkv, N, hd), 31)
+    V = _bf16((B, hkv, N, hd), 32)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32)
+    out = ops.attention(q.to(DEV), K.to(DEV), V.to(DEV), off.to(DEV), dims, max(counts), splits=splits)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    qd = _f64(q).reshape(-1, hq, hd)
+    for b in range(B):
+        s, e = int(off[b]), int(off[b + 1])
+        ref = om.attention(qd[s:e], _f64(K[b]), _f64(V[b])).reshape(e - s, -1)
+        err = _rowrel(got[s:e], ref)
+        assert err < TOL_ATTN_TC, (b, err)
+
+
 # ------------------------------------------------------------------ LM head
 
 @pytest.mark.parametrize("rows,V,count", [(7, 1024, None), (32, 4096, 20), (3, 126464 // 4, None)])

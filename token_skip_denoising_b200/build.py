@@ -12,7 +12,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libdllm.so")
-SOURCES = ["gemm_tc.cu", "attention.cu", "rowops.cu", "engine.cu", "ops.cu", "noalloc.cu", "fused_layer.cu"]
+SOURCES = ["gemm_tc.cu", "attention.cu", "attn_tc.cu", "rowops.cu", "engine.cu", "ops.cu", "noalloc.cu", "fused_layer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-rdc=true", "-Xcompiler", "-fPIC,-O2",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

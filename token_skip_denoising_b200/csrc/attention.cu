@@ -51,13 +51,24 @@ __global__ void attn_combine_kernel(AttnParams p) {
   attn_merge<HD>(p, row, h, lane);
 }
 
+// Merge of the split partials: one warp per (row, head).
+int combine_launch(const AttnParams& p, int rows_cap, int hd, cudaStream_t st) {
+  const int warps = rows_cap * p.Hq;
+  const int blocks = (warps * 32 + 255) / 256;
+  return hd == 128 ? launch_pdl(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, p)
+                   : launch_pdl(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, p);
+}
+
 }  // namespace
+
+int attn_tc_run(const attn::AttnParams& p, int rows_per_seq_cap, cudaStream_t st);
 
 size_t attn_partial_floats(int rows_cap, int Hq, int hd, int splits) {
   return static_cast<size_t>(splits) * rows_cap * Hq * hd;
 }
 
-int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N) {
+int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N, int hd) {
+  if (attn_use_tc(hd, G, rows_per_seq)) return attn_tc_pick_splits(B, Hkv, G, rows_per_seq, N);
   const int qtiles = (rows_per_seq * G + kUnitsPerCta - 1) / kUnitsPerCta;
   const int ctas = qtiles * B * Hkv;
   const int n_blocks = (N + kKeysPerBlock - 1) / kKeysPerBlock;
@@ -83,8 +94,11 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
   if (hd != 64 && hd != 128) return DLLM_ERR_UNSUPPORTED;
   if (rows_cap <= 0 || rows_per_seq_cap <= 0) return DLLM_OK;
   const int G = Hq / Hkv;
-  const int n_blocks = (N + kKeysPerBlock - 1) / kKeysPerBlock;
-  if (splits <= 0) splits = attn_pick_splits(B, Hkv, G, rows_per_seq_cap, N);
+  const bool tc = attn_use_tc(hd, G, rows_per_seq_cap);
+  // key blocks of the chosen path: 128 keys on the tensor cores, 64 on the CUDA cores
+  const int kblk = tc ? 128 : kKeysPerBlock;
+  const int n_blocks = (N + kblk - 1) / kblk;
+  if (splits <= 0) splits = attn_pick_splits(B, Hkv, G, rows_per_seq_cap, N, hd);
   splits = std::min(splits, n_blocks);
   if (splits > 1 && (!opart || !ml || partial_floats < attn_partial_floats(rows_cap, Hq, hd, splits))) splits = 1;
   const int bps = (n_blocks + splits - 1) / splits;
@@ -95,6 +109,11 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
   p.splits = splits; p.blocks_per_split = bps;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(hd));
   p.opart = opart; p.ml = ml;
+  if (tc) {
+    const int rc = attn_tc_run(p, rows_per_seq_cap, st);
+    if (rc) return rc;
+    return splits > 1 ? combine_launch(p, rows_cap, hd, st) : DLLM_OK;
+  }
   const int qtiles = (rows_per_seq_cap * G + kUnitsPerCta - 1) / kUnitsPerCta;
   dim3 grid(qtiles, B * Hkv, splits);
   const size_t smem = 4 * kKeysPerBlock * hd * 2;
@@ -112,14 +131,7 @@ int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bflo
     const int rc = launch_pdl(attn_kernel<64>, grid, dim3(128), smem, st, p);
     if (rc) return rc;
   }
-  if (splits > 1) {
-    const int warps = rows_cap * Hq;
-    const int blocks = (warps * 32 + 255) / 256;
-    const int rc = hd == 128 ? launch_pdl(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, p)
-                             : launch_pdl(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, p);
-    if (rc) return rc;
-  }
-  return DLLM_OK;
+  return splits > 1 ? combine_launch(p, rows_cap, hd, st) : DLLM_OK;
 }
 
 }  // namespace dllm

@@ -368,7 +368,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   const int G = c.n_heads / c.n_kv_heads;
   for (int cap_seq : {x->N, x->n_cand, x->k_keep, x->n_resp}) {
     if (cap_seq <= 0) continue;
-    const int sp = attn_pick_splits(x->B, c.n_kv_heads, G, cap_seq, x->N);
+    const int sp = attn_pick_splits(x->B, c.n_kv_heads, G, cap_seq, x->N, x->hd);
     if (sp > 1) af = std::max(af, attn_partial_floats(x->B * cap_seq, c.n_heads, x->hd, sp));
   }
   x->attn_opart = w.take<float>(af);
@@ -1214,7 +1214,7 @@ int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t ro
                         gemm_partial_floats(rows_cap, F / 64, d), gemm_partial_floats(rows_cap, d / 128, F)});
   w.take<float>(pf);
   const int B = cfg->batch, N = cfg->prompt_len + cfg->gen_len;
-  const int sp = attn_pick_splits(B, cfg->n_kv_heads, cfg->n_heads / cfg->n_kv_heads, rows_per_seq_cap, N);
+  const int sp = attn_pick_splits(B, cfg->n_kv_heads, cfg->n_heads / cfg->n_kv_heads, rows_per_seq_cap, N, cfg->head_dim);
   const size_t af = sp > 1 ? attn_partial_floats(rows_cap, cfg->n_heads, cfg->head_dim, sp) : 0;
   w.take<float>(af);
   w.take<float2>(af / cfg->head_dim);
@@ -1259,7 +1259,7 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
                         gemm_partial_floats(rows_cap, L.F / 64, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.F)});
   L.gs.partial = w.take<float>(pf);
   L.gs.partial_floats = pf;
-  const int sp = attn_pick_splits(L.B, L.Hkv, L.Hq / L.Hkv, rows_per_seq_cap, L.N);
+  const int sp = attn_pick_splits(L.B, L.Hkv, L.Hq / L.Hkv, rows_per_seq_cap, L.N, L.hd);
   L.attn_floats = sp > 1 ? attn_partial_floats(rows_cap, L.Hq, L.hd, sp) : 0;
   L.attn_opart = w.take<float>(L.attn_floats);
   L.attn_ml = w.take<float2>(L.attn_floats / L.hd);

@@ -146,7 +146,7 @@ int dllm_op_attention(const void* q, const void* kcache, const void* vcache, voi
   if (n_kv_heads <= 0 || n_heads % n_kv_heads) OP_FAIL(DLLM_ERR_SHAPE, "n_heads must be a multiple of n_kv_heads");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = n_heads / n_kv_heads;
-  int sp = splits > 0 ? splits : attn_pick_splits(B, n_kv_heads, G, rows_per_seq_cap, N);
+  int sp = splits > 0 ? splits : attn_pick_splits(B, n_kv_heads, G, rows_per_seq_cap, N, head_dim);
   float* opart = nullptr;
   float2* ml = nullptr;
   int* ctr = nullptr;

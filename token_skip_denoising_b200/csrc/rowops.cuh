@@ -84,7 +84,12 @@ int unmask_launch(int* tokens, const float* conf, const int* amax, int B, int N,
                   int* n_out, int max_out, int* remain, cudaStream_t st);
 
 size_t attn_partial_floats(int rows_cap, int Hq, int hd, int splits);
-int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N);
+// Key splits attn_launch uses when given none (the tensor-core or the CUDA-core path).
+int attn_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N, int hd);
+// Query units per (sequence, KV head) from which head dimension 128 runs on tcgen05 (attn_tc.cu).
+constexpr int kAttnTcMinUnits = 64;
+bool attn_use_tc(int hd, int G, int rows_per_seq);
+int attn_tc_pick_splits(int B, int Hkv, int G, int rows_per_seq, int N);
 int attn_counters_needed(int B, int Hkv, int G, int rows_per_seq);
 // counters: zero on entry, left at zero.
 int attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, __nv_bfloat16* out,
