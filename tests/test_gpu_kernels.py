@@ -234,6 +234,29 @@ def test_attention_tensor_core_vs_oracle(B, counts, N, hq, hkv, splits):
         assert err < TOL_ATTN_TC, (b, err)
 
 
+@pytest.mark.parametrize("ramp", [0.05, -0.05])
+def test_attention_tensor_core_rescale(ramp):
+    """Scores that climb (or fall) along the keys: every query shares a direction d with
+    |d|^2 = 16 and key n carries n * ramp * d, so S' moves by ~13 per 128-key tile.  Climbing,
+    each tile's maximum exceeds the running offset by more than the slack and O, l are
+    rescaled at every tile; falling, the first tile holds the maximum and nothing is."""
+    hd, hq, hkv, N, rows = 128, 2, 2, 1000, 200
+    dims = ModelDims(n_layers=1, d_model=hq * hd, n_heads=hq, n_kv_heads=hkv, head_dim=hd, ffn_dim=64, vocab=128,
+                     mask_id=127)
+    g = torch.Generator().manual_seed(40)
+    d = torch.zeros(hd)
+    d[:16] = 1.0
+    q = (torch.randn((rows, hq, hd), generator=g) * 0.3 + d).reshape(rows, hq * hd).to(torch.bfloat16)
+    pos = torch.arange(N, dtype=torch.float32)[:, None]
+    K = (torch.randn((1, hkv, N, hd), generator=g) * 0.3 + (pos * ramp) * d).to(torch.bfloat16)
+    V = _bf16((1, hkv, N, hd), 41)
+    off = torch.tensor([0, rows], dtype=torch.int32)
+    out = ops.attention(q.to(DEV), K.to(DEV), V.to(DEV), off.to(DEV), dims, rows)
+    torch.cuda.synchronize()
+    ref = om.attention(_f64(q).reshape(rows, hq, hd), _f64(K[0]), _f64(V[0])).reshape(rows, -1)
+    assert _rowrel(out.float().cpu().numpy(), ref) < TOL_ATTN_TC
+
+
 # ------------------------------------------------------------------ LM head
 
 @pytest.mark.parametrize("rows,V,count", [(7, 1024, None), (32, 4096, 20), (3, 126464 // 4, None)])

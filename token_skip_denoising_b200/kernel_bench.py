@@ -329,6 +329,7 @@ CASES = {
     "attn_m7": lambda **kw: attn_case(7, **kw),
     "attn_m32": lambda **kw: attn_case(32, **kw),
     "attn_m768": lambda **kw: attn_case(768, **kw),
+    "attn_m5120": lambda **kw: attn_case(5120, N=5120, **kw),
     "fused_m7_l3": lambda **kw: fused_case(7, **kw),
     "fused_m32_l3": lambda **kw: fused_case(32, **kw),
     "score_es_n8192": lambda **kw: score_es_case(8192, **kw),
