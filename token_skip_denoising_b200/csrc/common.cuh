@@ -76,7 +76,6 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 enum EpiKind : int {
   EPI_STORE_F32 = 0,   // out_f32[j * ldo + n]
   EPI_STORE_BF16 = 1,  // out_bf16[r * ldo + n], r = row_map ? row_map[j] : j
-  EPI_QKV_ROPE = 2,    // RoPE on q/k, q -> q_out, k/v -> cache rows of row_map[j]
   EPI_RESID_ADD = 3,   // h[row_map[j] * ldh + n] += C
   EPI_SWIGLU = 4,      // act[j * F + f] = silu(gate) * up   (W tile = 64 gate + 64 up rows)
   EPI_LMHEAD = 5,      // per (row, 128-vocab tile): max, sum exp, argmax (mask id excluded)
@@ -86,14 +85,7 @@ struct EpiParams {
   int kind = EPI_STORE_F32;
   void* out = nullptr;
   int64_t ldo = 0;
-  // QKV + RoPE + K/V scatter
-  __nv_bfloat16* q_out = nullptr;   // [rows, q_dim]
-  __nv_bfloat16* kcache = nullptr;  // this layer: [B, Hkv, N, hd]
-  __nv_bfloat16* vcache = nullptr;
-  const int* row_map = nullptr;     // row j -> b * N + pos
-  int seq_n = 0, n_kv = 0, head_dim = 0, q_dim = 0, kv_dim = 0;
-  const float* rope_cos = nullptr;  // [N, hd/2]
-  const float* rope_sin = nullptr;
+  const int* row_map = nullptr;     // row j -> output row (scatter kinds)
   // residual
   float* h = nullptr;
   int64_t ldh = 0;

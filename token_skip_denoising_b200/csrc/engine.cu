@@ -237,6 +237,7 @@ struct dllm_handle {
   size_t const_bytes = 0, state_total = 0;
   Prof prof;
   __nv_bfloat16 *z, *q, *attn, *act;
+  float* yqkv;             // [rows, qkvd] fp32 QKV products of the kernel-per-step layer
   float* vnew;
   float4* lm_part;
   GemmScratch gs;
@@ -343,6 +344,7 @@ void carve(dllm_handle* x, void* state, void* ws, size_t* state_bytes, size_t* w
   x->q = w.take<__nv_bfloat16>(R * x->qd);
   x->attn = w.take<__nv_bfloat16>(R * x->qd);
   x->act = w.take<__nv_bfloat16>(R * x->F);
+  x->yqkv = w.take<float>(R * x->qkvd);
   x->vnew = c.policy == DLLM_POLICY_DLLM_CACHE ? w.take<float>(static_cast<size_t>(x->B) * x->n_resp * x->kvd) : nullptr;
   const int lm_cap = lm_cap_of(x);
   x->lm_part = w.take<float4>(c.policy == DLLM_POLICY_SURELOCK ? 0 : static_cast<size_t>(lm_cap) * (x->V / 128));
@@ -429,6 +431,7 @@ struct LayerCtx {
   __nv_bfloat16 *kc, *vc;
   const float *rope_cos, *rope_sin;
   __nv_bfloat16 *z, *q, *attn, *act;
+  float* yqkv;             // [rows, qkvd] fp32 QKV products of the kernel-per-step layer
   GemmScratch gs;
   float* attn_opart;
   float2* attn_ml;
@@ -519,10 +522,12 @@ int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, con
   GemmArgs g;
   g.W = x.Wqkv; g.w_rows_total = x.qkvd; g.X = x.z; g.rows_cap = rows_cap; g.rows_dev = n; g.K = x.d;
   g.n_tiles_w = x.qkvd / 128;
-  g.epi.kind = EPI_QKV_ROPE; g.epi.q_out = x.q; g.epi.kcache = x.kc; g.epi.vcache = x.vc; g.epi.row_map = rows;
-  g.epi.seq_n = x.N; g.epi.n_kv = x.Hkv; g.epi.head_dim = x.hd; g.epi.q_dim = x.qd; g.epi.kv_dim = x.kvd;
-  g.epi.rope_cos = x.rope_cos; g.epi.rope_sin = x.rope_sin;
-  DLLM_TRY(timed_gemm(x.prof, g, x.gs, st, 2.0 * x.qkvd));
+  // fp32 products, then RoPE and the K/V scatter as one coalesced pass (a rotation inside the
+  // GEMM epilogue waits on the row map and the cos/sin table in every 16-column chunk)
+  g.epi.kind = EPI_STORE_F32; g.epi.out = x.yqkv; g.epi.ldo = x.qkvd;
+  DLLM_TRY(timed_gemm(x.prof, g, x.gs, st, 4.0 * x.qkvd));
+  DLLM_TRY(rope_scatter_launch(x.yqkv, rows_cap, n, rows, x.qkvd, x.qd, x.kvd, x.hd, x.N, x.Hkv, x.rope_cos,
+                               x.rope_sin, x.q, x.kc, x.vc, st));
   {
     cudaEvent_t a = nullptr;
     if (x.prof) x.prof->begin(st, &a, 1);
@@ -567,7 +572,7 @@ LayerCtx layer_ctx(const dllm_handle* x, int l) {
   L.kc = x->kcache + l * kvl;
   L.vc = x->vcache + l * kvl;
   L.rope_cos = x->rope_cos; L.rope_sin = x->rope_sin;
-  L.z = x->z; L.q = x->q; L.attn = x->attn; L.act = x->act;
+  L.z = x->z; L.q = x->q; L.attn = x->attn; L.act = x->act; L.yqkv = x->yqkv;
   L.gs = x->gs;
   L.attn_opart = x->attn_opart; L.attn_ml = x->attn_ml; L.attn_floats = x->attn_floats;
   L.attn_ctr = x->attn_ctr; L.n_attn_ctr = x->n_attn_ctr;
@@ -1210,6 +1215,7 @@ int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t ro
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * qd);
   w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * F);
+  w.take<float>(static_cast<size_t>(rows_cap) * qkvd);
   size_t pf = std::max({gemm_partial_floats(rows_cap, qkvd / 128, d), gemm_partial_floats(rows_cap, d / 128, qd),
                         gemm_partial_floats(rows_cap, F / 64, d), gemm_partial_floats(rows_cap, d / 128, F)});
   w.take<float>(pf);
@@ -1255,6 +1261,7 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
   L.q = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
   L.attn = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.qd);
   L.act = w.take<__nv_bfloat16>(static_cast<size_t>(rows_cap) * L.F);
+  L.yqkv = w.take<float>(static_cast<size_t>(rows_cap) * L.qkvd);
   size_t pf = std::max({gemm_partial_floats(rows_cap, L.qkvd / 128, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.qd),
                         gemm_partial_floats(rows_cap, L.F / 64, L.d), gemm_partial_floats(rows_cap, L.d / 128, L.F)});
   L.gs.partial = w.take<float>(pf);

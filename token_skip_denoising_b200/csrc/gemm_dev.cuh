@@ -108,62 +108,6 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
         if (rr[i] >= 0) atomicAdd(e.h + static_cast<int64_t>(rr[i]) * e.ldh + n, v[i]);
       break;
     }
-    case EPI_QKV_ROPE: {
-      // rotate-half pairs (i, i + hd/2) of a head sit in lanes t and t ^ (hd/2)
-#pragma unroll
-      for (int i = 0; i < 16; ++i) xb[t * XP + i] = v[i];
-      const int hd = e.head_dim;
-      const int half = hd >> 1;
-      const int i_in_head = n % hd;
-      const int fi = i_in_head % half;
-      const bool lo = i_in_head < half;
-      const int region = n < e.q_dim ? 0 : (n < e.q_dim + e.kv_dim ? 1 : 2);
-      // gather every index and table entry of the chunk first
-      int pos[16], bb[16];
-      float cs[16], sn[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int j = jbase + i;
-        const int flat = j < m_rows ? __ldg(e.row_map + j) : 0;
-        bb[i] = flat / e.seq_n;
-        pos[i] = flat - bb[i] * e.seq_n;
-      }
-      if (region < 2) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          cs[i] = __ldg(e.rope_cos + static_cast<int64_t>(pos[i]) * half + fi);
-          sn[i] = __ldg(e.rope_sin + static_cast<int64_t>(pos[i]) * half + fi);
-        }
-      }
-      grp_bar(bar);
-      const int partner = t ^ half;
-      float out[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float x = v[i];
-        if (region < 2) {
-          const float y = xb[partner * XP + i];
-          x = lo ? (x * cs[i] - y * sn[i]) : (x * cs[i] + y * sn[i]);
-        }
-        out[i] = x;
-      }
-      if (region == 0) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (jbase + i < m_rows) e.q_out[static_cast<int64_t>(jbase + i) * e.q_dim + n] = __float2bfloat16(out[i]);
-      } else {
-        const int nn = n - e.q_dim - (region == 2 ? e.kv_dim : 0);
-        const int kvh = nn / hd;
-        __nv_bfloat16* dst = region == 1 ? e.kcache : e.vcache;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (jbase + i < m_rows)
-            dst[((static_cast<int64_t>(bb[i]) * e.n_kv + kvh) * e.seq_n + pos[i]) * hd + (nn % hd)] =
-                __float2bfloat16(out[i]);
-      }
-      grp_bar(bar);
-      break;
-    }
     case EPI_SWIGLU: {
       // lanes 0-63 hold gate rows, lanes 64-127 the matching up rows
 #pragma unroll

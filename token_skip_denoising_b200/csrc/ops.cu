@@ -112,14 +112,17 @@ int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32
   GemmScratch gs;
   const int rc = gemm_scratch(cv, rows_cap, qkvd / 128, d, gs);
   if (rc) return rc;
+  float* y = cv.take<float>(static_cast<size_t>(rows_cap) * qkvd);
+  if (!cv.ok) OP_FAIL(DLLM_ERR_SHAPE, "workspace too small for the fp32 QKV products");
   GemmArgs g;
   g.W = W; g.w_rows_total = qkvd; g.X = X; g.rows_cap = rows_cap; g.rows_dev = count; g.K = d;
   g.n_tiles_w = qkvd / 128;
-  g.epi.kind = EPI_QKV_ROPE; g.epi.q_out = static_cast<__nv_bfloat16*>(q_out);
-  g.epi.kcache = static_cast<__nv_bfloat16*>(kcache); g.epi.vcache = static_cast<__nv_bfloat16*>(vcache);
-  g.epi.row_map = rows_map; g.epi.seq_n = N; g.epi.n_kv = n_kv_heads; g.epi.head_dim = head_dim;
-  g.epi.q_dim = qd; g.epi.kv_dim = kvd; g.epi.rope_cos = rope_cos; g.epi.rope_sin = rope_sin;
-  return gemm_launch(g, gs, st, splits, 0);
+  g.epi.kind = EPI_STORE_F32; g.epi.out = y; g.epi.ldo = qkvd;
+  const int rc2 = gemm_launch(g, gs, st, splits, 0);
+  if (rc2) return rc2;
+  return rope_scatter_launch(y, rows_cap, count, rows_map, qkvd, qd, kvd, head_dim, N, n_kv_heads, rope_cos,
+                             rope_sin, static_cast<__nv_bfloat16*>(q_out), static_cast<__nv_bfloat16*>(kcache),
+                             static_cast<__nv_bfloat16*>(vcache), st);
 }
 
 int dllm_op_gate_up(const void* W, int32_t F, const void* X, int32_t rows_cap, const int32_t* count, int32_t d,

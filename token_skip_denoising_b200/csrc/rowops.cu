@@ -663,6 +663,82 @@ int embed_rows_launch(const __nv_bfloat16* E, int V, const int* tokens, const in
   return DLLM_OK;
 }
 
+namespace {
+// RoPE (rotate-half pairs i, i + hd/2 of every q and k head, by pos theta^(-2i/hd) from the
+// cos/sin table) on the rows' fp32 QKV products, rounded once to bf16: q to its row of q_out,
+// k and v into the cache rows of their positions.  A thread takes four consecutive i of one
+// head of one row (16-byte loads of both halves and of the table).
+__global__ void rope_scatter_kernel(const float* __restrict__ y, int rows_cap, const int* count_dev,
+                                    const int* __restrict__ row_map, int qkvd, int qd, int kvd, int hd, int N,
+                                    int Hkv, const float* __restrict__ rope_cos, const float* __restrict__ rope_sin,
+                                    __nv_bfloat16* q_out, __nv_bfloat16* kc, __nv_bfloat16* vc) {
+  pdl_trigger();
+  pdl_wait();
+  const int m_rows = count_dev ? min(*count_dev, rows_cap) : rows_cap;
+  const int half = hd >> 1;
+  const int per_row = qkvd >> 3;                            // threads per row: 4 pairs each
+  const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int j = static_cast<int>(gi / per_row);
+  if (j >= m_rows) return;
+  const int r = static_cast<int>(gi - static_cast<int64_t>(j) * per_row);
+  const int head = r / (half >> 2);                         // head slot over q, k, v heads
+  const int i = (r - head * (half >> 2)) * 4;
+  const int n_lo = head * hd + i;                           // feature of the low half
+  const float* yr = y + static_cast<int64_t>(j) * qkvd;
+  const float4 a = __ldg(reinterpret_cast<const float4*>(yr + n_lo));
+  const float4 bq = __ldg(reinterpret_cast<const float4*>(yr + n_lo + half));
+  const int flat = __ldg(row_map + j);
+  const int b = flat / N, pos = flat - b * N;
+  float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {bq.x, bq.y, bq.z, bq.w};
+  if (n_lo < qd + kvd) {
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(rope_cos + static_cast<int64_t>(pos) * half + i));
+    const float4 s4 = __ldg(reinterpret_cast<const float4*>(rope_sin + static_cast<int64_t>(pos) * half + i));
+    const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x = lo[e], z = hi[e];
+      lo[e] = x * cs[e] - z * sn[e];
+      hi[e] = z * cs[e] + x * sn[e];
+    }
+  }
+  __nv_bfloat16* dst;
+  if (n_lo < qd) {
+    dst = q_out + static_cast<int64_t>(j) * qd + n_lo;
+  } else {
+    int nn = n_lo - qd;
+    __nv_bfloat16* cache = kc;
+    if (nn >= kvd) {
+      nn -= kvd;
+      cache = vc;
+    }
+    const int kvh = nn / hd;
+    dst = cache + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd + (nn - kvh * hd);
+  }
+  uint2 w0, w1;
+  __nv_bfloat162 t0 = __floats2bfloat162_rn(lo[0], lo[1]), t1 = __floats2bfloat162_rn(lo[2], lo[3]);
+  __nv_bfloat162 t2 = __floats2bfloat162_rn(hi[0], hi[1]), t3 = __floats2bfloat162_rn(hi[2], hi[3]);
+  w0.x = *reinterpret_cast<uint32_t*>(&t0);
+  w0.y = *reinterpret_cast<uint32_t*>(&t1);
+  w1.x = *reinterpret_cast<uint32_t*>(&t2);
+  w1.y = *reinterpret_cast<uint32_t*>(&t3);
+  *reinterpret_cast<uint2*>(dst) = w0;
+  *reinterpret_cast<uint2*>(dst + half) = w1;
+}
+}  // namespace
+
+int rope_scatter_launch(const float* y, int rows_cap, const int* count_dev, const int* row_map, int qkvd, int qd,
+                        int kvd, int hd, int N, int Hkv, const float* rope_cos, const float* rope_sin,
+                        __nv_bfloat16* q_out, __nv_bfloat16* kc, __nv_bfloat16* vc, cudaStream_t st) {
+  if (rows_cap <= 0) return DLLM_OK;
+  if (hd % 8 || qd % hd || kvd % hd || qkvd != qd + 2 * kvd) return DLLM_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(rope_cos) % 16 ||
+      reinterpret_cast<uintptr_t>(rope_sin) % 16)
+    return DLLM_ERR_INVALID_ARG;
+  const int64_t threads = static_cast<int64_t>(rows_cap) * (qkvd >> 3);
+  return launch_pdl(rope_scatter_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st, y,
+                    rows_cap, count_dev, row_map, qkvd, qd, kvd, hd, N, Hkv, rope_cos, rope_sin, q_out, kc, vc);
+}
+
 int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
                         float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;

@@ -32,6 +32,11 @@ struct SelectParams {
 int rope_table_launch(float* cos_t, float* sin_t, int N, int hd, double theta, cudaStream_t st);
 int embed_rows_launch(const __nv_bfloat16* E, int V, const int* tokens, const int* row_map, const int* count_dev,
                       int rows_cap, int d, float* h, cudaStream_t st);
+// RoPE and K/V scatter of the rows' fp32 QKV products y [rows_cap, qkvd] (row j at position
+// row_map[j] = b N + pos): q rotated to q_out [rows, qd], k rotated and v into the caches.
+int rope_scatter_launch(const float* y, int rows_cap, const int* count_dev, const int* row_map, int qkvd, int qd,
+                        int kvd, int hd, int N, int Hkv, const float* rope_cos, const float* rope_sin,
+                        __nv_bfloat16* q_out, __nv_bfloat16* kc, __nv_bfloat16* vc, cudaStream_t st);
 int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
                         float eps, __nv_bfloat16* z, int64_t ldz, cudaStream_t st);
 int score_es_launch(float* h, float* h_prev, const float* conf, uint8_t* masked_prev, const int* tokens,
