@@ -132,7 +132,8 @@ def test_embed_rows_rejects_token_ids_outside_the_vocabulary():
 
 # ------------------------------------------------------------------ QKV + RoPE, SwiGLU
 
-@pytest.mark.parametrize("hq,hkv,hd,rows,splits", [(4, 4, 64, 9, 0), (8, 2, 128, 37, 1), (28, 4, 128, 5, 3)])
+@pytest.mark.parametrize("hq,hkv,hd,rows,splits", [(4, 4, 64, 9, 0), (8, 2, 128, 37, 1), (28, 4, 128, 5, 3),
+                                                   (8, 2, 128, 100, 0), (28, 4, 128, 180, 0)])
 def test_qkv_rope_and_cache_scatter(hq, hkv, hd, rows, splits):
     d = 512 if hq * hd <= 1024 else 3584
     dims = ModelDims(n_layers=1, d_model=d, n_heads=hq, n_kv_heads=hkv, head_dim=hd, ffn_dim=256, vocab=256,

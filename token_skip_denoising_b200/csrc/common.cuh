@@ -107,6 +107,9 @@ struct GemmArgs {
   int K = 0;
   int n_tiles_w = 0;             // 128-row output tiles (SwiGLU: F / 64)
   bool swiglu = false;
+  // the activation tile may be 256 wide for 129-256 rows (one tile instead of two): faster for
+  // a weight matrix of many 128-row tiles whose epilogue is a plain store (QKV), not for the rest
+  bool wide_ok = false;
   EpiParams epi;
 };
 

@@ -524,7 +524,7 @@ int run_layer(const LayerCtx& x, float* hbuf, const int* rows, const int* n, con
   g.n_tiles_w = x.qkvd / 128;
   // fp32 products, then RoPE and the K/V scatter as one coalesced pass (a rotation inside the
   // GEMM epilogue waits on the row map and the cos/sin table in every 16-column chunk)
-  g.epi.kind = EPI_STORE_F32; g.epi.out = x.yqkv; g.epi.ldo = x.qkvd;
+  g.epi.kind = EPI_STORE_F32; g.epi.out = x.yqkv; g.epi.ldo = x.qkvd; g.wide_ok = true;
   DLLM_TRY(timed_gemm(x.prof, g, x.gs, st, 4.0 * x.qkvd));
   DLLM_TRY(rope_scatter_launch(x.yqkv, rows_cap, n, rows, x.qkvd, x.qd, x.kvd, x.hd, x.N, x.Hkv, x.rope_cos,
                                x.rope_sin, x.q, x.kc, x.vc, st));

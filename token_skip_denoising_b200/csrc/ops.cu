@@ -117,7 +117,7 @@ int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32
   GemmArgs g;
   g.W = W; g.w_rows_total = qkvd; g.X = X; g.rows_cap = rows_cap; g.rows_dev = count; g.K = d;
   g.n_tiles_w = qkvd / 128;
-  g.epi.kind = EPI_STORE_F32; g.epi.out = y; g.epi.ldo = qkvd;
+  g.epi.kind = EPI_STORE_F32; g.epi.out = y; g.epi.ldo = qkvd; g.wide_ok = true;
   const int rc2 = gemm_launch(g, gs, st, splits, 0);
   if (rc2) return rc2;
   return rope_scatter_launch(y, rows_cap, count, rows_map, qkvd, qd, kvd, head_dim, N, n_kv_heads, rope_cos,
