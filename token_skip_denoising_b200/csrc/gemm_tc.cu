@@ -517,11 +517,13 @@ int pick_grid(int tiles, int KB) {
   return static_cast<int>(std::min<int64_t>(num_sms(), T));
 }
 
-// One 128-wide activation tile (65-128 rows): every CTA takes whole tiles, or one of p equal
+// Grid for 128- and 256-wide activation tiles: every CTA takes whole tiles, or one of p equal
 // pieces of a tile (p divides the k blocks, a piece at least 32 of them), never the uneven
-// stream-K share.  Measured per GEMM at 65 and 128 rows (LLaDA-8B shapes): QKV 39.7 -> 24.7 us
-// (96 tiles, 96 CTAs), O 29.7 -> 20.3 us (32 CTAs), down 40.8 -> 33.5 us (3 pieces of 32 tiles),
-// gate/up 54.1 -> 46.3 us (2 of 192 tiles per CTA).
+// stream-K share, whose split tiles cost a partial-sum round trip and a serial fix-up at the
+// end.  Measured (LLaDA-8B shapes): at 65-128 rows QKV 39.7 -> 24.7 us (96 tiles, 96 CTAs),
+// O 29.7 -> 20.3 us (32 CTAs), down 40.8 -> 33.5 us (3 pieces of 32 tiles), gate/up 54.1 ->
+// 46.3 us (2 of 192 tiles per CTA); a whole 768-row layer 507 -> 441 us; O at 1536 rows 101 ->
+// 69 us.
 int whole_piece_grid(int tiles, int KB) {
   const int sms = num_sms();
   if (tiles >= sms) {
@@ -602,7 +604,7 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   const int ksub = pick_ksub(a.K, bn);
   const int KB = a.K / (kBK * ksub);
   int grid = force_grid > 0 ? force_grid : pick_grid(tiles, KB);
-  if (force_grid <= 0 && bn >= 128 && tiles_act == 1) grid = whole_piece_grid(a.n_tiles_w, KB);
+  if (force_grid <= 0 && bn >= 128) grid = whole_piece_grid(tiles, KB);
   grid = static_cast<int>(std::min<int64_t>(grid, static_cast<int64_t>(tiles) * KB));
   // split tiles need the partial buffer and one counter per tile; without them every
   // CTA takes whole tiles only (grid = number of tiles divides the work exactly)
