@@ -667,62 +667,59 @@ namespace {
 // RoPE (rotate-half pairs i, i + hd/2 of every q and k head, by pos theta^(-2i/hd) from the
 // cos/sin table) on the rows' fp32 QKV products, rounded once to bf16: q to its row of q_out,
 // k and v into the cache rows of their positions.  A thread takes four consecutive i of one
-// head of one row (16-byte loads of both halves and of the table).
+// head (16-byte loads of both halves and of the table) in the rows of its grid row.
 __global__ void rope_scatter_kernel(const float* __restrict__ y, int rows_cap, const int* count_dev,
-                                    const int* __restrict__ row_map, int qkvd, int qd, int kvd, int hd, int N,
+                                    const int* __restrict__ row_map, int qkvd, int qd, int kvd, int hd_log2, int N,
                                     int Hkv, const float* __restrict__ rope_cos, const float* __restrict__ rope_sin,
                                     __nv_bfloat16* q_out, __nv_bfloat16* kc, __nv_bfloat16* vc) {
   pdl_trigger();
   pdl_wait();
   const int m_rows = count_dev ? min(*count_dev, rows_cap) : rows_cap;
-  const int half = hd >> 1;
-  const int per_row = qkvd >> 3;                            // threads per row: 4 pairs each
-  const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int j = static_cast<int>(gi / per_row);
-  if (j >= m_rows) return;
-  const int r = static_cast<int>(gi - static_cast<int64_t>(j) * per_row);
-  const int head = r / (half >> 2);                         // head slot over q, k, v heads
-  const int i = (r - head * (half >> 2)) * 4;
-  const int n_lo = head * hd + i;                           // feature of the low half
-  const float* yr = y + static_cast<int64_t>(j) * qkvd;
-  const float4 a = __ldg(reinterpret_cast<const float4*>(yr + n_lo));
-  const float4 bq = __ldg(reinterpret_cast<const float4*>(yr + n_lo + half));
-  const int flat = __ldg(row_map + j);
-  const int b = flat / N, pos = flat - b * N;
-  float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {bq.x, bq.y, bq.z, bq.w};
-  if (n_lo < qd + kvd) {
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(rope_cos + static_cast<int64_t>(pos) * half + i));
-    const float4 s4 = __ldg(reinterpret_cast<const float4*>(rope_sin + static_cast<int64_t>(pos) * half + i));
-    const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+  const int hd = 1 << hd_log2, half = hd >> 1;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;      // 4-pair group within a row
+  if (r >= (qkvd >> 3)) return;
+  const int head = r >> (hd_log2 - 3);                      // head slot over q, k, v heads (hd / 8 groups each)
+  const int i = (r - (head << (hd_log2 - 3))) * 4;
+  const int n_lo = (head << hd_log2) + i;                   // feature of the low half
+  const bool rotate = n_lo < qd + kvd;
+  int nn = n_lo - qd;                                       // feature within K (or V) when not a q feature
+  __nv_bfloat16* cache = kc;
+  if (nn >= kvd) {
+    nn -= kvd;
+    cache = vc;
+  }
+  const int kvh = nn >> hd_log2;
+  for (int j = blockIdx.y; j < m_rows; j += gridDim.y) {    // rows
+    const float* yr = y + static_cast<int64_t>(j) * qkvd;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(yr + n_lo));
+    const float4 bq = __ldg(reinterpret_cast<const float4*>(yr + n_lo + half));
+    const int flat = __ldg(row_map + j);
+    const int b = flat / N, pos = flat - b * N;
+    float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {bq.x, bq.y, bq.z, bq.w};
+    if (rotate) {
+      const float4 c4 = __ldg(reinterpret_cast<const float4*>(rope_cos + static_cast<int64_t>(pos) * half + i));
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(rope_sin + static_cast<int64_t>(pos) * half + i));
+      const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x = lo[e], z = hi[e];
-      lo[e] = x * cs[e] - z * sn[e];
-      hi[e] = z * cs[e] + x * sn[e];
+      for (int e = 0; e < 4; ++e) {
+        const float x = lo[e], z = hi[e];
+        lo[e] = x * cs[e] - z * sn[e];
+        hi[e] = z * cs[e] + x * sn[e];
+      }
     }
+    __nv_bfloat16* dst = n_lo < qd ? q_out + static_cast<int64_t>(j) * qd + n_lo
+                                   : cache + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd +
+                                         (nn - (kvh << hd_log2));
+    uint2 w0, w1;
+    __nv_bfloat162 t0 = __floats2bfloat162_rn(lo[0], lo[1]), t1 = __floats2bfloat162_rn(lo[2], lo[3]);
+    __nv_bfloat162 t2 = __floats2bfloat162_rn(hi[0], hi[1]), t3 = __floats2bfloat162_rn(hi[2], hi[3]);
+    w0.x = *reinterpret_cast<uint32_t*>(&t0);
+    w0.y = *reinterpret_cast<uint32_t*>(&t1);
+    w1.x = *reinterpret_cast<uint32_t*>(&t2);
+    w1.y = *reinterpret_cast<uint32_t*>(&t3);
+    *reinterpret_cast<uint2*>(dst) = w0;
+    *reinterpret_cast<uint2*>(dst + half) = w1;
   }
-  __nv_bfloat16* dst;
-  if (n_lo < qd) {
-    dst = q_out + static_cast<int64_t>(j) * qd + n_lo;
-  } else {
-    int nn = n_lo - qd;
-    __nv_bfloat16* cache = kc;
-    if (nn >= kvd) {
-      nn -= kvd;
-      cache = vc;
-    }
-    const int kvh = nn / hd;
-    dst = cache + ((static_cast<int64_t>(b) * Hkv + kvh) * N + pos) * hd + (nn - kvh * hd);
-  }
-  uint2 w0, w1;
-  __nv_bfloat162 t0 = __floats2bfloat162_rn(lo[0], lo[1]), t1 = __floats2bfloat162_rn(lo[2], lo[3]);
-  __nv_bfloat162 t2 = __floats2bfloat162_rn(hi[0], hi[1]), t3 = __floats2bfloat162_rn(hi[2], hi[3]);
-  w0.x = *reinterpret_cast<uint32_t*>(&t0);
-  w0.y = *reinterpret_cast<uint32_t*>(&t1);
-  w1.x = *reinterpret_cast<uint32_t*>(&t2);
-  w1.y = *reinterpret_cast<uint32_t*>(&t3);
-  *reinterpret_cast<uint2*>(dst) = w0;
-  *reinterpret_cast<uint2*>(dst + half) = w1;
 }
 }  // namespace
 
@@ -730,13 +727,15 @@ int rope_scatter_launch(const float* y, int rows_cap, const int* count_dev, cons
                         int kvd, int hd, int N, int Hkv, const float* rope_cos, const float* rope_sin,
                         __nv_bfloat16* q_out, __nv_bfloat16* kc, __nv_bfloat16* vc, cudaStream_t st) {
   if (rows_cap <= 0) return DLLM_OK;
-  if (hd % 8 || qd % hd || kvd % hd || qkvd != qd + 2 * kvd) return DLLM_ERR_SHAPE;
+  int hd_log2 = 0;
+  while ((1 << hd_log2) < hd) ++hd_log2;
+  if (hd < 8 || (1 << hd_log2) != hd || qd % hd || kvd % hd || qkvd != qd + 2 * kvd) return DLLM_ERR_SHAPE;
   if (reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(rope_cos) % 16 ||
       reinterpret_cast<uintptr_t>(rope_sin) % 16)
     return DLLM_ERR_INVALID_ARG;
-  const int64_t threads = static_cast<int64_t>(rows_cap) * (qkvd >> 3);
-  return launch_pdl(rope_scatter_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st, y,
-                    rows_cap, count_dev, row_map, qkvd, qd, kvd, hd, N, Hkv, rope_cos, rope_sin, q_out, kc, vc);
+  const int per_row = qkvd >> 3;
+  return launch_pdl(rope_scatter_kernel, dim3((per_row + 255) / 256, std::min(rows_cap, 65535)), dim3(256), 0, st, y, rows_cap,
+                    count_dev, row_map, qkvd, qd, kvd, hd_log2, N, Hkv, rope_cos, rope_sin, q_out, kc, vc);
 }
 
 int rmsnorm_rows_launch(const float* h, const int* row_map, const int* count_dev, int rows_cap, int d, const float* g,
