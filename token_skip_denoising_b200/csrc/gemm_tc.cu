@@ -524,10 +524,16 @@ int pick_grid(int tiles, int KB) {
 // O 29.7 -> 20.3 us (32 CTAs), down 40.8 -> 33.5 us (3 pieces of 32 tiles), gate/up 54.1 ->
 // 46.3 us (2 of 192 tiles per CTA); a whole 768-row layer 507 -> 441 us; O at 1536 rows 101 ->
 // 69 us.
+// Above kMaxWholePerCta tiles per CTA the stream-K share wins (0 returned) unless rounding up
+// to whole tiles costs under a quarter tile per CTA: its two split tiles per CTA cost little
+// against many whole ones, while the rounding idles SMs (Dream-7B O at 12288 rows: 1344 tiles
+// on 135 CTAs of 10; batch-8 SureLock step 223 -> 244 ms with whole tiles at any count).
+constexpr int kMaxWholePerCta = 4;
 int whole_piece_grid(int tiles, int KB) {
   const int sms = num_sms();
   if (tiles >= sms) {
     const int per = (tiles + sms - 1) / sms;
+    if (per > kMaxWholePerCta && 4 * (static_cast<int64_t>(per) * sms - tiles) >= sms) return 0;
     return (tiles + per - 1) / per;
   }
   int p = std::max(1, std::min(sms / tiles, KB / 32));
@@ -604,7 +610,10 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   const int ksub = pick_ksub(a.K, bn);
   const int KB = a.K / (kBK * ksub);
   int grid = force_grid > 0 ? force_grid : pick_grid(tiles, KB);
-  if (force_grid <= 0 && bn >= 128) grid = whole_piece_grid(tiles, KB);
+  if (force_grid <= 0 && bn >= 128) {
+    const int wg = whole_piece_grid(tiles, KB);
+    if (wg > 0) grid = wg;
+  }
   grid = static_cast<int>(std::min<int64_t>(grid, static_cast<int64_t>(tiles) * KB));
   // split tiles need the partial buffer and one counter per tile; without them every
   // CTA takes whole tiles only (grid = number of tiles divides the work exactly)
