@@ -290,7 +290,8 @@ def run_ours(args, rank, world, local_rank):
 # ---------------------------------------------------------------- active-ratio sweep (single layer)
 def micro_sweep(peaks, reps=20):
     """Single-layer step at N = 2048 (d 4096, 32 heads, FFN 12288): score -> top-k ->
-    gathered QKV/O/FFN -> active-query attention -> K/V scatter, for each active ratio."""
+    gathered QKV/O/FFN -> active-query attention -> K/V scatter, for each active ratio; the
+    step's launches replay as one CUDA graph after an L2 flush."""
     import torch
 
     from synth import get_config, make_weights
@@ -334,18 +335,34 @@ def micro_sweep(peaks, reps=20):
             cnt = torch.tensor([k], dtype=torch.int32, device="cuda")
             off = torch.tensor([0, k], dtype=torch.int32, device="cuda")
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-            times = []
-            for it in range(reps + 3):
-                flush.zero_()
-                ev[0].record()
+
+            def step():
                 s = ops.score_es(h, hp, hin["conf"], 0.5, masked_prev=hin["masked_prev"])
                 ops.select(s, 1, N, ops.SEL_TOPK_DESC, k)
                 # the layer runs on the fixed index pattern so both patterns are measured
                 ops.layer(ccfg, lw, kc, vc, cos, sin, h, act_idx, cnt, off, k, k, ws=ws)
+
+            # the three launches replay as one CUDA graph, so the host's per-call marshalling
+            # does not pace the GPU (at 62 rows it would add ~100 us of idle device time)
+            step()
+            torch.cuda.synchronize()
+            cs = torch.cuda.Stream()
+            cs.wait_stream(torch.cuda.current_stream())
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(cs):
+                with torch.cuda.graph(graph, stream=cs):
+                    step()
+            torch.cuda.synchronize()
+            times = []
+            for it in range(reps + 3):
+                flush.zero_()
+                ev[0].record()
+                graph.replay()
                 ev[1].record()
                 torch.cuda.synchronize()
                 if it >= 3:
                     times.append(ev[0].elapsed_time(ev[1]))
+            del graph
             t = statistics.median(times)
             kv_bytes = 2 * N * m.kv_dim * 2
             byts = P * 2 + kv_bytes + k * (2 * m.kv_dim + 2 * d) * 2 + 2 * N * d * 4
