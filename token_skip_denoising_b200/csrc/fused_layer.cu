@@ -95,8 +95,9 @@ struct FParams {
   __nv_bfloat16* z2;      // [rows_cap, d]  g_ffn * h (gate/up operand)
   float* s_qkv;           // [kMaxRows, qkvd] fp32 QKV sums
   float* s_gu;            // [kMaxRows, 2F]   fp32 gate/up sums
-  float* ssp1;            // [grid, kMaxRows] per-CTA partial sums of h^2 before attention (RMSNorm)
-  float* ssp2;            // [grid, kMaxRows] the same before the FFN
+  float* ss1;             // [kMaxRows] sums of h^2 per row before attention (RMSNorm); zero
+                          // between uses: CTA 0 clears it once every CTA has read it
+  float* ss2;             // [kMaxRows] the same before the FFN
   int qkvd, qd, kvd, hd, Hkv, N, F;
   const float* rope_cos;
   const float* rope_sin;
@@ -438,9 +439,9 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
     };
 
     // GEMM operand X = bf16(gain * h) over every row, each CTA a slice of the columns, and
-    // the CTA's partial sums of h^2 per row into ssp[c][j] (RMSNorm is a per-row scale: the
+    // the CTA's partial sums of h^2 per row added into ss[j] (RMSNorm is a per-row scale: the
     // GEMM sums are multiplied by 1/rms afterwards)
-    auto gain_operand = [&](const float* gain, __nv_bfloat16* X, float* ssp) {
+    auto gain_operand = [&](const float* gain, __nv_bfloat16* X, float* ss) {
       const int n4 = p.d >> 2;
       const int q0 = static_cast<int>(static_cast<int64_t>(n4) * c / G);
       const int q1 = static_cast<int>(static_cast<int64_t>(n4) * (c + 1) / G);
@@ -461,19 +462,12 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         atomicAdd(&s_ss[jj], v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w);
       }
       epi_bar();
-      if (t < m_rows) ssp[c * kMaxRows + t] = s_ss[t];
+      if (t < m_rows) atomicAdd(ss + t, s_ss[t]);
     };
-    // 1/rms of every row from the partials of all CTAs (after the phase that wrote them)
-    auto rinv_from = [&](const float* ssp, float* rinv) {
-      const int jj = t % kMaxRows;
-      float acc = 0.f;
-      if (jj < m_rows)
-        for (int cc = t / kMaxRows; cc < G; cc += 128 / kMaxRows) acc += __ldcg(ssp + cc * kMaxRows + jj);
-      if (t < kMaxRows) s_ss[t] = 0.f;
-      epi_bar();
-      if (jj < m_rows) atomicAdd(&s_ss[jj], acc);
-      epi_bar();
-      if (t < m_rows) rinv[t] = rsqrtf(s_ss[t] / static_cast<float>(p.d) + p.eps);
+    // 1/rms of every row from the sums all CTAs added (after the phase that added them): one
+    // L2 round trip, where summing 148 per-CTA partials was a chain of dependent loads
+    auto rinv_from = [&](const float* ss, float* rinv) {
+      if (t < m_rows) rinv[t] = rsqrtf(__ldcg(ss + t) / static_cast<float>(p.d) + p.eps);
       epi_bar();
     };
 
@@ -565,15 +559,16 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int64_t x = gt; x < nq; x += gstride) reinterpret_cast<float4*>(p.s_qkv)[x] = z;
         for (int64_t x = gt; x < ng; x += gstride) reinterpret_cast<float4*>(p.s_gu)[x] = z;
-        gain_operand(p.g_attn + static_cast<int64_t>(l) * p.d, p.z1, p.ssp1);   // QKV operand
+        gain_operand(p.g_attn + static_cast<int64_t>(l) * p.d, p.z1, p.ss1);    // QKV operand
       }
       signal_phase(p.sync + S_X1, t);
-      if (epi_wait_phase(p.sync + S_X1, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ssp1, s_rinv1);   // while QKV streams
+      if (epi_wait_phase(p.sync + S_X1, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ss1, s_rinv1);   // while QKV streams
       gemm_epilogues(0, li);                                       // QKV sums
       signal_phase(p.sync + S_QKV, t);
       // RMSNorm scale and RoPE (rotate-half pairs i, i + hd/2) on q and k; q to the attention
       // operand, k and v scattered into the cache rows of their positions
       if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
+        if (c == 0 && t < kMaxRows) p.ss1[t] = 0.f;    // every CTA has read this layer's sums
         const int pairs = p.qkvd >> 1;
         const int64_t total = static_cast<int64_t>(m_rows) * pairs;
         constexpr int U = 4;                    // pairs per thread in flight: their loads go out together
@@ -694,13 +689,14 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       signal_phase(p.sync + S_O, t);
       // gate/up operand g_ffn * h once every O sum is in h
       if (epi_wait_phase(p.sync + S_O, target, s_flag, t, p.spin_limit, p.sync + S_ABORT))
-        gain_operand(p.g_ffn + static_cast<int64_t>(l) * p.d, p.z2, p.ssp2);
+        gain_operand(p.g_ffn + static_cast<int64_t>(l) * p.d, p.z2, p.ss2);
       signal_phase(p.sync + S_X2, t);
-      if (epi_wait_phase(p.sync + S_X2, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ssp2, s_rinv2);   // while gate/up streams
+      if (epi_wait_phase(p.sync + S_X2, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) rinv_from(p.ss2, s_rinv2);   // while gate/up streams
       gemm_epilogues(2, li);                                       // gate/up sums
       signal_phase(p.sync + S_GU, t);
       // SwiGLU on the RMSNorm-scaled sums: act = silu(gate) * up
       if (epi_wait_phase(p.sync + S_GU, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
+        if (c == 0 && t < kMaxRows) p.ss2[t] = 0.f;
         const int f4 = p.F >> 2;
         const int64_t total = static_cast<int64_t>(m_rows) * f4;
         constexpr int U = 4;                    // groups per thread in flight: their loads go out together
@@ -757,6 +753,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         for (int q = 0; q < p.n_attn_ctr; ++q) p.attn_ctr[q] = 0;
         if (p.es.on)
           for (int q = 0; q < 2 * p.es.B * p.es.n_cand; ++q) p.es_acc[q] = 0.f;
+        for (int q = 0; q < kMaxRows; ++q) p.ss1[q] = p.ss2[q] = 0.f;
       }
       for (int q = 0; q <= S_ABORT; ++q) atomicExch(p.sync + q, 0);
       __threadfence();
@@ -851,8 +848,8 @@ int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   p.z2 = a.z2;
   p.s_qkv = s_qkv;
   p.s_gu = s_gu;
-  p.ssp1 = ssp;
-  p.ssp2 = ssp + static_cast<size_t>(grid) * kMaxRows;
+  p.ss1 = ssp;
+  p.ss2 = ssp + kMaxRows;
   p.es_acc = ssp + 2 * static_cast<size_t>(a.max_ctas) * kMaxRows;
   p.n_attn_ctr = a.n_attn_ctr;
   p.spin_limit = a.spin_limit ? a.spin_limit : kSpinLimit;
