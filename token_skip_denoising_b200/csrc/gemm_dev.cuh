@@ -97,8 +97,8 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& e, const float (&v)[1
       break;
     }
     case EPI_RESID_ADD: {
-      // one writer per element (the tile's owner), so a reduction adds exactly once and the
-      // result is the same as a load and a store, without waiting for the load
+      // a reduction, not a load and a store, so nothing waits for the load; the tile's owner
+      // adds the whole sum, or (from 128-wide tiles on) each k piece of a split tile adds its own
       int rr[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)

@@ -69,6 +69,7 @@ struct KParams {
   int n_tiles_w;
   int tiles_act;
   int wt_fastest;      // tile numbering: 1 weight tile fastest, 0 activation tile fastest
+  int add_pieces;      // the epilogue adds into its target: a split tile's piece adds its own partial
   int swiglu;
   int ffn;
   float* partial;      // [gridDim.x][2][BN * 128]
@@ -295,7 +296,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       const int row0 = p.swiglu ? tw * 64 : tw * kTileM;
       const int row1 = p.swiglu ? p.ffn + tw * 64 : tw * kTileM + 64;
       const int n = t < 64 ? row0 + t : row1 + (t - 64);
-      const bool whole = (kb0 == 0 && kb1 == KB);
+      const bool whole = (kb0 == 0 && kb1 == KB) || p.add_pieces;
       if (whole) {
         for (int cc = c0; cc < c1; cc += 16) {
           float v[16];
@@ -610,7 +611,14 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   const int ksub = pick_ksub(a.K, bn);
   const int KB = a.K / (kBK * ksub);
   int grid = force_grid > 0 ? force_grid : pick_grid(tiles, KB);
-  if (force_grid <= 0 && bn >= 128) {
+  // The residual add is a reduction: when whole tiles would leave more than half the SMs idle
+  // (O and down at 65-256 rows: 32 or 64 tiles), each piece of a split tile adds its own partial
+  // sums into h, so the stream-K share over every SM needs no partial buffer and no fix-up
+  // (layers over 2048 positions: 65 rows 179 -> 161 us, 205 rows 240 -> 228 us; with 96 or 512
+  // tiles the extra reductions cost more than they gain: 384 rows 288 -> 298 us).  Narrower
+  // tiles keep the fixed-order fix-up, so layers of up to 64 rows stay bit-reproducible.
+  const bool add_pieces = a.epi.kind == EPI_RESID_ADD && bn >= 128 && 2 * tiles <= num_sms();
+  if (force_grid <= 0 && bn >= 128 && !add_pieces) {
     const int wg = whole_piece_grid(tiles, KB);
     if (wg > 0) grid = wg;
   }
@@ -618,7 +626,7 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   // split tiles need the partial buffer and one counter per tile; without them every
   // CTA takes whole tiles only (grid = number of tiles divides the work exactly)
   const size_t need = static_cast<size_t>(grid) * 2 * bn * 128;
-  if (!s.partial || s.partial_floats < need || !s.counters || s.n_counters < tiles) {
+  if (!add_pieces && (!s.partial || s.partial_floats < need || !s.counters || s.n_counters < tiles)) {
     if (static_cast<int64_t>(tiles) * KB % grid != 0 || tiles % grid != 0) grid = std::min(grid, tiles);
     while (grid > 1 && tiles % grid != 0) --grid;
   }
@@ -638,6 +646,7 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
     return e ? atoi(e) : -1;
   }();
   kp.wt_fastest = order_env >= 0 ? order_env : (tiles_act <= kMaxActTilesWtFastest ? 1 : 0);
+  kp.add_pieces = add_pieces ? 1 : 0;
   kp.swiglu = a.swiglu ? 1 : 0;
   kp.ffn = a.epi.ffn;
   kp.partial = s.partial;
