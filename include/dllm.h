@@ -421,8 +421,11 @@ int dllm_op_gemm(int32_t kind, const void* W, int32_t n_out, const void* X, int3
 int dllm_op_gemm_noalloc(int32_t kind, const void* W, int32_t n_out, const void* X, int32_t rows_cap,
                          const int32_t* count, int32_t K, void* out, const int32_t* rows_map, void* stream);
 
-/* Fused QKV projection: RoPE on q and k, q -> q_out bf16 [rows, Hq*hd], k and v -> the
- * cache rows (b, :, pos) of rows_map[j] = b * N + pos.  W = one layer of w_qkv. */
+/* QKV projection with RoPE on q and k: q -> q_out bf16 [rows, Hq*hd], k and v -> the cache
+ * rows (b, :, pos) of rows_map[j] = b * N + pos.  W = one layer of w_qkv.  The products are
+ * kept in fp32 in the workspace (rows_cap * (Hq + 2 Hkv) * hd * 4 bytes after the GEMM
+ * scratch; DLLM_ERR_SHAPE when it does not fit) and one coalesced pass rotates and
+ * scatters them; head_dim a power of two. */
 int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32_t* count, int32_t d,
                      int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t N, const int32_t* rows_map,
                      const float* rope_cos, const float* rope_sin, void* q_out, void* kcache, void* vcache,
@@ -433,7 +436,9 @@ int dllm_op_gate_up(const void* W, int32_t F, const void* X, int32_t rows_cap, c
                     void* act, int32_t splits, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Attention of the rows of each sequence (seq_off device int32 [B+1]) over all N cached keys.
- * q, out bf16 [rows, Hq*hd]; caches bf16 [B, Hkv, N, hd]; splits 0 = automatic. */
+ * q, out bf16 [rows, Hq*hd]; caches bf16 [B, Hkv, N, hd] (16-byte aligned); splits 0 = automatic
+ * (key splits, merged afterwards).  Head dim 128 with at least 64 query units per sequence and
+ * KV head (a unit is a (row, query head) pair) runs on the tensor cores, else on CUDA cores. */
 int dllm_op_attention(const void* q, const void* kcache, const void* vcache, void* out, const int32_t* seq_off,
                       int32_t B, int32_t rows_cap, int32_t rows_per_seq_cap, int32_t N, int32_t n_heads,
                       int32_t n_kv_heads, int32_t head_dim, int32_t splits, void* workspace, size_t workspace_bytes,
