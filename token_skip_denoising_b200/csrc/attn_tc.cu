@@ -137,16 +137,16 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 2^x by the MUFU instruction (relative error about 2^-22, inputs <= 0 here; P is rounded to
-// bf16 afterwards, 2^-9).
+// 2^x by the MUFU instruction (relative error about 2^-22; the inputs here are at most the
+// rescale slack, 8, and results below 2^-126 flush to 0; P is rounded to bf16 afterwards, 2^-9).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// Bounded wait of the softmax threads: between polls they sleep, so the 256 waiting
-// threads leave the issue slots of their SM sub-partitions to the TMA and MMA warps.
+// Bounded wait of the softmax threads: between polls they sleep, so waiting softmax warps
+// leave the issue slots of their SM sub-partitions to the TMA and MMA warps.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -218,8 +218,6 @@ __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t aq, uint32_t ak, uin
     tc_mma_f16(d, make_desc_k_sw128(aq + o), make_desc_k_sw128(ak + o), idesc, kk > 0 ? 1u : 0u);
   }
 }
-// O[d] (+)= P V over 128 keys: P K-major (keys contiguous), V MN-major (hd contiguous);
-// a K = 16 step is 16 key rows of V, 2048 B into each of its two hd panels.
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A is 128 lanes x 16 bf16 (eight columns).
 __device__ __forceinline__ void tc_mma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate) {
@@ -230,6 +228,9 @@ __device__ __forceinline__ void tc_mma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, 
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// O[d] (+)= P V over 128 keys: P from TMEM (two keys per 32-bit column, eight columns per
+// 16-key step), V MN-major (hd contiguous): a step is 16 key rows of V, 2048 B into each of
+// its two hd panels.
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t ap_tmem, uint32_t av, uint32_t idesc, bool acc) {
 #pragma unroll
   for (int kk = 0; kk < kTk / 16; ++kk)
