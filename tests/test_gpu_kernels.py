@@ -84,6 +84,29 @@ def test_gemm_residual_scatter(splits):
     np.testing.assert_array_equal(got[untouched], _f64(h0)[untouched])
 
 
+@pytest.mark.parametrize("rows,n_out,K,count", [(100, 1024, 2048, None), (205, 1024, 4096, 190), (768, 4096, 1024, None)])
+def test_gemm_residual_wide_tiles(rows, n_out, K, count):
+    """The residual add from 128-wide tiles on: at 100 and 205 rows (8 and 16 tiles, at most half
+    the SMs) each piece of a split tile adds its own partial into h; at 768 rows with 4096 outputs
+    the 128-wide tiles would outnumber the SMs, so it runs as 96 whole 256-wide tiles."""
+    W = _bf16((n_out, K), 12, 0.05)
+    X = _bf16((rows, K), 13)
+    g = _gen(14)
+    n_h = rows + 37
+    h0 = torch.randn((n_h, n_out), generator=g)
+    rmap = torch.randperm(n_h, generator=g)[:rows].to(torch.int32)
+    cnt = None if count is None else torch.tensor([count], dtype=torch.int32, device=DEV)
+    h = h0.clone().to(DEV)
+    ops.gemm(W.to(DEV), X.to(DEV), kind=3, count=cnt, out=h, rows_map=rmap.to(DEV))
+    m = rows if count is None else count
+    ref = _f64(h0)
+    ref[rmap[:m].numpy()] += _f64(X[:m]) @ _f64(W).T
+    got = h.cpu().double().numpy()
+    assert _rowrel(got, ref) < 1e-5
+    untouched = np.setdiff1d(np.arange(n_h), rmap[:m].numpy())
+    np.testing.assert_array_equal(got[untouched], _f64(h0)[untouched])
+
+
 def test_gemm_split_k_is_deterministic():
     W = _bf16((512, 4096), 6, 0.05).to(DEV)
     X = _bf16((11, 4096), 7).to(DEV)
