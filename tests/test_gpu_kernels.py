@@ -190,6 +190,31 @@ def test_qkv_rope_and_cache_scatter(hq, hkv, hd, rows, splits):
         assert np.all(kg[b, :, p] == 0)
 
 
+def test_qkv_rope_beyond_the_grid_height():
+    """70000 rows: the RoPE pass covers rows past the 65535-row grid height by striding."""
+    hq, hkv, hd, d, rows = 2, 2, 64, 64, 70000
+    dims = ModelDims(n_layers=1, d_model=d, n_heads=hq, n_kv_heads=hkv, head_dim=hd, ffn_dim=256, vocab=256,
+                     mask_id=255, rope_theta=10000.0)
+    N = rows
+    W = _bf16((dims.qkv_dim, d), 15, 0.1)
+    X = _bf16((rows, d), 16)
+    flat = np.random.default_rng(17).permutation(N).astype(np.int32)
+    cos, sin = ops.rope_table(N, hd, dims.rope_theta)
+    kc = torch.zeros((1, hkv, N, hd), dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    ws = torch.zeros(512 << 20, dtype=torch.uint8, device=DEV)
+    q = ops.qkv_rope(W.to(DEV), X.to(DEV), dims, N, torch.tensor(flat, device=DEV), cos, sin, kc, vc, ws=ws)
+    torch.cuda.synchronize()
+    y = _f64(X) @ _f64(W).T
+    qr = om.apply_rope(y[:, :dims.q_dim].reshape(rows, hq, hd), flat, dims.rope_theta)
+    kr = om.apply_rope(y[:, dims.q_dim:dims.q_dim + dims.kv_dim].reshape(rows, hkv, hd), flat, dims.rope_theta)
+    assert _rowrel(q.float().cpu().numpy(), qr.reshape(rows, -1)) < 1e-2
+    kg = kc[0].float().cpu().numpy().transpose(1, 0, 2)[flat]          # [rows, hkv, hd] in row order
+    vg = vc[0].float().cpu().numpy().transpose(1, 0, 2)[flat]
+    assert _rowrel(kg.reshape(rows, -1), kr.reshape(rows, -1)) < 1e-2
+    assert _rowrel(vg.reshape(rows, -1), y[:, dims.q_dim + dims.kv_dim:]) < 1e-2
+
+
 @pytest.mark.parametrize("rows,F,splits", [(3, 256, 0), (40, 1024, 1), (130, 512, 0), (8, 18944 // 4, 2)])
 def test_gate_up_swiglu(rows, F, splits):
     d = 512
