@@ -569,58 +569,74 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
       // operand, k and v scattered into the cache rows of their positions
       if (epi_wait_phase(p.sync + S_QKV, target, s_flag, t, p.spin_limit, p.sync + S_ABORT)) {
         if (c == 0 && t < kMaxRows) p.ss1[t] = 0.f;    // every CTA has read this layer's sums
-        const int pairs = p.qkvd >> 1;
-        const int64_t total = static_cast<int64_t>(m_rows) * pairs;
-        constexpr int U = 4;                    // pairs per thread in flight: their loads go out together
+        // an item is 4 consecutive pairs of one head of one row: 16-byte loads of both halves
+        // and of the cos/sin table, 8-byte stores
+        const int groups = p.qkvd >> 3;         // items per row
+        const int gph = half >> 2;              // items per head
+        const int64_t total = static_cast<int64_t>(m_rows) * groups;
+        constexpr int U = 4;                    // items per thread in flight: their loads go out together
         for (int64_t u0 = gt; u0 < total; u0 += U * gstride) {
-          float xl[U], xh[U], cs[U], sn[U];
+          float4 xl[U], xh[U], cs[U], sn[U];
           int jrs[U], nlo[U], pis[U];
 #pragma unroll
           for (int e = 0; e < U; ++e) {
             const int64_t uu = u0 + e * gstride < total ? u0 + e * gstride : 0;   // in bounds either way
-            const int jr = static_cast<int>(uu / pairs);
-            const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * pairs);
-            pis[e] = rr % half;
-            nlo[e] = (rr / half) * p.hd + pis[e];
+            const int jr = static_cast<int>(uu / groups);
+            const int rr = static_cast<int>(uu - static_cast<int64_t>(jr) * groups);
+            const int head = rr / gph;
+            pis[e] = (rr - head * gph) * 4;
+            nlo[e] = head * p.hd + pis[e];
             jrs[e] = jr;
             const float* srow = p.s_qkv + static_cast<int64_t>(jr) * p.qkvd;
-            xl[e] = __ldcg(srow + nlo[e]);
-            xh[e] = __ldcg(srow + nlo[e] + half);
+            xl[e] = __ldcg(reinterpret_cast<const float4*>(srow + nlo[e]));
+            xh[e] = __ldcg(reinterpret_cast<const float4*>(srow + nlo[e] + half));
             const int flat = s_rows[jr];
             const int pos = flat - (flat / p.N) * p.N;
-            cs[e] = __ldg(p.rope_cos + static_cast<int64_t>(pos) * half + pis[e]);
-            sn[e] = __ldg(p.rope_sin + static_cast<int64_t>(pos) * half + pis[e]);
+            cs[e] = __ldg(reinterpret_cast<const float4*>(p.rope_cos + static_cast<int64_t>(pos) * half + pis[e]));
+            sn[e] = __ldg(reinterpret_cast<const float4*>(p.rope_sin + static_cast<int64_t>(pos) * half + pis[e]));
           }
 #pragma unroll
           for (int e = 0; e < U; ++e) {
-          if (u0 + e * gstride >= total) break;
-          const int jr = jrs[e], n_lo = nlo[e], pi = pis[e];
-          const float ri = s_rinv1[jr];
-          const float x_l = xl[e] * ri, x_h = xh[e] * ri;
-          const int flat = s_rows[jr];
-          const int b = flat / p.N;
-          const int pos = flat - b * p.N;
-          float yl = x_l, yh = x_h;
-          if (n_lo < p.qd + p.kvd) {
-            yl = x_l * cs[e] - x_h * sn[e];
-            yh = x_h * cs[e] + x_l * sn[e];
-          }
-          if (n_lo < p.qd) {
-            __nv_bfloat16* dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
-            dst[0] = __float2bfloat16(yl);
-            dst[half] = __float2bfloat16(yh);
-          } else {
-            int nn = n_lo - p.qd;
-            __nv_bfloat16* cache = kc;
-            if (nn >= p.kvd) {
-              nn -= p.kvd;
-              cache = vc;
+            if (u0 + e * gstride >= total) break;
+            const int jr = jrs[e], n_lo = nlo[e], pi = pis[e];
+            const float ri = s_rinv1[jr];
+            float lo[4] = {xl[e].x * ri, xl[e].y * ri, xl[e].z * ri, xl[e].w * ri};
+            float hi[4] = {xh[e].x * ri, xh[e].y * ri, xh[e].z * ri, xh[e].w * ri};
+            if (n_lo < p.qd + p.kvd) {
+              const float c4[4] = {cs[e].x, cs[e].y, cs[e].z, cs[e].w};
+              const float s4[4] = {sn[e].x, sn[e].y, sn[e].z, sn[e].w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float x_l = lo[k], x_h = hi[k];
+                lo[k] = x_l * c4[k] - x_h * s4[k];
+                hi[k] = x_h * c4[k] + x_l * s4[k];
+              }
             }
-            const int kvh = nn / p.hd;
-            __nv_bfloat16* dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
-            dst[0] = __float2bfloat16(yl);
-            dst[half] = __float2bfloat16(yh);
-          }
+            const int flat = s_rows[jr];
+            const int b = flat / p.N;
+            const int pos = flat - b * p.N;
+            __nv_bfloat16* dst;
+            if (n_lo < p.qd) {
+              dst = p.q + static_cast<int64_t>(jr) * p.qd + n_lo;
+            } else {
+              int nn = n_lo - p.qd;
+              __nv_bfloat16* cache = kc;
+              if (nn >= p.kvd) {
+                nn -= p.kvd;
+                cache = vc;
+              }
+              const int kvh = nn / p.hd;
+              dst = cache + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + pos) * p.hd + pi;
+            }
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(lo[0], lo[1]), t1 = __floats2bfloat162_rn(lo[2], lo[3]);
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(hi[0], hi[1]), t3 = __floats2bfloat162_rn(hi[2], hi[3]);
+            uint2 w0, w1;
+            w0.x = *reinterpret_cast<uint32_t*>(&t0);
+            w0.y = *reinterpret_cast<uint32_t*>(&t1);
+            w1.x = *reinterpret_cast<uint32_t*>(&t2);
+            w1.y = *reinterpret_cast<uint32_t*>(&t3);
+            *reinterpret_cast<uint2*>(dst) = w0;
+            *reinterpret_cast<uint2*>(dst + half) = w1;
           }
         }
       }
@@ -699,7 +715,7 @@ fused_layer_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_consta
         if (c == 0 && t < kMaxRows) p.ss2[t] = 0.f;
         const int f4 = p.F >> 2;
         const int64_t total = static_cast<int64_t>(m_rows) * f4;
-        constexpr int U = 4;                    // groups per thread in flight: their loads go out together
+        constexpr int U = 8;                    // groups per thread in flight: their loads go out together
         for (int64_t u0 = gt; u0 < total; u0 += U * gstride) {
           float4 g4s[U], u4s[U];
 #pragma unroll
@@ -802,6 +818,10 @@ int fused_attn_counters(int B, int Hq, int Hkv, int rows_cap) {
 int fused_layer_launch(const FusedLayerArgs& a, cudaStream_t st) {
   if (a.rows_cap <= 0 || a.rows_cap > kMaxRows) return DLLM_ERR_UNSUPPORTED;
   if (a.d % 128 || a.qd % 128 || a.F % 128 || a.qkvd % 128 || a.hd > 128) return DLLM_ERR_UNSUPPORTED;
+  // the RoPE phase moves 4 pairs per item: 16-byte table loads, 8-byte operand and cache stores
+  if (a.hd % 8 || reinterpret_cast<uintptr_t>(a.rope_cos) % 16 || reinterpret_cast<uintptr_t>(a.rope_sin) % 16 ||
+      reinterpret_cast<uintptr_t>(a.kc) % 8 || reinterpret_cast<uintptr_t>(a.vc) % 8)
+    return DLLM_ERR_UNSUPPORTED;
   if (a.n_layers <= 0 || a.l0 < 0 || a.l0 + a.n_layers > a.L) return DLLM_ERR_INVALID_ARG;
   const int bn = a.rows_cap <= 16 ? 16 : (a.rows_cap <= 32 ? 32 : 64);
   if (a.max_ctas <= 0) return DLLM_ERR_INVALID_ARG;
