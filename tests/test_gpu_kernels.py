@@ -52,6 +52,7 @@ def _rowrel(a, b):
     (7, None, 384, 512, 0, 0), (16, None, 256, 256, 1, 0), (33, 29, 512, 1024, 3, 0),
     (100, None, 384, 512, 0, 0), (300, 257, 256, 512, 1, 0), (5, None, 128, 4096, 9, 0),
     (64, 50, 256, 512, 2, 128), (200, None, 128, 192, 0, 256),
+    (600, 577, 256, 512, 0, 0), (520, None, 384, 1024, 0, 0),
 ])
 def test_gemm_store_f32(rows, count, n_out, K, splits, bn):
     W = _bf16((n_out, K), 1, 0.05)
@@ -156,12 +157,13 @@ def test_embed_rows_rejects_token_ids_outside_the_vocabulary():
 # ------------------------------------------------------------------ QKV + RoPE, SwiGLU
 
 @pytest.mark.parametrize("hq,hkv,hd,rows,splits", [(4, 4, 64, 9, 0), (8, 2, 128, 37, 1), (28, 4, 128, 5, 3),
-                                                   (8, 2, 128, 100, 0), (28, 4, 128, 180, 0)])
+                                                   (8, 2, 128, 100, 0), (28, 4, 128, 180, 0),
+                                                   (8, 2, 128, 600, 0)])
 def test_qkv_rope_and_cache_scatter(hq, hkv, hd, rows, splits):
     d = 512 if hq * hd <= 1024 else 3584
     dims = ModelDims(n_layers=1, d_model=d, n_heads=hq, n_kv_heads=hkv, head_dim=hd, ffn_dim=256, vocab=256,
                      mask_id=255, rope_theta=10000.0)
-    B, N = 2, 96
+    B, N = 2, max(96, rows)
     W = _bf16((dims.qkv_dim, d), 12, 0.03)
     X = _bf16((rows, d), 13)
     rng = np.random.default_rng(14)
@@ -215,7 +217,8 @@ def test_qkv_rope_beyond_the_grid_height():
     assert _rowrel(vg.reshape(rows, -1), y[:, dims.q_dim + dims.kv_dim:]) < 1e-2
 
 
-@pytest.mark.parametrize("rows,F,splits", [(3, 256, 0), (40, 1024, 1), (130, 512, 0), (8, 18944 // 4, 2)])
+@pytest.mark.parametrize("rows,F,splits", [(3, 256, 0), (40, 1024, 1), (130, 512, 0), (8, 18944 // 4, 2),
+                                           (400, 512, 0), (700, 256, 0)])
 def test_gate_up_swiglu(rows, F, splits):
     d = 512
     W = _bf16((2 * F, d), 15, 0.04)

@@ -490,11 +490,12 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 
 namespace {
 
-// Activation-tile width.  Up to 768 rows the 128-wide tile: it keeps twice the weight bytes
+// Activation-tile width.  Up to 512 rows the 128-wide tile: it keeps twice the weight bytes
 // in flight per stage (two 64-column k-blocks: 96 KB of weights in the ring against 64 KB at
-// 256 wide), and a 256-wide tile's epilogue (RoPE and K/V scatter, SwiGLU, the residual add)
-// outlasts its MMAs.  Whole 768-row layers, weight tile fastest, eight epilogue warps:
-// 583 us at 128 wide, 594 us at 256 wide; QKV with its RoPE epilogue 120 vs 162 us.
+// 256 wide) and fills more SMs with whole tiles.  Above, the 256-wide tile halves the weight
+// tile rereads and the shared-memory operand traffic per MMA (LLaDA-8B shapes, 128 vs 256 wide:
+// QKV 84 vs 71 us at 640 rows, 88 vs 75 us at 768; gate/up + SwiGLU 147 vs 126 and 156 vs 131 us;
+// the 768-row layer over 2048 positions 452 -> 408 us).  Gate/up goes wide from 385 rows (below).
 int pick_bn(int rows) {
   static const int wide = [] {
     const char* e = getenv("DLLM_GEMM_WIDE_BN");   // A/B switch for measurements: width above 64 rows
@@ -504,7 +505,7 @@ int pick_bn(int rows) {
   if (rows <= 32) return 32;
   if (rows <= 64) return 64;
   if (wide == 128 || wide == 256) return wide;
-  if (rows <= 768) return 128;
+  if (rows <= 512) return 128;
   return 256;
 }
 // Weight tile fastest up to 8 activation tiles (whole 768-row layers: 583 us against 638 us
@@ -605,6 +606,9 @@ int gemm_launch(const GemmArgs& a, const GemmScratch& s, cudaStream_t st, int fo
   // 129-256 rows as one 256-wide activation tile when the caller allows it (QKV at 205 rows:
   // 41.6 -> 32.3 us; gate/up, O and down are not faster that way)
   if (!force_bn && a.wide_ok && bn == 128 && a.rows_cap > 128 && a.rows_cap <= 256) bn = 256;
+  // gate/up + SwiGLU at 385-512 rows: two 256-wide tiles beat three or four 128-wide ones
+  // (512 rows: 115.6 -> 98.3 us; at 384 rows 85.3 against 93.7 us the narrow tile still wins)
+  if (!force_bn && a.swiglu && bn == 128 && a.rows_cap > 384) bn = 256;
   // O and down (residual add): when 128-wide tiles outnumber the SMs, so that a CTA takes two
   // or more of them anyway, one 256-wide tile per weight tile instead (768 rows: O 44.6 ->
   // 40.4 us, down 106 -> 90 us; at 384-512 rows the 128-wide tiles fill more SMs and win)
