@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 # DRAM bytes (read + write) per layer of fused_layer_kernel, from one ncu capture of the kernel on three
 # LLaDA-8B-shaped layers (kernel_bench case fused_m7_l3); roofline.traffic scales it by the layers a launch runs
-FUSED_DRAM_BYTES_PER_LAYER = 451.11e6
+FUSED_DRAM_BYTES_PER_LAYER = 451.21e6
 METRIC = "generated tokens/s, LLaDA-8B shape, 1×B200; step latency & roofline % vs active ratio"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
