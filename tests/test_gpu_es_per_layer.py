@@ -176,7 +176,8 @@ def test_fused_per_layer_run_matches_oracle_teacher_forced(w4, batch):
     """dllm_select_layers_forward: on skip steps one persistent launch scores and chooses the
     rows at the start of every layer itself.  With the oracle's per-layer scores forced, the
     chosen rows are exact and outputs, confidences and caches agree within tolerance; the
-    scores it computes (the last layer's are kept) agree with Eq. 1 on the score scale."""
+    scores it computes (the last layer's are kept) agree element by element with Eq. 1 evaluated
+    on the GPU's own inputs of that layer."""
     cfg = PL.replace(batch=batch)
     tok0 = make_tokens(cfg)
     orc = OracleRun(cfg, w4, tok0.numpy())
