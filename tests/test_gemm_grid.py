@@ -178,3 +178,24 @@ def test_tile_width_rule():
     assert [width(r, F // 64, d, EPI_SWIGLU) for r in (384, 385, 512)] == [128, 256, 256]
     assert [width(r, d // 128, F, EPI_RESID_ADD) for r in (512, 513)] == [128, 256]
     assert width(384, 64, 8192, EPI_RESID_ADD) == 256          # 64 x 3 = 192 tiles > 148 SMs
+
+
+def test_restated_rule_matches_the_source():
+    """The thresholds restated above are the ones gemm_tc.cu uses (a change there must be
+    carried here, or these checks would test a stale rule)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "token_skip_denoising_b200", "csrc",
+                            "gemm_tc.cu")).read()
+    assert re.search(r"if \(rows <= 512\) return 128;\s*return 256;", src)
+    assert "a.wide_ok && bn == 128 && a.rows_cap > 128 && a.rows_cap <= 256) bn = 256;" in src
+    assert "a.swiglu && bn == 128 && a.rows_cap > 384) bn = 256;" in src
+    assert "a.epi.kind == EPI_RESID_ADD && bn == 128 &&" in src
+    assert "a.epi.kind == EPI_RESID_ADD && bn >= 128 && 2 * tiles <= num_sms();" in src
+    assert "constexpr int kMaxWholePerCta = 4;" in src
+    assert "per > kMaxWholePerCta && 4 * (static_cast<int64_t>(per) * sms - tiles) >= sms" in src
+    assert "std::max(1, std::min(sms / tiles, KB / 32));" in src
+    assert "constexpr int max_ksub(int bn) { return bn <= 64 ? 4 : (bn <= 128 ? 2 : 1); }" in src
+    dev = open(os.path.join(os.path.dirname(__file__), "..", "token_skip_denoising_b200", "csrc",
+                            "gemm_dev.cuh")).read()
+    assert "return T * c / G;" in dev and "((x + 1) * G + T - 1) / T - 1" in dev
