@@ -12,6 +12,8 @@ sweep around them, the property the kernel relies on:
   chunks, for any number of slices;
 * the attention key splits cover every 64-key block once and the query tiles
   every (row, head) unit once;
+* the RoPE step's 4-pair items rotate every (low, high) pair of a row once,
+  inside one head, with their vector loads and stores aligned;
 * choosing the k candidates whose rank (higher score first, ties to the lower
   position) is below k picks the same set, in ascending positions, as the
   selection kernel's rule "the k highest scores, ties to the lower position"
@@ -154,3 +156,49 @@ def test_rank_count_choice_is_the_selection_rule(seed):
         assert got == want
     else:
         assert got == stable_topk(s, k)
+
+
+def rope_items(qkvd, hd):
+    """The fused kernel's RoPE items of one row: item rr covers pairs pi..pi+3 of head rr / (hd/8),
+    element nlo (low half) and nlo + hd/2 (high half) of the row's QKV sums."""
+    half, groups, gph = hd // 2, qkvd >> 3, (hd // 2) >> 2
+    out = []
+    for rr in range(groups):
+        head = rr // gph
+        pi = (rr - head * gph) * 4
+        out.append((head * hd + pi, pi))
+    return out, half
+
+
+@pytest.mark.parametrize("Hq,Hkv,hd", [(4, 4, 64), (8, 2, 128), (28, 4, 128), (32, 32, 128), (4, 2, 64)])
+def test_rope_items_cover_each_pair_once_aligned(Hq, Hkv, hd):
+    """Every (low, high) element pair of a row is rotated exactly once; a 4-pair item never
+    crosses a head, and its 16-byte loads (fp32 sums, cos/sin rows) and 8-byte stores (bf16 q and
+    cache rows) start on their alignment for every row and position."""
+    qd, kvd = Hq * hd, Hkv * hd
+    qkvd = qd + 2 * kvd
+    items, half = rope_items(qkvd, hd)
+    seen = np.zeros(qkvd, dtype=int)
+    for nlo, pi in items:
+        assert nlo % 4 == 0 and pi % 4 == 0 and pi + 3 < half
+        assert nlo // hd == (nlo + half + 3) // hd          # both halves in one head
+        for k in range(4):
+            seen[nlo + k] += 1
+            seen[nlo + half + k] += 1
+        # q / K / V destination: the slot holds whole heads, so the 4 lanes stay in one of them
+        seg = 0 if nlo < qd else (1 if nlo < qd + kvd else 2)
+        assert seg == (0 if nlo + half + 3 < qd else (1 if nlo + half + 3 < qd + kvd else 2))
+    assert np.all(seen == 1)
+    # byte offsets of a row's first element are multiples of the row pitches: fp32 qkvd, bf16 qd,
+    # the cache row hd; with those, element offsets that are multiples of 4 keep the alignment
+    assert (qkvd * 4) % 16 == 0 and (qd * 2) % 8 == 0 and (hd * 2) % 8 == 0 and (half * 4) % 16 == 0
+
+
+def test_rope_items_match_the_kernel_source():
+    import os
+    src = open(os.path.join(os.path.dirname(__file__), "..", "token_skip_denoising_b200", "csrc",
+                            "fused_layer.cu")).read()
+    assert "const int groups = p.qkvd >> 3;" in src and "const int gph = half >> 2;" in src
+    assert "const int head = rr / gph;" in src and "pis[e] = (rr - head * gph) * 4;" in src
+    assert "nlo[e] = head * p.hd + pis[e];" in src
+    assert "if (a.hd % 8 || reinterpret_cast<uintptr_t>(a.rope_cos) % 16" in src
