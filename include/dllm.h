@@ -425,7 +425,8 @@ int dllm_op_gemm_noalloc(int32_t kind, const void* W, int32_t n_out, const void*
  * rows (b, :, pos) of rows_map[j] = b * N + pos.  W = one layer of w_qkv.  The products are
  * kept in fp32 in the workspace (rows_cap * (Hq + 2 Hkv) * hd * 4 bytes after the GEMM
  * scratch; DLLM_ERR_SHAPE when it does not fit) and one coalesced pass rotates and
- * scatters them; head_dim a power of two. */
+ * scatters them; head_dim a power of two.  rope_cos / rope_sin 16-byte aligned, q_out and
+ * the caches 8-byte aligned, else DLLM_ERR_INVALID_ARG. */
 int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32_t* count, int32_t d,
                      int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t N, const int32_t* rows_map,
                      const float* rope_cos, const float* rope_sin, void* q_out, void* kcache, void* vcache,

@@ -79,6 +79,18 @@ def test_null_arguments_are_rejected_without_a_gpu(lib):
     assert lib.dllm_op_select(None, 1, 4, 0, 2, 0.0, 0, 4, None, None, 0, None, None, None, None) == 1
 
 
+def test_qkv_rope_rejects_misaligned_tables_and_caches_before_any_launch(lib):
+    # the RoPE pass moves 16-byte table rows and 8-byte groups of q / cache elements; the op
+    # checks the caller's pointers on the host first (these addresses are never dereferenced)
+    base = 1 << 20
+    args = lambda cos, kc: (base, base, 16, None, 256, 4, 4, 64, 32, base, cos, base, base, kc, base, 0,
+                            base, 1 << 24, None)
+    assert lib.dllm_op_qkv_rope(*args(base + 8, base)) == 1       # cos table on an 8-byte boundary
+    assert lib.dllm_op_qkv_rope(*args(base, base + 2)) == 1       # K cache on a 2-byte boundary
+    ok = args(base, base)
+    assert lib.dllm_op_qkv_rope(*ok[:5], 1, *ok[6:]) == 2          # one 64-wide q head: not a multiple of 128
+
+
 def test_per_layer_selection_needs_a_layer_after_the_skip_layer(lib):
     run = get_config("tiny").replace(es_per_layer=True)
     sb, wb = ctypes.c_size_t(), ctypes.c_size_t()

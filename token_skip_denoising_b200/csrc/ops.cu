@@ -106,6 +106,9 @@ int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32
   if (head_dim != 64 && head_dim != 128) OP_FAIL(DLLM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   const int qd = n_heads * head_dim, kvd = n_kv_heads * head_dim;
   if (qd % 128 || kvd % 128 || d % 64) OP_FAIL(DLLM_ERR_SHAPE, "q / kv widths must be multiples of 128");
+  if ((reinterpret_cast<uintptr_t>(rope_cos) | reinterpret_cast<uintptr_t>(rope_sin)) % 16 ||
+      (reinterpret_cast<uintptr_t>(q_out) | reinterpret_cast<uintptr_t>(kcache) | reinterpret_cast<uintptr_t>(vcache)) % 8)
+    OP_FAIL(DLLM_ERR_INVALID_ARG, "cos/sin tables must be 16-byte aligned, q and the caches 8-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int qkvd = qd + 2 * kvd;
   OpCarver cv(workspace, workspace_bytes);

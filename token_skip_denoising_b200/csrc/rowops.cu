@@ -729,10 +729,18 @@ int rope_scatter_launch(const float* y, int rows_cap, const int* count_dev, cons
   if (rows_cap <= 0) return DLLM_OK;
   int hd_log2 = 0;
   while ((1 << hd_log2) < hd) ++hd_log2;
-  if (hd < 8 || (1 << hd_log2) != hd || qd % hd || kvd % hd || qkvd != qd + 2 * kvd) return DLLM_ERR_SHAPE;
-  if (reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(rope_cos) % 16 ||
-      reinterpret_cast<uintptr_t>(rope_sin) % 16)
+  if (hd < 8 || (1 << hd_log2) != hd || qd % hd || kvd % hd || qkvd != qd + 2 * kvd) {
+    set_last_error("rope_scatter: head_dim a power of two >= 8, q/kv widths whole heads", __FILE__, __LINE__);
+    return DLLM_ERR_SHAPE;
+  }
+  // 16-byte loads of the fp32 products and of the cos/sin rows, 8-byte stores of 4 bf16 values
+  if ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(rope_cos) |
+       reinterpret_cast<uintptr_t>(rope_sin)) % 16 ||
+      (reinterpret_cast<uintptr_t>(q_out) | reinterpret_cast<uintptr_t>(kc) | reinterpret_cast<uintptr_t>(vc)) % 8) {
+    set_last_error("rope_scatter: products and cos/sin tables 16-byte aligned, q and caches 8-byte aligned",
+                   __FILE__, __LINE__);
     return DLLM_ERR_INVALID_ARG;
+  }
   const int per_row = qkvd >> 3;
   return launch_pdl(rope_scatter_kernel, dim3((per_row + 255) / 256, std::min(rows_cap, 65535)), dim3(256), 0, st, y, rows_cap,
                     count_dev, row_map, qkvd, qd, kvd, hd_log2, N, Hkv, rope_cos, rope_sin, q_out, kc, vc);
