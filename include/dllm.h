@@ -164,8 +164,9 @@ int dllm_state_bytes(const dllm_config* cfg, size_t* state_bytes, size_t* worksp
  * The start of a generation as the pages describe it: the prompt is followed
  * by masked positions that the iterations unmask (ES-dLLM sec. 1; Plan for
  * Speed sec. 2, blocks generated in order).  state / workspace must hold the
- * sizes dllm_state_bytes gives, 256-byte aligned, else DLLM_ERR_INVALID_ARG;
- * every pointer must stay valid until dllm_destroy.  Synchronises `stream`
+ * sizes dllm_state_bytes gives, 256-byte aligned, every weight pointer 16-byte
+ * aligned and tokens 4-byte aligned, else DLLM_ERR_INVALID_ARG (checked before
+ * anything is enqueued); every pointer must stay valid until dllm_destroy.  Synchronises `stream`
  * once (the host copy of the DUS round masks must outlive its upload). */
 int dllm_step_init(dllm_handle** out, const dllm_config* cfg, const dllm_weights* w, void* state, void* workspace,
                    int32_t* tokens, void* stream);
@@ -379,7 +380,13 @@ void dllm_destroy(dllm_handle* h);
  * `workspace` (where taken) is caller scratch: zero it before its first use;
  * its first 256 KB hold GEMM tile counters that every call leaves at zero, so
  * calls on one stream may share it; calls that overlap on the GPU may not.
- * After dllm_device_status reports DLLM_DEV_TIMEOUT, zero it again.  */
+ * After dllm_device_status reports DLLM_DEV_TIMEOUT, zero it again.
+ * Alignment (the kernels move 16-byte vectors): workspaces 256-byte aligned;
+ * embedding tables, fp32 rows (h, h_prev, gains), caches, q and attention
+ * outputs and RoPE tables 16-byte aligned; bf16 outputs written 4 values at a
+ * time (RMSNorm z, q and cache rows of the QKV op) 8-byte aligned.  A pointer
+ * that misses its alignment is refused with DLLM_ERR_INVALID_ARG before
+ * anything is launched.  */
 
 /* RoPE tables cos/sin fp32 [N, hd/2] with angle pos * theta^(-2i/hd). */
 int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, double theta, void* stream);
@@ -495,7 +502,9 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
                   int32_t rows_cap, int32_t rows_per_seq_cap, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes dllm_op_layer needs for rows_cap rows (zero it before its first use;
- * the GEMM tile counters at its start are left at zero by every call). */
+ * the GEMM tile counters at its start are left at zero by every call).  dllm_op_layer
+ * takes its weights, gains, caches, RoPE tables and h 16-byte aligned and the workspace
+ * 256-byte aligned, else DLLM_ERR_INVALID_ARG. */
 int dllm_op_layer_workspace(const dllm_config* cfg, int32_t rows_cap, int32_t rows_per_seq_cap, size_t* bytes);
 
 #ifdef __cplusplus

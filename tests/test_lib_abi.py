@@ -91,6 +91,31 @@ def test_qkv_rope_rejects_misaligned_tables_and_caches_before_any_launch(lib):
     assert lib.dllm_op_qkv_rope(*ok[:5], 1, *ok[6:]) == 2          # one 64-wide q head: not a multiple of 128
 
 
+def test_misaligned_operands_are_refused_before_any_launch(lib):
+    # every kernel moves 16-byte (some 8-byte) vectors; each entry point checks the caller's
+    # pointers on the host first, so these addresses are never dereferenced
+    A = 1 << 20                                   # a 256-byte aligned stand-in address
+    assert lib.dllm_op_embed_rows(A, 1024, A, A, None, 4, 256, A + 4, None) == 1
+    assert lib.dllm_op_embed_rows(A + 8, 1024, A, A, None, 4, 256, A, None) == 1
+    assert lib.dllm_op_rmsnorm_rows(A, A, None, 4, 256, A, 1e-5, A + 2, None) == 1
+    assert lib.dllm_op_rmsnorm_rows(A, A, None, 4, 256, A + 4, 1e-5, A, None) == 1
+    assert lib.dllm_op_score_es(A, A + 4, A, None, None, 0, None, 4, 256, 0.5, 0, A, None) == 1
+    assert lib.dllm_op_attention(A + 8, A, A, A, A, 1, 4, 4, 64, 4, 4, 128, 1, A, 1 << 20, None) == 1
+    assert lib.dllm_op_attention(A, A, A + 2, A, A, 1, 4, 4, 64, 4, 4, 128, 1, A, 1 << 20, None) == 1
+    assert lib.dllm_op_gemm(0, A, 128, A, 4, None, 256, A, None, 0, 0, A + 16, 1 << 24, None) == 1
+    cfg = _lib.make_config(get_config("tiny"))
+    op = lambda kc, ws: lib.dllm_op_layer(ctypes.byref(cfg), A, A, A, A, A, A, kc, A, A, A, A, A, A, A, 4, 4,
+                                          ws, 1 << 30, None)
+    assert op(A + 8, A) == 1                      # K cache on an 8-byte boundary
+    assert op(A, A + 16) == 1                     # workspace not 256-byte aligned
+    w = _lib.DllmWeights(A, A, A, A + 2, A, A, A, A, A)
+    h = ctypes.c_void_p()
+    assert lib.dllm_step_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(w), A, A, A, None) == 1
+    w = _lib.DllmWeights(A, A, A, A, A, A, A, A, A)
+    assert lib.dllm_step_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(w), A, A, A + 2, None) == 1
+    assert not h.value                            # no handle was made
+
+
 def test_per_layer_selection_needs_a_layer_after_the_skip_layer(lib):
     run = get_config("tiny").replace(es_per_layer=True)
     sb, wb = ctypes.c_size_t(), ctypes.c_size_t()

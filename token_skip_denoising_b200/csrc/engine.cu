@@ -748,6 +748,11 @@ int dllm_step_init(dllm_handle** out, const dllm_config* cfg, const dllm_weights
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null weight pointer");
   if ((reinterpret_cast<uintptr_t>(state) | reinterpret_cast<uintptr_t>(workspace)) & 255)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "state and workspace must be 256-byte aligned");
+  // the kernels read weights and gains as 16-byte vectors (and through TMA)
+  const void* wp[9] = {w->embed, w->lm_head, w->w_qkv, w->w_o, w->w_gu, w->w_down, w->g_attn, w->g_ffn, w->g_final};
+  for (const void* p : wp)
+    if (reinterpret_cast<uintptr_t>(p) & 15) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "weights must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(tokens) & 3) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "tokens must be 4-byte aligned");
   dllm_handle* x = new (std::nothrow) dllm_handle();
   if (!x) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "out of host memory");
   fill_dims(x, cfg);
@@ -1237,6 +1242,13 @@ int dllm_op_layer(const dllm_config* cfg, const void* w_qkv, const void* w_o, co
   if (!w_qkv || !w_o || !w_gu || !w_down || !g_attn || !g_ffn || !kcache || !vcache || !rope_cos || !rope_sin || !h ||
       !rows || !seq_off || !workspace)
     DLLM_FAIL(DLLM_ERR_INVALID_ARG, "null argument");
+  {
+    // 16-byte vector and TMA access to the weights, gains, caches, tables and h
+    const void* ap[11] = {w_qkv, w_o, w_gu, w_down, g_attn, g_ffn, kcache, vcache, rope_cos, rope_sin, h};
+    for (const void* p : ap)
+      if (reinterpret_cast<uintptr_t>(p) & 15) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "layer operands must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) DLLM_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
   size_t need = 0;
   DLLM_TRY(dllm_op_layer_workspace(cfg, rows_cap, rows_per_seq_cap, &need));
   if (workspace_bytes < need) DLLM_FAIL(DLLM_ERR_SHAPE, "workspace too small for the layer");

@@ -1,6 +1,8 @@
 // C ABI of single kernels (dllm_op_*): argument checks, workspace carving and
 // one launch each.  Used by the parity tests and the single-layer benchmark.
 #include <algorithm>
+#include <cstdint>
+#include <initializer_list>
 #include <vector>
 
 #include "common.cuh"
@@ -34,6 +36,13 @@ struct OpCarver {
 // Scratch of one GEMM launched through an op: the tile counters live at the start of the
 // workspace (the caller zeroes the workspace once; every GEMM leaves its counters at zero),
 // the partial tiles of split work follow.
+// Whether every pointer is a multiple of `a` bytes: the kernels move 16-byte (and 8-byte) vectors.
+bool aligned_to(size_t a, std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (reinterpret_cast<uintptr_t>(q) % a) return false;
+  return true;
+}
+
 constexpr int kOpCounters = 65536;
 
 int gemm_scratch(OpCarver& cv, int rows_cap, int tiles, int K, GemmScratch& gs) {
@@ -62,6 +71,7 @@ int dllm_op_embed_rows(const void* embed, int32_t vocab, const int32_t* tokens, 
                        const int32_t* count, int32_t rows_cap, int32_t d, float* h, void* stream) {
   if (!embed || !tokens || !rows || !h || rows_cap < 0 || d <= 0 || vocab <= 0)
     OP_FAIL(DLLM_ERR_INVALID_ARG, "bad embed args");
+  if (!aligned_to(16, {embed, h})) OP_FAIL(DLLM_ERR_INVALID_ARG, "embedding table and h must be 16-byte aligned");
   return embed_rows_launch(static_cast<const __nv_bfloat16*>(embed), vocab, tokens, rows, count, rows_cap, d, h,
                            static_cast<cudaStream_t>(stream));
 }
@@ -69,6 +79,8 @@ int dllm_op_embed_rows(const void* embed, int32_t vocab, const int32_t* tokens, 
 int dllm_op_rmsnorm_rows(const float* h, const int32_t* rows, const int32_t* count, int32_t rows_cap, int32_t d,
                          const float* g, float eps, void* z, void* stream) {
   if (!h || !g || !z || rows_cap < 0 || d <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad rmsnorm args");
+  if (!aligned_to(16, {h, g}) || !aligned_to(8, {z}))
+    OP_FAIL(DLLM_ERR_INVALID_ARG, "h and g must be 16-byte aligned, z 8-byte aligned");
   return rmsnorm_rows_launch(h, rows, count, rows_cap, d, g, eps, static_cast<__nv_bfloat16*>(z), d,
                              static_cast<cudaStream_t>(stream));
 }
@@ -81,6 +93,7 @@ int dllm_op_gemm(int32_t kind, const void* W, int32_t n_out, const void* X, int3
   if (kind != EPI_STORE_F32 && kind != EPI_STORE_BF16 && kind != EPI_RESID_ADD)
     OP_FAIL(DLLM_ERR_INVALID_ARG, "kind must be 0, 1 or 3");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!aligned_to(256, {workspace})) OP_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
   const int rc = gemm_scratch(cv, rows_cap, n_out / 128, K, gs);
@@ -106,11 +119,11 @@ int dllm_op_qkv_rope(const void* W, const void* X, int32_t rows_cap, const int32
   if (head_dim != 64 && head_dim != 128) OP_FAIL(DLLM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   const int qd = n_heads * head_dim, kvd = n_kv_heads * head_dim;
   if (qd % 128 || kvd % 128 || d % 64) OP_FAIL(DLLM_ERR_SHAPE, "q / kv widths must be multiples of 128");
-  if ((reinterpret_cast<uintptr_t>(rope_cos) | reinterpret_cast<uintptr_t>(rope_sin)) % 16 ||
-      (reinterpret_cast<uintptr_t>(q_out) | reinterpret_cast<uintptr_t>(kcache) | reinterpret_cast<uintptr_t>(vcache)) % 8)
+  if (!aligned_to(16, {rope_cos, rope_sin}) || !aligned_to(8, {q_out, kcache, vcache}))
     OP_FAIL(DLLM_ERR_INVALID_ARG, "cos/sin tables must be 16-byte aligned, q and the caches 8-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int qkvd = qd + 2 * kvd;
+  if (!aligned_to(256, {workspace})) OP_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
   const int rc = gemm_scratch(cv, rows_cap, qkvd / 128, d, gs);
@@ -133,6 +146,7 @@ int dllm_op_gate_up(const void* W, int32_t F, const void* X, int32_t rows_cap, c
   if (!W || !X || !act || rows_cap <= 0 || F <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad gate_up args");
   if (F % 64 || d % 64) OP_FAIL(DLLM_ERR_SHAPE, "F and d must be multiples of 64");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!aligned_to(256, {workspace})) OP_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
   const int rc = gemm_scratch(cv, rows_cap, F / 64, d, gs);
@@ -149,6 +163,8 @@ int dllm_op_attention(const void* q, const void* kcache, const void* vcache, voi
                       int32_t n_kv_heads, int32_t head_dim, int32_t splits, void* workspace, size_t workspace_bytes,
                       void* stream) {
   if (!q || !kcache || !vcache || !out || !seq_off) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad attention args");
+  if (!aligned_to(16, {q, kcache, vcache, out}))
+    OP_FAIL(DLLM_ERR_INVALID_ARG, "q, the caches and out must be 16-byte aligned");
   if (n_kv_heads <= 0 || n_heads % n_kv_heads) OP_FAIL(DLLM_ERR_SHAPE, "n_heads must be a multiple of n_kv_heads");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = n_heads / n_kv_heads;
@@ -159,6 +175,7 @@ int dllm_op_attention(const void* q, const void* kcache, const void* vcache, voi
   int nctr = 0;
   size_t pf = 0;
   if (sp > 1) {
+    if (!aligned_to(256, {workspace})) OP_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     OpCarver cv(workspace, workspace_bytes);
     nctr = attn_counters_needed(B, n_kv_heads, G, rows_per_seq_cap);
     ctr = cv.take<int>(kOpCounters);        // the zeroed counter region at the workspace start
@@ -179,6 +196,7 @@ int dllm_op_lm_head(const void* W, int32_t V, const void* X, int32_t rows_cap, c
   if (!W || !X || rows_cap <= 0 || V <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad lm_head args");
   if (V % 128 || d % 64) OP_FAIL(DLLM_ERR_SHAPE, "V must be a multiple of 128 and d of 64");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!aligned_to(256, {workspace})) OP_FAIL(DLLM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   OpCarver cv(workspace, workspace_bytes);
   GemmScratch gs;
   const int rc = gemm_scratch(cv, rows_cap, V / 128, d, gs);
@@ -198,6 +216,7 @@ int dllm_op_score_es(const float* h, float* h_prev, const float* conf, uint8_t* 
                      float* score, void* stream) {
   if (!h || !h_prev || !conf || !score || n_rows < 0 || d <= 0) OP_FAIL(DLLM_ERR_INVALID_ARG, "bad score_es args");
   if (update && (!masked_prev || !tokens)) OP_FAIL(DLLM_ERR_INVALID_ARG, "update needs masked_prev and tokens");
+  if (!aligned_to(16, {h, h_prev})) OP_FAIL(DLLM_ERR_INVALID_ARG, "h and h_prev must be 16-byte aligned");
   // without a previous-layer choice (act_prev null) the kernel only reads h
   return score_es_launch(const_cast<float*>(h), h_prev, conf, masked_prev, tokens, mask_id, rows, n_rows, d, alpha,
                          update, nullptr, score, static_cast<cudaStream_t>(stream));
