@@ -386,9 +386,9 @@ void dllm_destroy(dllm_handle* h);
  * outputs and RoPE tables 16-byte aligned; bf16 outputs written 4 values at a
  * time (RMSNorm z, q and cache rows of the QKV op) 8-byte aligned.  A pointer
  * that misses its alignment is refused with DLLM_ERR_INVALID_ARG before
- * anything is launched.  Device-resident index arrays (rows, rows_map, seq_off,
- * counts) are read by the kernels as given, apart from token ids: each index
- * must lie inside the buffer it addresses.  */
+ * anything is launched.  Device-resident index arrays (rows, rows_map, seq_off)
+ * are read by the kernels as given: each index must lie inside the buffer it
+ * addresses (device counts are clamped to rows_cap, token ids are checked).  */
 
 /* RoPE tables cos/sin fp32 [N, hd/2] with angle pos * theta^(-2i/hd). */
 int dllm_op_rope_table(float* cos_t, float* sin_t, int32_t N, int32_t head_dim, double theta, void* stream);
